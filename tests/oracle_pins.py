@@ -1,0 +1,330 @@
+"""Pins that tie the fp64 oracle to what the pages and the mathematics fix.
+
+Each ``pin_*`` function takes the oracle module (``oracle.infini_ref`` or a
+deliberately broken copy of it) and returns a list of failure messages
+(empty when the pin holds).  ``test_oracle.py`` runs them against the real
+oracle; ``test_oracle_mutations.py`` plants plausible mistakes in the oracle
+and checks that at least one pin catches each.
+
+Sources, all on the explainer page "Leave No Context Behind: Efficient
+Infinite Context Transformers with Infini-attention" (section 3, Technical
+Approach) unless stated: Eq. 6 (local causal attention), Eq. 7 (retrieval),
+the closed forms of M_{s-1} and z_{s-1}, Eq. 8 / Eq. 9 (updates), Eq. 10
+(gate), Eq. 4 (recurrent contract), the delta rule's "binding already
+exists" property (also on the paperlayer.ai summary, section 3), and the
+per-layer footprint of d_key x d_value + d_key per head.
+"""
+
+from __future__ import annotations
+
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import torch
+
+from oracle import brute
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _expr(s: str) -> float:
+    """Evaluate a golden-file input expression built from numbers, ln(), sqrt() and unary minus."""
+    return float(eval(s, {"__builtins__": {}}, {"ln": math.log, "sqrt": math.sqrt}))
+
+
+def _frac(s: str) -> float:
+    return float(Fraction(s))
+
+
+def _rand(shape, seed, scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return (scale * torch.randn(*shape, generator=g, dtype=torch.float64)).numpy()
+
+
+def _close(a, b, tol, what):
+    a, b = np.asarray(a, np.float64), np.asarray(b, np.float64)
+    if a.shape != b.shape:
+        return [f"{what}: shape {a.shape} vs {b.shape}"]
+    if not np.all(np.isfinite(a)):
+        return [f"{what}: non-finite values"]
+    err = float(np.max(np.abs(a - b))) if a.size else 0.0
+    return [] if err <= tol else [f"{what}: max abs err {err:.3e} > {tol:.1e}"]
+
+
+# ---------------------------------------------------------------------------
+def pin_hand_examples(ref):
+    """Hand-derived worked examples (tests/golden/hand_examples.json)."""
+    with open(os.path.join(GOLDEN, "hand_examples.json")) as f:
+        data = json.load(f)
+    fails = []
+    for ex in data["examples"]:
+        q = np.array([[_expr(x) for x in row] for row in ex["q"]])[None, None]
+        k = np.array([[_expr(x) for x in row] for row in ex["k"]])[None, None]
+        v = np.array([[_expr(x) for x in row] for row in ex["v"]])[None, None]
+        beta = np.array([_expr(ex["beta"])])
+        want_out = np.array([[_frac(x) for x in row] for row in ex["out"]])
+        for mode, key in ((ref.LINEAR, "linear"), (ref.DELTA, "delta")):
+            out, M, z = ref.forward(q, k, v, beta, ex["N"], mode=mode)
+            fails += _close(out[0, 0], want_out, 1e-12, f"{ex['name']}/{key} out")
+            fails += _close(M[0, 0], np.array([[_frac(x) for x in r] for r in ex[key]["M"]]), 1e-12,
+                            f"{ex['name']}/{key} M")
+            fails += _close(z[0, 0], np.array([_frac(x) for x in ex[key]["z"]]), 1e-12, f"{ex['name']}/{key} z")
+    return fails
+
+
+def pin_sigma(ref):
+    """sigma = ELU + 1 (alpha = 1): identity + 1 above 0, exp at and below 0, continuous, positive."""
+    x = np.array([-30.0, -2.0, -math.log(2.0), -1e-9, 0.0, 1e-9, 0.5, 3.0])
+    want = np.array([math.exp(-30.0), math.exp(-2.0), 0.5, math.exp(-1e-9), 1.0, 1.0 + 1e-9, 1.5, 4.0])
+    fails = _close(ref.elu_plus_one(x), want, 1e-15, "sigma values")
+    if not np.all(ref.elu_plus_one(np.linspace(-50, 50, 1001)) > 0):
+        fails.append("sigma not positive")
+    return fails
+
+
+def pin_gate_zero_is_sdpa(ref):
+    """beta -> -inf gives g = 0: out equals per-segment causal softmax attention
+    computed by torch's scaled_dot_product_attention in float64 (Eq. 6, Eq. 10)."""
+    fails = []
+    B, H, L, dk, dv = 2, 3, 23, 8, 5
+    q, k, v = _rand((B, H, L, dk), 1), _rand((B, H, L, dk), 2), _rand((B, H, L, dv), 3)
+    beta = np.full(H, -np.inf)
+    for N in (L, 7, 4, 1):
+        scale = 1.0 / math.sqrt(dk)
+        out, _, _ = ref.forward(q, k, v, beta, N, mode=ref.LINEAR)
+        want = np.zeros_like(out)
+        for s0 in range(0, L, N):
+            s1 = min(L, s0 + N)
+            want[:, :, s0:s1] = torch.nn.functional.scaled_dot_product_attention(
+                torch.from_numpy(q[:, :, s0:s1]), torch.from_numpy(k[:, :, s0:s1]),
+                torch.from_numpy(v[:, :, s0:s1]), is_causal=True, scale=scale).numpy()
+        fails += _close(out, want, 1e-12, f"g=0 vs SDPA (N={N})")
+        out_d, _, _ = ref.forward(q, k, v, beta, N, mode=ref.DELTA)
+        fails += _close(out_d, want, 1e-12, f"g=0 delta vs SDPA (N={N})")
+    return fails
+
+
+def pin_linear_closed_form(ref):
+    """Linear rule: M_S = sum_t sigma(k_t)^T v_t and z_S = sum_t sigma(k_t) over every token,
+    hence independent of the segment length N (closed forms under Eq. 7)."""
+    fails = []
+    B, H, L, dk, dv = 1, 2, 24, 6, 4
+    q, k, v = _rand((B, H, L, dk), 4), _rand((B, H, L, dk), 5), _rand((B, H, L, dv), 6)
+    beta = _rand((H,), 7)
+    sk = np.where(k > 0, k + 1.0, np.exp(np.minimum(k, 0)))  # ELU + 1, written out independently
+    want_M = np.einsum("bhti,bhtj->bhij", sk, v)
+    want_z = sk.sum(axis=2)
+    for N in (24, 12, 6, 5, 1):
+        _, M, z = ref.forward(q, k, v, beta, N, mode=ref.LINEAR)
+        fails += _close(M, want_M, 1e-11, f"linear M closed form (N={N})")
+        fails += _close(z, want_z, 1e-11, f"linear z closed form (N={N})")
+    return fails
+
+
+def pin_brute_linear(ref):
+    """Segmentwise oracle == token-by-token normalised linear attention over earlier segments."""
+    fails = []
+    B, H, L, dk, dv = 1, 2, 13, 3, 2
+    q, k, v = _rand((B, H, L, dk), 8), _rand((B, H, L, dk), 9), _rand((B, H, L, dv), 10)
+    beta = _rand((H,), 11)
+    for N in (4, 5):
+        out, M, z = ref.forward(q, k, v, beta, N, mode=ref.LINEAR)
+        bo, bM, bz = brute.forward_linear_closed_form(q.tolist(), k.tolist(), v.tolist(), beta.tolist(), N)
+        fails += _close(out, np.array(bo), 1e-12, f"brute linear out (N={N})")
+        fails += _close(M, np.array(bM), 1e-12, f"brute linear M (N={N})")
+        fails += _close(z, np.array(bz), 1e-12, f"brute linear z (N={N})")
+    # memory read alone: beta -> +inf makes out = A_mem
+    big = np.full(H, np.inf)
+    out, _, _ = ref.forward(q, k, v, big, 4, mode=ref.LINEAR)
+    bo, _, _ = brute.forward_linear_closed_form(q.tolist(), k.tolist(), v.tolist(), big.tolist(), 4)
+    fails += _close(out, np.array(bo), 1e-12, "brute A_mem (g=1)")
+    return fails
+
+
+def pin_brute_delta(ref):
+    """Segmentwise oracle == element-loop evaluation of the delta rule on tiny inputs."""
+    fails = []
+    B, H, L, dk, dv = 1, 2, 11, 3, 2
+    q, k, v = _rand((B, H, L, dk), 12), _rand((B, H, L, dk), 13), _rand((B, H, L, dv), 14)
+    beta = _rand((H,), 15)
+    for N in (3, 4, 11):
+        out, M, z = ref.forward(q, k, v, beta, N, mode=ref.DELTA)
+        bo, bM, bz = brute.forward_delta_loops(q.tolist(), k.tolist(), v.tolist(), beta.tolist(), N)
+        fails += _close(out, np.array(bo), 1e-12, f"brute delta out (N={N})")
+        fails += _close(M, np.array(bM), 1e-12, f"brute delta M (N={N})")
+        fails += _close(z, np.array(bz), 1e-12, f"brute delta z (N={N})")
+    return fails
+
+
+def pin_delta_fixed_point(ref):
+    """Delta rule leaves M unchanged when V already equals what the memory returns for K,
+    while z still grows by sum_t sigma(K_t)."""
+    fails = []
+    dk, dv, n = 5, 4, 9
+    M0 = _rand((dk, dv), 16)
+    z0 = np.abs(_rand((dk,), 17)) + 3.0
+    Ks = _rand((n, dk), 18)
+    sk = np.where(Ks > 0, Ks + 1.0, np.exp(np.minimum(Ks, 0)))
+    Vs = (sk @ M0) / (sk @ z0)[:, None]
+    M1, z1 = ref.delta_update(M0, z0, ref.elu_plus_one(Ks), Vs)
+    fails += _close(M1, M0, 1e-12, "delta fixed point M")
+    fails += _close(z1, z0 + sk.sum(axis=0), 1e-12, "delta fixed point z")
+    # and through the full segment recurrence with a non-empty starting memory
+    q = _rand((1, 1, n, dk), 19)
+    _, M2, z2 = ref.forward(q, Ks[None, None], Vs[None, None], np.zeros(1), n, mode=ref.DELTA,
+                            M0=M0[None, None], z0=z0[None, None])
+    fails += _close(M2[0, 0], M0, 1e-12, "delta fixed point via forward M")
+    fails += _close(z2[0, 0], z0 + sk.sum(axis=0), 1e-12, "delta fixed point via forward z")
+    return fails
+
+
+def pin_delta_first_segment(ref):
+    """From empty memory, one segment of the delta rule equals the linear rule: M = sigma(K)^T V."""
+    fails = []
+    n, dk, dv = 7, 4, 3
+    q, k, v = _rand((1, 1, n, dk), 20), _rand((1, 1, n, dk), 21), _rand((1, 1, n, dv), 22)
+    sk = np.where(k > 0, k + 1.0, np.exp(np.minimum(k, 0)))[0, 0]
+    for mode in (ref.LINEAR, ref.DELTA):
+        _, M, z = ref.forward(q, k, v, np.zeros(1), n, mode=mode)
+        fails += _close(M[0, 0], sk.T @ v[0, 0], 1e-12, f"first segment M (mode {mode})")
+        fails += _close(z[0, 0], sk.sum(axis=0), 1e-12, f"first segment z (mode {mode})")
+    return fails
+
+
+def pin_gate_extremes(ref):
+    """g = 1 gives pure memory (0 in the first segment); g = 1/2 averages A_mem and A_dot (Eq. 10)."""
+    fails = []
+    B, H, L, dk, dv, N = 1, 2, 12, 4, 4, 4
+    q, k, v = _rand((B, H, L, dk), 23), _rand((B, H, L, dk), 24), _rand((B, H, L, dv), 25)
+    for mode in (ref.LINEAR, ref.DELTA):
+        out1, _, _ = ref.forward(q, k, v, np.full(H, np.inf), N, mode=mode)
+        out0, _, _ = ref.forward(q, k, v, np.full(H, -np.inf), N, mode=mode)
+        outh, _, _ = ref.forward(q, k, v, np.zeros(H), N, mode=mode)
+        fails += _close(out1[:, :, :N], np.zeros((B, H, N, dv)), 0.0, "g=1 first segment")
+        fails += _close(outh, 0.5 * (out0 + out1), 1e-12, "g=1/2 average")
+        if np.max(np.abs(out1[:, :, N:])) == 0.0:
+            fails.append("g=1 later segments are all zero")
+    return fails
+
+
+def pin_streaming_resume(ref):
+    """Eq. 4 contract: forward(L) == S single-segment steps == forward(L1) then forward(L - L1)."""
+    fails = []
+    B, H, L, dk, dv, N = 2, 2, 20, 4, 3, 5
+    q, k, v = _rand((B, H, L, dk), 26), _rand((B, H, L, dk), 27), _rand((B, H, L, dv), 28)
+    beta = _rand((H,), 29)
+    for mode in (ref.LINEAR, ref.DELTA):
+        out, M, z = ref.forward(q, k, v, beta, N, mode=mode)
+        Ms, zs = np.zeros((B, H, dk, dv)), np.zeros((B, H, dk))
+        outs = []
+        for s0 in range(0, L, N):
+            o, Ms, zs = ref.segment_step(q[:, :, s0:s0 + N], k[:, :, s0:s0 + N], v[:, :, s0:s0 + N], beta, Ms, zs,
+                                         mode=mode)
+            outs.append(o)
+        fails += _close(np.concatenate(outs, axis=2), out, 1e-12, f"streaming out (mode {mode})")
+        fails += _close(Ms, M, 1e-12, f"streaming M (mode {mode})")
+        L1 = 10
+        o1, M1, z1 = ref.forward(q[:, :, :L1], k[:, :, :L1], v[:, :, :L1], beta, N, mode=mode)
+        o2, M2, z2 = ref.forward(q[:, :, L1:], k[:, :, L1:], v[:, :, L1:], beta, N, mode=mode, M0=M1, z0=z1)
+        fails += _close(np.concatenate([o1, o2], axis=2), out, 1e-12, f"resume out (mode {mode})")
+        fails += _close(M2, M, 1e-12, f"resume M (mode {mode})")
+        fails += _close(z2, z, 1e-12, f"resume z (mode {mode})")
+    return fails
+
+
+def pin_head_permutation(ref):
+    """Heads are independent (multi-head section, Eq. 11): permuting heads permutes outputs and state."""
+    B, H, L, dk, dv, N = 1, 4, 9, 3, 3, 4
+    q, k, v = _rand((B, H, L, dk), 30), _rand((B, H, L, dk), 31), _rand((B, H, L, dv), 32)
+    beta = _rand((H,), 33)
+    perm = np.array([2, 0, 3, 1])
+    fails = []
+    for mode in (ref.LINEAR, ref.DELTA):
+        out, M, z = ref.forward(q, k, v, beta, N, mode=mode)
+        po, pM, pz = ref.forward(q[:, perm], k[:, perm], v[:, perm], beta[perm], N, mode=mode)
+        fails += _close(po, out[:, perm], 1e-13, f"permuted heads (mode {mode})")
+        fails += _close(pM, M[:, perm], 1e-13, f"permuted heads M (mode {mode})")
+    return fails
+
+
+def pin_state_size(ref):
+    """Memory of H (d_key d_value + d_key) numbers per layer, independent of L; the page's figures."""
+    with open(os.path.join(GOLDEN, "memory_footprint.json")) as f:
+        g = json.load(f)
+    fails = []
+    n = ref.state_numbers(g["H"], g["dk"], g["dv"])
+    if n != g["matrix_numbers_per_layer"] + g["normaliser_numbers_per_layer"]:
+        fails.append(f"state numbers {n}")
+    total = n * g["layers"] / 1e6
+    if abs(total - g["total_memory_parameters_millions_approx"]) > 0.05:
+        fails.append(f"12-layer total {total}M")
+    if abs(n * 4 / 2**20 - g["fp32_bytes_per_layer_approx_MB"]) > 0.01:
+        fails.append("fp32 bytes per layer")
+    ratio = g["memorizing_transformer_memory_parameters_millions"] / g["total_memory_parameters_millions_approx"]
+    if round(ratio) != g["compression_vs_memorizing_transformer_approx"]:
+        fails.append(f"compression ratio {ratio}")
+    if len(ref.segment_bounds(g["training_length"], g["segment_length"])) != g["segments_per_training_sequence"]:
+        fails.append("segments per training sequence")
+    # state shapes after forwards of different lengths
+    for L in (4, 17, 40):
+        q = _rand((1, 2, L, 3), 34)
+        _, M, z = ref.forward(q, q, q[..., :2], np.zeros(2), 4, mode=ref.DELTA)
+        if M.shape != (1, 2, 3, 2) or z.shape != (1, 2, 3):
+            fails.append(f"state shape depends on L={L}")
+    return fails
+
+
+def pin_tail_segment(ref):
+    """A short last segment is causal inside itself and updates M, z over its own tokens only."""
+    fails = []
+    B, H, L, dk, dv, N = 1, 1, 11, 3, 2, 4
+    q, k, v = _rand((B, H, L, dk), 35), _rand((B, H, L, dk), 36), _rand((B, H, L, dv), 37)
+    beta = _rand((H,), 38)
+    for mode in (ref.LINEAR, ref.DELTA):
+        out, M, z = ref.forward(q, k, v, beta, N, mode=mode)
+        o8, M8, z8 = ref.forward(q[:, :, :8], k[:, :, :8], v[:, :, :8], beta, N, mode=mode)
+        ot, Mt, zt = ref.segment_step(q[:, :, 8:], k[:, :, 8:], v[:, :, 8:], beta, M8, z8, mode=mode)
+        fails += _close(np.concatenate([o8, ot], axis=2), out, 1e-12, f"tail segment out (mode {mode})")
+        fails += _close(Mt, M, 1e-12, f"tail segment M (mode {mode})")
+    return fails
+
+
+def pin_flop_count(ref):
+    """Algorithmic FLOPs: 2(dk+dv) per unmasked (query, key) pair plus 2 dk dv per token for each
+    memory product (2 products for linear, 3 for delta), counted by brute force over the mask."""
+    fails = []
+    for (B, H, L, N, dk, dv) in ((1, 2, 10, 4, 3, 5), (2, 1, 9, 9, 2, 2)):
+        for mode, prods in ((ref.LINEAR, 2), (ref.DELTA, 3)):
+            pairs = 0
+            for s0 in range(0, L, N):
+                n = min(N, L - s0)
+                pairs += sum(1 for i in range(n) for j in range(n) if j <= i)
+            want = B * H * (pairs * 2 * (dk + dv) + L * prods * 2 * dk * dv)
+            got = ref.forward_flops(B, H, L, N, dk, dv, mode)
+            if got != want:
+                fails.append(f"flops {got} != {want}")
+    return fails
+
+
+ALL_PINS = [
+    pin_hand_examples, pin_sigma, pin_gate_zero_is_sdpa, pin_linear_closed_form, pin_brute_linear,
+    pin_brute_delta, pin_delta_fixed_point, pin_delta_first_segment, pin_gate_extremes,
+    pin_streaming_resume, pin_head_permutation, pin_state_size, pin_tail_segment, pin_flop_count,
+]
+
+
+def run_all(ref):
+    """Run every pin; returns {pin name: [failures]} for the pins that failed or raised."""
+    bad = {}
+    for pin in ALL_PINS:
+        try:
+            with np.errstate(all="ignore"):
+                f = pin(ref)
+        except Exception as e:  # a broken oracle may raise instead of returning wrong numbers
+            f = [f"raised {type(e).__name__}: {e}"]
+        if f:
+            bad[pin.__name__] = f
+    return bad
