@@ -1,0 +1,188 @@
+"""ctypes binding of libinfini_attn (argument marshalling only).
+
+Every function here has the name of the C entry point it calls and does no
+arithmetic of its own: it reads shapes, data pointers and the current CUDA
+stream from torch tensors and passes them on.  Importing this module loads
+the in-tree shared library and raises ``ImportError`` when it has not been
+built -- there is no CPU fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from . import DELTA, F32, LINEAR  # noqa: F401
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libinfini_attn.so")
+
+INFINI_OK = 0
+INFINI_ERR_INVALID_ARG = -1
+INFINI_ERR_UNSUPPORTED = -2
+INFINI_ERR_WORKSPACE = -3
+INFINI_ERR_LAUNCH = -4
+INFINI_ERR_TIMEOUT = -5
+INFINI_ERR_DEVICE = -6
+FLAG_FORCE_SIMT = 0x1
+
+EXPORTED = (
+    "infini_attn_forward", "infini_attn_segment_step", "infini_attn_forward_ex", "infini_attn_workspace_size",
+    "infini_attn_error_string", "infini_attn_device_status", "infini_attn_selftest_timeout",
+    "infini_attn_params_size", "infini_attn_path",
+)
+
+
+def _load():
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"libinfini_attn.so is not built ({_LIB_PATH}); run "
+                          "`python -m compressive_memory_transformer_sm_b200.build`")
+    return ctypes.CDLL(_LIB_PATH)
+
+
+lib = _load()
+_vp, _i, _l, _ll = ctypes.c_void_p, ctypes.c_int, ctypes.c_long, ctypes.c_longlong
+lib.infini_attn_forward.argtypes = [_vp] * 7 + [_i, _i, _l, _i, _i, _i, _i, _vp]
+lib.infini_attn_forward.restype = _i
+lib.infini_attn_segment_step.argtypes = [_vp] * 7 + [_i, _i, _i, _i, _i, _i, _vp]
+lib.infini_attn_segment_step.restype = _i
+lib.infini_attn_workspace_size.argtypes = [_i, _i, _l, _i, _i, _i, _i]
+lib.infini_attn_workspace_size.restype = ctypes.c_size_t
+lib.infini_attn_error_string.argtypes = [_i]
+lib.infini_attn_error_string.restype = ctypes.c_char_p
+lib.infini_attn_device_status.argtypes = [_i]
+lib.infini_attn_device_status.restype = _i
+lib.infini_attn_selftest_timeout.argtypes = [ctypes.c_uint, _vp]
+lib.infini_attn_selftest_timeout.restype = _i
+lib.infini_attn_params_size.argtypes = []
+lib.infini_attn_params_size.restype = ctypes.c_size_t
+lib.infini_attn_path.argtypes = [_i, _i, _i, _i]
+lib.infini_attn_path.restype = _i
+
+
+class InfiniAttnParams(ctypes.Structure):
+    """Mirror of ``infini_attn_params`` (include/infini_attn.h)."""
+
+    _fields_ = [
+        ("q", _vp), ("k", _vp), ("v", _vp), ("beta", _vp), ("M", _vp), ("z", _vp), ("out", _vp),
+        ("B", _i), ("H", _i), ("L", _ll), ("N", _i), ("dk", _i), ("dv", _i), ("mode", _i),
+        ("scale", ctypes.c_float),
+        ("q_stride", _ll * 3), ("k_stride", _ll * 3), ("v_stride", _ll * 3), ("o_stride", _ll * 3),
+        ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t), ("flags", _i), ("stream", _vp),
+    ]
+
+
+lib.infini_attn_forward_ex.argtypes = [ctypes.POINTER(InfiniAttnParams)]
+lib.infini_attn_forward_ex.restype = _i
+
+
+class InfiniAttnError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {infini_attn_error_string(code)} ({code})")
+
+
+def infini_attn_error_string(code: int) -> str:
+    return lib.infini_attn_error_string(int(code)).decode()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _mode(mode: int, t: torch.Tensor) -> int:
+    return int(mode) | (F32 if t.dtype == torch.float32 else 0)
+
+
+def _check(rc: int, where: str, raise_on_error: bool):
+    if rc != INFINI_OK and raise_on_error:
+        raise InfiniAttnError(rc, where)
+    return rc
+
+
+def infini_attn_forward(q, k, v, beta, M, z, out, N: int, mode: int = LINEAR, stream=None, raise_on_error=True):
+    """q, k [B,H,L,dk], v, out [B,H,L,dv] (bf16 or fp32, contiguous); beta [H]; M [B,H,dk,dv]; z [B,H,dk]."""
+    B, H, L, dk = q.shape
+    dv = v.shape[3]
+    rc = lib.infini_attn_forward(q.data_ptr(), k.data_ptr(), v.data_ptr(), beta.data_ptr(), M.data_ptr(),
+                                 z.data_ptr(), out.data_ptr(), B, H, L, int(N), dk, dv, _mode(mode, q),
+                                 _stream(stream))
+    return _check(rc, "infini_attn_forward", raise_on_error)
+
+
+def infini_attn_segment_step(q, k, v, beta, M, z, out, mode: int = LINEAR, stream=None, raise_on_error=True):
+    """One segment of n tokens per (b, h): q, k [B,H,n,dk], v, out [B,H,n,dv]."""
+    B, H, n, dk = q.shape
+    dv = v.shape[3]
+    rc = lib.infini_attn_segment_step(q.data_ptr(), k.data_ptr(), v.data_ptr(), beta.data_ptr(), M.data_ptr(),
+                                      z.data_ptr(), out.data_ptr(), B, H, n, dk, dv, _mode(mode, q),
+                                      _stream(stream))
+    return _check(rc, "infini_attn_segment_step", raise_on_error)
+
+
+def _bhl_strides(t: torch.Tensor):
+    """Element strides of the (B, H, L) dimensions of a [B, H, L, d] view with d contiguous."""
+    if t.stride(3) != 1:
+        raise ValueError("the last dimension must be contiguous")
+    return (t.stride(0), t.stride(1), t.stride(2))
+
+
+def infini_attn_forward_ex(q, k, v, beta, M, z, out, N: int, mode: int = LINEAR, scale: float = 0.0,
+                           workspace=None, flags: int = 0, stream=None, raise_on_error=True):
+    """Extended call: [B,H,L,d] views with any (B, H, L) strides, explicit scale, caller workspace, flags."""
+    B, H, L, dk = q.shape
+    dv = v.shape[3]
+    p = InfiniAttnParams()
+    p.q, p.k, p.v, p.beta = q.data_ptr(), k.data_ptr(), v.data_ptr(), beta.data_ptr()
+    p.M, p.z, p.out = M.data_ptr(), z.data_ptr(), out.data_ptr()
+    p.B, p.H, p.L, p.N, p.dk, p.dv = B, H, L, int(N), dk, dv
+    p.mode = _mode(mode, q)
+    p.scale = float(scale)
+    for name, t in (("q_stride", q), ("k_stride", k), ("v_stride", v), ("o_stride", out)):
+        getattr(p, name)[:] = _bhl_strides(t)
+    if workspace is not None:
+        p.workspace = workspace.data_ptr()
+        p.workspace_bytes = workspace.numel() * workspace.element_size()
+    p.flags = int(flags)
+    p.stream = _stream(stream)
+    rc = lib.infini_attn_forward_ex(ctypes.byref(p))
+    return _check(rc, "infini_attn_forward_ex", raise_on_error)
+
+
+def infini_attn_workspace_size(B, H, L, N, dk, dv, mode=LINEAR) -> int:
+    return int(lib.infini_attn_workspace_size(B, H, L, N, dk, dv, mode))
+
+
+def infini_attn_device_status(reset: bool = False) -> int:
+    return int(lib.infini_attn_device_status(1 if reset else 0))
+
+
+def infini_attn_selftest_timeout(limit_us: int, stream=None) -> int:
+    return int(lib.infini_attn_selftest_timeout(int(limit_us), _stream(stream)))
+
+
+def infini_attn_path(dk: int, dv: int, mode: int, flags: int = 0) -> int:
+    return int(lib.infini_attn_path(dk, dv, mode, flags))
+
+
+def forward_host(q, k, v, beta, M, z, N: int, mode: int = LINEAR, device="cuda", out=None, stream=None):
+    """End-to-end call with HOST tensors: copy inputs to the device, run, copy the output and state back.
+
+    q, k, v, beta, M, z are CPU tensors (pinned for asynchronous copies); returns (out, M, z) on the host.
+    """
+    dev = torch.device(device)
+    s = torch.cuda.current_stream(dev) if stream is None else stream
+    with torch.cuda.stream(s):
+        qd, kd, vd = (t.to(dev, non_blocking=True) for t in (q, k, v))
+        bd, Md, zd = (t.to(dev, non_blocking=True) for t in (beta, M, z))
+        od = torch.empty(q.shape[:3] + (v.shape[3],), dtype=q.dtype, device=dev)
+        infini_attn_forward(qd, kd, vd, bd, Md, zd, od, N, mode, stream=s)
+        if out is None:
+            out = torch.empty(od.shape, dtype=od.dtype, pin_memory=True)
+        out.copy_(od, non_blocking=True)
+        M.copy_(Md, non_blocking=True)
+        z.copy_(zd, non_blocking=True)
+    return out, M, z

@@ -1,0 +1,382 @@
+// Host side of libinfini_attn: the C ABI declared in include/infini_attn.h.
+//
+// A forward runs, on the caller's stream:
+//   linear rule (Eq. 8): update partials for every (b, h, segment, group) in
+//     one launch, then one state launch that scans the segments in order,
+//     writing the snapshots (M_{s-1}, z_{s-1}) and the final (M_S, z_S);
+//   delta rule (Eq. 9): a snapshot of (M_0, z_0), then per segment one
+//     update launch (reads M_{s-1}) and one state launch (adds the partials
+//     and snapshots M_s);
+//   then one attention launch (Eq. 6, 7, 10) over every (b, h, segment,
+//     query tile), reading the snapshots.
+// The order "read with M_{s-1}, then update" of the pages holds because the
+// attention kernel reads the snapshot of M_{s-1}, never the running state.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "../../include/infini_attn.h"
+#include "common.cuh"
+#include "simt.cuh"
+#include "sm100.cuh"
+
+namespace infini {
+namespace {
+
+constexpr int kChunk = 128;        // tokens per update chunk
+constexpr int kTargetCtas = 592;   // 4 x 148 SMs: aim of the update grid size
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+struct Plan {
+  int B, H, N, dk, dv, mode, S, G, cpb, nseg_part;
+  long long L;
+  bool delta, f32, tc;
+  size_t off_snapM, off_snapz, off_part, total;
+};
+
+// Workspace: per-segment snapshots of M_{s-1} (bf16 transposed for the tensor
+// cores, fp32 otherwise) and z_{s-1} (fp32), and the update partials
+// ([BH][S][G] for the linear scan, [BH][1][G] reused per segment for delta).
+int make_plan(int B, int H, long long L, int N, int dk, int dv, int mode, int flags, Plan* p) {
+  if (B <= 0 || H <= 0 || L <= 0 || N <= 0 || dk <= 0 || dv <= 0) return INFINI_ERR_INVALID_ARG;
+  if ((mode & ~(INFINI_DELTA | INFINI_F32)) != 0) return INFINI_ERR_UNSUPPORTED;
+  if (dk > 128 || dv > 128) return INFINI_ERR_UNSUPPORTED;
+  p->B = B; p->H = H; p->L = L; p->N = N; p->dk = dk; p->dv = dv; p->mode = mode;
+  p->delta = (mode & INFINI_DELTA) != 0;
+  p->f32 = (mode & INFINI_F32) != 0;
+  p->tc = !p->f32 && dk == 128 && dv == 128 && !(flags & INFINI_FLAG_FORCE_SIMT);
+  const long long S = (L + N - 1) / N;
+  const long long BH = (long long)B * H;
+  if (S > (1 << 30) || BH * S > (1LL << 31) / 4 || L > (1LL << 31) - 1) return INFINI_ERR_UNSUPPORTED;
+  p->S = (int)S;
+  const int chunks_per_seg = (std::min<long long>(N, L) + kChunk - 1) / kChunk;
+  const long long units = p->delta ? BH : BH * S;  // CTAs per launch before grouping
+  long long cpb = (units * chunks_per_seg + kTargetCtas - 1) / kTargetCtas;
+  cpb = std::max<long long>(1, std::min<long long>(cpb, chunks_per_seg));
+  p->cpb = (int)cpb;
+  p->G = (int)((chunks_per_seg + cpb - 1) / cpb);
+  p->nseg_part = p->delta ? 1 : p->S;
+  const size_t E = (size_t)dk * dv;
+  size_t off = 0;
+  p->off_snapM = off;
+  off = align_up(off + (size_t)BH * S * E * (p->tc ? 2 : 4));
+  p->off_snapz = off;
+  off = align_up(off + (size_t)BH * S * dk * 4);
+  p->off_part = off;
+  off = align_up(off + (size_t)BH * p->nseg_part * p->G * (E + dk) * 4);
+  p->total = off;
+  return INFINI_OK;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+// 4-D map over a [B, H, L, 128] bf16 tensor with element strides st[0..2]
+// (d contiguous); box 64 x 128 tokens, 128-byte swizzle.
+bool encode_bhld(CUtensorMap* m, const void* ptr, int B, int H, long long L, const long long st[3]) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {128, (cuuint64_t)L, (cuuint64_t)H, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)st[2] * 2, (cuuint64_t)st[1] * 2, (cuuint64_t)st[0] * 2};
+  cuuint32_t box[4] = {64, 128, 1, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+// 2-D map over rows x 128 bf16 (row-major), box 64 x 128 rows, 128-byte swizzle.
+bool encode_rows(CUtensorMap* m, const void* ptr, long long rows) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {128, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {256};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool ranges_overlap(const void* a, size_t an, const void* b, size_t bn) {
+  const char* x = static_cast<const char*>(a);
+  const char* y = static_cast<const char*>(b);
+  return x < y + bn && y < x + an;
+}
+size_t extent_bytes(const long long st[3], int B, int H, long long L, int d, size_t es) {
+  return (size_t)(((long long)(B - 1) * st[0] + (long long)(H - 1) * st[1] + (L - 1) * st[2] + d) * (long long)es);
+}
+
+int check_device(bool need_tc) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return INFINI_ERR_DEVICE;
+  int major = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return INFINI_ERR_DEVICE;
+  (void)need_tc;
+  return major == 10 ? INFINI_OK : INFINI_ERR_DEVICE;
+}
+
+int launch_status() { return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_LAUNCH; }
+
+template <typename T>
+int run_simt(const infini_attn_params& p, const Plan& pl, char* ws, float scale) {
+  Geo g;
+  g.B = p.B; g.H = p.H; g.L = p.L; g.N = p.N; g.dk = p.dk; g.dv = p.dv; g.S = pl.S;
+  for (int i = 0; i < 3; ++i) {
+    g.qs[i] = p.q_stride[i]; g.ks[i] = p.k_stride[i]; g.vs[i] = p.v_stride[i]; g.os[i] = p.o_stride[i];
+  }
+  float* snapM = reinterpret_cast<float*>(ws + pl.off_snapM);
+  float* snapz = reinterpret_cast<float*>(ws + pl.off_snapz);
+  float* part = reinterpret_cast<float*>(ws + pl.off_part);
+  const int BH = p.B * p.H, E = p.dk * p.dv;
+  const dim3 sgrid((E + p.dk + 255) / 256, BH);
+  const size_t upd_smem = (size_t)(32 * p.dk + 32 * p.dv + 32 + E + p.dk) * 4;
+  cudaFuncSetAttribute(simt_update_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)upd_smem);
+  const T* k = static_cast<const T*>(p.k);
+  const T* v = static_cast<const T*>(p.v);
+  if (!pl.delta) {
+    simt_update_kernel<T><<<BH * pl.S * pl.G, 256, upd_smem, p.stream>>>(k, v, g, 0, pl.S, pl.G, pl.cpb, nullptr,
+                                                                          nullptr, part);
+    state_kernel<<<sgrid, 256, 0, p.stream>>>(p.M, p.z, part, p.dk, p.dv, pl.S, 0, 0, pl.S, pl.G, snapM, nullptr,
+                                              snapz);
+  } else {
+    state_kernel<<<sgrid, 256, 0, p.stream>>>(p.M, p.z, part, p.dk, p.dv, pl.S, 2, 0, 1, pl.G, snapM, nullptr,
+                                              snapz);
+    for (int s = 0; s < pl.S; ++s) {
+      simt_update_kernel<T><<<BH * pl.G, 256, upd_smem, p.stream>>>(k, v, g, s, 1, pl.G, pl.cpb, snapM, snapz, part);
+      state_kernel<<<sgrid, 256, 0, p.stream>>>(p.M, p.z, part, p.dk, p.dv, pl.S, 1, s, 1, pl.G, snapM, nullptr,
+                                                snapz);
+    }
+  }
+  const int QT = (p.N + 31) / 32;
+  const size_t attn_smem = (size_t)(32 * (p.dk + 1) + 32 * p.dv + 32 * p.dk) * 4;
+  cudaFuncSetAttribute(simt_attn_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)attn_smem);
+  simt_attn_kernel<T><<<(unsigned)((long long)QT * BH * pl.S), 256, attn_smem, p.stream>>>(
+      static_cast<const T*>(p.q), k, v, p.beta, static_cast<T*>(p.out), g, scale, QT, snapM, snapz);
+  return launch_status();
+}
+
+int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale) {
+  CUtensorMap tm_q, tm_k, tm_v, tm_mt;
+  __nv_bfloat16* snapMt = reinterpret_cast<__nv_bfloat16*>(ws + pl.off_snapM);
+  float* snapz = reinterpret_cast<float*>(ws + pl.off_snapz);
+  float* part = reinterpret_cast<float*>(ws + pl.off_part);
+  const int BH = p.B * p.H, E = 128 * 128;
+  if (!encode_bhld(&tm_q, p.q, p.B, p.H, p.L, p.q_stride) || !encode_bhld(&tm_k, p.k, p.B, p.H, p.L, p.k_stride) ||
+      !encode_bhld(&tm_v, p.v, p.B, p.H, p.L, p.v_stride) || !encode_rows(&tm_mt, snapMt, (long long)BH * pl.S * 128))
+    return INFINI_ERR_LAUNCH;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kAttnSmem);
+    cudaFuncSetAttribute(tc::mem_update_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kUpdSmem);
+  });
+  const dim3 sgrid((E + 128 + 255) / 256, BH);
+  tc::UpdArgs ua;
+  ua.snapz = snapz; ua.partial = part; ua.B = p.B; ua.H = p.H; ua.S = pl.S; ua.N = p.N; ua.L = p.L;
+  ua.G = pl.G; ua.cpb = pl.cpb; ua.delta = pl.delta ? 1 : 0;
+  if (!pl.delta) {
+    ua.seg0 = 0; ua.nseg = pl.S;
+    tc::mem_update_tc_kernel<<<BH * pl.S * pl.G, 160, tc::kUpdSmem, p.stream>>>(tm_k, tm_v, tm_mt, ua);
+    state_kernel<<<sgrid, 256, 0, p.stream>>>(p.M, p.z, part, 128, 128, pl.S, 0, 0, pl.S, pl.G, nullptr, snapMt,
+                                              snapz);
+  } else {
+    state_kernel<<<sgrid, 256, 0, p.stream>>>(p.M, p.z, part, 128, 128, pl.S, 2, 0, 1, pl.G, nullptr, snapMt, snapz);
+    ua.nseg = 1;
+    for (int s = 0; s < pl.S; ++s) {
+      ua.seg0 = s;
+      tc::mem_update_tc_kernel<<<BH * pl.G, 160, tc::kUpdSmem, p.stream>>>(tm_k, tm_v, tm_mt, ua);
+      state_kernel<<<sgrid, 256, 0, p.stream>>>(p.M, p.z, part, 128, 128, pl.S, 1, s, 1, pl.G, nullptr, snapMt,
+                                                snapz);
+    }
+  }
+  tc::AttnArgs aa;
+  aa.beta = p.beta; aa.snapz = snapz; aa.out = static_cast<__nv_bfloat16*>(p.out);
+  aa.B = p.B; aa.H = p.H; aa.S = pl.S; aa.T = (p.N + 127) / 128; aa.L = p.L; aa.N = p.N;
+  aa.scale_log2 = scale * 1.4426950408889634f;
+  for (int i = 0; i < 3; ++i) aa.os[i] = p.o_stride[i];
+  tc::attn_tc_kernel<<<(unsigned)((long long)aa.T * BH * pl.S), 192, tc::kAttnSmem, p.stream>>>(tm_q, tm_k, tm_v,
+                                                                                               tm_mt, aa);
+  return launch_status();
+}
+
+bool tc_layout_ok(const infini_attn_params& p) {
+  const void* ptrs[4] = {p.q, p.k, p.v, p.out};
+  const long long* sts[4] = {p.q_stride, p.k_stride, p.v_stride, p.o_stride};
+  for (int t = 0; t < 4; ++t) {
+    if (reinterpret_cast<uintptr_t>(ptrs[t]) % 16 != 0) return false;
+    for (int i = 0; i < 3; ++i)
+      if (sts[t][i] <= 0 || (sts[t][i] * 2) % 16 != 0 || sts[t][i] * 2 >= (1LL << 40)) return false;
+  }
+  return true;
+}
+
+int forward_impl(infini_attn_params p) {
+  if (!p.q || !p.k || !p.v || !p.beta || !p.M || !p.z || !p.out) return INFINI_ERR_INVALID_ARG;
+  Plan pl;
+  int rc = make_plan(p.B, p.H, p.L, p.N, p.dk, p.dv, p.mode, p.flags, &pl);
+  if (rc != INFINI_OK) return rc;
+  // default contiguous strides
+  auto fill = [&](long long st[3], int d) {
+    if (st[0] == 0 && st[1] == 0 && st[2] == 0) {
+      st[2] = d;
+      st[1] = p.L * d;
+      st[0] = (long long)p.H * p.L * d;
+    }
+  };
+  fill(p.q_stride, p.dk);
+  fill(p.k_stride, p.dk);
+  fill(p.v_stride, p.dv);
+  fill(p.o_stride, p.dv);
+  for (int i = 0; i < 3; ++i)
+    if (p.q_stride[i] < 0 || p.k_stride[i] < 0 || p.v_stride[i] < 0 || p.o_stride[i] <= 0)
+      return INFINI_ERR_INVALID_ARG;
+  const size_t es = pl.f32 ? 4 : 2;
+  const size_t out_ext = extent_bytes(p.o_stride, p.B, p.H, p.L, p.dv, es);
+  if (ranges_overlap(p.out, out_ext, p.q, extent_bytes(p.q_stride, p.B, p.H, p.L, p.dk, es)) ||
+      ranges_overlap(p.out, out_ext, p.k, extent_bytes(p.k_stride, p.B, p.H, p.L, p.dk, es)) ||
+      ranges_overlap(p.out, out_ext, p.v, extent_bytes(p.v_stride, p.B, p.H, p.L, p.dv, es)) ||
+      ranges_overlap(p.out, out_ext, p.M, (size_t)p.B * p.H * p.dk * p.dv * 4) ||
+      ranges_overlap(p.out, out_ext, p.z, (size_t)p.B * p.H * p.dk * 4) ||
+      ranges_overlap(p.out, out_ext, p.beta, (size_t)p.H * 4) ||
+      ranges_overlap(p.M, (size_t)p.B * p.H * p.dk * p.dv * 4, p.z, (size_t)p.B * p.H * p.dk * 4))
+    return INFINI_ERR_INVALID_ARG;
+  if (pl.tc && !tc_layout_ok(p)) {
+    // The tensor-core kernels need TMA-compatible strides; other layouts run on CUDA cores.
+    rc = make_plan(p.B, p.H, p.L, p.N, p.dk, p.dv, p.mode, p.flags | INFINI_FLAG_FORCE_SIMT, &pl);
+    if (rc != INFINI_OK) return rc;
+  }
+  if (p.workspace) {
+    if (p.workspace_bytes < pl.total || reinterpret_cast<uintptr_t>(p.workspace) % kAlign != 0)
+      return INFINI_ERR_WORKSPACE;
+  }
+  rc = check_device(pl.tc);
+  if (rc != INFINI_OK) return rc;
+  if (pl.tc && !get_encode()) return INFINI_ERR_DEVICE;
+  const float scale = p.scale != 0.f ? p.scale : 1.f / sqrtf((float)p.dk);
+  char* ws = static_cast<char*>(p.workspace);
+  bool own = false;
+  if (!ws) {
+    void* w = nullptr;
+    if (cudaMallocAsync(&w, pl.total, p.stream) != cudaSuccess) {
+      cudaGetLastError();
+      return INFINI_ERR_WORKSPACE;
+    }
+    ws = static_cast<char*>(w);
+    own = true;
+  }
+  if (pl.tc)
+    rc = run_tc(p, pl, ws, scale);
+  else if (pl.f32)
+    rc = run_simt<float>(p, pl, ws, scale);
+  else
+    rc = run_simt<__nv_bfloat16>(p, pl, ws, scale);
+  if (own && cudaFreeAsync(ws, p.stream) != cudaSuccess && rc == INFINI_OK) rc = INFINI_ERR_WORKSPACE;
+  return rc;
+}
+
+__global__ void selftest_wait_kernel(unsigned long long limit_ns) {
+  __shared__ __align__(8) unsigned long long bar;
+  const uint32_t b = smem_u32(&bar);
+  mbar_init(b, 1);
+  fence_barrier_init();
+  // Nothing arrives on this barrier: the wait must give up after limit_ns.
+  mbar_wait(b, 0, limit_ns);
+}
+
+}  // namespace
+}  // namespace infini
+
+using namespace infini;
+
+extern "C" {
+
+int infini_attn_forward(const void* q, const void* k, const void* v, const float* beta, float* M, float* z, void* out,
+                        int B, int H, long L, int N, int dk, int dv, int mode, cudaStream_t stream) {
+  infini_attn_params p;
+  memset(&p, 0, sizeof(p));
+  p.q = q; p.k = k; p.v = v; p.beta = beta; p.M = M; p.z = z; p.out = out;
+  p.B = B; p.H = H; p.L = L; p.N = N; p.dk = dk; p.dv = dv; p.mode = mode; p.stream = stream;
+  return forward_impl(p);
+}
+
+int infini_attn_segment_step(const void* q, const void* k, const void* v, const float* beta, float* M, float* z,
+                             void* out, int B, int H, int n, int dk, int dv, int mode, cudaStream_t stream) {
+  if (n <= 0) return INFINI_ERR_INVALID_ARG;
+  return infini_attn_forward(q, k, v, beta, M, z, out, B, H, n, n, dk, dv, mode, stream);
+}
+
+int infini_attn_forward_ex(const infini_attn_params* p) {
+  if (!p) return INFINI_ERR_INVALID_ARG;
+  return forward_impl(*p);
+}
+
+size_t infini_attn_workspace_size(int B, int H, long L, int N, int dk, int dv, int mode) {
+  Plan pl;
+  if (make_plan(B, H, L, N, dk, dv, mode, 0, &pl) != INFINI_OK) return 0;
+  Plan pl2;  // a layout that falls back to CUDA cores needs the fp32 snapshots
+  if (make_plan(B, H, L, N, dk, dv, mode, INFINI_FLAG_FORCE_SIMT, &pl2) != INFINI_OK) return 0;
+  return std::max(pl.total, pl2.total);
+}
+
+const char* infini_attn_error_string(int code) {
+  switch (code) {
+    case INFINI_OK: return "ok";
+    case INFINI_ERR_INVALID_ARG: return "invalid argument (null pointer, non-positive size, or aliasing buffers)";
+    case INFINI_ERR_UNSUPPORTED: return "unsupported head size, mode, layout or size";
+    case INFINI_ERR_WORKSPACE: return "workspace too small, misaligned, or allocation failed";
+    case INFINI_ERR_LAUNCH: return "CUDA launch or runtime call failed";
+    case INFINI_ERR_TIMEOUT: return "a bounded device-side wait ran out";
+    case INFINI_ERR_DEVICE: return "no usable CUDA device (sm_100 required)";
+    default: return "unknown error code";
+  }
+}
+
+int infini_attn_device_status(int reset) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return INFINI_ERR_LAUNCH;
+  unsigned st = 0;
+  if (cudaMemcpyFromSymbol(&st, g_status, sizeof(st)) != cudaSuccess) return INFINI_ERR_LAUNCH;
+  if (reset) {
+    const unsigned zero = 0;
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return INFINI_ERR_LAUNCH;
+  }
+  return (st & kStatusTimeout) ? INFINI_ERR_TIMEOUT : INFINI_OK;
+}
+
+int infini_attn_selftest_timeout(unsigned limit_us, cudaStream_t stream) {
+  if (limit_us < 1 || limit_us > 1000000) return INFINI_ERR_INVALID_ARG;
+  int rc = check_device(false);
+  if (rc != INFINI_OK) return rc;
+  selftest_wait_kernel<<<1, 1, 0, stream>>>((unsigned long long)limit_us * 1000ull);
+  if (cudaGetLastError() != cudaSuccess) return INFINI_ERR_LAUNCH;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return INFINI_ERR_LAUNCH;
+  return infini_attn_device_status(0);
+}
+
+int infini_attn_path(int dk, int dv, int mode, int flags) {
+  Plan pl;
+  int rc = make_plan(1, 1, 1, 1, dk, dv, mode, flags, &pl);
+  if (rc != INFINI_OK) return rc;
+  return pl.tc ? 1 : 0;
+}
+
+size_t infini_attn_params_size(void) { return sizeof(infini_attn_params); }
+
+}  // extern "C"

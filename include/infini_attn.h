@@ -1,0 +1,174 @@
+/*
+ * infini_attn.h -- C ABI of the Infini-attention forward for NVIDIA B200 (sm_100a).
+ *
+ * The operation is the Infini-attention layer of "Leave No Context Behind:
+ * Efficient Infinite Context Transformers with Infini-attention" (arXiv
+ * 2404.07143), as laid out on the explainer page of that title
+ * (paper-graph-ui.vercel.app), section 3 "Technical Approach":
+ *
+ *   per (batch b, head h), the sequence of L tokens is cut into S = ceil(L/N)
+ *   segments of N tokens (the last one may be shorter; section 3, "Training
+ *   infrastructure: segment chunking at each layer").  For segment s with
+ *   rows Q, K, V:
+ *     A_dot = softmax_causal(scale * Q K^T) V                       (Eq. 6)
+ *     A_mem = sigma(Q) M_{s-1} / (sigma(Q) z_{s-1}),  sigma = ELU+1  (Eq. 7)
+ *     A     = sigmoid(beta_h) A_mem + (1 - sigmoid(beta_h)) A_dot  (Eq. 10)
+ *   then the memory is updated, linear rule (Eq. 8):
+ *     M_s = M_{s-1} + sigma(K)^T V,          z_s = z_{s-1} + sum_t sigma(K_t)
+ *   or delta rule (Eq. 9):
+ *     M_s = M_{s-1} + sigma(K)^T (V - sigma(K) M_{s-1} / (sigma(K) z_{s-1})),
+ *     z_s as in the linear rule.
+ *
+ * Conventions where the pages leave a step open:
+ *   - scale defaults to 1/sqrt(dk);
+ *   - a retrieval row whose denominator sigma(q) z is exactly 0 (empty
+ *     memory, M_0 = 0 and z_0 = 0) is the zero row, for A_mem and for the
+ *     delta rule's retrieval term alike;
+ *   - ELU uses alpha = 1; the causal mask includes the diagonal; A_dot never
+ *     looks across a segment boundary;
+ *   - M and z are fp32 throughout; products run with fp32 accumulation.
+ *
+ * Layouts (row-major, element strides; "contiguous" = the default):
+ *   q, k   [B, H, L, dk]   v, out [B, H, L, dv]    element type bf16, or fp32
+ *                                                  when mode has INFINI_F32
+ *   beta   [H]        fp32, shared by every batch row
+ *   M      [B, H, dk, dv] fp32, z [B, H, dk] fp32: on entry M_0, z_0; on
+ *          return M_S, z_S (updated in place)
+ *
+ * Ownership: every pointer is caller-owned DEVICE memory on the current
+ * device.  q, k, v and beta are read only; M and z are read and written;
+ * out is written and must not alias any input.  The library keeps no state
+ * between calls apart from a per-device error word (see
+ * infini_attn_device_status).  Temporary workspace is taken with
+ * cudaMallocAsync on `stream` and released on `stream` before the call
+ * returns, unless infini_attn_forward_ex is handed a caller workspace.
+ *
+ * Errors: every call returns INFINI_OK (0) or a negative INFINI_ERR_* code
+ * after validating its arguments on the host; nothing is launched when
+ * validation fails.  Work is asynchronous on `stream`: faults of the
+ * launched kernels surface on the caller's next synchronisation, and a
+ * bounded device-side wait that ran out is reported by
+ * infini_attn_device_status.  No kernel traps.
+ */
+#ifndef INFINI_ATTN_H
+#define INFINI_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define INFINI_API __attribute__((visibility("default")))
+#else
+#define INFINI_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* update rule, low bits of `mode` */
+#define INFINI_LINEAR 0x0 /* Eq. 8 */
+#define INFINI_DELTA 0x1  /* Eq. 9 */
+/* element type of q, k, v and out: bf16 unless this bit is set */
+#define INFINI_F32 0x10
+/* infini_attn_params.flags: run the CUDA-core (SIMT) kernels even where the
+ * tensor-core kernels apply -- a second GPU implementation, for testing */
+#define INFINI_FLAG_FORCE_SIMT 0x1
+
+enum {
+  INFINI_OK = 0,
+  INFINI_ERR_INVALID_ARG = -1, /* null pointer, size <= 0, n > N, aliasing */
+  INFINI_ERR_UNSUPPORTED = -2, /* head size, mode bits, stride or alignment not handled */
+  INFINI_ERR_WORKSPACE = -3,   /* workspace too small, or cudaMallocAsync failed */
+  INFINI_ERR_LAUNCH = -4,      /* a CUDA launch or runtime call failed */
+  INFINI_ERR_TIMEOUT = -5,     /* a bounded device-side wait ran out */
+  INFINI_ERR_DEVICE = -6       /* no CUDA device, or not sm_100 */
+};
+
+/*
+ * Whole-sequence forward over L tokens in segments of N (Eq. 4 applied
+ * S = ceil(L/N) times per (b, h)).  q, k, v, out contiguous [B, H, L, d].
+ * mode = INFINI_LINEAR or INFINI_DELTA, optionally | INFINI_F32.
+ * Supported: 1 <= dk, dv <= 128 (bf16 with dk = dv = 128 runs on the
+ * tensor cores, everything else on CUDA cores); B, H, N >= 1; L >= 1.
+ */
+INFINI_API int infini_attn_forward(const void* q, const void* k, const void* v, const float* beta, float* M, float* z,
+                        void* out, int B, int H, long L, int N, int dk, int dv, int mode, cudaStream_t stream);
+
+/*
+ * One streaming step (Eq. 4 once): every (b, h) consumes one segment of
+ * n tokens, 1 <= n.  q, k, v, out contiguous [B, H, n, d].  Reads the live
+ * M, z as M_{s-1}, z_{s-1} and leaves M_s, z_s in them.  S calls of this
+ * function give the same result as one infini_attn_forward over S*n tokens
+ * with N = n.
+ */
+INFINI_API int infini_attn_segment_step(const void* q, const void* k, const void* v, const float* beta, float* M, float* z,
+                             void* out, int B, int H, int n, int dk, int dv, int mode, cudaStream_t stream);
+
+/* Extended call: explicit scale, strides, workspace and flags. */
+typedef struct infini_attn_params {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* beta;
+  float* M;
+  float* z;
+  void* out;
+  int B, H;
+  long long L; /* tokens per (b, h) */
+  int N;       /* segment length */
+  int dk, dv;
+  int mode;    /* INFINI_LINEAR | INFINI_DELTA, optionally | INFINI_F32 */
+  float scale; /* softmax scale; 0 selects 1/sqrt(dk) */
+  /* element strides of the (B, H, L) dimensions of q, k, v, out; the last
+   * dimension is always contiguous.  All zero selects the contiguous
+   * [B, H, L, d] layout.  A layout such as [B, L, H, d] is
+   * {L*H*d, d, H*d}.  Tensor-core kernels need every stride times the
+   * element size to be a multiple of 16 bytes and 16-byte aligned bases. */
+  long long q_stride[3], k_stride[3], v_stride[3], o_stride[3];
+  /* caller workspace of at least infini_attn_workspace_size(...) bytes,
+   * 256-byte aligned; NULL lets the call allocate and free its own on
+   * `stream` (cudaMallocAsync / cudaFreeAsync). */
+  void* workspace;
+  size_t workspace_bytes;
+  int flags; /* INFINI_FLAG_* */
+  cudaStream_t stream;
+} infini_attn_params;
+
+INFINI_API int infini_attn_forward_ex(const infini_attn_params* p);
+
+/* Bytes of workspace a forward of this shape needs (0 if the shape is invalid). */
+INFINI_API size_t infini_attn_workspace_size(int B, int H, long L, int N, int dk, int dv, int mode);
+
+/* Static English text for a return code; never NULL. */
+INFINI_API const char* infini_attn_error_string(int code);
+
+/*
+ * Synchronises the current device and returns INFINI_ERR_TIMEOUT if any
+ * kernel of this library gave up a bounded wait since the last reset,
+ * else INFINI_OK (or INFINI_ERR_LAUNCH if the synchronisation failed).
+ * reset != 0 clears the error word.
+ */
+INFINI_API int infini_attn_device_status(int reset);
+
+/*
+ * Self-test of the bounded-wait machinery: launches one block that waits on
+ * an mbarrier nothing will ever complete, with a limit of `limit_us`
+ * microseconds (1 .. 1000000).  The kernel must give up, record
+ * INFINI_ERR_TIMEOUT in the error word and return; the call synchronises
+ * and returns what infini_attn_device_status(0) then reports.
+ */
+INFINI_API int infini_attn_selftest_timeout(unsigned limit_us, cudaStream_t stream);
+
+/* sizeof(infini_attn_params), for bindings that build the struct themselves. */
+INFINI_API size_t infini_attn_params_size(void);
+
+/* Which kernels the given arguments would run: 1 tensor-core, 0 CUDA-core, <0 error code. */
+INFINI_API int infini_attn_path(int dk, int dv, int mode, int flags);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* INFINI_ATTN_H */

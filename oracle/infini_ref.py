@@ -202,3 +202,32 @@ def forward_flops(B: int, H: int, L: int, N: int, dk: int, dv: int, mode: int) -
         n = s1 - s0
         total += n * (n + 1) * (dk + dv) + per_mem * n
     return B * H * total
+
+
+def memory_trajectory(K, V, N, mode=LINEAR, M0=None, z0=None):
+    """States (M_{s-1}, z_{s-1}) entering each segment of one head, and the final (M_S, z_S).
+
+    The update steps of Eq. 8 / Eq. 9 alone, for sampled checks of long inputs
+    where the attention of every segment would be too slow on the CPU.
+    K: [L, dk], V: [L, dv].
+    """
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    dk, dv = K.shape[1], V.shape[1]
+    M = np.zeros((dk, dv)) if M0 is None else np.array(M0, dtype=np.float64)
+    z = np.zeros(dk) if z0 is None else np.array(z0, dtype=np.float64)
+    states = []
+    for s0, s1 in segment_bounds(K.shape[0], N):
+        states.append((M.copy(), z.copy()))
+        sig_k = elu_plus_one(K[s0:s1])
+        if mode == LINEAR:
+            M, z = linear_update(M, z, sig_k, V[s0:s1])
+        else:
+            M, z = delta_update(M, z, sig_k, V[s0:s1])
+    return states, (M, z)
+
+
+def segment_output(Qs, Ks, Vs, M, z, beta_h, scale=None):
+    """Output A of one segment of one head given the memory (M_{s-1}, z_{s-1}) it reads (Eq. 6, 7, 10)."""
+    A, _, _, _ = infini_attention_segment(Qs, Ks, Vs, M, z, beta_h, LINEAR, scale)
+    return A

@@ -328,3 +328,23 @@ def run_all(ref):
         if f:
             bad[pin.__name__] = f
     return bad
+
+
+def pin_trajectory(ref):
+    """The update-only trajectory and per-segment outputs reproduce the full forward."""
+    fails = []
+    L, dk, dv, N = 19, 4, 3, 5
+    q, k, v = _rand((1, 1, L, dk), 40), _rand((1, 1, L, dk), 41), _rand((1, 1, L, dv), 42)
+    beta = _rand((1,), 43)
+    for mode in (ref.LINEAR, ref.DELTA):
+        out, M, z = ref.forward(q, k, v, beta, N, mode=mode)
+        states, (Mf, zf) = ref.memory_trajectory(k[0, 0], v[0, 0], N, mode)
+        fails += _close(Mf, M[0, 0], 1e-12, f"trajectory M (mode {mode})")
+        fails += _close(zf, z[0, 0], 1e-12, f"trajectory z (mode {mode})")
+        for si, (s0, s1) in enumerate(ref.segment_bounds(L, N)):
+            A = ref.segment_output(q[0, 0, s0:s1], k[0, 0, s0:s1], v[0, 0, s0:s1], *states[si], beta[0])
+            fails += _close(A, out[0, 0, s0:s1], 1e-12, f"segment output {si} (mode {mode})")
+    return fails
+
+
+ALL_PINS.append(pin_trajectory)
