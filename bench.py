@@ -1,0 +1,492 @@
+"""Benchmark of the Infini-attention forward on B200.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--mode linear|delta]
+                [--impl ours|reference]
+
+A step is one pass of the whole forward (segment chunking, memory update,
+local attention, memory read, gate) over one batch of the workload with the
+inputs resident in HBM: one ``infini_attn_forward`` call, or for the
+streaming workload one ``infini_attn_segment_step`` call per segment.  The
+default workload is the 1B-shaped layer (B=1, H=8, d=128, N=2048,
+L=32768, bf16, linear rule).  Under torchrun each rank runs its own copy of
+the workload on its own GPU (independent (batch, head) problems, no
+collective on the data path): weak scaling, value = tokens of all ranks /
+max over ranks of the step time.
+
+Timing: W warm-up steps, then K steps, each bracketed by CUDA events on the
+launching stream, with a 256 MB buffer written between steps (outside the
+events) so that no step starts with its inputs in the 126 MB L2; a barrier
+and a device synchronisation on both sides of the timed region.
+
+``--impl reference`` times the fp64 CPU oracle on the host cores instead
+(each step a bounded sample of the same workload); under torchrun only
+rank 0 runs it.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from compressive_memory_transformer_sm_b200 import DELTA, LINEAR  # noqa: E402
+from compressive_memory_transformer_sm_b200 import workloads as W  # noqa: E402
+
+METRIC = "Infini-attn fwd tokens/s per layer; TFLOP/s and % of B200 bf16 tensor peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FLUSH_BYTES = 256 << 20
+
+
+# ------------------------------------------------------------------ work model
+def algorithmic_flops(w: W.Workload, mode: int):
+    """(attention kernel FLOPs, memory-update FLOPs) per step.
+
+    Attention: n(n+1)(dk+dv) per segment for the unmasked causal half of
+    Q K^T and P V, plus 2 n dk dv for sigma(Q) M_{s-1}.  Update: 2 n dk dv for
+    sigma(K)^T U, plus 2 n dk dv for sigma(K) M_{s-1} under the delta rule.
+    """
+    attn = upd = 0
+    for s0 in range(0, w.L, w.N):
+        n = min(w.N, w.L - s0)
+        attn += n * (n + 1) * (w.dk + w.dv) + 2 * n * w.dk * w.dv
+        upd += (2 if mode == LINEAR else 4) * n * w.dk * w.dv
+    return w.B * w.H * attn, w.B * w.H * upd
+
+
+def algorithmic_bytes(w: W.Workload):
+    """q, k, v read once and out written once in the input dtype, M and z read and written once (fp32)."""
+    es = torch.finfo(w.dtype).bits // 8
+    return w.B * w.H * (w.L * (2 * w.dk + 2 * w.dv) * es + 2 * (w.dk * w.dv + w.dk) * 4)
+
+
+# ------------------------------------------------------------------ ranks
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def init_dist(backend: str, timeout_s: float = 120.0):
+    import datetime
+
+    import torch.distributed as dist
+
+    rank, world, _ = dist_env()
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=timeout_s))
+    return rank, world
+
+
+def max_over_ranks(x: float, device) -> float:
+    """The slowest rank's value (every rank takes the same collective step)."""
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device):
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        if device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def rank_seed(w: W.Workload, rank: int) -> int:
+    """Each rank solves its own independent problem of the same shape."""
+    return w.seed + 7 * rank
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock, power and throttle reasons while the GPU works."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.gpu = gpu_index
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(gpu_index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 10:
+                continue
+            try:
+                rows.append((float(f[1]), float(f[2]), float(f[3]) if f[3] not in ("[N/A]", "N/A") else None,
+                             float(f[4]), f[6], f[7], f[8], f[9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        busy = [r for r in rows if r[3] > 0] or rows
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({names[i] for r in busy for i, v in enumerate(r[4:8]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in busy), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows), "samples_under_load": len([r for r in rows if r[3] > 0]),
+                "power_w_max": max((r[2] for r in rows if r[2] is not None), default=None)}
+
+
+# ------------------------------------------------------------------ peaks / traffic
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    with open(os.path.join(ROOT, "compressive_memory_transformer_sm_b200", "csrc", "sm100.cuh"), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def measured_traffic(workload: str, mode: str):
+    """DRAM bytes per attention launch from the committed ncu summary, if it matches the current kernel."""
+    path = os.path.join(ROOT, "profiles", "attn_tc_kernel_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if d.get("kernel_source_sha256_16") != kernel_source_hash():
+        return None
+    e = d.get("per_launch_bytes", {}).get(f"{workload}/{mode}")
+    return None if e is None else float(e)
+
+
+# ------------------------------------------------------------------ oracle timing (CPU)
+def oracle_sample(w: W.Workload, mode: int, q, k, v, beta, budget_s: float, max_segments=None):
+    """Runs the fp64 oracle over consecutive segments of head (0, 0) until the time budget is spent.
+
+    Returns (tokens processed, seconds, segments).  Inputs are one head's [L, d] host tensors.
+    """
+    from oracle import infini_ref as R
+
+    Q, K, V = (t.double().numpy() for t in (q, k, v))
+    M = np.zeros((w.dk, w.dv))
+    z = np.zeros(w.dk)
+    tokens = segs = 0
+    t0 = time.perf_counter()
+    for s0, s1 in R.segment_bounds(w.L, w.N):
+        _, M, z, _ = R.infini_attention_segment(Q[s0:s1], K[s0:s1], V[s0:s1], M, z, float(beta), mode)
+        tokens += s1 - s0
+        segs += 1
+        if time.perf_counter() - t0 >= budget_s or (max_segments and segs >= max_segments):
+            break
+    return tokens, time.perf_counter() - t0, segs
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def one_head_host(w: W.Workload, seed: int):
+    """Head (0, 0) of the workload's inputs, generated on the CPU with the same recipe."""
+    one = w.with_(B=1, H=1)
+    q, k, v, beta = W.make_inputs(one, device="cpu", seed=seed)
+    return q[0, 0], k[0, 0], v[0, 0], beta[0]
+
+
+def cpu_baseline(w: W.Workload, mode: int, budget_s: float):
+    q, k, v, beta = one_head_host(w, w.seed)
+    tokens, secs, segs = oracle_sample(w, mode, q, k, v, beta, budget_s)
+    # tokens/s of the whole workload = one head's tokens/s divided by the B*H heads it must serve
+    per_head = tokens / secs
+    return {"value": per_head / (w.B * w.H), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"fp64 NumPy oracle, head (0,0), first {segs} segment(s) ({tokens} tokens) in {secs:.2f} s; "
+                      f"tokens/s scaled by 1/(B*H) = 1/{w.B * w.H} to the whole workload"}
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, w: W.Workload, mode: int):
+    from compressive_memory_transformer_sm_b200 import api
+
+    rank, world = init_dist("nccl")
+    _, _, local = dist_env()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    q, k, v, beta = W.make_inputs(w, device=dev, seed=rank_seed(w, rank))
+    M, z = W.empty_state(w, device=dev)
+    out = torch.empty_like(v)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flags = api.FLAG_FORCE_SIMT if args.force_simt else 0
+    if w.streaming:
+        S = w.segments
+        seg = lambda t: t.view(w.B, w.H, S, w.N, t.shape[3]).permute(2, 0, 1, 3, 4).contiguous()  # noqa: E731
+        q, k, v = seg(q), seg(k), seg(v)
+        out = torch.empty_like(v)
+
+    def step():
+        M.zero_()
+        z.zero_()
+        if w.streaming:
+            for s in range(w.segments):
+                api.infini_attn_segment_step(q[s], k[s], v[s], beta, M, z, out[s], mode, stream=stream)
+        elif flags:
+            api.infini_attn_forward_ex(q, k, v, beta, M, z, out, w.N, mode, flags=flags, stream=stream)
+        else:
+            api.infini_attn_forward(q, k, v, beta, M, z, out, w.N, mode, stream=stream)
+
+    sampler = ClockSampler(local)
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize(dev)
+    api.infini_attn_profile_read(reset=True)
+
+    # ---------------------------------------------------------------- timed region
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    api.infini_attn_profile_enable(1 << api.PHASE_ATTN)
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    launches0 = api.infini_attn_launch_count()
+    wall0 = time.perf_counter()
+    for i in range(args.steps):
+        flush.fill_(i & 0xff)
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    wall = time.perf_counter() - wall0
+    launches = api.infini_attn_launch_count() - launches0
+    api.infini_attn_profile_enable(0)
+    clocks = sampler.stop() if sampler else None
+    if api.infini_attn_device_status() != api.INFINI_OK:
+        raise RuntimeError("a device-side wait timed out during the benchmark")
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    ms_local = sum(step_ms) / len(step_ms)
+    attn_ms, attn_n = api.infini_attn_profile_read(reset=True)
+    attn_ms_per_launch_local = attn_ms[api.PHASE_ATTN] / max(1, attn_n[api.PHASE_ATTN])
+
+    # per-phase breakdown: a second pass of K steps with every launch bracketed
+    api.infini_attn_profile_enable(7)
+    for i in range(args.steps):
+        flush.fill_(i & 0xff)
+        step()
+    torch.cuda.synchronize(dev)
+    api.infini_attn_profile_enable(0)
+    phase_ms, phase_n = api.infini_attn_profile_read(reset=True)
+
+    ms = max_over_ranks(ms_local, dev)
+    attn_ms_per_launch = max_over_ranks(attn_ms_per_launch_local, dev)
+
+    # ---------------------------------------------------------------- end to end, host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, w, mode, dev, stream, rank)
+
+    tokens = w.B * w.L * world
+    f_attn, f_upd = algorithmic_flops(w, mode)
+    peaks, peak_src = load_peaks()
+    per_launch_attn_flops = f_attn / (w.segments if w.streaming else 1)
+    achieved = per_launch_attn_flops / (attn_ms_per_launch * 1e-3) / 1e12
+    sustained = attn_ms_per_launch > 10.0
+    peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    traffic = measured_traffic(w.name, W.MODE_NAMES[mode])
+    result = {
+        "metric": METRIC, "value": tokens / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "N": w.N, "dk": w.dk, "dv": w.dv,
+                   "mode": W.MODE_NAMES[mode], "path": "simt" if args.force_simt else "tensor",
+                   "streaming_steps": w.segments if w.streaming else 0,
+                   "l2": "256 MB buffer written between timed steps (outside the step events)",
+                   "parallelism": f"independent problem per rank x{world}"},
+        "tflops": (f_attn + f_upd) * world / (ms * 1e-3) / 1e12,
+        "pct_of_bf16_peak": 100.0 * (f_attn + f_upd) / (ms * 1e-3) / 1e12 / peak,
+        "hbm_gbs": algorithmic_bytes(w) * world / (ms * 1e-3) / 1e9,
+        "roofline": {"kernel": "attn_tc_kernel" if not args.force_simt else "simt_attn_kernel", "bound": "tensor",
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "traffic": traffic,
+                     "peak_source": f"{peak_src} {'bf16_tflops_sustained' if sustained else 'bf16_tflops'}",
+                     "launch_ms": attn_ms_per_launch, "flops_per_launch": per_launch_attn_flops},
+        "phases_ms_per_step": {name: phase_ms[i] / args.steps for i, name in enumerate(("update", "state",
+                                                                                          "attention"))},
+        "phase_launches_per_step": {name: phase_n[i] / args.steps for i, name in enumerate(("update", "state",
+                                                                                              "attention"))},
+        "gpu_launches": int(launches),
+        "clocks": clocks, "wall_s_timed_region": wall,
+    }
+    if e2e is not None:
+        result["e2e"] = e2e
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(w, mode, args.cpu_budget)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    import torch.distributed as dist
+
+    if dist.is_initialized():
+        dist.destroy_process_group()
+
+
+def run_e2e(args, w: W.Workload, mode: int, dev, stream, rank):
+    """Same metric through the public call with pinned HOST buffers: H2D of the step's inputs,
+    the forward, D2H of the output and the state, all inside each step's events."""
+    from compressive_memory_transformer_sm_b200 import api
+
+    q, k, v, beta = W.make_inputs(w, device=dev, seed=rank_seed(w, rank))
+    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+    hb = beta.cpu().pin_memory()
+    del q, k, v
+    hM = torch.zeros(w.B, w.H, w.dk, w.dv).pin_memory()
+    hz = torch.zeros(w.B, w.H, w.dk).pin_memory()
+    ho = torch.empty(w.B, w.H, w.L, w.dv, dtype=w.dtype).pin_memory()
+    dq, dk_, dv_ = (torch.empty(t.shape, dtype=t.dtype, device=dev) for t in (hq, hk, hv))
+    db = torch.empty(w.H, device=dev)
+    dM = torch.empty(hM.shape, device=dev)
+    dz = torch.empty(hz.shape, device=dev)
+    do = torch.empty(ho.shape, dtype=w.dtype, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hb, hM, hz))
+    d2h = sum(t.numel() * t.element_size() for t in (ho, hM, hz))
+
+    def step():
+        for d, h in ((dq, hq), (dk_, hk), (dv_, hv), (db, hb), (dM, hM), (dz, hz)):
+            d.copy_(h, non_blocking=True)
+        if w.streaming:
+            S = w.segments
+            for s in range(S):
+                sl = slice(s * w.N, (s + 1) * w.N)
+                api.infini_attn_forward_ex(dq[:, :, sl], dk_[:, :, sl], dv_[:, :, sl], db, dM, dz, do[:, :, sl],
+                                           w.N, mode, stream=stream)
+        else:
+            api.infini_attn_forward(dq, dk_, dv_, db, dM, dz, do, w.N, mode, stream=stream)
+        for h, d in ((ho, do), (hM, dM), (hz, dz)):
+            h.copy_(d, non_blocking=True)
+
+    for _ in range(max(1, min(args.warmup, 3))):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize(dev)
+    n = max(1, min(args.steps, 10))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    barrier(dev)
+    for i in range(n):
+        flush.fill_(i & 0xff)
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / n, dev)
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    return {"value": w.B * w.L * world / (ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": n,
+            "path": "pinned host -> device, forward, device -> pinned host, per step"}
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args, w: W.Workload, mode: int):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return  # only rank 0 times the CPU oracle
+    q, k, v, beta = one_head_host(w, w.seed)
+    budget = args.ref_step_budget
+    for _ in range(args.warmup):
+        oracle_sample(w, mode, q, k, v, beta, budget, max_segments=1)
+    tokens = 0
+    secs = 0.0
+    segs = 0
+    for _ in range(args.steps):
+        t, s, n = oracle_sample(w, mode, q, k, v, beta, budget, max_segments=1)
+        tokens += t
+        secs += s
+        segs += n
+    per_head = tokens / secs
+    value = per_head / (w.B * w.H)
+    cores = blas_threads()
+    sample = (f"each step: fp64 NumPy oracle on the first segment ({w.N if w.N < w.L else w.L} tokens) of head "
+              f"(0,0); tokens/s scaled by 1/(B*H) = 1/{w.B * w.H} to the whole workload")
+    f_attn, f_upd = algorithmic_flops(w, mode)
+    result = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "N": w.N, "dk": w.dk, "dv": w.dv,
+                   "mode": W.MODE_NAMES[mode]},
+        "tflops": value / (w.B * w.L) * (f_attn + f_upd) / 1e12,
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(result), flush=True)
+
+
+def parse(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", choices=sorted(W.WORKLOADS), default=W.LAYER_1B.name)
+    ap.add_argument("--mode", choices=("linear", "delta"), default=None)
+    ap.add_argument("--force-simt", action="store_true", help="time the CUDA-core kernels instead")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--ref-step-budget", type=float, default=5.0)
+    return ap.parse_args(argv)
+
+
+def main(argv=None):
+    args = parse(argv)
+    w = W.WORKLOADS[args.workload]
+    mode = {"linear": LINEAR, "delta": DELTA}[args.mode] if args.mode else w.modes[0]
+    if args.warmup < 3 and args.impl == "ours":
+        raise SystemExit("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args, w, mode)
+    else:
+        run_ours(args, w, mode)
+
+
+if __name__ == "__main__":
+    main()

@@ -30,7 +30,8 @@ FLAG_FORCE_SIMT = 0x1
 EXPORTED = (
     "infini_attn_forward", "infini_attn_segment_step", "infini_attn_forward_ex", "infini_attn_workspace_size",
     "infini_attn_error_string", "infini_attn_device_status", "infini_attn_selftest_timeout",
-    "infini_attn_params_size", "infini_attn_path",
+    "infini_attn_params_size", "infini_attn_path", "infini_attn_profile_enable", "infini_attn_profile_read",
+    "infini_attn_launch_count",
 )
 
 
@@ -59,6 +60,14 @@ lib.infini_attn_params_size.argtypes = []
 lib.infini_attn_params_size.restype = ctypes.c_size_t
 lib.infini_attn_path.argtypes = [_i, _i, _i, _i]
 lib.infini_attn_path.restype = _i
+lib.infini_attn_profile_enable.argtypes = [_i]
+lib.infini_attn_profile_enable.restype = _i
+lib.infini_attn_profile_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_ll), _i]
+lib.infini_attn_profile_read.restype = _i
+lib.infini_attn_launch_count.argtypes = []
+lib.infini_attn_launch_count.restype = _ll
+
+PHASE_UPDATE, PHASE_STATE, PHASE_ATTN = 0, 1, 2
 
 
 class InfiniAttnParams(ctypes.Structure):
@@ -166,6 +175,24 @@ def infini_attn_selftest_timeout(limit_us: int, stream=None) -> int:
 
 def infini_attn_path(dk: int, dv: int, mode: int, flags: int = 0) -> int:
     return int(lib.infini_attn_path(dk, dv, mode, flags))
+
+
+def infini_attn_profile_enable(phase_mask: int) -> int:
+    return int(lib.infini_attn_profile_enable(int(phase_mask)))
+
+
+def infini_attn_profile_read(reset: bool = True):
+    """Returns ([ms per phase], [timed launches per phase]) for phases update, state, attention."""
+    ms = (ctypes.c_double * 3)(0.0, 0.0, 0.0)
+    n = (_ll * 3)(0, 0, 0)
+    rc = lib.infini_attn_profile_read(ms, n, 1 if reset else 0)
+    if rc != INFINI_OK:
+        raise InfiniAttnError(rc, "infini_attn_profile_read")
+    return list(ms), list(n)
+
+
+def infini_attn_launch_count() -> int:
+    return int(lib.infini_attn_launch_count())
 
 
 def forward_host(q, k, v, beta, M, z, N: int, mode: int = LINEAR, device="cuda", out=None, stream=None):

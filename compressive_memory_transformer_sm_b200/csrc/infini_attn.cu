@@ -16,7 +16,9 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
+#include <vector>
 
 #include "../../include/infini_attn.h"
 #include "common.cuh"
@@ -31,6 +33,43 @@ constexpr int kTargetCtas = 592;   // 4 x 148 SMs: aim of the update grid size
 constexpr size_t kAlign = 256;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+// ------------------------------------------------------------ launch accounting
+enum Phase { kPhaseUpdate = 0, kPhaseState = 1, kPhaseAttn = 2 };
+std::atomic<long long> g_launches{0};
+std::atomic<int> g_profile_mask{0};
+struct EventPair {
+  int phase;
+  cudaEvent_t a, b;
+};
+std::mutex g_prof_mu;
+std::vector<EventPair> g_prof;
+
+// Counts one kernel launch and, when its phase is being timed, brackets it
+// with events on `stream`.  Construct right before the launch, destroy
+// right after it.
+struct LaunchScope {
+  int phase;
+  cudaStream_t stream;
+  cudaEvent_t a = nullptr, b = nullptr;
+  LaunchScope(int ph, cudaStream_t st) : phase(ph), stream(st) {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    if (g_profile_mask.load(std::memory_order_relaxed) & (1 << ph)) {
+      if (cudaEventCreate(&a) == cudaSuccess && cudaEventCreate(&b) == cudaSuccess) {
+        cudaEventRecord(a, stream);
+      } else {
+        a = b = nullptr;
+      }
+    }
+  }
+  ~LaunchScope() {
+    if (a && b) {
+      cudaEventRecord(b, stream);
+      std::lock_guard<std::mutex> lk(g_prof_mu);
+      g_prof.push_back({phase, a, b});
+    }
+  }
+};
 
 struct Plan {
   int B, H, N, dk, dv, mode, S, G, cpb, nseg_part;
@@ -153,15 +192,29 @@ int run_simt(const infini_attn_params& p, const Plan& pl, char* ws, float scale)
   const T* k = static_cast<const T*>(p.k);
   const T* v = static_cast<const T*>(p.v);
   if (!pl.delta) {
-    simt_update_kernel<T><<<BH * pl.S * pl.G, 256, upd_smem, p.stream>>>(k, v, g, 0, pl.S, pl.G, pl.cpb, nullptr,
-                                                                          nullptr, part);
-    state_kernel<<<sgrid, 256, 0, p.stream>>>(p.M, p.z, part, p.dk, p.dv, pl.S, 0, 0, pl.S, pl.G, snapM, nullptr,
-                                              snapz);
+    {
+      LaunchScope ls(kPhaseUpdate, p.stream);
+      simt_update_kernel<T><<<BH * pl.S * pl.G, 256, upd_smem, p.stream>>>(k, v, g, 0, pl.S, pl.G, pl.cpb, nullptr,
+                                                                            nullptr, part);
+    }
+    {
+      LaunchScope ls(kPhaseState, p.stream);
+      state_kernel<<<sgrid, 256, 0, p.stream>>>(p.M, p.z, part, p.dk, p.dv, pl.S, 0, 0, pl.S, pl.G, snapM, nullptr,
+                                                snapz);
+    }
   } else {
-    state_kernel<<<sgrid, 256, 0, p.stream>>>(p.M, p.z, part, p.dk, p.dv, pl.S, 2, 0, 1, pl.G, snapM, nullptr,
-                                              snapz);
+    {
+      LaunchScope ls(kPhaseState, p.stream);
+      state_kernel<<<sgrid, 256, 0, p.stream>>>(p.M, p.z, part, p.dk, p.dv, pl.S, 2, 0, 1, pl.G, snapM, nullptr,
+                                                snapz);
+    }
     for (int s = 0; s < pl.S; ++s) {
-      simt_update_kernel<T><<<BH * pl.G, 256, upd_smem, p.stream>>>(k, v, g, s, 1, pl.G, pl.cpb, snapM, snapz, part);
+      {
+        LaunchScope ls(kPhaseUpdate, p.stream);
+        simt_update_kernel<T><<<BH * pl.G, 256, upd_smem, p.stream>>>(k, v, g, s, 1, pl.G, pl.cpb, snapM, snapz,
+                                                                       part);
+      }
+      LaunchScope ls(kPhaseState, p.stream);
       state_kernel<<<sgrid, 256, 0, p.stream>>>(p.M, p.z, part, p.dk, p.dv, pl.S, 1, s, 1, pl.G, snapM, nullptr,
                                                 snapz);
     }
@@ -169,6 +222,7 @@ int run_simt(const infini_attn_params& p, const Plan& pl, char* ws, float scale)
   const int QT = (p.N + 31) / 32;
   const size_t attn_smem = (size_t)(32 * (p.dk + 1) + 32 * p.dv + 32 * p.dk) * 4;
   cudaFuncSetAttribute(simt_attn_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)attn_smem);
+  LaunchScope ls(kPhaseAttn, p.stream);
   simt_attn_kernel<T><<<(unsigned)((long long)QT * BH * pl.S), 256, attn_smem, p.stream>>>(
       static_cast<const T*>(p.q), k, v, p.beta, static_cast<T*>(p.out), g, scale, QT, snapM, snapz);
   return launch_status();
@@ -194,15 +248,27 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale) {
   ua.G = pl.G; ua.cpb = pl.cpb; ua.delta = pl.delta ? 1 : 0;
   if (!pl.delta) {
     ua.seg0 = 0; ua.nseg = pl.S;
-    tc::mem_update_tc_kernel<<<BH * pl.S * pl.G, 160, tc::kUpdSmem, p.stream>>>(tm_k, tm_v, tm_mt, ua);
+    {
+      LaunchScope ls(kPhaseUpdate, p.stream);
+      tc::mem_update_tc_kernel<<<BH * pl.S * pl.G, 160, tc::kUpdSmem, p.stream>>>(tm_k, tm_v, tm_mt, ua);
+    }
+    LaunchScope ls(kPhaseState, p.stream);
     state_kernel<<<sgrid, 256, 0, p.stream>>>(p.M, p.z, part, 128, 128, pl.S, 0, 0, pl.S, pl.G, nullptr, snapMt,
                                               snapz);
   } else {
-    state_kernel<<<sgrid, 256, 0, p.stream>>>(p.M, p.z, part, 128, 128, pl.S, 2, 0, 1, pl.G, nullptr, snapMt, snapz);
+    {
+      LaunchScope ls(kPhaseState, p.stream);
+      state_kernel<<<sgrid, 256, 0, p.stream>>>(p.M, p.z, part, 128, 128, pl.S, 2, 0, 1, pl.G, nullptr, snapMt,
+                                                snapz);
+    }
     ua.nseg = 1;
     for (int s = 0; s < pl.S; ++s) {
       ua.seg0 = s;
-      tc::mem_update_tc_kernel<<<BH * pl.G, 160, tc::kUpdSmem, p.stream>>>(tm_k, tm_v, tm_mt, ua);
+      {
+        LaunchScope ls(kPhaseUpdate, p.stream);
+        tc::mem_update_tc_kernel<<<BH * pl.G, 160, tc::kUpdSmem, p.stream>>>(tm_k, tm_v, tm_mt, ua);
+      }
+      LaunchScope ls(kPhaseState, p.stream);
       state_kernel<<<sgrid, 256, 0, p.stream>>>(p.M, p.z, part, 128, 128, pl.S, 1, s, 1, pl.G, nullptr, snapMt,
                                                 snapz);
     }
@@ -212,6 +278,7 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale) {
   aa.B = p.B; aa.H = p.H; aa.S = pl.S; aa.T = (p.N + 127) / 128; aa.L = p.L; aa.N = p.N;
   aa.scale_log2 = scale * 1.4426950408889634f;
   for (int i = 0; i < 3; ++i) aa.os[i] = p.o_stride[i];
+  LaunchScope ls(kPhaseAttn, p.stream);
   tc::attn_tc_kernel<<<(unsigned)((long long)aa.T * BH * pl.S), 192, tc::kAttnSmem, p.stream>>>(tm_q, tm_k, tm_v,
                                                                                                tm_mt, aa);
   return launch_status();
@@ -378,5 +445,41 @@ int infini_attn_path(int dk, int dv, int mode, int flags) {
 }
 
 size_t infini_attn_params_size(void) { return sizeof(infini_attn_params); }
+
+int infini_attn_profile_enable(int phase_mask) {
+  if (phase_mask < 0 || phase_mask > 7) return INFINI_ERR_INVALID_ARG;
+  g_profile_mask.store(phase_mask);
+  return INFINI_OK;
+}
+
+int infini_attn_profile_read(double* ms, long long* launches, int reset) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  int rc = INFINI_OK;
+  double acc[3] = {0, 0, 0};
+  long long cnt[3] = {0, 0, 0};
+  for (const EventPair& e : g_prof) {
+    float t = 0.f;
+    if (cudaEventSynchronize(e.b) != cudaSuccess || cudaEventElapsedTime(&t, e.a, e.b) != cudaSuccess) {
+      rc = INFINI_ERR_LAUNCH;
+      continue;
+    }
+    acc[e.phase] += t;
+    cnt[e.phase] += 1;
+  }
+  for (int i = 0; i < 3; ++i) {
+    if (ms) ms[i] += acc[i];
+    if (launches) launches[i] += cnt[i];
+  }
+  if (reset) {
+    for (const EventPair& e : g_prof) {
+      cudaEventDestroy(e.a);
+      cudaEventDestroy(e.b);
+    }
+    g_prof.clear();
+  }
+  return rc;
+}
+
+long long infini_attn_launch_count(void) { return g_launches.load(); }
 
 }  // extern "C"

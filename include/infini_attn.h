@@ -161,6 +161,23 @@ INFINI_API int infini_attn_device_status(int reset);
  */
 INFINI_API int infini_attn_selftest_timeout(unsigned limit_us, cudaStream_t stream);
 
+/*
+ * Kernel timing for benchmarks.  phase_mask selects phases (bit 0 = memory
+ * update kernels, bit 1 = state/snapshot kernels, bit 2 = attention
+ * kernel); while a bit is set, every launch of that phase is bracketed by
+ * two CUDA events recorded on the launch's stream.  0 turns timing off.
+ */
+INFINI_API int infini_attn_profile_enable(int phase_mask);
+/*
+ * Synchronises the recorded events and adds, per phase p in 0..2, the
+ * elapsed milliseconds to ms[p] and the number of timed launches to
+ * launches[p], for everything recorded since the last reset; reset != 0
+ * then drops the records.  Either array may be NULL.
+ */
+INFINI_API int infini_attn_profile_read(double* ms, long long* launches, int reset);
+/* Number of kernels this library has launched in this process (all phases). */
+INFINI_API long long infini_attn_launch_count(void);
+
 /* sizeof(infini_attn_params), for bindings that build the struct themselves. */
 INFINI_API size_t infini_attn_params_size(void);
 
