@@ -25,13 +25,15 @@ INFINI_ERR_WORKSPACE = -3
 INFINI_ERR_LAUNCH = -4
 INFINI_ERR_TIMEOUT = -5
 INFINI_ERR_DEVICE = -6
+INFINI_ERR_SCRATCH_LIMIT = -7
+NOALLOC_SCRATCH_BYTES = 32 << 20
 FLAG_FORCE_SIMT = 0x1
 
 EXPORTED = (
     "infini_attn_forward", "infini_attn_segment_step", "infini_attn_forward_ex", "infini_attn_workspace_size",
     "infini_attn_error_string", "infini_attn_device_status", "infini_attn_selftest_timeout",
     "infini_attn_params_size", "infini_attn_path", "infini_attn_profile_enable", "infini_attn_profile_read",
-    "infini_attn_launch_count",
+    "infini_attn_launch_count", "infini_attn_forward_noalloc",
 )
 
 
@@ -46,6 +48,8 @@ lib = _load()
 _vp, _i, _l, _ll = ctypes.c_void_p, ctypes.c_int, ctypes.c_long, ctypes.c_longlong
 lib.infini_attn_forward.argtypes = [_vp] * 7 + [_i, _i, _l, _i, _i, _i, _i, _vp]
 lib.infini_attn_forward.restype = _i
+lib.infini_attn_forward_noalloc.argtypes = [_vp] * 7 + [_i, _i, _l, _i, _i, _i, _i, _vp]
+lib.infini_attn_forward_noalloc.restype = _i
 lib.infini_attn_segment_step.argtypes = [_vp] * 7 + [_i, _i, _i, _i, _i, _i, _vp]
 lib.infini_attn_segment_step.restype = _i
 lib.infini_attn_workspace_size.argtypes = [_i, _i, _l, _i, _i, _i, _i]
@@ -120,6 +124,22 @@ def infini_attn_forward(q, k, v, beta, M, z, out, N: int, mode: int = LINEAR, st
                                  z.data_ptr(), out.data_ptr(), B, H, L, int(N), dk, dv, _mode(mode, q),
                                  _stream(stream))
     return _check(rc, "infini_attn_forward", raise_on_error)
+
+
+def infini_attn_forward_noalloc(q, k, v, beta, M, z, out, N: int, mode: int = LINEAR, stream=None,
+                                raise_on_error=True):
+    """infini_attn_forward for callers that must not allocate device memory during the call.
+
+    The workspace comes from the library's fixed 32 MiB device buffer instead of
+    cudaMallocAsync; shapes needing more are refused (INFINI_ERR_SCRATCH_LIMIT).  Calls that
+    overlap on the GPU share that buffer and race, so keep them on one stream.
+    """
+    B, H, L, dk = q.shape
+    dv = v.shape[3]
+    rc = lib.infini_attn_forward_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), beta.data_ptr(), M.data_ptr(),
+                                         z.data_ptr(), out.data_ptr(), B, H, L, int(N), dk, dv, _mode(mode, q),
+                                         _stream(stream))
+    return _check(rc, "infini_attn_forward_noalloc", raise_on_error)
 
 
 def infini_attn_segment_step(q, k, v, beta, M, z, out, mode: int = LINEAR, stream=None, raise_on_error=True):

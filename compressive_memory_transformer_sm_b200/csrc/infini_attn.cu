@@ -368,6 +368,36 @@ __global__ void selftest_wait_kernel(unsigned long long limit_ns) {
   mbar_wait(b, 0, limit_ns);
 }
 
+// ------------------------------------------------------------ fixed scratch
+// Workspace of infini_attn_forward_noalloc: one buffer per device, part of
+// the module image, so it exists from load to exit and no call allocates.
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of the buffer on the current device.  The symbol's name is
+// only a host-side handle; the address comes from cudaGetSymbolAddress, once
+// per device, with that device current.
+int noalloc_scratch(void** out) {
+  static std::mutex mu;
+  static void* addr[256] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) {
+    cudaGetLastError();
+    return INFINI_ERR_DEVICE;
+  }
+  std::lock_guard<std::mutex> lk(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return INFINI_ERR_LAUNCH;
+    }
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return INFINI_OK;
+}
+
 }  // namespace
 }  // namespace infini
 
@@ -388,6 +418,28 @@ int infini_attn_segment_step(const void* q, const void* k, const void* v, const 
                              void* out, int B, int H, int n, int dk, int dv, int mode, cudaStream_t stream) {
   if (n <= 0) return INFINI_ERR_INVALID_ARG;
   return infini_attn_forward(q, k, v, beta, M, z, out, B, H, n, n, dk, dv, mode, stream);
+}
+
+int infini_attn_forward_noalloc(const void* q, const void* k, const void* v, const float* beta, float* M, float* z,
+                                void* out, int B, int H, long L, int N, int dk, int dv, int mode,
+                                cudaStream_t stream) {
+  if (!q || !k || !v || !beta || !M || !z || !out) return INFINI_ERR_INVALID_ARG;
+  Plan pl;
+  int rc = make_plan(B, H, L, N, dk, dv, mode, 0, &pl);
+  if (rc != INFINI_OK) return rc;
+  if (pl.total > kNoAllocScratchBytes) return INFINI_ERR_SCRATCH_LIMIT;
+  rc = check_device(pl.tc);
+  if (rc != INFINI_OK) return rc;
+  void* scratch = nullptr;
+  rc = noalloc_scratch(&scratch);
+  if (rc != INFINI_OK) return rc;
+  infini_attn_params p;
+  memset(&p, 0, sizeof(p));
+  p.q = q; p.k = k; p.v = v; p.beta = beta; p.M = M; p.z = z; p.out = out;
+  p.B = B; p.H = H; p.L = L; p.N = N; p.dk = dk; p.dv = dv; p.mode = mode; p.stream = stream;
+  p.workspace = scratch;
+  p.workspace_bytes = kNoAllocScratchBytes;
+  return forward_impl(p);
 }
 
 int infini_attn_forward_ex(const infini_attn_params* p) {
@@ -412,6 +464,8 @@ const char* infini_attn_error_string(int code) {
     case INFINI_ERR_LAUNCH: return "CUDA launch or runtime call failed";
     case INFINI_ERR_TIMEOUT: return "a bounded device-side wait ran out";
     case INFINI_ERR_DEVICE: return "no usable CUDA device (sm_100 required)";
+    case INFINI_ERR_SCRATCH_LIMIT:
+      return "shape needs more workspace than the 32 MiB fixed scratch of infini_attn_forward_noalloc";
     default: return "unknown error code";
   }
 }

@@ -83,7 +83,8 @@ enum {
   INFINI_ERR_WORKSPACE = -3,   /* workspace too small, or cudaMallocAsync failed */
   INFINI_ERR_LAUNCH = -4,      /* a CUDA launch or runtime call failed */
   INFINI_ERR_TIMEOUT = -5,     /* a bounded device-side wait ran out */
-  INFINI_ERR_DEVICE = -6       /* no CUDA device, or not sm_100 */
+  INFINI_ERR_DEVICE = -6,      /* no CUDA device, or not sm_100 */
+  INFINI_ERR_SCRATCH_LIMIT = -7 /* shape needs more than infini_attn_forward_noalloc's fixed scratch */
 };
 
 /*
@@ -105,6 +106,31 @@ INFINI_API int infini_attn_forward(const void* q, const void* k, const void* v, 
  */
 INFINI_API int infini_attn_segment_step(const void* q, const void* k, const void* v, const float* beta, float* M, float* z,
                              void* out, int B, int H, int n, int dk, int dv, int mode, cudaStream_t stream);
+
+/*
+ * infini_attn_forward without any device allocation.  The paper has no
+ * counterpart: this exists for callers that must not allocate device memory
+ * while they run -- for example a serving loop that forbids allocation after
+ * start-up, or code under a memory budget fixed in advance -- and so can
+ * neither let the call take its workspace with cudaMallocAsync nor hand it a
+ * buffer of their own.  Same arguments, layouts, results and errors as
+ * infini_attn_forward; the workspace instead comes from one fixed 32 MiB
+ * buffer in device memory that belongs to this library (every GPU that
+ * loads the library holds it until the process exits).
+ *   - Shapes whose workspace (infini_attn_workspace_size) exceeds 32 MiB are
+ *     rejected with INFINI_ERR_SCRATCH_LIMIT before anything is launched.
+ *   - The first call on a device looks up that device's address of the
+ *     buffer (with the device current); make that first call before any
+ *     stream capture.  Nothing else is set up, and no call allocates.
+ *   - All calls on a device share the one buffer and it keeps the previous
+ *     call's contents; nothing in it has to start at zero, since a call reads
+ *     only what it wrote earlier in the same call.  Calls whose work overlaps
+ *     on the GPU (different streams without ordering between them) race on
+ *     the buffer and give wrong results: order them on one stream.
+ */
+INFINI_API int infini_attn_forward_noalloc(const void* q, const void* k, const void* v, const float* beta, float* M,
+                                           float* z, void* out, int B, int H, long L, int N, int dk, int dv,
+                                           int mode, cudaStream_t stream);
 
 /* Extended call: explicit scale, strides, workspace and flags. */
 typedef struct infini_attn_params {
