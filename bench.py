@@ -173,7 +173,7 @@ def load_peaks():
 
 
 def kernel_source_hash() -> str:
-    with open(os.path.join(ROOT, "compressive_memory_transformer_sm_b200", "csrc", "sm100.cuh"), "rb") as f:
+    with open(os.path.join(ROOT, "compressive_memory_transformer_sm_b200", "csrc", "sm100_attn.cuh"), "rb") as f:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 

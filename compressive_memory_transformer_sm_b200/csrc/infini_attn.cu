@@ -23,7 +23,8 @@
 #include "../../include/infini_attn.h"
 #include "common.cuh"
 #include "simt.cuh"
-#include "sm100.cuh"
+#include "sm100_attn.cuh"
+#include "sm100_update.cuh"
 
 namespace infini {
 namespace {
@@ -275,12 +276,19 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale) {
   }
   tc::AttnArgs aa;
   aa.beta = p.beta; aa.snapz = snapz; aa.out = static_cast<__nv_bfloat16*>(p.out);
-  aa.B = p.B; aa.H = p.H; aa.S = pl.S; aa.T = (p.N + 127) / 128; aa.L = p.L; aa.N = p.N;
+  aa.B = p.B; aa.H = p.H; aa.S = pl.S; aa.T = (p.N + 127) / 128; aa.P = (aa.T + 1) / 2; aa.L = p.L; aa.N = p.N;
   aa.scale_log2 = scale * 1.4426950408889634f;
   for (int i = 0; i < 3; ++i) aa.os[i] = p.o_stride[i];
+  // Scheduling groups of GS segments: about one wave of CTAs per group.
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    sms = 148;
+  const long long NS = (long long)BH * pl.S;
+  aa.GS = (int)std::max<long long>(1, std::min<long long>(NS, (sms + aa.P - 1) / aa.P));
+  const long long groups = (NS + aa.GS - 1) / aa.GS;
   LaunchScope ls(kPhaseAttn, p.stream);
-  tc::attn_tc_kernel<<<(unsigned)((long long)aa.T * BH * pl.S), 192, tc::kAttnSmem, p.stream>>>(tm_q, tm_k, tm_v,
-                                                                                               tm_mt, aa);
+  tc::attn_tc_kernel<<<(unsigned)(groups * aa.GS * aa.P), tc::kAttnThreads, tc::kAttnSmem, p.stream>>>(
+      tm_q, tm_k, tm_v, tm_mt, aa);
   return launch_status();
 }
 

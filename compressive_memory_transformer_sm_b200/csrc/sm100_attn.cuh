@@ -1,0 +1,344 @@
+// attn_tc_kernel: A_dot (Eq. 6) + A_mem (Eq. 7) + gate (Eq. 10) of the
+// Infini-attention forward, fused, on the sm_100a tensor cores: one CTA per
+// (b, h, segment, pair of 128-row query tiles).
+#pragma once
+
+#include "sm100_common.cuh"
+
+namespace infini {
+namespace tc {
+
+struct AttnArgs {
+  const float* beta;
+  const float* snapz;     // [BH][S][128] fp32: z_{s-1}
+  __nv_bfloat16* out;
+  int B, H, S, T;         // T = query tiles per full segment
+  int P;                  // query-tile pairs per full segment = ceil(T / 2)
+  int GS;                 // segments per scheduling group
+  long long L;
+  int N;
+  float scale_log2;       // softmax scale * log2(e)
+  long long os[3];        // element strides of out
+};
+
+// Shared memory of the attention kernel (offsets from a 1024-aligned base).
+constexpr uint32_t kA_Q0 = 0;
+constexpr uint32_t kA_Q1 = 32768;
+constexpr uint32_t kA_K0 = 65536;    // K ring: 2 stages of 32 KB
+constexpr uint32_t kA_V0 = 131072;   // V ring: 2 stages of 32 KB
+constexpr uint32_t kA_Z = 196608;
+constexpr uint32_t kA_BAR = kA_Z + 512;
+constexpr uint32_t kA_TMEMSLOT = kA_BAR + 256;
+constexpr uint32_t kAttnSmem = kA_TMEMSLOT + 16 + 1024;  // + alignment slack
+constexpr int kAttnThreads = 320;
+
+// Barrier indices.
+enum : int {
+  B_Q = 0,
+  B_KF0 = 1,   // K stage full (2)
+  B_VF0 = 3,   // V stage full (2)
+  B_KVE0 = 5,  // K/V stage free (2)
+  B_SF0 = 7,   // S of query tile k ready (2)
+  B_PF0 = 9,   // P of query tile k written (2, 128 arrivals)
+  B_SQ0 = 11,  // sigma(Q) of query tile k written (2, 128 arrivals)
+  B_MEM0 = 13, // sigma(Q_k) M_{s-1} ready (2)
+  B_COUNT = 15
+};
+
+// One CTA computes two adjacent 128-row query tiles (2m, 2m+1) of one
+// (b, h, segment), sharing every K/V tile load between them.
+// Warps 0-3: softmax warpgroup of query tile 2m; warps 4-7: of tile 2m+1
+// (thread = query row = TMEM lane).  Warp 8 loads (TMA), warp 9 issues the
+// MMAs and owns TMEM.  TMEM columns: S of tile 2m [0,128), S of tile 2m+1
+// [128,256), O of tile 2m [256,384), O of tile 2m+1 [384,512).  P (bf16)
+// overwrites the first 64 columns of its S buffer and feeds the P V product
+// from TMEM; after the last P V product the S buffer receives sigma(Q) M_{s-1}.
+//
+// MMA issue order (k = query tile): S_0(0) S_1(0) | PV_0(j-1) S_0(j) PV_1(j-1)
+// S_1(j) | ... so that one softmax warpgroup works while the tensor cores
+// serve the other, and "S_k(j) complete" implies "PV_k(j-1) complete": the
+// O rescale of the softmax needs no extra wait.
+//
+// CTAs are ordered by groups of GS segments (about one wave of CTAs per
+// group, so the group's K/V stays in L2), heaviest pair first inside a group.
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_mt,
+                   const AttnArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+
+  // ---- work item: (pair m, segment) from the grouped schedule
+  const int NS = a.B * a.H * a.S;
+  const int per_group = a.GS * a.P;
+  const int grp = (int)(blockIdx.x / per_group);
+  const int r = (int)(blockIdx.x % per_group);
+  const int gsz = min(a.GS, NS - grp * a.GS);
+  if (r >= gsz * a.P) return;  // padding of the last group
+  const int m = a.P - 1 - r / gsz;
+  const int seg = grp * a.GS + r % gsz;  // = bh * S + s
+  const int bh = seg / a.S, s = seg % a.S;
+  const int b = bh / a.H, h = bh % a.H;
+  const long long seg0 = (long long)s * a.N;
+  const int n_s = (int)min((long long)a.N, a.L - seg0);
+  if (2 * m * kTile >= n_s) return;  // tail segment: both tiles empty
+  const int nk1 = 2 * m + 2;         // K/V tiles of query tile 2m+1 (tile 2m uses one fewer)
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  auto sQ = [&](int k) { return base + (k ? kA_Q1 : kA_Q0); };
+  auto sK = [&](int st) { return base + kA_K0 + (uint32_t)st * kTileBytes; };
+  auto sV = [&](int st) { return base + kA_V0 + (uint32_t)st * kTileBytes; };
+  auto bar = [&](int i) { return base + kA_BAR + 8u * (uint32_t)i; };
+  float* zs = reinterpret_cast<float*>(gbase + kA_Z);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kA_TMEMSLOT);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(B_Q), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(B_KF0 + i), 1);
+      mbar_init(bar(B_VF0 + i), 1);
+      mbar_init(bar(B_KVE0 + i), 1);
+      mbar_init(bar(B_SF0 + i), 1);
+      mbar_init(bar(B_PF0 + i), 128);
+      mbar_init(bar(B_SQ0 + i), 128);
+      mbar_init(bar(B_MEM0 + i), 1);
+    }
+    fence_barrier_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  if (threadIdx.x < 128) zs[threadIdx.x] = a.snapz[(long long)seg * 128 + threadIdx.x];
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer
+      prefetch_tensormap(&tm_q);
+      prefetch_tensormap(&tm_k);
+      prefetch_tensormap(&tm_v);
+      prefetch_tensormap(&tm_mt);
+      const int lq = (int)(seg0 + (long long)(2 * m) * kTile);
+      mbar_expect_tx(bar(B_Q), 2 * kTileBytes);
+      tma_load_4d(sQ(0), &tm_q, bar(B_Q), 0, lq, h, b);
+      tma_load_4d(sQ(0) + kBox, &tm_q, bar(B_Q), 64, lq, h, b);
+      tma_load_4d(sQ(1), &tm_q, bar(B_Q), 0, lq + kTile, h, b);
+      tma_load_4d(sQ(1) + kBox, &tm_q, bar(B_Q), 64, lq + kTile, h, b);
+      for (int j = 0; j < nk1; ++j) {
+        const int st = j & 1;
+        if (j >= 2) mbar_wait(bar(B_KVE0 + st), ((j - 2) >> 1) & 1);
+        const int lk = (int)(seg0 + (long long)j * kTile);
+        mbar_expect_tx(bar(B_KF0 + st), kTileBytes);
+        tma_load_4d(sK(st), &tm_k, bar(B_KF0 + st), 0, lk, h, b);
+        tma_load_4d(sK(st) + kBox, &tm_k, bar(B_KF0 + st), 64, lk, h, b);
+        mbar_expect_tx(bar(B_VF0 + st), kTileBytes);
+        tma_load_4d(sV(st), &tm_v, bar(B_VF0 + st), 0, lk, h, b);
+        tma_load_4d(sV(st) + kBox, &tm_v, bar(B_VF0 + st), 64, lk, h, b);
+      }
+      // M_{s-1}^T (bf16 snapshot) enters the K ring as tile nk1.
+      const int st = nk1 & 1;
+      mbar_wait(bar(B_KVE0 + st), ((nk1 - 2) >> 1) & 1);
+      mbar_expect_tx(bar(B_KF0 + st), kTileBytes);
+      tma_load_2d(sK(st), &tm_mt, bar(B_KF0 + st), 0, seg * 128);
+      tma_load_2d(sK(st) + kBox, &tm_mt, bar(B_KF0 + st), 64, seg * 128);
+    }
+  } else if (warp == 9) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      constexpr uint32_t idesc_kk = idesc_bf16(128, 128, 0, 0);
+      constexpr uint32_t idesc_pv = idesc_bf16(128, 128, 0, 1);
+      const int nk0 = nk1 - 1;
+      auto issue_s = [&](int k, int j) {
+        const int st = j & 1;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem + (uint32_t)k * 128u, kmajor_desc(sQ(k), kk), kmajor_desc(sK(st), kk), idesc_kk,
+                 kk > 0 ? 1u : 0u);
+        mma_commit(bar(B_SF0 + k));
+      };
+      auto issue_pv = [&](int k, int j) {  // P of tile k, key tile j; call in order j = 0, 1, ...
+        const int st = j & 1;
+        mbar_wait(bar(B_PF0 + k), j & 1);
+        mbar_wait(bar(B_VF0 + st), (j >> 1) & 1);
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + 256u + (uint32_t)k * 128u, tmem + (uint32_t)k * 128u + (uint32_t)kk * 8u,
+                 mnmajor_desc(sV(st), kk), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+      };
+      mbar_wait(bar(B_Q), 0);
+      mbar_wait(bar(B_KF0), 0);
+      tc_fence_after();
+      issue_s(0, 0);
+      issue_s(1, 0);
+      for (int j = 1; j < nk1; ++j) {
+        const int st = j & 1;
+        mbar_wait(bar(B_KF0 + st), (j >> 1) & 1);
+        tc_fence_after();
+        if (j - 1 < nk0) issue_pv(0, j - 1);
+        if (j < nk0) issue_s(0, j);
+        issue_pv(1, j - 1);
+        mma_commit(bar(B_KVE0 + ((j - 1) & 1)));
+        issue_s(1, j);
+      }
+      issue_pv(1, nk1 - 1);
+      mma_commit(bar(B_KVE0 + ((nk1 - 1) & 1)));
+      // memory read: sigma(Q_k) (written over Q_k by the softmax warps) times M_{s-1}
+      const int stm = nk1 & 1;
+      mbar_wait(bar(B_KF0 + stm), (nk1 >> 1) & 1);
+#pragma unroll 1
+      for (int k = 0; k < 2; ++k) {
+        mbar_wait(bar(B_SQ0 + k), 0);
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem + (uint32_t)k * 128u, kmajor_desc(sQ(k), kk), kmajor_desc(sK(stm), kk), idesc_kk,
+                 kk > 0 ? 1u : 0u);
+        mma_commit(bar(B_MEM0 + k));
+      }
+    }
+  } else {
+    // -------------------------------------------------------------- softmax WGs
+    const int k = warp >> 2;            // query tile 2m + k
+    const int row = (warp & 3) * 32 + lane;  // query row in the tile = TMEM lane
+    const uint32_t lrow = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lrow + (uint32_t)k * 128u;
+    const uint32_t tO = tmem + lrow + 256u + (uint32_t)k * 128u;
+    const int nk = nk1 - 1 + k;
+    const float c = a.scale_log2;
+    float m_ref = 0.f, l = 0.f;
+    for (int j = 0; j < nk; ++j) {
+      mbar_wait(bar(B_SF0 + k), j & 1);
+      tc_fence_after();
+      uint32_t x[128];
+      {
+        uint32_t (&x0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&x[0]);
+        uint32_t (&x1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&x[32]);
+        uint32_t (&x2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&x[64]);
+        uint32_t (&x3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&x[96]);
+        tmem_ld32(tS, x0);
+        tmem_ld32(tS + 32u, x1);
+        tmem_ld32(tS + 64u, x2);
+        tmem_ld32(tS + 96u, x3);
+        tmem_ld_wait();
+      }
+      if (j == nk - 1) {  // diagonal tile: key e is visible to query row iff e <= row
+#pragma unroll
+        for (int e = 0; e < 128; ++e)
+          if (e > row) x[e] = __float_as_uint(-INFINITY);
+      }
+      float mx[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) mx[i] = __uint_as_float(x[i]);
+#pragma unroll
+      for (int e = 4; e < 128; ++e) mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(x[e]));
+      const float mxs = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * c;
+      // Move the reference max only when the row max grows by more than 2^8:
+      // O / l stays exact for any reference, and p stays below 256.
+      const float m_new = (j == 0) ? mxs : (mxs > m_ref + 8.f ? mxs : m_ref);
+      const bool resc = (j > 0) && (m_new != m_ref);
+      if (__any_sync(0xffffffffu, resc)) {
+        // S_k(j) complete implies P V of tile j-1 complete (issue order), so O is final here.
+        const float alpha = resc ? ex2_approx(m_ref - m_new) : 1.f;
+        l *= alpha;
+        uint32_t o[16];
+#pragma unroll 1
+        for (int cc = 0; cc < 8; ++cc) {
+          tmem_ld16(tO + 16u * cc, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st16(tO + 16u * cc, o);
+        }
+        tmem_st_wait();
+      }
+      m_ref = m_new;
+      const float nm = -m_ref;
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int e = 0; e < 64; ++e) {
+        const float p0 = ex2_approx(fmaf(__uint_as_float(x[2 * e]), c, nm));
+        const float p1 = ex2_approx(fmaf(__uint_as_float(x[2 * e + 1]), c, nm));
+        ls[e & 3] += p0 + p1;
+        x[e] = pack_bf16x2(p0, p1);
+      }
+      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      {
+        uint32_t (&p0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&x[0]);
+        uint32_t (&p1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&x[32]);
+        tmem_st32(tS, p0);
+        tmem_st32(tS + 32u, p1);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar(B_PF0 + k));
+    }
+    // Every Q_k K^T product has completed: overwrite this row of Q_k with
+    // sigma(Q_k) (bf16) for the memory read, and form the fp32 denominator
+    // sigma(q) . z_{s-1} from the unrounded sigma.
+    float den = 0.f;
+    {
+      const uint32_t q = sQ(k);
+#pragma unroll
+      for (int cc = 0; cc < 16; ++cc) {
+        const uint32_t ad = q + swz_chunk(row, cc);
+        uint4 w = lds128(ad);
+        uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float s0 = elu1(bf16_lo(wp[e])), s1 = elu1(bf16_hi(wp[e]));
+          den = fmaf(s0, zs[8 * cc + 2 * e], den);
+          den = fmaf(s1, zs[8 * cc + 2 * e + 1], den);
+          wp[e] = pack_bf16x2(s0, s1);
+        }
+        sts128(ad, w);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(bar(B_SQ0 + k));
+    }
+    // ---------------------------------------------------------------- epilogue
+    mbar_wait(bar(B_MEM0 + k), 0);  // also implies the last P V product of tile k is complete
+    tc_fence_after();
+    const float gw = 1.f / (1.f + __expf(-a.beta[h]));
+    const float wdot = (1.f - gw) / l;
+    const float wmem = den != 0.f ? gw / den : 0.f;
+    const int qrow = (2 * m + k) * kTile + row;
+    const bool valid = qrow < n_s;
+    __nv_bfloat16* orow = a.out + b * a.os[0] + h * a.os[1] + (seg0 + qrow) * a.os[2];
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+      uint32_t ro[32], rm[32];
+      tmem_ld32(tO + 32u * cc, ro);
+      tmem_ld32(tS + 32u * cc, rm);
+      tmem_ld_wait();
+      uint32_t pk[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float v0 = wmem * __uint_as_float(rm[2 * e]) + wdot * __uint_as_float(ro[2 * e]);
+        const float v1 = wmem * __uint_as_float(rm[2 * e + 1]) + wdot * __uint_as_float(ro[2 * e + 1]);
+        pk[e] = pack_bf16x2(v0, v1);
+      }
+      if (valid) {
+        uint4* dst = reinterpret_cast<uint4*>(orow + 32 * cc);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace tc
+}  // namespace infini
