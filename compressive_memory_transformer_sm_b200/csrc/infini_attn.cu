@@ -30,7 +30,8 @@ namespace infini {
 namespace {
 
 constexpr int kChunk = 128;        // tokens per update chunk
-constexpr int kTargetCtas = 592;   // 4 x 148 SMs: aim of the update grid size
+constexpr int kSms = 148;          // B200 SM count: grid sizing (device independent, so plans are too)
+constexpr int kTargetCtas = 4 * kSms;  // CUDA-core update grid size aim
 constexpr size_t kAlign = 256;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
@@ -96,8 +97,18 @@ int make_plan(int B, int H, long long L, int N, int dk, int dv, int mode, int fl
   p->S = (int)S;
   const int chunks_per_seg = (std::min<long long>(N, L) + kChunk - 1) / kChunk;
   const long long units = p->delta ? BH : BH * S;  // CTAs per launch before grouping
-  long long cpb = (units * chunks_per_seg + kTargetCtas - 1) / kTargetCtas;
-  cpb = std::max<long long>(1, std::min<long long>(cpb, chunks_per_seg));
+  long long cpb;
+  if (p->tc) {
+    // Tensor cores: long CTAs (the chunk pipeline hides load latency), about one
+    // wave; the delta rule's G CTAs of a head form one cluster of at most 8.
+    long long G = std::max<long long>(1, kSms / units);
+    G = std::min<long long>(G, p->delta ? tc::kMaxDeltaCluster : chunks_per_seg);
+    G = std::min<long long>(G, chunks_per_seg);
+    cpb = (chunks_per_seg + G - 1) / G;
+  } else {
+    cpb = (units * chunks_per_seg + kTargetCtas - 1) / kTargetCtas;
+    cpb = std::max<long long>(1, std::min<long long>(cpb, chunks_per_seg));
+  }
   p->cpb = (int)cpb;
   p->G = (int)((chunks_per_seg + cpb - 1) / cpb);
   p->nseg_part = p->delta ? 1 : p->S;
@@ -241,17 +252,22 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale) {
   static std::once_flag once;
   std::call_once(once, [] {
     cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kAttnSmem);
-    cudaFuncSetAttribute(tc::mem_update_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kUpdSmem);
+    cudaFuncSetAttribute(tc::mem_update_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)tc::UpdSmem<false>::BYTES);
+    cudaFuncSetAttribute(tc::mem_update_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)tc::UpdSmem<true>::BYTES);
   });
   const dim3 sgrid((E + 128 + 255) / 256, BH);
   tc::UpdArgs ua;
-  ua.snapz = snapz; ua.partial = part; ua.B = p.B; ua.H = p.H; ua.S = pl.S; ua.N = p.N; ua.L = p.L;
-  ua.G = pl.G; ua.cpb = pl.cpb; ua.delta = pl.delta ? 1 : 0;
+  ua.snapz = snapz; ua.partial = part; ua.M = p.M; ua.z = p.z; ua.snapMt = snapMt; ua.snapzw = snapz;
+  ua.B = p.B; ua.H = p.H; ua.S = pl.S; ua.N = p.N; ua.L = p.L;
+  ua.G = pl.G; ua.cpb = pl.cpb;
   if (!pl.delta) {
     ua.seg0 = 0; ua.nseg = pl.S;
     {
       LaunchScope ls(kPhaseUpdate, p.stream);
-      tc::mem_update_tc_kernel<<<BH * pl.S * pl.G, 160, tc::kUpdSmem, p.stream>>>(tm_k, tm_v, tm_mt, ua);
+      tc::mem_update_tc_kernel<false><<<BH * pl.S * pl.G, tc::kUpdThreads, tc::UpdSmem<false>::BYTES, p.stream>>>(
+          tm_k, tm_v, tm_mt, ua);
     }
     LaunchScope ls(kPhaseState, p.stream);
     state_kernel<<<sgrid, 256, 0, p.stream>>>(p.M, p.z, part, 128, 128, pl.S, 0, 0, pl.S, pl.G, nullptr, snapMt,
@@ -263,15 +279,26 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale) {
                                                 snapz);
     }
     ua.nseg = 1;
+    // one cluster of G CTAs per head; G <= 8 (plan)
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = pl.G;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(BH * pl.G);
+    cfg.blockDim = dim3(tc::kUpdThreads);
+    cfg.dynamicSmemBytes = tc::UpdSmem<true>::BYTES;
+    cfg.stream = p.stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     for (int s = 0; s < pl.S; ++s) {
+      // partials of segment s, reduced inside each head's cluster into M, z and
+      // the snapshot of M_s for segment s + 1
       ua.seg0 = s;
-      {
-        LaunchScope ls(kPhaseUpdate, p.stream);
-        tc::mem_update_tc_kernel<<<BH * pl.G, 160, tc::kUpdSmem, p.stream>>>(tm_k, tm_v, tm_mt, ua);
-      }
-      LaunchScope ls(kPhaseState, p.stream);
-      state_kernel<<<sgrid, 256, 0, p.stream>>>(p.M, p.z, part, 128, 128, pl.S, 1, s, 1, pl.G, nullptr, snapMt,
-                                                snapz);
+      LaunchScope ls(kPhaseUpdate, p.stream);
+      if (cudaLaunchKernelEx(&cfg, tc::mem_update_tc_kernel<true>, tm_k, tm_v, tm_mt, ua) != cudaSuccess)
+        return INFINI_ERR_LAUNCH;
     }
   }
   tc::AttnArgs aa;
@@ -293,6 +320,8 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale) {
 }
 
 bool tc_layout_ok(const infini_attn_params& p) {
+  // the cluster reduction of the delta rule moves M and z in 16-byte vectors
+  if (reinterpret_cast<uintptr_t>(p.M) % 16 != 0 || reinterpret_cast<uintptr_t>(p.z) % 16 != 0) return false;
   const void* ptrs[4] = {p.q, p.k, p.v, p.out};
   const long long* sts[4] = {p.q_stride, p.k_stride, p.v_stride, p.o_stride};
   for (int t = 0; t < 4; ++t) {
@@ -435,7 +464,9 @@ int infini_attn_forward_noalloc(const void* q, const void* k, const void* v, con
   Plan pl;
   int rc = make_plan(B, H, L, N, dk, dv, mode, 0, &pl);
   if (rc != INFINI_OK) return rc;
-  if (pl.total > kNoAllocScratchBytes) return INFINI_ERR_SCRATCH_LIMIT;
+  // the documented limit: infini_attn_workspace_size, which also covers the
+  // CUDA-core kernels a misaligned layout falls back to
+  if (infini_attn_workspace_size(B, H, L, N, dk, dv, mode) > kNoAllocScratchBytes) return INFINI_ERR_SCRATCH_LIMIT;
   rc = check_device(pl.tc);
   if (rc != INFINI_OK) return rc;
   void* scratch = nullptr;

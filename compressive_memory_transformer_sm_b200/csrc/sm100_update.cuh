@@ -10,40 +10,72 @@ namespace infini {
 namespace tc {
 
 // ------------------------------------------------------------------------
-// Memory update.  Grid: BH * nseg * G CTAs of 160 threads; CTA (bh, segment
-// seg0 + sl, group grp) covers tokens [grp*cpb*128, min((grp+1)*cpb*128, n_s))
-// of the segment in 128-token chunks.  Warp 0 lane 0 loads (TMA) and issues
-// MMAs; warps 1-4 (thread = token row of the chunk = TMEM lane) apply sigma,
-// split it into bf16 hi + lo parts and, for the delta rule, form
-// U = V - R / den with R = sigma(K)_hi M_{s-1} from the tensor cores and
-// den = sigma(K) . z_{s-1} in fp32, again split into hi + lo.  The products
-//   dM += sK_hi^T U_hi + sK_lo^T U_hi (+ sK_hi^T U_lo)       (fp32 in TMEM)
-//   dz += sK_hi^T 1 + sK_lo^T 1                            (N = 16 ones block)
-// keep the update within ~2^-16 relative of fp32 arithmetic.
+// Memory update.  Grid: BH * nseg * G CTAs; CTA (bh, segment seg0 + sl,
+// group grp) covers tokens [grp*cpb*128, min((grp+1)*cpb*128, n_s)) of the
+// segment in 128-token chunks.
+//
+// Warps 0-7: thread (row r of the chunk = TMEM lane, half hh = warp / 4)
+// handles value columns [64 hh, 64 hh + 64) of its token: sigma(K) split into
+// bf16 hi + lo parts, and for the delta rule U = V - R / den with
+// R = sigma(K)_hi M_{s-1} from the tensor cores and den = sigma(K) . z_{s-1}
+// in fp32, again split into hi + lo.  Warp 8 loads (TMA: K ring of 2 stages,
+// V ring of 2 stages (linear) or 1 (delta, where U overwrites V in place)),
+// warp 9 issues the MMAs:
+//   dM += sK_hi^T U_hi + sK_lo^T U_hi (+ sK_hi^T U_lo)   (fp32 in TMEM)
+//   dz += sK_hi^T 1 + sK_lo^T 1                        (N = 16 block of ones)
+// which keeps the update within ~2^-16 relative of fp32 arithmetic.  The lo
+// parts of the next chunk wait in registers until the MMAs of the previous
+// chunk have released the lo buffers, so the CUDA-core pass overlaps them.
+//
+// Delta rule: the G CTAs of a head form one thread-block cluster (G <= 8).
+// Each stages its partial [dM | dz] in its own shared memory; after a cluster
+// barrier, CTA g adds slice g of every partial, read from the peers' shared
+// memory in rank order (deterministic), to the running M, z and writes the
+// snapshot of M_s for the next segment.  A second cluster barrier keeps every
+// CTA's shared memory alive until its peers have read it.
 struct UpdArgs {
-  const float* snapz;  // [BH][S][128]
-  float* partial;      // [BH][nseg][G][128*128 + 128]
+  const float* snapz;           // [BH][S][128]
+  float* partial;               // [BH][nseg][G][128*128 + 128] (linear)
+  float* M;                     // running state (delta)
+  float* z;
+  __nv_bfloat16* snapMt;        // [BH][S][128][128] (delta: M_s^T for segment s+1)
+  float* snapzw;                // [BH][S][128] (delta: z_s for segment s+1)
   int B, H, S, N;
   long long L;
-  int seg0, nseg, G, cpb, delta;
+  int seg0, nseg, G, cpb;
+};
+constexpr int kMaxDeltaCluster = 8;
+
+template <bool DELTA>
+struct UpdSmem {
+  static constexpr int VST = DELTA ? 1 : 2;
+  static constexpr uint32_t K0 = 0;           // K ring (2 x 32 KB); sigma(K)_hi in place
+  static constexpr uint32_t V0 = 65536;       // V ring; U_hi in place (delta)
+  static constexpr uint32_t KLO = V0 + VST * 32768u;
+  static constexpr uint32_t ULO = KLO + 32768u;                 // delta
+  static constexpr uint32_t MT = ULO + 32768u;                  // delta
+  static constexpr uint32_t ONES = DELTA ? MT + 32768u : KLO + 32768u;
+  static constexpr uint32_t Z = ONES + 4096u;
+  static constexpr uint32_t DENP = Z + 512u;  // [2 buffers][2 halves][128]
+  static constexpr uint32_t BAR = DENP + 2048u;
+  static constexpr uint32_t SLOT = BAR + 256u;
+  static constexpr uint32_t BYTES = SLOT + 16u + 1024u;
+  // delta: [dM (128 x 128) | dz (128)] fp32 staged for the cluster reduction,
+  // over the K and V rings once every chunk has been consumed
+  static constexpr uint32_t RED = 0;
 };
 
-constexpr uint32_t kU_K = 0;         // sigma(K) hi (in place over K)
-constexpr uint32_t kU_KLO = 32768;   // sigma(K) lo
-constexpr uint32_t kU_V = 65536;     // U hi (in place over V)
-constexpr uint32_t kU_ULO = 98304;   // U lo
-constexpr uint32_t kU_MT = 131072;   // M_{s-1}^T
-constexpr uint32_t kU_ONES = 163840; // 4 KB of bf16 ones
-constexpr uint32_t kU_Z = 167936;
-constexpr uint32_t kU_BAR = kU_Z + 512;
-constexpr uint32_t kU_TMEMSLOT = kU_BAR + 128;
-constexpr uint32_t kUpdSmem = kU_TMEMSLOT + 16 + 1024;
+enum : int {
+  U_KF0 = 0, U_KE0 = 2, U_VF0 = 4, U_VE0 = 6, U_MT = 8, U_SK = 9, U_R = 10, U_U = 11, U_MMA = 12, U_COUNT = 13
+};
+constexpr int kUpdThreads = 320;
 
-enum : int { U_LD = 0, U_MT = 1, U_SK = 2, U_R = 3, U_U = 4, U_MMA = 5, U_COUNT = 6 };
-
-__global__ void __launch_bounds__(160, 1)
+template <bool DELTA>
+__global__ void __launch_bounds__(kUpdThreads, 1)
     mem_update_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                          const __grid_constant__ CUtensorMap tm_mt, const UpdArgs a) {
+  using SL = UpdSmem<DELTA>;
+  constexpr int VST = SL::VST;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -62,181 +94,260 @@ __global__ void __launch_bounds__(160, 1)
   const int t_end = min(n_s, t_begin + a.cpb * kTile);
   float* part = a.partial + (((long long)bh * a.nseg + sl) * a.G + grp) * (long long)(128 * 128 + 128);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (t_begin >= t_end) {  // group past the end of a short segment: contributes nothing
-    for (int e = threadIdx.x; e < 128 * 128 + 128; e += blockDim.x) part[e] = 0.f;
-    return;
-  }
-  const int nchunks = (t_end - t_begin + kTile - 1) / kTile;
-  const bool delta = a.delta != 0;
+  const int nchunks = t_begin < t_end ? (t_end - t_begin + kTile - 1) / kTile : 0;
 
-  auto bar = [&](int i) { return base + kU_BAR + 8u * (uint32_t)i; };
-  float* zs = reinterpret_cast<float*>(gbase + kU_Z);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kU_TMEMSLOT);
-  if (threadIdx.x == 0) {
-    mbar_init(bar(U_LD), 1);
-    mbar_init(bar(U_MT), 1);
-    mbar_init(bar(U_SK), 128);
-    mbar_init(bar(U_R), 1);
-    mbar_init(bar(U_U), 128);
-    mbar_init(bar(U_MMA), 1);
-    fence_barrier_init();
-  }
-  {
-    uint32_t* ones = reinterpret_cast<uint32_t*>(gbase + kU_ONES);
-    for (int e = threadIdx.x; e < 1024; e += blockDim.x) ones[e] = 0x3f803f80u;  // bf16 1.0 pairs
-  }
-  if (warp >= 1) zs[threadIdx.x - 32] = delta ? a.snapz[((long long)bh * a.S + s) * 128 + (threadIdx.x - 32)] : 0.f;
-  if (warp == 0) {
-    tmem_alloc(smem_u32(tmem_slot), 512);
-    tmem_relinquish();
-  }
-  fence_proxy_async_smem();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const uint32_t tR = tmem, tM = tmem + 128, tZ = tmem + 256;
-  const uint32_t sKt = base + kU_K, sKlo = base + kU_KLO, sVt = base + kU_V, sUlo = base + kU_ULO,
-                 sMt = base + kU_MT, sOnes = base + kU_ONES;
-
-  if (warp == 0) {
-    if (lane == 0) {
-      prefetch_tensormap(&tm_k);
-      prefetch_tensormap(&tm_v);
-      if (delta) {
-        prefetch_tensormap(&tm_mt);
-        const int row = (bh * a.S + s) * 128;
-        mbar_expect_tx(bar(U_MT), kTileBytes);
-        tma_load_2d(sMt, &tm_mt, bar(U_MT), 0, row);
-        tma_load_2d(sMt + kBox, &tm_mt, bar(U_MT), 64, row);
-      }
-      constexpr uint32_t idesc_r = idesc_bf16(128, 128, 0, 0);
-      constexpr uint32_t idesc_m = idesc_bf16(128, 128, 1, 1);
-      constexpr uint32_t idesc_z = idesc_bf16(128, 16, 1, 0);
-      for (int c = 0; c < nchunks; ++c) {
-        if (c > 0) mbar_wait(bar(U_MMA), (c - 1) & 1);
-        const int lt = (int)(seg_start + t_begin + (long long)c * kTile);
-        mbar_expect_tx(bar(U_LD), 2 * kTileBytes);
-        tma_load_4d(sKt, &tm_k, bar(U_LD), 0, lt, h, b);
-        tma_load_4d(sKt + kBox, &tm_k, bar(U_LD), 64, lt, h, b);
-        tma_load_4d(sVt, &tm_v, bar(U_LD), 0, lt, h, b);
-        tma_load_4d(sVt + kBox, &tm_v, bar(U_LD), 64, lt, h, b);
-        if (delta) {
-          mbar_wait(bar(U_SK), c & 1);
-          if (c == 0) mbar_wait(bar(U_MT), 0);
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tR, kmajor_desc(sKt, kk), kmajor_desc(sMt, kk), idesc_r, kk > 0 ? 1u : 0u);
-          mma_commit(bar(U_R));
-        }
-        mbar_wait(bar(U_U), c & 1);
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t acc = (c > 0 || kk > 0) ? 1u : 0u;
-          const uint64_t aH = mnmajor_desc(sKt, kk), aL = mnmajor_desc(sKlo, kk);
-          const uint64_t bH = mnmajor_desc(sVt, kk);
-          mma_ss(tM, aH, bH, idesc_m, acc);
-          mma_ss(tM, aL, bH, idesc_m, 1u);
-          if (delta) mma_ss(tM, aH, mnmajor_desc(sUlo, kk), idesc_m, 1u);
-          const uint64_t bO = ones_desc(sOnes, kk);
-          mma_ss(tZ, aH, bO, idesc_z, acc);
-          mma_ss(tZ, aL, bO, idesc_z, 1u);
-        }
-        mma_commit(bar(U_MMA));
-      }
+  float* red = reinterpret_cast<float*>(gbase + SL::RED);
+  if (nchunks == 0) {  // group past the end of a short segment: contributes nothing
+    if (DELTA) {
+      for (int e = threadIdx.x; e < 128 * 128 + 128; e += blockDim.x) red[e] = 0.f;
+    } else {
+      for (int e = threadIdx.x; e < 128 * 128 + 128; e += blockDim.x) part[e] = 0.f;
     }
   } else {
-    const int wq = warp & 3;
-    const int row = wq * 32 + lane;
-    const uint32_t lrow = (uint32_t)(wq * 32) << 16;
-    for (int c = 0; c < nchunks; ++c) {
-      mbar_wait(bar(U_LD), c & 1);
-      const bool valid = t_begin + c * kTile + row < t_end;
-      float den = 0.f;
-#pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {
-        const uint32_t off = swz_chunk(row, ch);
-        uint4 w = lds128(sKt + off);
-        uint4 wl;
-        uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
-        uint32_t* lp = reinterpret_cast<uint32_t*>(&wl);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float s0 = valid ? elu1(bf16_lo(wp[e])) : 0.f;
-          float s1 = valid ? elu1(bf16_hi(wp[e])) : 0.f;
-          den = fmaf(s0, zs[8 * ch + 2 * e], den);
-          den = fmaf(s1, zs[8 * ch + 2 * e + 1], den);
-          const uint32_t hi = pack_bf16x2(s0, s1);
-          wp[e] = hi;
-          lp[e] = pack_bf16x2(s0 - bf16_lo(hi), s1 - bf16_hi(hi));
-        }
-        sts128(sKt + off, w);
-        sts128(sKlo + off, wl);
+    auto bar = [&](int i) { return base + SL::BAR + 8u * (uint32_t)i; };
+    auto sK = [&](int st) { return base + SL::K0 + (uint32_t)st * kTileBytes; };
+    auto sV = [&](int st) { return base + SL::V0 + (uint32_t)st * kTileBytes; };
+    const uint32_t sKlo = base + SL::KLO, sUlo = base + SL::ULO, sMt = base + SL::MT, sOnes = base + SL::ONES;
+    float* zs = reinterpret_cast<float*>(gbase + SL::Z);
+    float* denp = reinterpret_cast<float*>(gbase + SL::DENP);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + SL::SLOT);
+    if (threadIdx.x == 0) {
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(bar(U_KF0 + i), 1);
+        mbar_init(bar(U_KE0 + i), 1);
+        mbar_init(bar(U_VF0 + i), 1);
+        mbar_init(bar(U_VE0 + i), 1);
       }
-      fence_proxy_async_smem();
-      if (delta) {
+      mbar_init(bar(U_MT), 1);
+      mbar_init(bar(U_SK), 256);
+      mbar_init(bar(U_R), 1);
+      mbar_init(bar(U_U), 256);
+      mbar_init(bar(U_MMA), 1);
+      fence_barrier_init();
+    }
+    {
+      uint32_t* ones = reinterpret_cast<uint32_t*>(gbase + SL::ONES);
+      for (int e = threadIdx.x; e < 1024; e += blockDim.x) ones[e] = 0x3f803f80u;  // bf16 1.0 pairs
+    }
+    if (threadIdx.x < 128) zs[threadIdx.x] = DELTA ? a.snapz[((long long)bh * a.S + s) * 128 + threadIdx.x] : 0.f;
+    if (warp == 9) {
+      tmem_alloc(smem_u32(tmem_slot), 512);
+      tmem_relinquish();
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tR = tmem, tM = tmem + 128, tZ = tmem + 256;
+
+    if (warp == 8) {
+      if (lane == 0) {
+        // ---------------------------------------------------------- producer
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+        if (DELTA) {
+          const int row = (bh * a.S + s) * 128;
+          mbar_expect_tx(bar(U_MT), kTileBytes);
+          tma_load_2d(sMt, &tm_mt, bar(U_MT), 0, row);
+          tma_load_2d(sMt + kBox, &tm_mt, bar(U_MT), 64, row);
+        }
+        for (int c = 0; c < nchunks; ++c) {
+          const int lt = (int)(seg_start + t_begin + (long long)c * kTile);
+          const int kst = c & 1;
+          if (c >= 2) mbar_wait(bar(U_KE0 + kst), ((c - 2) >> 1) & 1);
+          mbar_expect_tx(bar(U_KF0 + kst), kTileBytes);
+          tma_load_4d(sK(kst), &tm_k, bar(U_KF0 + kst), 0, lt, h, b);
+          tma_load_4d(sK(kst) + kBox, &tm_k, bar(U_KF0 + kst), 64, lt, h, b);
+          const int vst = c % VST;
+          if (c >= VST) mbar_wait(bar(U_VE0 + vst), ((c - VST) / VST) & 1);
+          mbar_expect_tx(bar(U_VF0 + vst), kTileBytes);
+          tma_load_4d(sV(vst), &tm_v, bar(U_VF0 + vst), 0, lt, h, b);
+          tma_load_4d(sV(vst) + kBox, &tm_v, bar(U_VF0 + vst), 64, lt, h, b);
+        }
+      }
+    } else if (warp == 9) {
+      if (lane == 0) {
+        // ---------------------------------------------------------- MMA issuer
+        constexpr uint32_t idesc_r = idesc_bf16(128, 128, 0, 0);
+        constexpr uint32_t idesc_m = idesc_bf16(128, 128, 1, 1);
+        constexpr uint32_t idesc_z = idesc_bf16(128, 16, 1, 0);
+        for (int c = 0; c < nchunks; ++c) {
+          const int kst = c & 1, vst = c % VST;
+          mbar_wait(bar(U_SK), c & 1);
+          if (DELTA) {
+            if (c == 0) mbar_wait(bar(U_MT), 0);
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ss(tR, kmajor_desc(sK(kst), kk), kmajor_desc(sMt, kk), idesc_r, kk > 0 ? 1u : 0u);
+            mma_commit(bar(U_R));
+            mbar_wait(bar(U_U), c & 1);
+          } else {
+            mbar_wait(bar(U_VF0 + vst), (c / VST) & 1);
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t acc = (c > 0 || kk > 0) ? 1u : 0u;
+            const uint64_t aH = mnmajor_desc(sK(kst), kk), aL = mnmajor_desc(sKlo, kk);
+            const uint64_t bH = mnmajor_desc(sV(vst), kk);
+            mma_ss(tM, aH, bH, idesc_m, acc);
+            mma_ss(tM, aL, bH, idesc_m, 1u);
+            if (DELTA) mma_ss(tM, aH, mnmajor_desc(sUlo, kk), idesc_m, 1u);
+            const uint64_t bO = ones_desc(sOnes, kk);
+            mma_ss(tZ, aH, bO, idesc_z, acc);
+            mma_ss(tZ, aL, bO, idesc_z, 1u);
+          }
+          mma_commit(bar(U_MMA));
+          mma_commit(bar(U_KE0 + kst));
+          mma_commit(bar(U_VE0 + vst));
+        }
+      }
+    } else {
+      // ------------------------------------------------------------ compute warps
+      const int row = (warp & 3) * 32 + lane;
+      const int hh = warp >> 2;
+      const uint32_t lrow = (uint32_t)((warp & 3) * 32) << 16;
+      for (int c = 0; c < nchunks; ++c) {
+        const int kst = c & 1, vst = c % VST;
+        mbar_wait(bar(U_KF0 + kst), (c >> 1) & 1);
+        const bool valid = t_begin + c * kTile + row < t_end;
+        float dpart = 0.f;
+        uint32_t lo[32];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint32_t off = swz_chunk(row, 8 * hh + i);
+          uint4 w = lds128(sK(kst) + off);
+          uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float s0 = valid ? elu1(bf16_lo(wp[e])) : 0.f;
+            const float s1 = valid ? elu1(bf16_hi(wp[e])) : 0.f;
+            if (DELTA) {
+              dpart = fmaf(s0, zs[64 * hh + 8 * i + 2 * e], dpart);
+              dpart = fmaf(s1, zs[64 * hh + 8 * i + 2 * e + 1], dpart);
+            }
+            const uint32_t hi = pack_bf16x2(s0, s1);
+            wp[e] = hi;
+            lo[4 * i + e] = pack_bf16x2(s0 - bf16_lo(hi), s1 - bf16_hi(hi));
+          }
+          sts128(sK(kst) + off, w);
+        }
+        if (c > 0) mbar_wait(bar(U_MMA), (c - 1) & 1);  // MMAs of chunk c-1 released the lo buffers
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          sts128(sKlo + swz_chunk(row, 8 * hh + i), make_uint4(lo[4 * i], lo[4 * i + 1], lo[4 * i + 2], lo[4 * i + 3]));
+        float den = 0.f;
+        if (DELTA) {
+          denp[(c & 1) * 256 + hh * 128 + row] = dpart;
+          named_bar_sync(1, 256);
+          den = denp[(c & 1) * 256 + row] + denp[(c & 1) * 256 + 128 + row];
+        }
+        fence_proxy_async_smem();
         mbar_arrive(bar(U_SK));
-        mbar_wait(bar(U_R), c & 1);
-        tc_fence_after();
-        const float rinv = den != 0.f ? 1.f / den : 0.f;
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          uint32_t r[32];
-          tmem_ld32(tR + lrow + 32u * q4, r);
+        if (DELTA) {
+          mbar_wait(bar(U_R), c & 1);
+          tc_fence_after();
+          const float rinv = den != 0.f ? 1.f / den : 0.f;
+          uint32_t r0[32], r1[32];
+          tmem_ld32(tR + lrow + 64u * hh, r0);
+          tmem_ld32(tR + lrow + 64u * hh + 32u, r1);
           tmem_ld_wait();
+          mbar_wait(bar(U_VF0 + vst), (c / VST) & 1);
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
-            const int ch = q4 * 4 + cc;  // 16-byte chunk = 8 value columns
-            const uint32_t off = swz_chunk(row, ch);
-            uint4 w = lds128(sVt + off);
+          for (int i = 0; i < 8; ++i) {
+            const uint32_t off = swz_chunk(row, 8 * hh + i);
+            uint4 w = lds128(sV(vst) + off);
             uint4 wl;
             uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
             uint32_t* lp = reinterpret_cast<uint32_t*>(&wl);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const float u0 = bf16_lo(wp[e]) - __uint_as_float(r[8 * cc + 2 * e]) * rinv;
-              const float u1 = bf16_hi(wp[e]) - __uint_as_float(r[8 * cc + 2 * e + 1]) * rinv;
+              const int col = 8 * i + 2 * e;  // within this thread's 64 columns
+              const float rr0 = __uint_as_float(col < 32 ? r0[col] : r1[col - 32]);
+              const float rr1 = __uint_as_float(col + 1 < 32 ? r0[col + 1] : r1[col + 1 - 32]);
+              const float u0 = bf16_lo(wp[e]) - rr0 * rinv;
+              const float u1 = bf16_hi(wp[e]) - rr1 * rinv;
               const uint32_t hi = pack_bf16x2(u0, u1);
               wp[e] = hi;
               lp[e] = pack_bf16x2(u0 - bf16_lo(hi), u1 - bf16_hi(hi));
             }
-            sts128(sVt + off, w);
+            sts128(sV(vst) + off, w);
             sts128(sUlo + off, wl);
           }
+          fence_proxy_async_smem();
+          tc_fence_before();
+          mbar_arrive(bar(U_U));
         }
-        fence_proxy_async_smem();
-        tc_fence_before();
       }
-      mbar_arrive(bar(U_U));
-    }
-    mbar_wait(bar(U_MMA), (nchunks - 1) & 1);
-    tc_fence_after();
-    float* prow = part + (long long)row * 128;
+      mbar_wait(bar(U_MMA), (nchunks - 1) & 1);
+      tc_fence_after();
+      // every load and MMA of this CTA is complete: the K/V rings can hold the partial
+      float* prow = (DELTA ? red : part) + (long long)row * 128 + 64 * hh;
 #pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4) {
-      uint32_t r[32];
-      tmem_ld32(tM + lrow + 32u * q4, r);
+      for (int q2 = 0; q2 < 2; ++q2) {
+        uint32_t rr[32];
+        tmem_ld32(tM + lrow + 64u * hh + 32u * q2, rr);
+        tmem_ld_wait();
+        float4* dst = reinterpret_cast<float4*>(prow + 32 * q2);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          dst[e] = make_float4(__uint_as_float(rr[4 * e]), __uint_as_float(rr[4 * e + 1]),
+                               __uint_as_float(rr[4 * e + 2]), __uint_as_float(rr[4 * e + 3]));
+      }
+      uint32_t zr;
+      tmem_ld1(tZ + lrow, zr);
       tmem_ld_wait();
-      float4* dst = reinterpret_cast<float4*>(prow + 32 * q4);
-#pragma unroll
-      for (int e = 0; e < 8; ++e)
-        dst[e] = make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]), __uint_as_float(r[4 * e + 2]),
-                             __uint_as_float(r[4 * e + 3]));
+      if (hh == 0) (DELTA ? red : part)[128 * 128 + row] = __uint_as_float(zr);
     }
-    uint32_t zr;
-    tmem_ld1(tZ + lrow, zr);
-    tmem_ld_wait();
-    part[128 * 128 + row] = __uint_as_float(zr);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 9) {
+      __syncwarp();
+      tc_fence_after();
+      tmem_dealloc(tmem, 512);
+    }
   }
-  tc_fence_before();
+  if (!DELTA) return;
+  // ------------------------------------------------------------ delta: cluster reduction
   __syncthreads();
-  if (warp == 0) {
-    __syncwarp();
-    tc_fence_after();
-    tmem_dealloc(tmem, 512);
+  cluster_sync();  // every CTA of the head has staged its partial
+  {
+    constexpr int E4 = (128 * 128 + 128) / 4;  // float4 elements of [M | z]
+    const int per = (E4 + a.G - 1) / a.G;
+    const int e4_begin = grp * per, e4_end = min(E4, e4_begin + per);
+    const uint32_t red_addr = smem_u32(red);
+    const bool snap_next = s + 1 < a.S;
+    const long long sb = (long long)bh * a.S + s + 1;
+    for (int e4 = e4_begin + (int)threadIdx.x; e4 < e4_end; e4 += blockDim.x) {
+      const int e = 4 * e4;
+      float4* st = e < 16384 ? reinterpret_cast<float4*>(&a.M[(long long)bh * 16384 + e])
+                             : reinterpret_cast<float4*>(&a.z[(long long)bh * 128 + (e - 16384)]);
+      float4 acc = *st;
+      for (int g = 0; g < a.G; ++g) {
+        const float4 v = ld_dsmem_f4(mapa_shared(red_addr + 16u * (uint32_t)e4, (uint32_t)g));
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+      }
+      *st = acc;
+      if (snap_next) {
+        if (e < 16384) {
+          const int i = e >> 7, j = e & 127;
+          __nv_bfloat16* d = a.snapMt + sb * 16384 + (long long)j * 128 + i;
+          d[0] = __float2bfloat16_rn(acc.x);
+          d[128] = __float2bfloat16_rn(acc.y);
+          d[256] = __float2bfloat16_rn(acc.z);
+          d[384] = __float2bfloat16_rn(acc.w);
+        } else {
+          *reinterpret_cast<float4*>(&a.snapzw[sb * 128 + (e - 16384)]) = acc;
+        }
+      }
+    }
   }
+  cluster_sync();  // peers have finished reading this CTA's shared memory
 }
 
 }  // namespace tc
