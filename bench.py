@@ -469,6 +469,7 @@ def parse(argv=None):
     ap.add_argument("--workload", choices=sorted(W.WORKLOADS), default=W.LAYER_1B.name)
     ap.add_argument("--mode", choices=("linear", "delta"), default=None)
     ap.add_argument("--force-simt", action="store_true", help="time the CUDA-core kernels instead")
+    ap.add_argument("--shape", default=None, help="B,H,L,N override of the workload's sizes (for profiling)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
@@ -479,6 +480,9 @@ def parse(argv=None):
 def main(argv=None):
     args = parse(argv)
     w = W.WORKLOADS[args.workload]
+    if args.shape:
+        B, H, L, N = (int(x) for x in args.shape.split(","))
+        w = w.with_(name=f"{w.name}@{B}x{H}x{L}x{N}", B=B, H=H, L=L, N=N)
     mode = {"linear": LINEAR, "delta": DELTA}[args.mode] if args.mode else w.modes[0]
     if args.warmup < 3 and args.impl == "ours":
         raise SystemExit("--warmup must be at least 3")

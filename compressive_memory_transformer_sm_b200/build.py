@@ -47,12 +47,36 @@ def build(force: bool = False, verbose: bool = False) -> str:
     cmd = [nvcc_path(), ARCH, "-O3", "-std=c++17", "-lineinfo", "-shared", "-Xcompiler", "-fPIC",
            "-Xcompiler", "-fvisibility=hidden", "-I", os.path.join(ROOT, "include"),
            "-o", tmp, os.path.join(CSRC, "infini_attn.cu")]
+    extra = os.environ.get("INFINI_NVCC_FLAGS", "").split()
+    cmd[1:1] = extra + ["-Xptxas=-v"]
     if verbose:
-        cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd), flush=True)
-    subprocess.run(cmd, check=True)
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    if res.returncode != 0:
+        sys.stderr.write(res.stdout + res.stderr)
+        raise RuntimeError(f"nvcc failed with exit code {res.returncode}")
+    if verbose:
+        print(res.stdout + res.stderr, flush=True)
+    check_register_split(res.stdout + res.stderr)
     os.replace(tmp, LIB)
     return LIB
+
+
+def check_register_split(ptxas_log: str, kernel: str = "attn_tc_kernel", want: int = 168) -> None:
+    """The attention kernel redistributes registers between warpgroups (setmaxnreg)
+    assuming it was launched with exactly `want` registers per thread; any other
+    allocation could make a register increase wait forever, so refuse to build."""
+    lines = ptxas_log.splitlines()
+    for i, line in enumerate(lines):
+        if "Compiling entry function" in line and kernel in line:
+            for nxt in lines[i + 1:i + 6]:
+                if "Used" in nxt and "registers" in nxt:
+                    used = int(nxt.split("Used")[1].split("registers")[0])
+                    if used != want:
+                        raise RuntimeError(f"{kernel} uses {used} registers per thread, its register split "
+                                           f"assumes {want}: refusing to build")
+                    return
+    raise RuntimeError(f"ptxas report for {kernel} not found: cannot verify its register split")
 
 
 if __name__ == "__main__":

@@ -396,6 +396,11 @@ int forward_impl(infini_attn_params p) {
   return rc;
 }
 
+__global__ void selftest_exp2_kernel(const float* x, float* y, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) y[i] = exp2_poly(x[i]);
+}
+
 __global__ void selftest_wait_kernel(unsigned long long limit_ns) {
   __shared__ __align__(8) unsigned long long bar;
   const uint32_t b = smem_u32(&bar);
@@ -530,6 +535,15 @@ int infini_attn_selftest_timeout(unsigned limit_us, cudaStream_t stream) {
   return infini_attn_device_status(0);
 }
 
+int infini_attn_selftest_exp2(const float* x, float* y, int n, cudaStream_t stream) {
+  if (!x || !y || n < 0) return INFINI_ERR_INVALID_ARG;
+  if (n == 0) return INFINI_OK;
+  int rc = check_device(false);
+  if (rc != INFINI_OK) return rc;
+  selftest_exp2_kernel<<<(n + 255) / 256, 256, 0, stream>>>(x, y, n);
+  return launch_status();
+}
+
 int infini_attn_path(int dk, int dv, int mode, int flags) {
   Plan pl;
   int rc = make_plan(1, 1, 1, 1, dk, dv, mode, flags, &pl);
@@ -538,6 +552,16 @@ int infini_attn_path(int dk, int dv, int mode, int flags) {
 }
 
 size_t infini_attn_params_size(void) { return sizeof(infini_attn_params); }
+
+#ifdef INFINI_ATTN_TRACE
+// Tuning builds only: copies the attention pipeline timestamps to the host.
+INFINI_API int infini_attn_debug_trace(unsigned long long* host, int n) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return INFINI_ERR_LAUNCH;
+  return cudaMemcpyFromSymbol(host, tc::g_attn_trace, sizeof(unsigned long long) * std::min(n, 4096)) == cudaSuccess
+             ? INFINI_OK
+             : INFINI_ERR_LAUNCH;
+}
+#endif
 
 int infini_attn_profile_enable(int phase_mask) {
   if (phase_mask < 0 || phase_mask > 7) return INFINI_ERR_INVALID_ARG;

@@ -5,8 +5,37 @@
 
 #include "sm100_common.cuh"
 
+// Softmax tuning knobs (compile time): every INFINI_POLY_EVERY-th pair of
+// exponentials runs on the FMA pipe (0 = none), and P is packed to bf16 on the
+// integer pipe when INFINI_PACK_ALU is 1.
+#ifndef INFINI_POLY_EVERY
+#define INFINI_POLY_EVERY 0
+#endif
+#ifndef INFINI_PACK_ALU
+#define INFINI_PACK_ALU 0
+#endif
+// 1: scale-and-subtract and the row sum use packed fp32x2 instructions.
+#ifndef INFINI_F32X2
+#define INFINI_F32X2 1
+#endif
+
 namespace infini {
 namespace tc {
+
+// Pipeline timestamps of one CTA (block INFINI_ATTN_TRACE) for tuning builds:
+// slot = 8 * (tile) + event; softmax warpgroup k writes at 1024 * k, the MMA
+// thread at 2048.  Compiled out unless INFINI_ATTN_TRACE is defined.
+#ifdef INFINI_ATTN_TRACE
+__device__ unsigned long long g_attn_trace[4096];
+#define ATTN_TRACE(cond, slot)                                                                   \
+  do {                                                                                           \
+    if ((cond) && blockIdx.x == INFINI_ATTN_TRACE && (slot) < 4096) g_attn_trace[(slot)] = clock64(); \
+  } while (0)
+#else
+#define ATTN_TRACE(cond, slot) \
+  do {                         \
+  } while (0)
+#endif
 
 struct AttnArgs {
   const float* beta;
@@ -22,42 +51,57 @@ struct AttnArgs {
 };
 
 // Shared memory of the attention kernel (offsets from a 1024-aligned base).
+constexpr int kKStages = 3;          // K ring depth (V ring: 2)
 constexpr uint32_t kA_Q0 = 0;
 constexpr uint32_t kA_Q1 = 32768;
-constexpr uint32_t kA_K0 = 65536;    // K ring: 2 stages of 32 KB
-constexpr uint32_t kA_V0 = 131072;   // V ring: 2 stages of 32 KB
-constexpr uint32_t kA_Z = 196608;
+constexpr uint32_t kA_K0 = 65536;    // K ring: 3 stages of 32 KB
+constexpr uint32_t kA_V0 = kA_K0 + kKStages * 32768u;  // V ring: 2 stages of 32 KB
+constexpr uint32_t kA_Z = kA_V0 + 2 * 32768u;
 constexpr uint32_t kA_BAR = kA_Z + 512;
-constexpr uint32_t kA_TMEMSLOT = kA_BAR + 256;
-constexpr uint32_t kAttnSmem = kA_TMEMSLOT + 16 + 1024;  // + alignment slack
-constexpr int kAttnThreads = 320;
+constexpr int kAttnThreads = 384;
+// Register split: the kernel launches with 168 registers per thread (384 x 168
+// = 64512); the load/MMA warpgroup gives back to 88 and the two softmax
+// warpgroups take 208: 2 x 128 x 208 + 128 x 88 = 64512 (the split with no
+// spills on either side).  The build checks
+// that ptxas allocated exactly kAttnLaunchRegs, else an increase could wait
+// forever.
+constexpr uint32_t kAttnLaunchRegs = 168, kAttnSoftmaxRegs = 208, kAttnOtherRegs = 88;
+static_assert(2 * 128 * kAttnSoftmaxRegs + 128 * kAttnOtherRegs == kAttnThreads * kAttnLaunchRegs,
+              "register split must add up to the launch allocation");
 
 // Barrier indices.
 enum : int {
   B_Q = 0,
   B_KF0 = 1,   // K stage full (2)
   B_VF0 = 3,   // V stage full (2)
-  B_KVE0 = 5,  // K/V stage free (2)
+  B_KE0 = 5,   // K stage free: both S products of that key tile done (2)
   B_SF0 = 7,   // S of query tile k ready (2)
   B_PF0 = 9,   // P of query tile k written (2, 128 arrivals)
   B_SQ0 = 11,  // sigma(Q) of query tile k written (2, 128 arrivals)
   B_MEM0 = 13, // sigma(Q_k) M_{s-1} ready (2)
-  B_COUNT = 15
+  B_VE0 = 15,  // V stage free: both P V products of that key tile done (2)
+  B_KF2 = 17,  // third K stage full
+  B_KE2 = 18,  // third K stage free
+  B_COUNT = 19
 };
+constexpr uint32_t kA_TMEMSLOT = kA_BAR + 8 * B_COUNT;
+constexpr uint32_t kAttnSmem = kA_TMEMSLOT + 16 + 1024;  // + alignment slack
+static_assert(kAttnSmem <= 232448, "attention kernel exceeds 227 KB of shared memory");
 
 // One CTA computes two adjacent 128-row query tiles (2m, 2m+1) of one
 // (b, h, segment), sharing every K/V tile load between them.
 // Warps 0-3: softmax warpgroup of query tile 2m; warps 4-7: of tile 2m+1
 // (thread = query row = TMEM lane).  Warp 8 loads (TMA), warp 9 issues the
-// MMAs and owns TMEM.  TMEM columns: S of tile 2m [0,128), S of tile 2m+1
+// MMAs and owns TMEM, warps 10-11 only complete their warpgroup.  TMEM columns: S of tile 2m [0,128), S of tile 2m+1
 // [128,256), O of tile 2m [256,384), O of tile 2m+1 [384,512).  P (bf16)
 // overwrites the first 64 columns of its S buffer and feeds the P V product
 // from TMEM; after the last P V product the S buffer receives sigma(Q) M_{s-1}.
 //
 // MMA issue order (k = query tile): S_0(0) S_1(0) | PV_0(j-1) S_0(j) PV_1(j-1)
-// S_1(j) | ... so that one softmax warpgroup works while the tensor cores
-// serve the other, and "S_k(j) complete" implies "PV_k(j-1) complete": the
-// O rescale of the softmax needs no extra wait.
+// S_1(j) | ... : the strict alternation keeps the two softmax warpgroups half
+// a period apart, so one works while the tensor cores serve the other, and
+// "S_k(j) complete" implies "PV_k(j-1) complete": the O rescale of the
+// softmax needs no extra wait.
 //
 // CTAs are ordered by groups of GS segments (about one wave of CTAs per
 // group, so the group's K/V stays in L2), heaviest pair first inside a group.
@@ -91,6 +135,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   auto sK = [&](int st) { return base + kA_K0 + (uint32_t)st * kTileBytes; };
   auto sV = [&](int st) { return base + kA_V0 + (uint32_t)st * kTileBytes; };
   auto bar = [&](int i) { return base + kA_BAR + 8u * (uint32_t)i; };
+  // K tile j lives in stage j % 3; its barriers (full / free) and their phase (j / 3) & 1
+  auto kfull = [&](int j) { const int st = j % kKStages; return bar(st < 2 ? B_KF0 + st : B_KF2); };
+  auto kfree = [&](int j) { const int st = j % kKStages; return bar(st < 2 ? B_KE0 + st : B_KE2); };
+  auto kph = [&](int j) { return (uint32_t)((j / kKStages) & 1); };
+  auto sKt = [&](int j) { return sK(j % kKStages); };
   float* zs = reinterpret_cast<float*>(gbase + kA_Z);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kA_TMEMSLOT);
 
@@ -99,7 +148,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(B_KF0 + i), 1);
       mbar_init(bar(B_VF0 + i), 1);
-      mbar_init(bar(B_KVE0 + i), 1);
+      mbar_init(bar(B_KE0 + i), 1);
+      mbar_init(bar(B_VE0 + i), 1);
+      if (i == 0) {
+        mbar_init(bar(B_KF2), 1);
+        mbar_init(bar(B_KE2), 1);
+      }
       mbar_init(bar(B_SF0 + i), 1);
       mbar_init(bar(B_PF0 + i), 128);
       mbar_init(bar(B_SQ0 + i), 128);
@@ -117,6 +171,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  if (warp >= 8) {
+  regs_decrease<kAttnOtherRegs>();
   if (warp == 8) {
     if (lane == 0) {
       // ------------------------------------------------------------ producer
@@ -130,23 +186,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tma_load_4d(sQ(0) + kBox, &tm_q, bar(B_Q), 64, lq, h, b);
       tma_load_4d(sQ(1), &tm_q, bar(B_Q), 0, lq + kTile, h, b);
       tma_load_4d(sQ(1) + kBox, &tm_q, bar(B_Q), 64, lq + kTile, h, b);
-      for (int j = 0; j < nk1; ++j) {
-        const int st = j & 1;
-        if (j >= 2) mbar_wait(bar(B_KVE0 + st), ((j - 2) >> 1) & 1);
-        const int lk = (int)(seg0 + (long long)j * kTile);
-        mbar_expect_tx(bar(B_KF0 + st), kTileBytes);
-        tma_load_4d(sK(st), &tm_k, bar(B_KF0 + st), 0, lk, h, b);
-        tma_load_4d(sK(st) + kBox, &tm_k, bar(B_KF0 + st), 64, lk, h, b);
-        mbar_expect_tx(bar(B_VF0 + st), kTileBytes);
-        tma_load_4d(sV(st), &tm_v, bar(B_VF0 + st), 0, lk, h, b);
-        tma_load_4d(sV(st) + kBox, &tm_v, bar(B_VF0 + st), 64, lk, h, b);
+      // K tile j goes in once the S products of key tile j-2 are done; V trails
+      // K by one tile (V tile j once the P V products of key tile j-2 are
+      // done), so that a pending V never holds back the next K.
+      for (int j = 0; j <= nk1; ++j) {
+        if (j < nk1) {
+          const int lk = (int)(seg0 + (long long)j * kTile);
+          if (j >= kKStages) mbar_wait(kfree(j), kph(j - kKStages));
+          mbar_expect_tx(kfull(j), kTileBytes);
+          tma_load_4d(sKt(j), &tm_k, kfull(j), 0, lk, h, b);
+          tma_load_4d(sKt(j) + kBox, &tm_k, kfull(j), 64, lk, h, b);
+        }
+        if (j >= 1) {
+          const int jv = j - 1, st = jv & 1;
+          const int lk = (int)(seg0 + (long long)jv * kTile);
+          if (jv >= 2) mbar_wait(bar(B_VE0 + st), ((jv - 2) >> 1) & 1);
+          mbar_expect_tx(bar(B_VF0 + st), kTileBytes);
+          tma_load_4d(sV(st), &tm_v, bar(B_VF0 + st), 0, lk, h, b);
+          tma_load_4d(sV(st) + kBox, &tm_v, bar(B_VF0 + st), 64, lk, h, b);
+        }
       }
       // M_{s-1}^T (bf16 snapshot) enters the K ring as tile nk1.
-      const int st = nk1 & 1;
-      mbar_wait(bar(B_KVE0 + st), ((nk1 - 2) >> 1) & 1);
-      mbar_expect_tx(bar(B_KF0 + st), kTileBytes);
-      tma_load_2d(sK(st), &tm_mt, bar(B_KF0 + st), 0, seg * 128);
-      tma_load_2d(sK(st) + kBox, &tm_mt, bar(B_KF0 + st), 64, seg * 128);
+      if (nk1 >= kKStages) mbar_wait(kfree(nk1), kph(nk1 - kKStages));
+      mbar_expect_tx(kfull(nk1), kTileBytes);
+      tma_load_2d(sKt(nk1), &tm_mt, kfull(nk1), 0, seg * 128);
+      tma_load_2d(sKt(nk1) + kBox, &tm_mt, kfull(nk1), 64, seg * 128);
     }
   } else if (warp == 9) {
     if (lane == 0) {
@@ -155,16 +219,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       constexpr uint32_t idesc_pv = idesc_bf16(128, 128, 0, 1);
       const int nk0 = nk1 - 1;
       auto issue_s = [&](int k, int j) {
-        const int st = j & 1;
+        const uint32_t kt = sKt(j);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + (uint32_t)k * 128u, kmajor_desc(sQ(k), kk), kmajor_desc(sK(st), kk), idesc_kk,
+          mma_ss(tmem + (uint32_t)k * 128u, kmajor_desc(sQ(k), kk), kmajor_desc(kt, kk), idesc_kk,
                  kk > 0 ? 1u : 0u);
         mma_commit(bar(B_SF0 + k));
       };
       auto issue_pv = [&](int k, int j) {  // P of tile k, key tile j; call in order j = 0, 1, ...
         const int st = j & 1;
         mbar_wait(bar(B_PF0 + k), j & 1);
+        ATTN_TRACE(true, 2048 + 8 * (j + 1) + 3 + k);
         mbar_wait(bar(B_VF0 + st), (j >> 1) & 1);
         tc_fence_after();
 #pragma unroll
@@ -173,37 +238,44 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                  mnmajor_desc(sV(st), kk), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
       };
       mbar_wait(bar(B_Q), 0);
-      mbar_wait(bar(B_KF0), 0);
+      mbar_wait(kfull(0), 0);
       tc_fence_after();
       issue_s(0, 0);
       issue_s(1, 0);
+      mma_commit(kfree(0));
       for (int j = 1; j < nk1; ++j) {
-        const int st = j & 1;
-        mbar_wait(bar(B_KF0 + st), (j >> 1) & 1);
+        mbar_wait(kfull(j), kph(j));
+        ATTN_TRACE(true, 2048 + 8 * j + 0);
         tc_fence_after();
         if (j - 1 < nk0) issue_pv(0, j - 1);
+        ATTN_TRACE(true, 2048 + 8 * j + 1);
         if (j < nk0) issue_s(0, j);
+        ATTN_TRACE(true, 2048 + 8 * j + 5);
         issue_pv(1, j - 1);
-        mma_commit(bar(B_KVE0 + ((j - 1) & 1)));
+        ATTN_TRACE(true, 2048 + 8 * j + 2);
+        mma_commit(bar(B_VE0 + ((j - 1) & 1)));
         issue_s(1, j);
+        mma_commit(kfree(j));
       }
       issue_pv(1, nk1 - 1);
-      mma_commit(bar(B_KVE0 + ((nk1 - 1) & 1)));
+      mma_commit(bar(B_VE0 + ((nk1 - 1) & 1)));
       // memory read: sigma(Q_k) (written over Q_k by the softmax warps) times M_{s-1}
-      const int stm = nk1 & 1;
-      mbar_wait(bar(B_KF0 + stm), (nk1 >> 1) & 1);
+      mbar_wait(kfull(nk1), kph(nk1));
+      const uint32_t mt = sKt(nk1);
 #pragma unroll 1
       for (int k = 0; k < 2; ++k) {
         mbar_wait(bar(B_SQ0 + k), 0);
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + (uint32_t)k * 128u, kmajor_desc(sQ(k), kk), kmajor_desc(sK(stm), kk), idesc_kk,
+          mma_ss(tmem + (uint32_t)k * 128u, kmajor_desc(sQ(k), kk), kmajor_desc(mt, kk), idesc_kk,
                  kk > 0 ? 1u : 0u);
         mma_commit(bar(B_MEM0 + k));
       }
     }
+  }
   } else {
+    regs_increase<kAttnSoftmaxRegs>();
     // -------------------------------------------------------------- softmax WGs
     const int k = warp >> 2;            // query tile 2m + k
     const int row = (warp & 3) * 32 + lane;  // query row in the tile = TMEM lane
@@ -213,8 +285,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int nk = nk1 - 1 + k;
     const float c = a.scale_log2;
     float m_ref = 0.f, l = 0.f;
+    const bool tr = (row == 0);
     for (int j = 0; j < nk; ++j) {
+      ATTN_TRACE(tr, 1024 * k + 8 * j + 0);
       mbar_wait(bar(B_SF0 + k), j & 1);
+      ATTN_TRACE(tr, 1024 * k + 8 * j + 1);
       tc_fence_after();
       uint32_t x[128];
       {
@@ -239,6 +314,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
       for (int e = 4; e < 128; ++e) mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(x[e]));
       const float mxs = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * c;
+      ATTN_TRACE(tr, 1024 * k + 8 * j + 2);
       // Move the reference max only when the row max grows by more than 2^8:
       // O / l stays exact for any reference, and p stays below 256.
       const float m_new = (j == 0) ? mxs : (mxs > m_ref + 8.f ? mxs : m_ref);
@@ -263,12 +339,34 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int e = 0; e < 64; ++e) {
-        const float p0 = ex2_approx(fmaf(__uint_as_float(x[2 * e]), c, nm));
-        const float p1 = ex2_approx(fmaf(__uint_as_float(x[2 * e + 1]), c, nm));
-        ls[e & 3] += p0 + p1;
-        x[e] = pack_bf16x2(p0, p1);
+        float a0, a1;
+        if (INFINI_F32X2) {
+          fma2(a0, a1, __uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1]), c, c, nm, nm);
+        } else {
+          a0 = fmaf(__uint_as_float(x[2 * e]), c, nm);
+          a1 = fmaf(__uint_as_float(x[2 * e + 1]), c, nm);
+        }
+        float p0, p1;
+        if (INFINI_POLY_EVERY > 0 && (e % (INFINI_POLY_EVERY > 0 ? INFINI_POLY_EVERY : 1)) == INFINI_POLY_EVERY - 1) {
+          p0 = exp2_poly(a0);
+          p1 = exp2_poly(a1);
+        } else {
+          p0 = ex2_approx(a0);
+          p1 = ex2_approx(a1);
+        }
+        if (INFINI_F32X2) {
+          if ((e & 1) == 0) {
+            add2(ls[0], ls[1], ls[0], ls[1], p0, p1);
+          } else {
+            add2(ls[2], ls[3], ls[2], ls[3], p0, p1);
+          }
+        } else {
+          ls[e & 3] += p0 + p1;
+        }
+        x[e] = INFINI_PACK_ALU ? pack_bf16x2_alu(p0, p1) : pack_bf16x2(p0, p1);
       }
       l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      ATTN_TRACE(tr, 1024 * k + 8 * j + 3);
       {
         uint32_t (&p0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&x[0]);
         uint32_t (&p1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&x[32]);
@@ -278,6 +376,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(B_PF0 + k));
+      ATTN_TRACE(tr, 1024 * k + 8 * j + 4);
     }
     // Every Q_k K^T product has completed: overwrite this row of Q_k with
     // sigma(Q_k) (bf16) for the memory read, and form the fp32 denominator

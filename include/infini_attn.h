@@ -204,6 +204,14 @@ INFINI_API int infini_attn_profile_read(double* ms, long long* launches, int res
 /* Number of kernels this library has launched in this process (all phases). */
 INFINI_API long long infini_attn_launch_count(void);
 
+/*
+ * Self-test of the polynomial 2^x used inside the attention kernel to take
+ * part of the exponentials off the exponential unit: y[i] = 2^x[i] for n
+ * device floats, asynchronously on `stream`.  Relative error <= 1e-4 for
+ * x in [-125, 125]; smaller x give about 2^-125.
+ */
+INFINI_API int infini_attn_selftest_exp2(const float* x, float* y, int n, cudaStream_t stream);
+
 /* sizeof(infini_attn_params), for bindings that build the struct themselves. */
 INFINI_API size_t infini_attn_params_size(void);
 

@@ -276,3 +276,18 @@ def test_workload_8b_long_both_rules():
         out, M, z = run(q, k, v, beta, w.N, mode)
         _sample_check_head(q, k, v, beta, out, M, z, w.B - 1, w.H - 1, w.N, mode, segments=[0, 1, w.segments - 1])
         del out
+
+
+def test_polynomial_exp2_error_bound():
+    """The FMA-pipe 2^x used for part of the softmax stays within its fitted error bound."""
+    x = torch.cat([torch.linspace(-125.0, 125.0, 1_000_001), torch.tensor([-126.5, -300.0, -float("inf")])])
+    xd = x.to(DEV)
+    y = torch.empty_like(xd)
+    assert api.infini_attn_selftest_exp2(xd, y) == api.INFINI_OK
+    torch.cuda.synchronize()
+    got = y.double().cpu().numpy()
+    want = np.exp2(x.double().numpy())
+    inner = slice(0, 1_000_001)
+    rel = np.abs(got[inner] / want[inner] - 1.0)
+    assert float(rel.max()) <= 1e-4, float(rel.max())
+    assert np.all(got[-3:] <= 2.0 ** -124) and np.all(got[-3:] >= 0.0)
