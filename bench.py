@@ -14,9 +14,11 @@ collective on the data path): weak scaling, value = tokens of all ranks /
 max over ranks of the step time.
 
 Timing: W warm-up steps, then K steps, each bracketed by CUDA events on the
-launching stream, with a 256 MB buffer written between steps (outside the
-events) so that no step starts with its inputs in the 126 MB L2; a barrier
-and a device synchronisation on both sides of the timed region.
+launching stream.  Between steps, outside the events, the initial state is
+reset to M_0 = 0, z_0 = 0 and a 1 GiB buffer is written so that no step
+starts with its inputs in the 126 MB L2 (the write also lets the host
+enqueue the step before the GPU reaches it).  A barrier and a device
+synchronisation on both sides of the timed region.
 
 ``--impl reference`` times the fp64 CPU oracle on the host cores instead
 (each step a bounded sample of the same workload); under torchrun only
@@ -46,7 +48,7 @@ from compressive_memory_transformer_sm_b200 import workloads as W  # noqa: E402
 
 METRIC = "Infini-attn fwd tokens/s per layer; TFLOP/s and % of B200 bf16 tensor peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-FLUSH_BYTES = 256 << 20
+FLUSH_BYTES = 1 << 30
 
 
 # ------------------------------------------------------------------ work model
@@ -262,9 +264,11 @@ def run_ours(args, w: W.Workload, mode: int):
         q, k, v = seg(q), seg(k), seg(v)
         out = torch.empty_like(v)
 
-    def step():
+    def reset_state():  # M_0 = 0, z_0 = 0 are inputs: set before a step's events
         M.zero_()
         z.zero_()
+
+    def step():
         if w.streaming:
             for s in range(w.segments):
                 api.infini_attn_segment_step(q[s], k[s], v[s], beta, M, z, out[s], mode, stream=stream)
@@ -275,6 +279,7 @@ def run_ours(args, w: W.Workload, mode: int):
 
     sampler = ClockSampler(local)
     for _ in range(args.warmup):
+        reset_state()
         flush.fill_(1)
         step()
     torch.cuda.synchronize(dev)
@@ -288,6 +293,7 @@ def run_ours(args, w: W.Workload, mode: int):
     launches0 = api.infini_attn_launch_count()
     wall0 = time.perf_counter()
     for i in range(args.steps):
+        reset_state()
         flush.fill_(i & 0xff)
         evs[i][0].record(stream)
         step()
@@ -308,6 +314,7 @@ def run_ours(args, w: W.Workload, mode: int):
     # per-phase breakdown: a second pass of K steps with every launch bracketed
     api.infini_attn_profile_enable(7)
     for i in range(args.steps):
+        reset_state()
         flush.fill_(i & 0xff)
         step()
     torch.cuda.synchronize(dev)
@@ -338,7 +345,7 @@ def run_ours(args, w: W.Workload, mode: int):
         "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "N": w.N, "dk": w.dk, "dv": w.dv,
                    "mode": W.MODE_NAMES[mode], "path": "simt" if args.force_simt else "tensor",
                    "streaming_steps": w.segments if w.streaming else 0,
-                   "l2": "256 MB buffer written between timed steps (outside the step events)",
+                   "l2": "1 GiB buffer written between timed steps (outside the step events)",
                    "parallelism": f"independent problem per rank x{world}"},
         "tflops": (f_attn + f_upd) * world / (ms * 1e-3) / 1e12,
         "pct_of_bf16_peak": 100.0 * (f_attn + f_upd) / (ms * 1e-3) / 1e12 / peak,
