@@ -80,7 +80,7 @@ struct Plan {
   size_t off_snapM, off_snapz, off_part, total;
 };
 
-// Workspace: per-segment snapshots of M_{s-1} (bf16 transposed for the tensor
+// Workspace: per-segment snapshots of M_{s-1} (bf16 [dk][dv] for the tensor
 // cores, fp32 otherwise) and z_{s-1} (fp32), and the update partials
 // ([BH][S][G] for the linear scan, [BH][1][G] reused per segment for delta).
 int make_plan(int B, int H, long long L, int N, int dk, int dv, int mode, int flags, Plan* p) {
@@ -242,12 +242,12 @@ int run_simt(const infini_attn_params& p, const Plan& pl, char* ws, float scale)
 
 int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale) {
   CUtensorMap tm_q, tm_k, tm_v, tm_mt;
-  __nv_bfloat16* snapMt = reinterpret_cast<__nv_bfloat16*>(ws + pl.off_snapM);
+  __nv_bfloat16* snapM16 = reinterpret_cast<__nv_bfloat16*>(ws + pl.off_snapM);
   float* snapz = reinterpret_cast<float*>(ws + pl.off_snapz);
   float* part = reinterpret_cast<float*>(ws + pl.off_part);
   const int BH = p.B * p.H, E = 128 * 128;
   if (!encode_bhld(&tm_q, p.q, p.B, p.H, p.L, p.q_stride) || !encode_bhld(&tm_k, p.k, p.B, p.H, p.L, p.k_stride) ||
-      !encode_bhld(&tm_v, p.v, p.B, p.H, p.L, p.v_stride) || !encode_rows(&tm_mt, snapMt, (long long)BH * pl.S * 128))
+      !encode_bhld(&tm_v, p.v, p.B, p.H, p.L, p.v_stride) || !encode_rows(&tm_mt, snapM16, (long long)BH * pl.S * 128))
     return INFINI_ERR_LAUNCH;
   static std::once_flag once;
   std::call_once(once, [] {
@@ -259,7 +259,7 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale) {
   });
   const dim3 sgrid((E + 128 + 255) / 256, BH);
   tc::UpdArgs ua;
-  ua.snapz = snapz; ua.partial = part; ua.M = p.M; ua.z = p.z; ua.snapMt = snapMt; ua.snapzw = snapz;
+  ua.snapz = snapz; ua.partial = part; ua.M = p.M; ua.z = p.z; ua.snapM = snapM16; ua.snapzw = snapz;
   ua.B = p.B; ua.H = p.H; ua.S = pl.S; ua.N = p.N; ua.L = p.L;
   ua.G = pl.G; ua.cpb = pl.cpb;
   if (!pl.delta) {
@@ -270,12 +270,12 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale) {
           tm_k, tm_v, tm_mt, ua);
     }
     LaunchScope ls(kPhaseState, p.stream);
-    state_kernel<<<sgrid, 256, 0, p.stream>>>(p.M, p.z, part, 128, 128, pl.S, 0, 0, pl.S, pl.G, nullptr, snapMt,
+    state_kernel<<<sgrid, 256, 0, p.stream>>>(p.M, p.z, part, 128, 128, pl.S, 0, 0, pl.S, pl.G, nullptr, snapM16,
                                               snapz);
   } else {
     {
       LaunchScope ls(kPhaseState, p.stream);
-      state_kernel<<<sgrid, 256, 0, p.stream>>>(p.M, p.z, part, 128, 128, pl.S, 2, 0, 1, pl.G, nullptr, snapMt,
+      state_kernel<<<sgrid, 256, 0, p.stream>>>(p.M, p.z, part, 128, 128, pl.S, 2, 0, 1, pl.G, nullptr, snapM16,
                                                 snapz);
     }
     ua.nseg = 1;

@@ -146,12 +146,12 @@ __global__ void __launch_bounds__(256) simt_update_kernel(const T* __restrict__ 
 //   op 1 (delta step of segment s): add the G partials of the one segment
 //        in `partial`, store, and snapshot as segment s + 1 if it exists.
 //   op 2 (snapshot only): snapshot the state as segment s.
-// Snapshots are fp32 [BH][S][dk][dv] (snapM32) or, for the tensor-core
-// kernels, bf16 transposed [BH][S][dv][dk] (snapMt16); z snapshots fp32.
+// Snapshots are fp32 [BH][S][dk][dv] (snapM32) and/or, for the tensor-core
+// kernels, bf16 [BH][S][dk][dv] (snapM16); z snapshots fp32.
 __global__ void __launch_bounds__(256) state_kernel(float* __restrict__ M, float* __restrict__ z,
                                                     const float* __restrict__ partial, int dk, int dv, int S, int op,
                                                     int s, int nseg, int G, float* __restrict__ snapM32,
-                                                    __nv_bfloat16* __restrict__ snapMt16,
+                                                    __nv_bfloat16* __restrict__ snapM16,
                                                     float* __restrict__ snapz) {
   const int bh = blockIdx.y;
   const int e = blockIdx.x * 256 + threadIdx.x;
@@ -164,10 +164,7 @@ __global__ void __launch_bounds__(256) state_kernel(float* __restrict__ M, float
     const long long base = (long long)bh * S + seg;
     if (e < E) {
       if (snapM32) snapM32[base * E + e] = val;
-      if (snapMt16) {
-        const int i = e / dv, j = e - i * dv;
-        snapMt16[base * E + (long long)j * dk + i] = __float2bfloat16_rn(val);
-      }
+      if (snapM16) snapM16[base * E + e] = __float2bfloat16_rn(val);
     } else {
       snapz[base * dk + (e - E)] = val;
     }

@@ -206,7 +206,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tma_load_4d(sV(st) + kBox, &tm_v, bar(B_VF0 + st), 64, lk, h, b);
         }
       }
-      // M_{s-1}^T (bf16 snapshot) enters the K ring as tile nk1.
+      // M_{s-1} (bf16 snapshot, [dk][dv]) enters the K ring as tile nk1.
       if (nk1 >= kKStages) mbar_wait(kfree(nk1), kph(nk1 - kKStages));
       mbar_expect_tx(kfull(nk1), kTileBytes);
       tma_load_2d(sKt(nk1), &tm_mt, kfull(nk1), 0, seg * 128);
@@ -261,14 +261,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mma_commit(bar(B_VE0 + ((nk1 - 1) & 1)));
       // memory read: sigma(Q_k) (written over Q_k by the softmax warps) times M_{s-1}
       mbar_wait(kfull(nk1), kph(nk1));
-      const uint32_t mt = sKt(nk1);
+      const uint32_t mt = sKt(nk1);  // M_{s-1} [dk][dv]: MN-major B operand (like V)
+      constexpr uint32_t idesc_mem = idesc_bf16(128, 128, 0, 1);
 #pragma unroll 1
       for (int k = 0; k < 2; ++k) {
         mbar_wait(bar(B_SQ0 + k), 0);
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + (uint32_t)k * 128u, kmajor_desc(sQ(k), kk), kmajor_desc(mt, kk), idesc_kk,
+          mma_ss(tmem + (uint32_t)k * 128u, kmajor_desc(sQ(k), kk), mnmajor_desc(mt, kk), idesc_mem,
                  kk > 0 ? 1u : 0u);
         mma_commit(bar(B_MEM0 + k));
       }

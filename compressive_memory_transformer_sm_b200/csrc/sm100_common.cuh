@@ -6,9 +6,9 @@
 // Operand tiles are 128 rows x 128 bf16 columns, held in shared memory as two
 // TMA boxes of 128 rows x 64 columns (16 KB each) with the 128-byte swizzle:
 // 16-byte chunk c of row r sits at chunk position c ^ (r % 8) of the row.
-// A tile is K-major when its rows are the MMA's M/N index (Q, K, sigma(Q),
-// M^T); it is MN-major when its rows are the MMA's K index (V, U, sigma(K)
-// read as sigma(K)^T).
+// A tile is K-major when its rows are the MMA's M/N index (Q, K, sigma(Q));
+// it is MN-major when its rows are the MMA's K index (V, U, the memory
+// snapshot M_{s-1} [dk][dv], sigma(K) read as sigma(K)^T).
 #pragma once
 
 #include "common.cuh"

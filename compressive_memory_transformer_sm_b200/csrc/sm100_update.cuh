@@ -38,7 +38,7 @@ struct UpdArgs {
   float* partial;               // [BH][nseg][G][128*128 + 128] (linear)
   float* M;                     // running state (delta)
   float* z;
-  __nv_bfloat16* snapMt;        // [BH][S][128][128] (delta: M_s^T for segment s+1)
+  __nv_bfloat16* snapM;         // [BH][S][128][128] bf16 [dk][dv] (delta: M_s for segment s+1)
   float* snapzw;                // [BH][S][128] (delta: z_s for segment s+1)
   int B, H, S, N;
   long long L;
@@ -53,7 +53,7 @@ struct UpdSmem {
   static constexpr uint32_t V0 = 65536;       // V ring; U_hi in place (delta)
   static constexpr uint32_t KLO = V0 + VST * 32768u;
   static constexpr uint32_t ULO = KLO + 32768u;                 // delta
-  static constexpr uint32_t MT = ULO + 32768u;                  // delta
+  static constexpr uint32_t MT = ULO + 32768u;                  // delta: M_{s-1} [dk][dv]
   static constexpr uint32_t ONES = DELTA ? MT + 32768u : KLO + 32768u;
   static constexpr uint32_t Z = ONES + 4096u;
   static constexpr uint32_t DENP = Z + 512u;  // [2 buffers][2 halves][128]
@@ -107,7 +107,7 @@ __global__ void __launch_bounds__(kUpdThreads, 1)
     auto bar = [&](int i) { return base + SL::BAR + 8u * (uint32_t)i; };
     auto sK = [&](int st) { return base + SL::K0 + (uint32_t)st * kTileBytes; };
     auto sV = [&](int st) { return base + SL::V0 + (uint32_t)st * kTileBytes; };
-    const uint32_t sKlo = base + SL::KLO, sUlo = base + SL::ULO, sMt = base + SL::MT, sOnes = base + SL::ONES;
+    const uint32_t sKlo = base + SL::KLO, sUlo = base + SL::ULO, sMs = base + SL::MT, sOnes = base + SL::ONES;
     float* zs = reinterpret_cast<float*>(gbase + SL::Z);
     float* denp = reinterpret_cast<float*>(gbase + SL::DENP);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + SL::SLOT);
@@ -149,8 +149,8 @@ __global__ void __launch_bounds__(kUpdThreads, 1)
         if (DELTA) {
           const int row = (bh * a.S + s) * 128;
           mbar_expect_tx(bar(U_MT), kTileBytes);
-          tma_load_2d(sMt, &tm_mt, bar(U_MT), 0, row);
-          tma_load_2d(sMt + kBox, &tm_mt, bar(U_MT), 64, row);
+          tma_load_2d(sMs, &tm_mt, bar(U_MT), 0, row);
+          tma_load_2d(sMs + kBox, &tm_mt, bar(U_MT), 64, row);
         }
         for (int c = 0; c < nchunks; ++c) {
           const int lt = (int)(seg_start + t_begin + (long long)c * kTile);
@@ -169,7 +169,7 @@ __global__ void __launch_bounds__(kUpdThreads, 1)
     } else if (warp == 9) {
       if (lane == 0) {
         // ---------------------------------------------------------- MMA issuer
-        constexpr uint32_t idesc_r = idesc_bf16(128, 128, 0, 0);
+        constexpr uint32_t idesc_r = idesc_bf16(128, 128, 0, 1);  // B = M_{s-1} [dk][dv], MN-major
         constexpr uint32_t idesc_m = idesc_bf16(128, 128, 1, 1);
         constexpr uint32_t idesc_z = idesc_bf16(128, 16, 1, 0);
         for (int c = 0; c < nchunks; ++c) {
@@ -180,7 +180,7 @@ __global__ void __launch_bounds__(kUpdThreads, 1)
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-              mma_ss(tR, kmajor_desc(sK(kst), kk), kmajor_desc(sMt, kk), idesc_r, kk > 0 ? 1u : 0u);
+              mma_ss(tR, kmajor_desc(sK(kst), kk), mnmajor_desc(sMs, kk), idesc_r, kk > 0 ? 1u : 0u);
             mma_commit(bar(U_R));
             mbar_wait(bar(U_U), c & 1);
           } else {
@@ -335,12 +335,8 @@ __global__ void __launch_bounds__(kUpdThreads, 1)
       *st = acc;
       if (snap_next) {
         if (e < 16384) {
-          const int i = e >> 7, j = e & 127;
-          __nv_bfloat16* d = a.snapMt + sb * 16384 + (long long)j * 128 + i;
-          d[0] = __float2bfloat16_rn(acc.x);
-          d[128] = __float2bfloat16_rn(acc.y);
-          d[256] = __float2bfloat16_rn(acc.z);
-          d[384] = __float2bfloat16_rn(acc.w);
+          *reinterpret_cast<uint2*>(a.snapM + sb * 16384 + e) =
+              make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
         } else {
           *reinterpret_cast<float4*>(&a.snapzw[sb * 128 + (e - 16384)]) = acc;
         }
