@@ -18,8 +18,9 @@ namespace tc {
 // handles value columns [64 hh, 64 hh + 64) of its token: sigma(K) split into
 // bf16 hi + lo parts, and for the delta rule U = V - R / den with
 // R = sigma(K)_hi M_{s-1} from the tensor cores and den = sigma(K) . z_{s-1}
-// in fp32, again split into hi + lo.  Warp 8 loads (TMA: K ring of 2 stages,
-// V ring of 2 stages (linear) or 1 (delta, where U overwrites V in place)),
+// in fp32, again split into hi + lo.  Warp 8 loads (TMA: K ring of 3 stages
+// (linear) or 2 (delta), V ring of 2 stages (linear) or 1 (delta, where U
+// overwrites V in place)),
 // warp 9 issues the MMAs:
 //   dM += sK_hi^T U_hi + sK_lo^T U_hi (+ sK_hi^T U_lo)   (fp32 in TMEM)
 //   dz += sK_hi^T 1 + sK_lo^T 1                        (N = 16 block of ones)
@@ -48,9 +49,10 @@ constexpr int kMaxDeltaCluster = 8;
 
 template <bool DELTA>
 struct UpdSmem {
-  static constexpr int VST = DELTA ? 1 : 2;
-  static constexpr uint32_t K0 = 0;           // K ring (2 x 32 KB); sigma(K)_hi in place
-  static constexpr uint32_t V0 = 65536;       // V ring; U_hi in place (delta)
+  static constexpr int KST = DELTA ? 2 : 3;   // K ring depth
+  static constexpr int VST = DELTA ? 1 : 2;   // V ring depth
+  static constexpr uint32_t K0 = 0;           // K ring (KST x 32 KB); sigma(K)_hi in place
+  static constexpr uint32_t V0 = KST * 32768u;  // V ring; U_hi in place (delta)
   static constexpr uint32_t KLO = V0 + VST * 32768u;
   static constexpr uint32_t ULO = KLO + 32768u;                 // delta
   static constexpr uint32_t MT = ULO + 32768u;                  // delta: M_{s-1} [dk][dv]
@@ -60,13 +62,14 @@ struct UpdSmem {
   static constexpr uint32_t BAR = DENP + 2048u;
   static constexpr uint32_t SLOT = BAR + 256u;
   static constexpr uint32_t BYTES = SLOT + 16u + 1024u;
+  static_assert(BYTES <= 232448, "update kernel exceeds 227 KB of shared memory");
   // delta: [dM (128 x 128) | dz (128)] fp32 staged for the cluster reduction,
   // over the K and V rings once every chunk has been consumed
   static constexpr uint32_t RED = 0;
 };
 
 enum : int {
-  U_KF0 = 0, U_KE0 = 2, U_VF0 = 4, U_VE0 = 6, U_MT = 8, U_SK = 9, U_R = 10, U_U = 11, U_MMA = 12, U_COUNT = 13
+  U_KF0 = 0, U_KE0 = 3, U_VF0 = 6, U_VE0 = 8, U_MT = 10, U_SK = 11, U_R = 12, U_U = 13, U_MMA = 14, U_COUNT = 15
 };
 constexpr int kUpdThreads = 320;
 
@@ -75,7 +78,7 @@ __global__ void __launch_bounds__(kUpdThreads, 1)
     mem_update_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                          const __grid_constant__ CUtensorMap tm_mt, const UpdArgs a) {
   using SL = UpdSmem<DELTA>;
-  constexpr int VST = SL::VST;
+  constexpr int KST = SL::KST, VST = SL::VST;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -112,9 +115,11 @@ __global__ void __launch_bounds__(kUpdThreads, 1)
     float* denp = reinterpret_cast<float*>(gbase + SL::DENP);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + SL::SLOT);
     if (threadIdx.x == 0) {
-      for (int i = 0; i < 2; ++i) {
+      for (int i = 0; i < 3; ++i) {
         mbar_init(bar(U_KF0 + i), 1);
         mbar_init(bar(U_KE0 + i), 1);
+      }
+      for (int i = 0; i < 2; ++i) {
         mbar_init(bar(U_VF0 + i), 1);
         mbar_init(bar(U_VE0 + i), 1);
       }
@@ -154,8 +159,8 @@ __global__ void __launch_bounds__(kUpdThreads, 1)
         }
         for (int c = 0; c < nchunks; ++c) {
           const int lt = (int)(seg_start + t_begin + (long long)c * kTile);
-          const int kst = c & 1;
-          if (c >= 2) mbar_wait(bar(U_KE0 + kst), ((c - 2) >> 1) & 1);
+          const int kst = c % KST;
+          if (c >= KST) mbar_wait(bar(U_KE0 + kst), ((c - KST) / KST) & 1);
           mbar_expect_tx(bar(U_KF0 + kst), kTileBytes);
           tma_load_4d(sK(kst), &tm_k, bar(U_KF0 + kst), 0, lt, h, b);
           tma_load_4d(sK(kst) + kBox, &tm_k, bar(U_KF0 + kst), 64, lt, h, b);
@@ -173,7 +178,7 @@ __global__ void __launch_bounds__(kUpdThreads, 1)
         constexpr uint32_t idesc_m = idesc_bf16(128, 128, 1, 1);
         constexpr uint32_t idesc_z = idesc_bf16(128, 16, 1, 0);
         for (int c = 0; c < nchunks; ++c) {
-          const int kst = c & 1, vst = c % VST;
+          const int kst = c % KST, vst = c % VST;
           mbar_wait(bar(U_SK), c & 1);
           if (DELTA) {
             if (c == 0) mbar_wait(bar(U_MT), 0);
@@ -210,8 +215,8 @@ __global__ void __launch_bounds__(kUpdThreads, 1)
       const int hh = warp >> 2;
       const uint32_t lrow = (uint32_t)((warp & 3) * 32) << 16;
       for (int c = 0; c < nchunks; ++c) {
-        const int kst = c & 1, vst = c % VST;
-        mbar_wait(bar(U_KF0 + kst), (c >> 1) & 1);
+        const int kst = c % KST, vst = c % VST;
+        mbar_wait(bar(U_KF0 + kst), (c / KST) & 1);
         const bool valid = t_begin + c * kTile + row < t_end;
         float dpart = 0.f;
         uint32_t lo[32];
