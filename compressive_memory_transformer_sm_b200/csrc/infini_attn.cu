@@ -303,7 +303,7 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale) {
   }
   tc::AttnArgs aa;
   aa.beta = p.beta; aa.snapz = snapz; aa.out = static_cast<__nv_bfloat16*>(p.out);
-  aa.B = p.B; aa.H = p.H; aa.S = pl.S; aa.T = (p.N + 127) / 128; aa.P = (aa.T + 1) / 2; aa.L = p.L; aa.N = p.N;
+  aa.B = p.B; aa.H = p.H; aa.S = pl.S; aa.T = (p.N + 127) / 128; aa.L = p.L; aa.N = p.N;
   aa.scale_log2 = scale * 1.4426950408889634f;
   for (int i = 0; i < 3; ++i) aa.os[i] = p.o_stride[i];
   // Scheduling groups of GS segments: about one wave of CTAs per group.
@@ -311,6 +311,12 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale) {
   if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     sms = 148;
   const long long NS = (long long)BH * pl.S;
+  // Pairs of query tiles per CTA, unless that leaves SMs idle (short streaming steps):
+  // then one query tile per CTA.
+  aa.single = NS * ((aa.T + 1) / 2) < sms ? 1 : 0;
+  if (p.flags & INFINI_FLAG_ATTN_SINGLE) aa.single = 1;
+  if (p.flags & INFINI_FLAG_ATTN_PAIRS) aa.single = 0;
+  aa.P = aa.single ? aa.T : (aa.T + 1) / 2;
   aa.GS = (int)std::max<long long>(1, std::min<long long>(NS, (sms + aa.P - 1) / aa.P));
   const long long groups = (NS + aa.GS - 1) / aa.GS;
   LaunchScope ls(kPhaseAttn, p.stream);

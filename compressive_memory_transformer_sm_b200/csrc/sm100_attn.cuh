@@ -42,8 +42,9 @@ struct AttnArgs {
   const float* snapz;     // [BH][S][128] fp32: z_{s-1}
   __nv_bfloat16* out;
   int B, H, S, T;         // T = query tiles per full segment
-  int P;                  // query-tile pairs per full segment = ceil(T / 2)
+  int P;                  // work items per full segment: ceil(T / 2) pairs, or T tiles when `single`
   int GS;                 // segments per scheduling group
+  int single;             // 1: one query tile per CTA (small grids), warpgroup 1 idle
   long long L;
   int N;
   float scale_log2;       // softmax scale * log2(e)
@@ -113,6 +114,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
+  ATTN_TRACE(threadIdx.x == 0, 3000);
 
   // ---- work item: (pair m, segment) from the grouped schedule
   const int NS = a.B * a.H * a.S;
@@ -121,14 +123,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int r = (int)(blockIdx.x % per_group);
   const int gsz = min(a.GS, NS - grp * a.GS);
   if (r >= gsz * a.P) return;  // padding of the last group
-  const int m = a.P - 1 - r / gsz;
+  const int m = a.P - 1 - r / gsz;       // pair index, or tile index when single
   const int seg = grp * a.GS + r % gsz;  // = bh * S + s
   const int bh = seg / a.S, s = seg % a.S;
   const int b = bh / a.H, h = bh % a.H;
   const long long seg0 = (long long)s * a.N;
   const int n_s = (int)min((long long)a.N, a.L - seg0);
-  if (2 * m * kTile >= n_s) return;  // tail segment: both tiles empty
-  const int nk1 = 2 * m + 2;         // K/V tiles of query tile 2m+1 (tile 2m uses one fewer)
+  const bool single = a.single != 0;
+  const int tq0 = single ? m : 2 * m;    // query tile of warpgroup 0 (warpgroup 1: tq0 + 1)
+  if (tq0 * kTile >= n_s) return;        // tail segment: the tile(s) are empty
+  const int nk1 = tq0 + (single ? 1 : 2); // K/V tiles of the CTA's last query tile
+  const int nk0 = tq0 + 1;               // K/V tiles of query tile tq0
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   auto sQ = [&](int k) { return base + (k ? kA_Q1 : kA_Q0); };
@@ -170,6 +175,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  ATTN_TRACE(threadIdx.x == 0, 3001);
 
   if (warp >= 8) {
   regs_decrease<kAttnOtherRegs>();
@@ -180,12 +186,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       prefetch_tensormap(&tm_k);
       prefetch_tensormap(&tm_v);
       prefetch_tensormap(&tm_mt);
-      const int lq = (int)(seg0 + (long long)(2 * m) * kTile);
-      mbar_expect_tx(bar(B_Q), 2 * kTileBytes);
+      const int lq = (int)(seg0 + (long long)tq0 * kTile);
+      mbar_expect_tx(bar(B_Q), (single ? 1 : 2) * kTileBytes);
       tma_load_4d(sQ(0), &tm_q, bar(B_Q), 0, lq, h, b);
       tma_load_4d(sQ(0) + kBox, &tm_q, bar(B_Q), 64, lq, h, b);
-      tma_load_4d(sQ(1), &tm_q, bar(B_Q), 0, lq + kTile, h, b);
-      tma_load_4d(sQ(1) + kBox, &tm_q, bar(B_Q), 64, lq + kTile, h, b);
+      if (!single) {
+        tma_load_4d(sQ(1), &tm_q, bar(B_Q), 0, lq + kTile, h, b);
+        tma_load_4d(sQ(1) + kBox, &tm_q, bar(B_Q), 64, lq + kTile, h, b);
+      }
       // K tile j goes in once the S products of key tile j-2 are done; V trails
       // K by one tile (V tile j once the P V products of key tile j-2 are
       // done), so that a pending V never holds back the next K.
@@ -217,7 +225,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // ------------------------------------------------------------ MMA issuer
       constexpr uint32_t idesc_kk = idesc_bf16(128, 128, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16(128, 128, 0, 1);
-      const int nk0 = nk1 - 1;
       auto issue_s = [&](int k, int j) {
         const uint32_t kt = sKt(j);
 #pragma unroll
@@ -241,7 +248,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_wait(kfull(0), 0);
       tc_fence_after();
       issue_s(0, 0);
-      issue_s(1, 0);
+      if (!single) issue_s(1, 0);
       mma_commit(kfree(0));
       for (int j = 1; j < nk1; ++j) {
         mbar_wait(kfull(j), kph(j));
@@ -251,20 +258,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         ATTN_TRACE(true, 2048 + 8 * j + 1);
         if (j < nk0) issue_s(0, j);
         ATTN_TRACE(true, 2048 + 8 * j + 5);
-        issue_pv(1, j - 1);
+        if (!single) issue_pv(1, j - 1);
         ATTN_TRACE(true, 2048 + 8 * j + 2);
         mma_commit(bar(B_VE0 + ((j - 1) & 1)));
-        issue_s(1, j);
+        if (!single) issue_s(1, j);
         mma_commit(kfree(j));
       }
-      issue_pv(1, nk1 - 1);
+      issue_pv(single ? 0 : 1, nk1 - 1);
       mma_commit(bar(B_VE0 + ((nk1 - 1) & 1)));
       // memory read: sigma(Q_k) (written over Q_k by the softmax warps) times M_{s-1}
       mbar_wait(kfull(nk1), kph(nk1));
       const uint32_t mt = sKt(nk1);  // M_{s-1} [dk][dv]: MN-major B operand (like V)
       constexpr uint32_t idesc_mem = idesc_bf16(128, 128, 0, 1);
 #pragma unroll 1
-      for (int k = 0; k < 2; ++k) {
+      for (int k = 0; k < (single ? 1 : 2); ++k) {
         mbar_wait(bar(B_SQ0 + k), 0);
         tc_fence_after();
 #pragma unroll
@@ -278,12 +285,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   } else {
     regs_increase<kAttnSoftmaxRegs>();
     // -------------------------------------------------------------- softmax WGs
-    const int k = warp >> 2;            // query tile 2m + k
+    const int k = warp >> 2;            // query tile tq0 + k
+    if (!(single && k == 1)) {
     const int row = (warp & 3) * 32 + lane;  // query row in the tile = TMEM lane
     const uint32_t lrow = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lrow + (uint32_t)k * 128u;
     const uint32_t tO = tmem + lrow + 256u + (uint32_t)k * 128u;
-    const int nk = nk1 - 1 + k;
+    const int nk = nk0 + k;             // its K/V tiles; the last one is its diagonal
     const float c = a.scale_log2;
     float m_ref = 0.f, l = 0.f;
     const bool tr = (row == 0);
@@ -401,14 +409,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       fence_proxy_async_smem();
       mbar_arrive(bar(B_SQ0 + k));
+      ATTN_TRACE(row == 0, 3008 + 8 * k + 0);
     }
     // ---------------------------------------------------------------- epilogue
     mbar_wait(bar(B_MEM0 + k), 0);  // also implies the last P V product of tile k is complete
+    ATTN_TRACE(row == 0, 3008 + 8 * k + 1);
     tc_fence_after();
     const float gw = 1.f / (1.f + __expf(-a.beta[h]));
     const float wdot = (1.f - gw) / l;
     const float wmem = den != 0.f ? gw / den : 0.f;
-    const int qrow = (2 * m + k) * kTile + row;
+    const int qrow = (tq0 + k) * kTile + row;
     const bool valid = qrow < n_s;
     __nv_bfloat16* orow = a.out + b * a.os[0] + h * a.os[1] + (seg0 + qrow) * a.os[2];
 #pragma unroll
@@ -429,6 +439,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
         for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
       }
+    }
+    ATTN_TRACE(row == 0, 3008 + 8 * k + 2);
     }
   }
   tc_fence_before();

@@ -75,6 +75,11 @@ extern "C" {
 /* infini_attn_params.flags: run the CUDA-core (SIMT) kernels even where the
  * tensor-core kernels apply -- a second GPU implementation, for testing */
 #define INFINI_FLAG_FORCE_SIMT 0x1
+/* tensor-core attention schedule: one query tile per CTA (the default for
+ * grids that would otherwise leave SMs idle) or pairs of query tiles per CTA
+ * (the default otherwise); these force one of them, for testing */
+#define INFINI_FLAG_ATTN_SINGLE 0x2
+#define INFINI_FLAG_ATTN_PAIRS 0x4
 
 enum {
   INFINI_OK = 0,

@@ -109,24 +109,27 @@ BF16_SHAPES = [
 ]
 
 
+PATH_FLAGS = {"tensor-pairs": api.FLAG_ATTN_PAIRS, "tensor-single": api.FLAG_ATTN_SINGLE,
+              "simt": api.FLAG_FORCE_SIMT}
+
+
 @pytest.mark.parametrize("shape", BF16_SHAPES)
 @pytest.mark.parametrize("mode", [LINEAR, DELTA])
-@pytest.mark.parametrize("path", ["tensor", "simt"])
+@pytest.mark.parametrize("path", list(PATH_FLAGS))
 def test_bf16_parity(shape, mode, path):
     B, H, L, N = shape
     q, k, v, beta = inputs(B, H, L, 128, 128, torch.bfloat16, 100 + L + N)
-    flags = api.FLAG_FORCE_SIMT if path == "simt" else 0
-    compare(q, k, v, beta, N, mode, False, f"{path} {shape} mode={mode}", flags=flags)
+    compare(q, k, v, beta, N, mode, False, f"{path} {shape} mode={mode}", flags=PATH_FLAGS[path])
 
 
 @pytest.mark.parametrize("mode", [LINEAR, DELTA])
-@pytest.mark.parametrize("path", ["tensor", "simt"])
+@pytest.mark.parametrize("path", list(PATH_FLAGS))
 def test_bf16_memory_read_alone(mode, path):
     """Gate forced to 1: out = A_mem, checked with the relative tolerance."""
     B, H, L, N = 1, 2, 1024, 256
     q, k, v, _ = inputs(B, H, L, 128, 128, torch.bfloat16, 7)
     beta = torch.full((H,), float("inf"), device=DEV)
-    flags = api.FLAG_FORCE_SIMT if path == "simt" else 0
+    flags = PATH_FLAGS[path]
     out, _, _ = run(q, k, v, beta, N, mode, flags=flags)
     wo, _, _ = oracle(q, k, v, beta, N, mode)
     got = np64(out)
@@ -146,13 +149,13 @@ def test_bf16_local_attention_alone(mode):
 
 
 @pytest.mark.parametrize("mode", [LINEAR, DELTA])
-@pytest.mark.parametrize("path", ["tensor", "simt"])
+@pytest.mark.parametrize("path", list(PATH_FLAGS))
 def test_bf16_nonempty_initial_state(mode, path):
     B, H, L, N = 2, 2, 512, 256
     q, k, v, beta = inputs(B, H, L, 128, 128, torch.bfloat16, 9)
     w = W.Workload("s", B=B, H=H, L=L, N=N, dk=128, dv=128, dtype=torch.bfloat16, modes=(mode,), seed=9)
     M0, z0 = (t.to(DEV) for t in W.random_state(w))
-    flags = api.FLAG_FORCE_SIMT if path == "simt" else 0
+    flags = PATH_FLAGS[path]
     compare(q, k, v, beta, N, mode, False, f"{path} state0 mode={mode}", M0=M0, z0=z0, flags=flags)
 
 
