@@ -27,10 +27,12 @@ template <typename T> __device__ __forceinline__ T from_f32(float x);
 template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
 template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
 
-// sigma(x) = ELU(x) + 1 with alpha = 1: x + 1 above zero, exp(x) at or below.
-__device__ __forceinline__ float elu1(float x) { return x > 0.f ? x + 1.f : __expf(x); }
+// sigma(x) = ELU(x) + 1 with alpha = 1: x + 1 above zero, exp(x) at or below,
+// written branch-free as max(x, 0) + exp(min(x, 0)) (a select per element
+// would diverge inside every warp of random-signed data).
+__device__ __forceinline__ float elu1(float x) { return fmaxf(x, 0.f) + __expf(fminf(x, 0.f)); }
 // Accurate variant for the fp32 CUDA-core path.
-__device__ __forceinline__ float elu1_accurate(float x) { return x > 0.f ? x + 1.f : expf(x); }
+__device__ __forceinline__ float elu1_accurate(float x) { return fmaxf(x, 0.f) + expf(fminf(x, 0.f)); }
 
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;

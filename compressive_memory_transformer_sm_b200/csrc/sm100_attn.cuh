@@ -57,8 +57,8 @@ constexpr uint32_t kA_Q0 = 0;
 constexpr uint32_t kA_Q1 = 32768;
 constexpr uint32_t kA_K0 = 65536;    // K ring: 3 stages of 32 KB
 constexpr uint32_t kA_V0 = kA_K0 + kKStages * 32768u;  // V ring: 2 stages of 32 KB
-constexpr uint32_t kA_Z = kA_V0 + 2 * 32768u;
-constexpr uint32_t kA_BAR = kA_Z + 512;
+constexpr uint32_t kA_Z = kA_V0 + 2 * 32768u;  // z_{s-1}, one copy per softmax warpgroup
+constexpr uint32_t kA_BAR = kA_Z + 1024;
 constexpr int kAttnThreads = 384;
 // Register split: the kernel launches with 168 registers per thread (384 x 168
 // = 64512); the load/MMA warpgroup gives back to 88 and the two softmax
@@ -170,7 +170,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
-  if (threadIdx.x < 128) zs[threadIdx.x] = a.snapz[(long long)seg * 128 + threadIdx.x];
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -295,6 +294,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const float c = a.scale_log2;
     float m_ref = 0.f, l = 0.f;
     const bool tr = (row == 0);
+    const float zrow = a.snapz[(long long)seg * 128 + row];  // used after the loop
     for (int j = 0; j < nk; ++j) {
       ATTN_TRACE(tr, 1024 * k + 8 * j + 0);
       mbar_wait(bar(B_SF0 + k), j & 1);
@@ -392,21 +392,32 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // sigma(q) . z_{s-1} from the unrounded sigma.
     float den = 0.f;
     {
+      float* zk = zs + 128 * k;
+      zk[row] = zrow;
+      named_bar_sync(1 + k, 128);
+      ATTN_TRACE(row == 0, 3008 + 8 * k + 3);
       const uint32_t q = sQ(k);
+      uint4 w[16];
+#pragma unroll
+      for (int cc = 0; cc < 16; ++cc) w[cc] = lds128(q + swz_chunk(row, cc));
+      ATTN_TRACE(row == 0, 3008 + 8 * k + 4);
+      float dp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int cc = 0; cc < 16; ++cc) {
-        const uint32_t ad = q + swz_chunk(row, cc);
-        uint4 w = lds128(ad);
-        uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
+        uint32_t* wp = reinterpret_cast<uint32_t*>(&w[cc]);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float s0 = elu1(bf16_lo(wp[e])), s1 = elu1(bf16_hi(wp[e]));
-          den = fmaf(s0, zs[8 * cc + 2 * e], den);
-          den = fmaf(s1, zs[8 * cc + 2 * e + 1], den);
+          dp[e] = fmaf(s0, zk[8 * cc + 2 * e], dp[e]);
+          dp[e] = fmaf(s1, zk[8 * cc + 2 * e + 1], dp[e]);
           wp[e] = pack_bf16x2(s0, s1);
         }
-        sts128(ad, w);
       }
+      ATTN_TRACE(row == 0, 3008 + 8 * k + 5);
+#pragma unroll
+      for (int cc = 0; cc < 16; ++cc) sts128(q + swz_chunk(row, cc), w[cc]);
+      den = (dp[0] + dp[1]) + (dp[2] + dp[3]);
+      ATTN_TRACE(row == 0, 3008 + 8 * k + 6);
       fence_proxy_async_smem();
       mbar_arrive(bar(B_SQ0 + k));
       ATTN_TRACE(row == 0, 3008 + 8 * k + 0);

@@ -218,27 +218,30 @@ __global__ void __launch_bounds__(kUpdThreads, 1)
         const int kst = c % KST, vst = c % VST;
         mbar_wait(bar(U_KF0 + kst), (c / KST) & 1);
         const bool valid = t_begin + c * kTile + row < t_end;
-        float dpart = 0.f;
+        float dp[4] = {0.f, 0.f, 0.f, 0.f};
         uint32_t lo[32];
+        uint4 w[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) w[i] = lds128(sK(kst) + swz_chunk(row, 8 * hh + i));
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const uint32_t off = swz_chunk(row, 8 * hh + i);
-          uint4 w = lds128(sK(kst) + off);
-          uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
+          uint32_t* wp = reinterpret_cast<uint32_t*>(&w[i]);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float s0 = valid ? elu1(bf16_lo(wp[e])) : 0.f;
             const float s1 = valid ? elu1(bf16_hi(wp[e])) : 0.f;
             if (DELTA) {
-              dpart = fmaf(s0, zs[64 * hh + 8 * i + 2 * e], dpart);
-              dpart = fmaf(s1, zs[64 * hh + 8 * i + 2 * e + 1], dpart);
+              dp[e] = fmaf(s0, zs[64 * hh + 8 * i + 2 * e], dp[e]);
+              dp[e] = fmaf(s1, zs[64 * hh + 8 * i + 2 * e + 1], dp[e]);
             }
             const uint32_t hi = pack_bf16x2(s0, s1);
             wp[e] = hi;
             lo[4 * i + e] = pack_bf16x2(s0 - bf16_lo(hi), s1 - bf16_hi(hi));
           }
-          sts128(sK(kst) + off, w);
         }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sts128(sK(kst) + swz_chunk(row, 8 * hh + i), w[i]);
+        const float dpart = (dp[0] + dp[1]) + (dp[2] + dp[3]);
         if (c > 0) mbar_wait(bar(U_MMA), (c - 1) & 1);  // MMAs of chunk c-1 released the lo buffers
 #pragma unroll
         for (int i = 0; i < 8; ++i)
