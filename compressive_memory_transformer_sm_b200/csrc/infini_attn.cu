@@ -266,7 +266,7 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale) {
     ua.seg0 = 0; ua.nseg = pl.S;
     {
       LaunchScope ls(kPhaseUpdate, p.stream);
-      tc::mem_update_tc_kernel<false><<<BH * pl.S * pl.G, tc::kUpdThreads, tc::UpdSmem<false>::BYTES, p.stream>>>(
+      tc::mem_update_tc_kernel<false><<<BH * pl.S * pl.G, tc::UpdWarps<false>::THREADS, tc::UpdSmem<false>::BYTES, p.stream>>>(
           tm_k, tm_v, tm_mt, ua);
     }
     LaunchScope ls(kPhaseState, p.stream);
@@ -287,7 +287,7 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale) {
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.gridDim = dim3(BH * pl.G);
-    cfg.blockDim = dim3(tc::kUpdThreads);
+    cfg.blockDim = dim3(tc::UpdWarps<true>::THREADS);
     cfg.dynamicSmemBytes = tc::UpdSmem<true>::BYTES;
     cfg.stream = p.stream;
     cfg.attrs = attr;

@@ -9,6 +9,19 @@
 namespace infini {
 namespace tc {
 
+// Per-chunk timestamps of one update CTA (block INFINI_UPD_TRACE) for tuning
+// builds; shares the attention kernel's trace array (slots 3200 and up).
+#if defined(INFINI_UPD_TRACE) && defined(INFINI_ATTN_TRACE)
+#define UPD_TRACE(cond, slot)                                                                          \
+  do {                                                                                                 \
+    if ((cond) && blockIdx.x == INFINI_UPD_TRACE && (slot) < 4096) g_attn_trace[(slot)] = clock64();  \
+  } while (0)
+#else
+#define UPD_TRACE(cond, slot) \
+  do {                        \
+  } while (0)
+#endif
+
 // ------------------------------------------------------------------------
 // Memory update.  Grid: BH * nseg * G CTAs; CTA (bh, segment seg0 + sl,
 // group grp) covers tokens [grp*cpb*128, min((grp+1)*cpb*128, n_s)) of the
@@ -71,14 +84,24 @@ struct UpdSmem {
 enum : int {
   U_KF0 = 0, U_KE0 = 3, U_VF0 = 6, U_VE0 = 8, U_MT = 10, U_SK = 11, U_R = 12, U_U = 13, U_MMA = 14, U_COUNT = 15
 };
-constexpr int kUpdThreads = 320;
+// Compute warps: 16 for the linear rule (four threads per token row, 32
+// columns each, to hide the latency of the sigma pass), 8 for the delta rule
+// (two per row: its U pass needs the registers).  Plus a TMA and an MMA warp.
+template <bool DELTA> struct UpdWarps {
+  static constexpr int NCW = DELTA ? 8 : 16;
+  static constexpr int PARTS = NCW / 4;        // threads per token row
+  static constexpr int CH = 16 / PARTS;        // 16-byte chunks (8 columns) per thread
+  static constexpr int THREADS = 32 * (NCW + 2);
+};
 
 template <bool DELTA>
-__global__ void __launch_bounds__(kUpdThreads, 1)
+__global__ void __launch_bounds__(UpdWarps<DELTA>::THREADS, 1)
     mem_update_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                          const __grid_constant__ CUtensorMap tm_mt, const UpdArgs a) {
   using SL = UpdSmem<DELTA>;
+  using WR = UpdWarps<DELTA>;
   constexpr int KST = SL::KST, VST = SL::VST;
+  constexpr int NCW = WR::NCW, PARTS = WR::PARTS, CH = WR::CH;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -124,9 +147,9 @@ __global__ void __launch_bounds__(kUpdThreads, 1)
         mbar_init(bar(U_VE0 + i), 1);
       }
       mbar_init(bar(U_MT), 1);
-      mbar_init(bar(U_SK), 256);
+      mbar_init(bar(U_SK), 32 * NCW);
       mbar_init(bar(U_R), 1);
-      mbar_init(bar(U_U), 256);
+      mbar_init(bar(U_U), 32 * NCW);
       mbar_init(bar(U_MMA), 1);
       fence_barrier_init();
     }
@@ -135,7 +158,7 @@ __global__ void __launch_bounds__(kUpdThreads, 1)
       for (int e = threadIdx.x; e < 1024; e += blockDim.x) ones[e] = 0x3f803f80u;  // bf16 1.0 pairs
     }
     if (threadIdx.x < 128) zs[threadIdx.x] = DELTA ? a.snapz[((long long)bh * a.S + s) * 128 + threadIdx.x] : 0.f;
-    if (warp == 9) {
+    if (warp == NCW + 1) {
       tmem_alloc(smem_u32(tmem_slot), 512);
       tmem_relinquish();
     }
@@ -146,7 +169,7 @@ __global__ void __launch_bounds__(kUpdThreads, 1)
     const uint32_t tmem = *tmem_slot;
     const uint32_t tR = tmem, tM = tmem + 128, tZ = tmem + 256;
 
-    if (warp == 8) {
+    if (warp == NCW) {
       if (lane == 0) {
         // ---------------------------------------------------------- producer
         prefetch_tensormap(&tm_k);
@@ -171,7 +194,7 @@ __global__ void __launch_bounds__(kUpdThreads, 1)
           tma_load_4d(sV(vst) + kBox, &tm_v, bar(U_VF0 + vst), 64, lt, h, b);
         }
       }
-    } else if (warp == 9) {
+    } else if (warp == NCW + 1) {
       if (lane == 0) {
         // ---------------------------------------------------------- MMA issuer
         constexpr uint32_t idesc_r = idesc_bf16(128, 128, 0, 1);  // B = M_{s-1} [dk][dv], MN-major
@@ -205,6 +228,7 @@ __global__ void __launch_bounds__(kUpdThreads, 1)
             mma_ss(tZ, aL, bO, idesc_z, 1u);
           }
           mma_commit(bar(U_MMA));
+          UPD_TRACE(c < 64, 3200 + 8 * c + 6);
           mma_commit(bar(U_KE0 + kst));
           mma_commit(bar(U_VE0 + vst));
         }
@@ -212,27 +236,29 @@ __global__ void __launch_bounds__(kUpdThreads, 1)
     } else {
       // ------------------------------------------------------------ compute warps
       const int row = (warp & 3) * 32 + lane;
-      const int hh = warp >> 2;
+      const int hh = warp >> 2;  // which PARTS-th of the row: chunks [CH * hh, CH * hh + CH)
       const uint32_t lrow = (uint32_t)((warp & 3) * 32) << 16;
       for (int c = 0; c < nchunks; ++c) {
         const int kst = c % KST, vst = c % VST;
+        const bool tr = threadIdx.x == 0 && c < 64;
         mbar_wait(bar(U_KF0 + kst), (c / KST) & 1);
+        UPD_TRACE(tr, 3200 + 8 * c + 0);
         const bool valid = t_begin + c * kTile + row < t_end;
         float dp[4] = {0.f, 0.f, 0.f, 0.f};
-        uint32_t lo[32];
-        uint4 w[8];
+        uint32_t lo[4 * CH];
+        uint4 w[CH];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) w[i] = lds128(sK(kst) + swz_chunk(row, 8 * hh + i));
+        for (int i = 0; i < CH; ++i) w[i] = lds128(sK(kst) + swz_chunk(row, CH * hh + i));
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < CH; ++i) {
           uint32_t* wp = reinterpret_cast<uint32_t*>(&w[i]);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float s0 = valid ? elu1(bf16_lo(wp[e])) : 0.f;
             const float s1 = valid ? elu1(bf16_hi(wp[e])) : 0.f;
             if (DELTA) {
-              dp[e] = fmaf(s0, zs[64 * hh + 8 * i + 2 * e], dp[e]);
-              dp[e] = fmaf(s1, zs[64 * hh + 8 * i + 2 * e + 1], dp[e]);
+              dp[e] = fmaf(s0, zs[8 * (CH * hh + i) + 2 * e], dp[e]);
+              dp[e] = fmaf(s1, zs[8 * (CH * hh + i) + 2 * e + 1], dp[e]);
             }
             const uint32_t hi = pack_bf16x2(s0, s1);
             wp[e] = hi;
@@ -240,22 +266,26 @@ __global__ void __launch_bounds__(kUpdThreads, 1)
           }
         }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) sts128(sK(kst) + swz_chunk(row, 8 * hh + i), w[i]);
+        for (int i = 0; i < CH; ++i) sts128(sK(kst) + swz_chunk(row, CH * hh + i), w[i]);
         const float dpart = (dp[0] + dp[1]) + (dp[2] + dp[3]);
+        UPD_TRACE(tr, 3200 + 8 * c + 1);
         if (c > 0) mbar_wait(bar(U_MMA), (c - 1) & 1);  // MMAs of chunk c-1 released the lo buffers
+        UPD_TRACE(tr, 3200 + 8 * c + 2);
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          sts128(sKlo + swz_chunk(row, 8 * hh + i), make_uint4(lo[4 * i], lo[4 * i + 1], lo[4 * i + 2], lo[4 * i + 3]));
+        for (int i = 0; i < CH; ++i)
+          sts128(sKlo + swz_chunk(row, CH * hh + i), make_uint4(lo[4 * i], lo[4 * i + 1], lo[4 * i + 2], lo[4 * i + 3]));
         float den = 0.f;
         if (DELTA) {
           denp[(c & 1) * 256 + hh * 128 + row] = dpart;
-          named_bar_sync(1, 256);
+          named_bar_sync(1, 32 * NCW);
           den = denp[(c & 1) * 256 + row] + denp[(c & 1) * 256 + 128 + row];
         }
         fence_proxy_async_smem();
         mbar_arrive(bar(U_SK));
+        UPD_TRACE(tr, 3200 + 8 * c + 3);
         if (DELTA) {
           mbar_wait(bar(U_R), c & 1);
+          UPD_TRACE(tr, 3200 + 8 * c + 4);
           tc_fence_after();
           const float rinv = den != 0.f ? 1.f / den : 0.f;
           uint32_t r0[32], r1[32];
@@ -287,16 +317,18 @@ __global__ void __launch_bounds__(kUpdThreads, 1)
           fence_proxy_async_smem();
           tc_fence_before();
           mbar_arrive(bar(U_U));
+          UPD_TRACE(tr, 3200 + 8 * c + 5);
         }
       }
       mbar_wait(bar(U_MMA), (nchunks - 1) & 1);
       tc_fence_after();
       // every load and MMA of this CTA is complete: the K/V rings can hold the partial
-      float* prow = (DELTA ? red : part) + (long long)row * 128 + 64 * hh;
+      constexpr int CPT = 128 / PARTS;  // value columns per thread
+      float* prow = (DELTA ? red : part) + (long long)row * 128 + CPT * hh;
 #pragma unroll
-      for (int q2 = 0; q2 < 2; ++q2) {
+      for (int q2 = 0; q2 < CPT / 32; ++q2) {
         uint32_t rr[32];
-        tmem_ld32(tM + lrow + 64u * hh + 32u * q2, rr);
+        tmem_ld32(tM + lrow + (uint32_t)(CPT * hh) + 32u * q2, rr);
         tmem_ld_wait();
         float4* dst = reinterpret_cast<float4*>(prow + 32 * q2);
 #pragma unroll
@@ -311,7 +343,7 @@ __global__ void __launch_bounds__(kUpdThreads, 1)
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 9) {
+    if (warp == NCW + 1) {
       __syncwarp();
       tc_fence_after();
       tmem_dealloc(tmem, 512);
