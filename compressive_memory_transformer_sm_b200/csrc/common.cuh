@@ -143,6 +143,34 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigne
     if (mbar_try_wait(bar, parity)) return true;
   return mbar_wait_slow(bar, parity, limit_ns);
 }
+// x, hidden from the optimiser: values derived from it are recomputed where
+// they are used instead of being hoisted out of loops and kept in registers.
+__device__ __forceinline__ uint32_t opaque_u32(uint32_t x) {
+  asm volatile("mov.b32 %0, %0;" : "+r"(x));
+  return x;
+}
+// True in exactly one lane of a fully active warp (the same lane every time).
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+// True once a bounded wait on this device has given up.
+__device__ __forceinline__ bool device_aborted() {
+  return (*reinterpret_cast<volatile unsigned*>(&g_status) & kStatusTimeout) != 0;
+}
+// Wait for a copy this thread issued (completing phase `parity` of `bar`)
+// even after the error word is set, for at most `limit_ns`: a kernel that
+// gives up drains its own copies in flight before it exits.
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity, unsigned long long limit_ns = 100000000ull) {
+  const unsigned long long t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer_ns() - t0 > limit_ns) return;
+}
 
 // ---------------------------------------------------------------- fences
 __device__ __forceinline__ void fence_proxy_async_smem() {

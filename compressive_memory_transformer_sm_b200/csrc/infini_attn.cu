@@ -77,7 +77,7 @@ struct Plan {
   int B, H, N, dk, dv, mode, S, G, cpb, nseg_part;
   long long L;
   bool delta, f32, tc;
-  size_t off_snapM, off_snapz, off_part, total;
+  size_t off_snapM, off_snapz, off_part, off_ctr, total;
 };
 
 // Workspace: per-segment snapshots of M_{s-1} (bf16 [dk][dv] for the tensor
@@ -120,6 +120,8 @@ int make_plan(int B, int H, long long L, int N, int dk, int dv, int mode, int fl
   off = align_up(off + (size_t)BH * S * dk * 4);
   p->off_part = off;
   off = align_up(off + (size_t)BH * p->nseg_part * p->G * (E + dk) * 4);
+  p->off_ctr = off;  // work counter of the persistent attention kernel
+  off = align_up(off + (p->tc ? 8 : 0));
   p->total = off;
   return INFINI_OK;
 }
@@ -319,8 +321,14 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale) {
   aa.P = aa.single ? aa.T : (aa.T + 1) / 2;
   aa.GS = (int)std::max<long long>(1, std::min<long long>(NS, (sms + aa.P - 1) / aa.P));
   const long long groups = (NS + aa.GS - 1) / aa.GS;
+  // persistent: one CTA per SM, or one per work item when there are fewer
+  const long long items = groups * aa.GS * aa.P;
+  if (items >= (1LL << 31)) return INFINI_ERR_UNSUPPORTED;
+  aa.work_counter = reinterpret_cast<unsigned int*>(ws + pl.off_ctr);
+  if (cudaMemsetAsync(aa.work_counter, 0, sizeof(unsigned int), p.stream) != cudaSuccess)
+    return INFINI_ERR_LAUNCH;
   LaunchScope ls(kPhaseAttn, p.stream);
-  tc::attn_tc_kernel<<<(unsigned)(groups * aa.GS * aa.P), tc::kAttnThreads, tc::kAttnSmem, p.stream>>>(
+  tc::attn_tc_kernel<<<(unsigned)std::min<long long>(items, sms), tc::kAttnThreads, tc::kAttnSmem, p.stream>>>(
       tm_q, tm_k, tm_v, tm_mt, aa);
   return launch_status();
 }

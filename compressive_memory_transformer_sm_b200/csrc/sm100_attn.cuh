@@ -1,6 +1,6 @@
 // attn_tc_kernel: A_dot (Eq. 6) + A_mem (Eq. 7) + gate (Eq. 10) of the
-// Infini-attention forward, fused, on the sm_100a tensor cores: one CTA per
-// (b, h, segment, pair of 128-row query tiles).
+// Infini-attention forward, fused, on the sm_100a tensor cores: a persistent
+// kernel whose work items are (b, h, segment, pair of 128-row query tiles).
 #pragma once
 
 #include "sm100_common.cuh"
@@ -23,28 +23,32 @@ namespace infini {
 namespace tc {
 
 // Pipeline timestamps of one CTA (block INFINI_ATTN_TRACE) for tuning builds:
-// slot = 8 * (tile) + event; softmax warpgroup k writes at 1024 * k, the MMA
-// thread at 2048.  Compiled out unless INFINI_ATTN_TRACE is defined.
+// item `it` of softmax warpgroup k at 1024 * k + 16 * it + event, of the MMA
+// thread at 2048 + 16 * it + event, of the TMA thread at 3072 + 16 * it +
+// event; kernel start / setup done at 4000 / 4001.  Compiled out unless
+// INFINI_ATTN_TRACE is defined.
 #ifdef INFINI_ATTN_TRACE
 __device__ unsigned long long g_attn_trace[4096];
-#define ATTN_TRACE(cond, slot)                                                                   \
-  do {                                                                                           \
-    if ((cond) && blockIdx.x == INFINI_ATTN_TRACE && (slot) < 4096) g_attn_trace[(slot)] = clock64(); \
+#define ATTN_TRACE_VAL(cond, slot, val)                                                           \
+  do {                                                                                            \
+    if ((cond) && blockIdx.x == INFINI_ATTN_TRACE && (slot) < 4096) g_attn_trace[(slot)] = (val); \
   } while (0)
 #else
-#define ATTN_TRACE(cond, slot) \
-  do {                         \
+#define ATTN_TRACE_VAL(cond, slot, val) \
+  do {                                  \
   } while (0)
 #endif
+#define ATTN_TRACE(cond, slot) ATTN_TRACE_VAL(cond, slot, clock64())
 
 struct AttnArgs {
   const float* beta;
   const float* snapz;     // [BH][S][128] fp32: z_{s-1}
   __nv_bfloat16* out;
+  unsigned int* work_counter;  // next unclaimed work item; zero at launch (items < 2^31)
   int B, H, S, T;         // T = query tiles per full segment
   int P;                  // work items per full segment: ceil(T / 2) pairs, or T tiles when `single`
   int GS;                 // segments per scheduling group
-  int single;             // 1: one query tile per CTA (small grids), warpgroup 1 idle
+  int single;             // 1: one query tile per work item (small grids), warpgroup 1 idle
   long long L;
   int N;
   float scale_log2;       // softmax scale * log2(e)
@@ -53,6 +57,7 @@ struct AttnArgs {
 
 // Shared memory of the attention kernel (offsets from a 1024-aligned base).
 constexpr int kKStages = 3;          // K ring depth (V ring: 2)
+constexpr int kItemSlots = 2;        // work items handed from the TMA thread to the consumers
 constexpr uint32_t kA_Q0 = 0;
 constexpr uint32_t kA_Q1 = 32768;
 constexpr uint32_t kA_K0 = 65536;    // K ring: 3 stages of 32 KB
@@ -83,14 +88,26 @@ enum : int {
   B_VE0 = 15,  // V stage free: both P V products of that key tile done (2)
   B_KF2 = 17,  // third K stage full
   B_KE2 = 18,  // third K stage free
-  B_COUNT = 19
+  B_OF0 = 19,  // TMEM S_k / O_k read out by the epilogue of query tile k (2, 128 arrivals)
+  B_IF0 = 21,  // work-item slot published (kItemSlots)
+  B_IE0 = 23,  // work-item slot read by every consumer (kItemSlots)
+  B_DONE = 25, // every product issued by the MMA thread complete (exit)
+  B_PH0 = 26,  // first half of P (keys 0-63) of query tile k written (2, 128 arrivals)
+  B_COUNT = 28
 };
-constexpr uint32_t kA_TMEMSLOT = kA_BAR + 8 * B_COUNT;
+constexpr uint32_t kA_ITEMS = kA_BAR + 8 * B_COUNT;  // kItemSlots x int64 work-item indices
+constexpr uint32_t kA_TMEMSLOT = kA_ITEMS + 8 * kItemSlots;
 constexpr uint32_t kAttnSmem = kA_TMEMSLOT + 16 + 1024;  // + alignment slack
 static_assert(kAttnSmem <= 232448, "attention kernel exceeds 227 KB of shared memory");
 
-// One CTA computes two adjacent 128-row query tiles (2m, 2m+1) of one
-// (b, h, segment), sharing every K/V tile load between them.
+// Persistent kernel, one CTA per SM.  A work item is two adjacent 128-row
+// query tiles (2m, 2m+1) of one (b, h, segment), sharing every K/V tile load
+// between them (or the single tile m when `single`).  The TMA thread claims
+// items from a global counter in the grouped order below and hands each to
+// the other roles through a two-slot ring in shared memory; every role keeps
+// running barrier phases across the CTA's items, so the loads and the first
+// products of the next item overlap the epilogue of the current one.
+//
 // Warps 0-3: softmax warpgroup of query tile 2m; warps 4-7: of tile 2m+1
 // (thread = query row = TMEM lane).  Warp 8 loads (TMA), warp 9 issues the
 // MMAs and owns TMEM, warps 10-11 only complete their warpgroup.  TMEM columns: S of tile 2m [0,128), S of tile 2m+1
@@ -104,8 +121,9 @@ static_assert(kAttnSmem <= 232448, "attention kernel exceeds 227 KB of shared me
 // "S_k(j) complete" implies "PV_k(j-1) complete": the O rescale of the
 // softmax needs no extra wait.
 //
-// CTAs are ordered by groups of GS segments (about one wave of CTAs per
-// group, so the group's K/V stays in L2), heaviest pair first inside a group.
+// Items are ordered by groups of GS segments (about one wave of items per
+// group, so the group's K/V stays in L2), heaviest pair first inside a group;
+// claiming them dynamically balances the CTAs.
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_mt,
@@ -114,38 +132,59 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
-  ATTN_TRACE(threadIdx.x == 0, 3000);
+  ATTN_TRACE(threadIdx.x == 0, 4000);
 
-  // ---- work item: (pair m, segment) from the grouped schedule
   const int NS = a.B * a.H * a.S;
   const int per_group = a.GS * a.P;
-  const int grp = (int)(blockIdx.x / per_group);
-  const int r = (int)(blockIdx.x % per_group);
-  const int gsz = min(a.GS, NS - grp * a.GS);
-  if (r >= gsz * a.P) return;  // padding of the last group
-  const int m = a.P - 1 - r / gsz;       // pair index, or tile index when single
-  const int seg = grp * a.GS + r % gsz;  // = bh * S + s
-  const int bh = seg / a.S, s = seg % a.S;
-  const int b = bh / a.H, h = bh % a.H;
-  const long long seg0 = (long long)s * a.N;
-  const int n_s = (int)min((long long)a.N, a.L - seg0);
+  const int total = ((NS + a.GS - 1) / a.GS) * per_group;  // the host keeps this below 2^31
   const bool single = a.single != 0;
-  const int tq0 = single ? m : 2 * m;    // query tile of warpgroup 0 (warpgroup 1: tq0 + 1)
-  if (tq0 * kTile >= n_s) return;        // tail segment: the tile(s) are empty
-  const int nk1 = tq0 + (single ? 1 : 2); // K/V tiles of the CTA's last query tile
-  const int nk0 = tq0 + 1;               // K/V tiles of query tile tq0
+  // Work item idx of the grouped heavy-first order -> (m, segment); false for
+  // the padding of the last group and for tiles past the end of a short
+  // (tail) segment.
+  struct Item {
+    int m, seg, b, h, n_s, tq0, nk0, nk1;
+    long long seg0;
+  };
+  auto decode = [&](int idx, Item& it) -> bool {
+    const int grp = idx / per_group;
+    const int r = idx - grp * per_group;
+    const int gsz = min(a.GS, NS - grp * a.GS);
+    if (r >= gsz * a.P) return false;
+    it.m = a.P - 1 - r / gsz;  // pair index, or tile index when single
+    it.seg = grp * a.GS + r % gsz;  // = bh * S + s
+    const int bh = it.seg / a.S, s = it.seg % a.S;
+    it.b = bh / a.H;
+    it.h = bh % a.H;
+    it.seg0 = (long long)s * a.N;
+    it.n_s = (int)min((long long)a.N, a.L - it.seg0);
+    it.tq0 = single ? it.m : 2 * it.m;        // query tile of warpgroup 0 (warpgroup 1: tq0 + 1)
+    it.nk0 = it.tq0 + 1;                      // K/V tiles of query tile tq0
+    it.nk1 = it.tq0 + (single ? 1 : 2);       // K/V tiles of the item's last query tile
+    return it.tq0 * kTile < it.n_s;
+  };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   auto sQ = [&](int k) { return base + (k ? kA_Q1 : kA_Q0); };
   auto sK = [&](int st) { return base + kA_K0 + (uint32_t)st * kTileBytes; };
   auto sV = [&](int st) { return base + kA_V0 + (uint32_t)st * kTileBytes; };
   auto bar = [&](int i) { return base + kA_BAR + 8u * (uint32_t)i; };
-  // K tile j lives in stage j % 3; its barriers (full / free) and their phase (j / 3) & 1
-  auto kfull = [&](int j) { const int st = j % kKStages; return bar(st < 2 ? B_KF0 + st : B_KF2); };
-  auto kfree = [&](int j) { const int st = j % kKStages; return bar(st < 2 ? B_KE0 + st : B_KE2); };
-  auto kph = [&](int j) { return (uint32_t)((j / kKStages) & 1); };
-  auto sKt = [&](int j) { return sK(j % kKStages); };
+  // The K ring is used in order: every item's K tiles, then its M_{s-1}
+  // snapshot.  Slot g (counted modulo 6 over all the CTA's items) lives in
+  // stage g % 3, and its barriers (full / free) complete a phase of parity
+  // g / 3 for it.  V-ring slot g (counted modulo 2^32): stage g % 2, parity
+  // (g / 2) % 2.  A producer waits for the free phase of the previous use,
+  // parity ^ 1, which a fresh barrier reports complete.
+  auto knext = [](uint32_t g, int j) { return (g + (uint32_t)(j % 6)) % 6u; };
+  auto kfull = [&](uint32_t g) { const uint32_t st = g % 3u; return bar(st < 2 ? B_KF0 + (int)st : B_KF2); };
+  auto kfree = [&](uint32_t g) { const uint32_t st = g % 3u; return bar(st < 2 ? B_KE0 + (int)st : B_KE2); };
+  auto kph = [](uint32_t g) { return g / 3u; };
+  auto sKt = [&](uint32_t g) { return sK((int)(g % 3u)); };
+  auto vfull = [&](uint32_t g) { return bar(B_VF0 + (int)(g & 1u)); };
+  auto vfree = [&](uint32_t g) { return bar(B_VE0 + (int)(g & 1u)); };
+  auto vph = [](uint32_t g) { return (g >> 1) & 1u; };
+  auto sVt = [&](uint32_t g) { return sV((int)(g & 1u)); };
   float* zs = reinterpret_cast<float*>(gbase + kA_Z);
+  int* slots = reinterpret_cast<int*>(gbase + kA_ITEMS);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kA_TMEMSLOT);
 
   if (threadIdx.x == 0) {
@@ -155,14 +194,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(bar(B_VF0 + i), 1);
       mbar_init(bar(B_KE0 + i), 1);
       mbar_init(bar(B_VE0 + i), 1);
-      if (i == 0) {
-        mbar_init(bar(B_KF2), 1);
-        mbar_init(bar(B_KE2), 1);
-      }
       mbar_init(bar(B_SF0 + i), 1);
       mbar_init(bar(B_PF0 + i), 128);
+      mbar_init(bar(B_PH0 + i), 128);
       mbar_init(bar(B_SQ0 + i), 128);
       mbar_init(bar(B_MEM0 + i), 1);
+      mbar_init(bar(B_OF0 + i), 128);
+    }
+    mbar_init(bar(B_KF2), 1);
+    mbar_init(bar(B_KE2), 1);
+    mbar_init(bar(B_DONE), 1);
+    for (int i = 0; i < kItemSlots; ++i) {
+      mbar_init(bar(B_IF0 + i), 1);
+      mbar_init(bar(B_IE0 + i), single ? 1 + 128 : 1 + 256);  // lane 0 of the MMA warp + the softmax threads
     }
     fence_barrier_init();
   }
@@ -173,8 +217,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  ATTN_TRACE(threadIdx.x == 0, 3001);
+  // The CTA owns all 512 columns of the SM's tensor memory, so its block
+  // starts at lane 0, column 0 and every TMEM address below is a constant.
+  if (*tmem_slot != 0u) {  // not expected: report and leave
+    if (threadIdx.x == 0) atomicOr(&g_status, kStatusTimeout);
+    if (warp == 9) tmem_dealloc(*tmem_slot, 512);
+    return;
+  }
+  constexpr uint32_t tmem = 0;
+  ATTN_TRACE(threadIdx.x == 0, 4001);
+
+  // Consumers take work item `it` of this CTA from slot it % kItemSlots
+  // (-1: no more work, or a wait on this device gave up).
+  auto take_item = [&](int it, bool arrive) -> int {
+    const int sl = it % kItemSlots;
+    mbar_wait(bar(B_IF0 + sl), (uint32_t)((it / kItemSlots) & 1));
+    const int idx = *reinterpret_cast<volatile int*>(&slots[sl]);
+    if (arrive) mbar_arrive(bar(B_IE0 + sl));
+    return device_aborted() ? -1 : idx;
+  };
 
   if (warp >= 8) {
   regs_decrease<kAttnOtherRegs>();
@@ -185,273 +246,403 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       prefetch_tensormap(&tm_k);
       prefetch_tensormap(&tm_v);
       prefetch_tensormap(&tm_mt);
-      const int lq = (int)(seg0 + (long long)tq0 * kTile);
-      mbar_expect_tx(bar(B_Q), (single ? 1 : 2) * kTileBytes);
-      tma_load_4d(sQ(0), &tm_q, bar(B_Q), 0, lq, h, b);
-      tma_load_4d(sQ(0) + kBox, &tm_q, bar(B_Q), 64, lq, h, b);
-      if (!single) {
-        tma_load_4d(sQ(1), &tm_q, bar(B_Q), 0, lq + kTile, h, b);
-        tma_load_4d(sQ(1) + kBox, &tm_q, bar(B_Q), 64, lq + kTile, h, b);
-      }
-      // K tile j goes in once the S products of key tile j-2 are done; V trails
-      // K by one tile (V tile j once the P V products of key tile j-2 are
-      // done), so that a pending V never holds back the next K.
-      for (int j = 0; j <= nk1; ++j) {
-        if (j < nk1) {
-          const int lk = (int)(seg0 + (long long)j * kTile);
-          if (j >= kKStages) mbar_wait(kfree(j), kph(j - kKStages));
-          mbar_expect_tx(kfull(j), kTileBytes);
-          tma_load_4d(sKt(j), &tm_k, kfull(j), 0, lk, h, b);
-          tma_load_4d(sKt(j) + kBox, &tm_k, kfull(j), 64, lk, h, b);
+      uint32_t gk = 0, gv = 0, nq = 0;  // next K-ring slot (mod 6), next V-ring slot, Q pairs loaded
+      uint32_t kn = 0, vn = 0;          // K / V fills issued, saturating at the ring depth
+      for (int it = 0;; ++it) {
+        int idx = total;
+        Item w;
+        if (!device_aborted()) {
+          do {
+            idx = (int)atomicAdd(a.work_counter, 1u);
+          } while (idx < total && !decode(idx, w));
         }
-        if (j >= 1) {
-          const int jv = j - 1, st = jv & 1;
-          const int lk = (int)(seg0 + (long long)jv * kTile);
-          if (jv >= 2) mbar_wait(bar(B_VE0 + st), ((jv - 2) >> 1) & 1);
-          mbar_expect_tx(bar(B_VF0 + st), kTileBytes);
-          tma_load_4d(sV(st), &tm_v, bar(B_VF0 + st), 0, lk, h, b);
-          tma_load_4d(sV(st) + kBox, &tm_v, bar(B_VF0 + st), 64, lk, h, b);
+        ATTN_TRACE(true, 3072 + 16 * it + 0);
+        ATTN_TRACE_VAL(true, 3072 + 16 * it + 8, (unsigned long long)idx);
+        const int sl = it % kItemSlots;
+        if (!mbar_wait(bar(B_IE0 + sl), (uint32_t)(((it / kItemSlots) & 1) ^ 1))) break;
+        slots[sl] = idx < total ? idx : -1;
+        mbar_arrive(bar(B_IF0 + sl));  // release: the consumers see the slot once the phase completes
+        ATTN_TRACE(true, 3072 + 16 * it + 1);
+        if (idx >= total) break;
+        // K tile j once the S products of the slot's previous use are done; V
+        // tile j-1 likewise after its P V products (V trails K by one tile, so
+        // a pending V never holds back the next K).  Q after the memory-read
+        // products of the previous item, which read sigma(Q) from the Q
+        // tiles: issued after K tile 0 of the new item.
+        for (int j = 0; j <= w.nk1; ++j) {
+          if (j < w.nk1) {
+            const int lk = (int)(w.seg0 + (long long)j * kTile);
+            if (!mbar_wait(kfree(gk), kph(gk) ^ 1u)) goto done;
+            mbar_expect_tx(kfull(gk), kTileBytes);
+            tma_load_4d(sKt(gk), &tm_k, kfull(gk), 0, lk, w.h, w.b);
+            tma_load_4d(sKt(gk) + kBox, &tm_k, kfull(gk), 64, lk, w.h, w.b);
+            gk = knext(gk, 1);
+            kn = min(kn + 1u, (uint32_t)kKStages);
+          }
+          if (j == 0) {
+            const uint32_t prev = (uint32_t)(it & 1) ^ 1u;  // previous item's phase (fresh: complete)
+            if (!mbar_wait(bar(B_MEM0), prev)) goto done;
+            if (!single && !mbar_wait(bar(B_MEM0 + 1), prev)) goto done;
+            const int lq = (int)(w.seg0 + (long long)w.tq0 * kTile);
+            mbar_expect_tx(bar(B_Q), (single ? 1 : 2) * kTileBytes);
+            tma_load_4d(sQ(0), &tm_q, bar(B_Q), 0, lq, w.h, w.b);
+            tma_load_4d(sQ(0) + kBox, &tm_q, bar(B_Q), 64, lq, w.h, w.b);
+            if (!single) {
+              tma_load_4d(sQ(1), &tm_q, bar(B_Q), 0, lq + kTile, w.h, w.b);
+              tma_load_4d(sQ(1) + kBox, &tm_q, bar(B_Q), 64, lq + kTile, w.h, w.b);
+            }
+            ++nq;
+            ATTN_TRACE(true, 3072 + 16 * it + 2);
+          }
+          if (j >= 1) {
+            const int lk = (int)(w.seg0 + (long long)(j - 1) * kTile);
+            if (!mbar_wait(vfree(gv), vph(gv) ^ 1u)) goto done;
+            mbar_expect_tx(vfull(gv), kTileBytes);
+            tma_load_4d(sVt(gv), &tm_v, vfull(gv), 0, lk, w.h, w.b);
+            tma_load_4d(sVt(gv) + kBox, &tm_v, vfull(gv), 64, lk, w.h, w.b);
+            ++gv;
+            vn = min(vn + 1u, 2u);
+          }
         }
+        // M_{s-1} (bf16 snapshot, [dk][dv]) enters the K ring after the item's K tiles.
+        if (!mbar_wait(kfree(gk), kph(gk) ^ 1u)) goto done;
+        mbar_expect_tx(kfull(gk), kTileBytes);
+        tma_load_2d(sKt(gk), &tm_mt, kfull(gk), 0, w.seg * 128);
+        tma_load_2d(sKt(gk) + kBox, &tm_mt, kfull(gk), 64, w.seg * 128);
+        ATTN_TRACE(true, 3072 + 16 * it + 3);
+        gk = knext(gk, 1);
+        kn = min(kn + 1u, (uint32_t)kKStages);
       }
-      // M_{s-1} (bf16 snapshot, [dk][dv]) enters the K ring as tile nk1.
-      if (nk1 >= kKStages) mbar_wait(kfree(nk1), kph(nk1 - kKStages));
-      mbar_expect_tx(kfull(nk1), kTileBytes);
-      tma_load_2d(sKt(nk1), &tm_mt, kfull(nk1), 0, seg * 128);
-      tma_load_2d(sKt(nk1) + kBox, &tm_mt, kfull(nk1), 64, seg * 128);
+    done:
+      if (device_aborted()) {
+        // a wait gave up: let the copies still in flight land before the CTA exits
+        for (uint32_t i = 1; i <= kn; ++i) {
+          const uint32_t g = knext(gk, 6 - (int)i);
+          mbar_drain(kfull(g), kph(g));
+        }
+        for (uint32_t i = 1; i <= vn; ++i) mbar_drain(vfull(gv - i), vph(gv - i));
+        if (nq > 0) mbar_drain(bar(B_Q), (nq - 1u) & 1u);
+      }
     }
   } else if (warp == 9) {
-    if (lane == 0) {
+    {
+      // The whole warp runs the issue loop (uniform control flow); one elected
+      // lane issues the MMAs and the commits.
       // ------------------------------------------------------------ MMA issuer
+      // Per key tile j of query tile k: P_k(j) (bf16, TMEM columns 0-63)
+      // feeds P V in two halves, the first while the softmax still computes
+      // the second; S_k(j+1) overwrites those columns after the second.
       constexpr uint32_t idesc_kk = idesc_bf16(128, 128, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16(128, 128, 0, 1);
-      auto issue_s = [&](int k, int j) {
-        const uint32_t kt = sKt(j);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + (uint32_t)k * 128u, kmajor_desc(sQ(k), kk), kmajor_desc(kt, kk), idesc_kk,
-                 kk > 0 ? 1u : 0u);
-        mma_commit(bar(B_SF0 + k));
-      };
-      auto issue_pv = [&](int k, int j) {  // P of tile k, key tile j; call in order j = 0, 1, ...
-        const int st = j & 1;
-        mbar_wait(bar(B_PF0 + k), j & 1);
-        ATTN_TRACE(true, 2048 + 8 * (j + 1) + 3 + k);
-        mbar_wait(bar(B_VF0 + st), (j >> 1) & 1);
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + 256u + (uint32_t)k * 128u, tmem + (uint32_t)k * 128u + (uint32_t)kk * 8u,
-                 mnmajor_desc(sV(st), kk), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-      };
-      mbar_wait(bar(B_Q), 0);
-      mbar_wait(kfull(0), 0);
-      tc_fence_after();
-      issue_s(0, 0);
-      if (!single) issue_s(1, 0);
-      mma_commit(kfree(0));
-      for (int j = 1; j < nk1; ++j) {
-        mbar_wait(kfull(j), kph(j));
-        ATTN_TRACE(true, 2048 + 8 * j + 0);
-        tc_fence_after();
-        if (j - 1 < nk0) issue_pv(0, j - 1);
-        ATTN_TRACE(true, 2048 + 8 * j + 1);
-        if (j < nk0) issue_s(0, j);
-        ATTN_TRACE(true, 2048 + 8 * j + 5);
-        if (!single) issue_pv(1, j - 1);
-        ATTN_TRACE(true, 2048 + 8 * j + 2);
-        mma_commit(bar(B_VE0 + ((j - 1) & 1)));
-        if (!single) issue_s(1, j);
-        mma_commit(kfree(j));
-      }
-      issue_pv(single ? 0 : 1, nk1 - 1);
-      mma_commit(bar(B_VE0 + ((nk1 - 1) & 1)));
-      // memory read: sigma(Q_k) (written over Q_k by the softmax warps) times M_{s-1}
-      mbar_wait(kfull(nk1), kph(nk1));
-      const uint32_t mt = sKt(nk1);  // M_{s-1} [dk][dv]: MN-major B operand (like V)
       constexpr uint32_t idesc_mem = idesc_bf16(128, 128, 0, 1);
-#pragma unroll 1
-      for (int k = 0; k < (single ? 1 : 2); ++k) {
-        mbar_wait(bar(B_SQ0 + k), 0);
-        tc_fence_after();
+      uint32_t gk = 0, gv = 0;           // next K / V ring slot
+      uint32_t nt0 = 0, nt1 = 0;         // P tiles of query tile 0 / 1 so far (PH / PF phases)
+      for (int it = 0;; ++it) {
+        const int idx = take_item(it, lane == 0);  // one arrival for the warp
+        if (idx < 0) break;
+        Item w;
+        decode(idx, w);
+        // the Q tile addresses are re-derived per item so that their
+        // descriptors are not kept live across the whole loop
+        const uint32_t q0 = opaque_u32(sQ(0));
+        auto sQi = [&](int k) { return q0 + (k ? kA_Q1 - kA_Q0 : 0u); };
+        // S_k(j) = Q_k K_j^T
+        auto issue_s = [&](int k, uint32_t g) {
+          const uint64_t da = kmajor_base(sQi(k)), db = kmajor_base(sKt(g));
+          if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + (uint32_t)k * 128u, kmajor_desc(sQ(k), kk), mnmajor_desc(mt, kk), idesc_mem,
-                 kk > 0 ? 1u : 0u);
-        mma_commit(bar(B_MEM0 + k));
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ss(tmem + (uint32_t)k * 128u, da + kmajor_step(kk), db + kmajor_step(kk), idesc_kk, kk > 0 ? 1u : 0u);
+          }
+          __syncwarp();
+        };
+        // O_k (+)= P_k V: K-steps [4h, 4h + 4) = keys [64h, 64h + 64)
+        auto issue_pv_half = [&](int k, uint32_t g, int h, bool first) {
+          const uint64_t db = mnmajor_base(sVt(g));
+          if (elect_one()) {
+#pragma unroll
+            for (int kk = 4 * h; kk < 4 * h + 4; ++kk)
+              mma_ts(tmem + 256u + (uint32_t)k * 128u, tmem + (uint32_t)k * 128u + (uint32_t)kk * 8u,
+                     db + mnmajor_step(kk), idesc_pv, (!first || kk > 0) ? 1u : 0u);
+          }
+          __syncwarp();
+        };
+        auto commit = [&](uint32_t b) {
+          if (elect_one()) mma_commit(b);
+          __syncwarp();
+        };
+        const uint32_t prev = (uint32_t)(it & 1) ^ 1u;  // previous item's phase (fresh: complete)
+        ATTN_TRACE(true, 2048 + 16 * it + 0);
+        mbar_wait(bar(B_Q), (uint32_t)(it & 1));
+        ATTN_TRACE(true, 2048 + 16 * it + 1);
+        mbar_wait(kfull(gk), kph(gk));
+        // S_k(0) overwrites the S_k / O_k columns the previous item's epilogue reads
+        mbar_wait(bar(B_OF0), prev);
+        tc_fence_after();
+        issue_s(0, gk);
+        commit(bar(B_SF0));
+        ATTN_TRACE(true, 2048 + 16 * it + 2);
+        if (!single) {
+          mbar_wait(bar(B_OF0 + 1), prev);
+          tc_fence_after();
+          issue_s(1, gk);
+          commit(bar(B_SF0 + 1));
+          ATTN_TRACE(true, 2048 + 16 * it + 3);
+        }
+        commit(kfree(gk));
+        // one step per key tile j: the P V products of tile j and S(j + 1), query tile 0 then 1
+        for (int j = 0; j < w.nk1; ++j) {
+          const uint32_t gvj = gv + (uint32_t)j, gn = knext(gk, j + 1);
+          const bool more = j + 1 < w.nk1;  // key tile j + 1 exists (for query tile 1)
+          if (more) mbar_wait(kfull(gn), kph(gn));
+          mbar_wait(vfull(gvj), vph(gvj));
+#pragma unroll 1
+          for (int k = 0; k < 2; ++k) {
+            const int nk = k ? w.nk1 : w.nk0;  // key tiles of query tile k
+            if ((k == 1 && single) || j >= nk) continue;
+            const bool next = j + 1 < nk;
+            uint32_t& nt = k ? nt1 : nt0;
+            mbar_wait(bar(B_PH0 + k), nt & 1u);
+            ATTN_TRACE(it == 0, 2560 + 8 * j + 3 * k + 1);
+            tc_fence_after();
+            issue_pv_half(k, gvj, 0, j == 0);
+            mbar_wait(bar(B_PF0 + k), nt & 1u);
+            ++nt;
+            ATTN_TRACE(it == 0, 2560 + 8 * j + 3 * k + 2);
+            tc_fence_after();
+            issue_pv_half(k, gvj, 1, j == 0);
+            if (next) {
+              issue_s(k, gn);
+              commit(bar(B_SF0 + k));
+            }
+          }
+          commit(vfree(gvj));
+          if (more) commit(kfree(gn));
+        }
+        ATTN_TRACE(true, 2048 + 16 * it + 4);
+        // memory read: sigma(Q_k) (written over Q_k by the softmax warps) times M_{s-1}
+        const uint32_t gm = knext(gk, w.nk1);
+        mbar_wait(kfull(gm), kph(gm));
+        const uint32_t mt = sKt(gm);  // M_{s-1} [dk][dv]: MN-major B operand (like V)
+#pragma unroll 1
+        for (int k = 0; k < (single ? 1 : 2); ++k) {
+          mbar_wait(bar(B_SQ0 + k), (uint32_t)(it & 1));
+          tc_fence_after();
+          const uint64_t da = kmajor_base(sQi(k)), db = mnmajor_base(mt);
+          if (elect_one()) {
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ss(tmem + (uint32_t)k * 128u, da + kmajor_step(kk), db + mnmajor_step(kk), idesc_mem, kk > 0 ? 1u : 0u);
+          }
+          __syncwarp();
+          commit(bar(B_MEM0 + k));
+          ATTN_TRACE(true, 2048 + 16 * it + 5 + k);
+        }
+        commit(kfree(gm));
+        gk = knext(gm, 1);
+        gv += (uint32_t)w.nk1;
       }
+      // every product issued has completed before TMEM is released
+      if (elect_one()) {
+        mma_commit(bar(B_DONE));
+        mbar_drain(bar(B_DONE), 0);
+      }
+      __syncwarp();
     }
   }
   } else {
     regs_increase<kAttnSoftmaxRegs>();
     // -------------------------------------------------------------- softmax WGs
-    const int k = warp >> 2;            // query tile tq0 + k
+    const int k = warp >> 2;  // query tile tq0 + k of each item
     if (!(single && k == 1)) {
     const int row = (warp & 3) * 32 + lane;  // query row in the tile = TMEM lane
     const uint32_t lrow = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lrow + (uint32_t)k * 128u;
     const uint32_t tO = tmem + lrow + 256u + (uint32_t)k * 128u;
-    const int nk = nk0 + k;             // its K/V tiles; the last one is its diagonal
     const float c = a.scale_log2;
-    float m_ref = 0.f, l = 0.f;
     const bool tr = (row == 0);
-    const float zrow = a.snapz[(long long)seg * 128 + row];  // used after the loop
-    for (int j = 0; j < nk; ++j) {
-      ATTN_TRACE(tr, 1024 * k + 8 * j + 0);
-      mbar_wait(bar(B_SF0 + k), j & 1);
-      ATTN_TRACE(tr, 1024 * k + 8 * j + 1);
-      tc_fence_after();
-      uint32_t x[128];
-      {
-        uint32_t (&x0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&x[0]);
-        uint32_t (&x1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&x[32]);
-        uint32_t (&x2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&x[64]);
-        uint32_t (&x3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&x[96]);
-        tmem_ld32(tS, x0);
-        tmem_ld32(tS + 32u, x1);
-        tmem_ld32(tS + 64u, x2);
-        tmem_ld32(tS + 96u, x3);
-        tmem_ld_wait();
-      }
-      if (j == nk - 1) {  // diagonal tile: key e is visible to query row iff e <= row
-#pragma unroll
-        for (int e = 0; e < 128; ++e)
-          if (e > row) x[e] = __float_as_uint(-INFINITY);
-      }
-      float mx[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) mx[i] = __uint_as_float(x[i]);
-#pragma unroll
-      for (int e = 4; e < 128; ++e) mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(x[e]));
-      const float mxs = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * c;
-      ATTN_TRACE(tr, 1024 * k + 8 * j + 2);
-      // Move the reference max only when the row max grows by more than 2^8:
-      // O / l stays exact for any reference, and p stays below 256.
-      const float m_new = (j == 0) ? mxs : (mxs > m_ref + 8.f ? mxs : m_ref);
-      const bool resc = (j > 0) && (m_new != m_ref);
-      if (__any_sync(0xffffffffu, resc)) {
-        // S_k(j) complete implies P V of tile j-1 complete (issue order), so O is final here.
-        const float alpha = resc ? ex2_approx(m_ref - m_new) : 1.f;
-        l *= alpha;
-        uint32_t o[16];
-#pragma unroll 1
-        for (int cc = 0; cc < 8; ++cc) {
-          tmem_ld16(tO + 16u * cc, o);
+    uint32_t ns = 0;  // S tiles of query tile k so far (phase of its S barrier)
+    for (int it = 0;; ++it) {
+      const int idx = take_item(it, true);
+      if (idx < 0) break;
+      Item w;
+      decode(idx, w);
+      const int nk = w.nk0 + k;  // its K/V tiles; the last one is its diagonal
+      ATTN_TRACE(tr, 1024 * k + 16 * it + 0);
+      ATTN_TRACE_VAL(tr, 1024 * k + 16 * it + 8, (unsigned long long)nk);
+      const float zrow = a.snapz[(long long)w.seg * 128 + row];  // used after the loop
+      float m_ref = 0.f, l = 0.f;
+      for (int j = 0; j < nk; ++j) {
+        mbar_wait(bar(B_SF0 + k), ns & 1u);
+        ++ns;
+        ATTN_TRACE(tr && j == 0, 1024 * k + 16 * it + 1);
+        ATTN_TRACE(tr && it == 0, 1024 * k + 512 + 8 * j + 0);
+        tc_fence_after();
+        uint32_t x[128];
+        {
+          uint32_t (&x0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&x[0]);
+          uint32_t (&x1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&x[32]);
+          uint32_t (&x2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&x[64]);
+          uint32_t (&x3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&x[96]);
+          tmem_ld32(tS, x0);
+          tmem_ld32(tS + 32u, x1);
+          tmem_ld32(tS + 64u, x2);
+          tmem_ld32(tS + 96u, x3);
           tmem_ld_wait();
+        }
+        ATTN_TRACE(tr && it == 0, 1024 * k + 512 + 8 * j + 2);
+        if (j == nk - 1) {  // diagonal tile: key e is visible to query row iff e <= row
 #pragma unroll
-          for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st16(tO + 16u * cc, o);
+          for (int e = 0; e < 128; ++e)
+            if (e > row) x[e] = __float_as_uint(-INFINITY);
+        }
+        float mx[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) mx[i] = __uint_as_float(x[i]);
+#pragma unroll
+        for (int e = 4; e < 128; ++e) mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(x[e]));
+        const float mxs = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * c;
+        // Move the reference max only when the row max grows by more than 2^8:
+        // O / l stays exact for any reference, and p stays below 256.
+        const float m_new = (j == 0) ? mxs : (mxs > m_ref + 8.f ? mxs : m_ref);
+        const bool resc = (j > 0) && (m_new != m_ref);
+        if (__any_sync(0xffffffffu, resc)) {
+          // S_k(j) complete implies P V of tile j-1 complete (issue order), so O is final here.
+          const float alpha = resc ? ex2_approx(m_ref - m_new) : 1.f;
+          l *= alpha;
+          uint32_t o[16];
+#pragma unroll 1
+          for (int cc = 0; cc < 8; ++cc) {
+            tmem_ld16(tO + 16u * cc, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st16(tO + 16u * cc, o);
+          }
+          tmem_st_wait();
+        }
+        m_ref = m_new;
+        const float nm = -m_ref;
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int e = 0; e < 64; ++e) {
+          float a0, a1;
+          if (INFINI_F32X2) {
+            fma2(a0, a1, __uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1]), c, c, nm, nm);
+          } else {
+            a0 = fmaf(__uint_as_float(x[2 * e]), c, nm);
+            a1 = fmaf(__uint_as_float(x[2 * e + 1]), c, nm);
+          }
+          float p0, p1;
+          if (INFINI_POLY_EVERY > 0 && (e % (INFINI_POLY_EVERY > 0 ? INFINI_POLY_EVERY : 1)) == INFINI_POLY_EVERY - 1) {
+            p0 = exp2_poly(a0);
+            p1 = exp2_poly(a1);
+          } else {
+            p0 = ex2_approx(a0);
+            p1 = ex2_approx(a1);
+          }
+          if (INFINI_F32X2) {
+            if ((e & 1) == 0) {
+              add2(ls[0], ls[1], ls[0], ls[1], p0, p1);
+            } else {
+              add2(ls[2], ls[3], ls[2], ls[3], p0, p1);
+            }
+          } else {
+            ls[e & 3] += p0 + p1;
+          }
+          x[e] = INFINI_PACK_ALU ? pack_bf16x2_alu(p0, p1) : pack_bf16x2(p0, p1);
+          if (e == 31) {  // keys 0-63 done: their P goes to TMEM while the rest is computed
+            uint32_t (&ph)[32] = *reinterpret_cast<uint32_t(*)[32]>(&x[0]);
+            tmem_st32(tS, ph);
+          }
+          if (e == 47) {
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(bar(B_PH0 + k));
+            ATTN_TRACE(tr && it == 0, 1024 * k + 512 + 8 * j + 4);
+          }
+        }
+        l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        ATTN_TRACE(tr && it == 0, 1024 * k + 512 + 8 * j + 3);
+        {
+          uint32_t (&p1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&x[32]);
+          tmem_st32(tS + 32u, p1);
         }
         tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar(B_PF0 + k));
+        ATTN_TRACE(tr && it == 0, 1024 * k + 512 + 8 * j + 1);
       }
-      m_ref = m_new;
-      const float nm = -m_ref;
-      float ls[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int e = 0; e < 64; ++e) {
-        float a0, a1;
-        if (INFINI_F32X2) {
-          fma2(a0, a1, __uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1]), c, c, nm, nm);
-        } else {
-          a0 = fmaf(__uint_as_float(x[2 * e]), c, nm);
-          a1 = fmaf(__uint_as_float(x[2 * e + 1]), c, nm);
-        }
-        float p0, p1;
-        if (INFINI_POLY_EVERY > 0 && (e % (INFINI_POLY_EVERY > 0 ? INFINI_POLY_EVERY : 1)) == INFINI_POLY_EVERY - 1) {
-          p0 = exp2_poly(a0);
-          p1 = exp2_poly(a1);
-        } else {
-          p0 = ex2_approx(a0);
-          p1 = ex2_approx(a1);
-        }
-        if (INFINI_F32X2) {
-          if ((e & 1) == 0) {
-            add2(ls[0], ls[1], ls[0], ls[1], p0, p1);
-          } else {
-            add2(ls[2], ls[3], ls[2], ls[3], p0, p1);
-          }
-        } else {
-          ls[e & 3] += p0 + p1;
-        }
-        x[e] = INFINI_PACK_ALU ? pack_bf16x2_alu(p0, p1) : pack_bf16x2(p0, p1);
-      }
-      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-      ATTN_TRACE(tr, 1024 * k + 8 * j + 3);
+      ATTN_TRACE(tr, 1024 * k + 16 * it + 2);
+      // Every Q_k K^T product of the item has completed: overwrite this row of
+      // Q_k with sigma(Q_k) (bf16) for the memory read, and form the fp32
+      // denominator sigma(q) . z_{s-1} from the unrounded sigma.  (The z copy
+      // is free again here: the warpgroup's last reads of it, in the previous
+      // item, precede its O-free arrival, which precedes this item's S.)
+      float den = 0.f;
       {
-        uint32_t (&p0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&x[0]);
-        uint32_t (&p1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&x[32]);
-        tmem_st32(tS, p0);
-        tmem_st32(tS + 32u, p1);
+        float* zk = zs + 128 * k;
+        zk[row] = zrow;
+        named_bar_sync(1 + k, 128);
+        ATTN_TRACE(tr, 1024 * k + 16 * it + 9);
+        const uint32_t q = sQ(k);
+        uint4 wq[16];
+#pragma unroll
+        for (int cc = 0; cc < 16; ++cc) wq[cc] = lds128(q + swz_chunk(row, cc));
+        float dp[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int cc = 0; cc < 16; ++cc) {
+          uint32_t* wp = reinterpret_cast<uint32_t*>(&wq[cc]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float s0 = elu1(bf16_lo(wp[e])), s1 = elu1(bf16_hi(wp[e]));
+            dp[e] = fmaf(s0, zk[8 * cc + 2 * e], dp[e]);
+            dp[e] = fmaf(s1, zk[8 * cc + 2 * e + 1], dp[e]);
+            wp[e] = pack_bf16x2(s0, s1);
+          }
+        }
+        ATTN_TRACE(tr, 1024 * k + 16 * it + 10);
+#pragma unroll
+        for (int cc = 0; cc < 16; ++cc) sts128(q + swz_chunk(row, cc), wq[cc]);
+        den = (dp[0] + dp[1]) + (dp[2] + dp[3]);
+        fence_proxy_async_smem();
+        mbar_arrive(bar(B_SQ0 + k));
       }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(bar(B_PF0 + k));
-      ATTN_TRACE(tr, 1024 * k + 8 * j + 4);
-    }
-    // Every Q_k K^T product has completed: overwrite this row of Q_k with
-    // sigma(Q_k) (bf16) for the memory read, and form the fp32 denominator
-    // sigma(q) . z_{s-1} from the unrounded sigma.
-    float den = 0.f;
-    {
-      float* zk = zs + 128 * k;
-      zk[row] = zrow;
-      named_bar_sync(1 + k, 128);
-      ATTN_TRACE(row == 0, 3008 + 8 * k + 3);
-      const uint32_t q = sQ(k);
-      uint4 w[16];
+      ATTN_TRACE(tr, 1024 * k + 16 * it + 3);
+      // ---------------------------------------------------------------- epilogue
+      mbar_wait(bar(B_MEM0 + k), (uint32_t)(it & 1));  // also implies the last P V of tile k
+      ATTN_TRACE(tr, 1024 * k + 16 * it + 4);
+      tc_fence_after();
+      const float gw = 1.f / (1.f + __expf(-a.beta[w.h]));
+      const float wdot = (1.f - gw) / l;
+      const float wmem = den != 0.f ? gw / den : 0.f;
+      uint32_t pk[64];
 #pragma unroll
-      for (int cc = 0; cc < 16; ++cc) w[cc] = lds128(q + swz_chunk(row, cc));
-      ATTN_TRACE(row == 0, 3008 + 8 * k + 4);
-      float dp[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t ro[32], rm[32];
+        tmem_ld32(tO + 32u * cc, ro);
+        tmem_ld32(tS + 32u * cc, rm);
+        tmem_ld_wait();
 #pragma unroll
-      for (int cc = 0; cc < 16; ++cc) {
-        uint32_t* wp = reinterpret_cast<uint32_t*>(&w[cc]);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float s0 = elu1(bf16_lo(wp[e])), s1 = elu1(bf16_hi(wp[e]));
-          dp[e] = fmaf(s0, zk[8 * cc + 2 * e], dp[e]);
-          dp[e] = fmaf(s1, zk[8 * cc + 2 * e + 1], dp[e]);
-          wp[e] = pack_bf16x2(s0, s1);
+        for (int e = 0; e < 16; ++e) {
+          const float v0 = wmem * __uint_as_float(rm[2 * e]) + wdot * __uint_as_float(ro[2 * e]);
+          const float v1 = wmem * __uint_as_float(rm[2 * e + 1]) + wdot * __uint_as_float(ro[2 * e + 1]);
+          pk[16 * cc + e] = pack_bf16x2(v0, v1);
         }
       }
-      ATTN_TRACE(row == 0, 3008 + 8 * k + 5);
+      // S_k and O_k are read out: the next item's products may overwrite them
+      // while this row goes to memory.
+      tc_fence_before();
+      mbar_arrive(bar(B_OF0 + k));
+      ATTN_TRACE(tr, 1024 * k + 16 * it + 5);
+      const int qrow = (w.tq0 + k) * kTile + row;
+      if (qrow < w.n_s) {
+        uint4* dst = reinterpret_cast<uint4*>(a.out + w.b * a.os[0] + w.h * a.os[1] + (w.seg0 + qrow) * a.os[2]);
 #pragma unroll
-      for (int cc = 0; cc < 16; ++cc) sts128(q + swz_chunk(row, cc), w[cc]);
-      den = (dp[0] + dp[1]) + (dp[2] + dp[3]);
-      ATTN_TRACE(row == 0, 3008 + 8 * k + 6);
-      fence_proxy_async_smem();
-      mbar_arrive(bar(B_SQ0 + k));
-      ATTN_TRACE(row == 0, 3008 + 8 * k + 0);
-    }
-    // ---------------------------------------------------------------- epilogue
-    mbar_wait(bar(B_MEM0 + k), 0);  // also implies the last P V product of tile k is complete
-    ATTN_TRACE(row == 0, 3008 + 8 * k + 1);
-    tc_fence_after();
-    const float gw = 1.f / (1.f + __expf(-a.beta[h]));
-    const float wdot = (1.f - gw) / l;
-    const float wmem = den != 0.f ? gw / den : 0.f;
-    const int qrow = (tq0 + k) * kTile + row;
-    const bool valid = qrow < n_s;
-    __nv_bfloat16* orow = a.out + b * a.os[0] + h * a.os[1] + (seg0 + qrow) * a.os[2];
-#pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
-      uint32_t ro[32], rm[32];
-      tmem_ld32(tO + 32u * cc, ro);
-      tmem_ld32(tS + 32u * cc, rm);
-      tmem_ld_wait();
-      uint32_t pk[16];
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const float v0 = wmem * __uint_as_float(rm[2 * e]) + wdot * __uint_as_float(ro[2 * e]);
-        const float v1 = wmem * __uint_as_float(rm[2 * e + 1]) + wdot * __uint_as_float(ro[2 * e + 1]);
-        pk[e] = pack_bf16x2(v0, v1);
+        for (int e = 0; e < 16; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
       }
-      if (valid) {
-        uint4* dst = reinterpret_cast<uint4*>(orow + 32 * cc);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
-      }
+      ATTN_TRACE(tr, 1024 * k + 16 * it + 6);
     }
-    ATTN_TRACE(row == 0, 3008 + 8 * k + 2);
     }
   }
   tc_fence_before();

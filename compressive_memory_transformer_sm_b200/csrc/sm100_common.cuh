@@ -20,14 +20,20 @@ constexpr int kTile = 128;
 constexpr uint32_t kBox = 16384;        // 128 rows x 128 B
 constexpr uint32_t kTileBytes = 32768;  // two boxes
 
-// Descriptor of K-step kk (16 elements along K) of a K-major tile.
-__device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int kk) {
-  return smem_desc_sw128(tile + (uint32_t)(kk >> 2) * kBox + (uint32_t)(kk & 3) * 32u, 16u, 1024u);
+// Descriptor of K-step kk (16 elements along K) of a K-major tile: the
+// descriptor of step 0 plus the step's offset in the start-address field.
+// Shared-memory addresses stay below 256 KB, so (address >> 4) fits the
+// 14-bit field and the addition never carries out of it; the base is then
+// computed once per tile and each step costs one add.
+__device__ __forceinline__ uint64_t kmajor_base(uint32_t tile) { return smem_desc_sw128(tile, 16u, 1024u); }
+__host__ __device__ constexpr uint64_t kmajor_step(int kk) {
+  return (uint64_t)((uint32_t)(kk >> 2) * (kBox >> 4) + (uint32_t)(kk & 3) * 2u);
 }
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int kk) { return kmajor_base(tile) + kmajor_step(kk); }
 // Descriptor of K-step kk (16 rows along K) of an MN-major tile.
-__device__ __forceinline__ uint64_t mnmajor_desc(uint32_t tile, int kk) {
-  return smem_desc_sw128(tile + (uint32_t)kk * 2048u, kBox, 1024u);
-}
+__device__ __forceinline__ uint64_t mnmajor_base(uint32_t tile) { return smem_desc_sw128(tile, kBox, 1024u); }
+__host__ __device__ constexpr uint64_t mnmajor_step(int kk) { return (uint64_t)((uint32_t)kk * (2048u >> 4)); }
+__device__ __forceinline__ uint64_t mnmajor_desc(uint32_t tile, int kk) { return mnmajor_base(tile) + mnmajor_step(kk); }
 // Descriptor of K-step kk of the 16-row K-major block of ones (two 2 KB boxes).
 __device__ __forceinline__ uint64_t ones_desc(uint32_t tile, int kk) {
   return smem_desc_sw128(tile + (uint32_t)(kk >> 2) * 2048u + (uint32_t)(kk & 3) * 32u, 16u, 1024u);
