@@ -586,24 +586,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         named_bar_sync(1 + k, 128);
         ATTN_TRACE(tr, 1024 * k + 16 * it + 9);
         const uint32_t q = sQ(k);
-        uint4 wq[16];
-#pragma unroll
-        for (int cc = 0; cc < 16; ++cc) wq[cc] = lds128(q + swz_chunk(row, cc));
         float dp[4] = {0.f, 0.f, 0.f, 0.f};
+        // Two batches of 8 chunks: the loads of a batch are in flight
+        // together and its 64 elements are independent, while the code stays
+        // small enough for the instruction cache (this runs once per item).
+#pragma unroll 1
+        for (int c8 = 0; c8 < 16; c8 += 8) {
+          uint4 v[8];
 #pragma unroll
-        for (int cc = 0; cc < 16; ++cc) {
-          uint32_t* wp = reinterpret_cast<uint32_t*>(&wq[cc]);
+          for (int i = 0; i < 8; ++i) v[i] = lds128(q + swz_chunk(row, c8 + i));
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float s0 = elu1(bf16_lo(wp[e])), s1 = elu1(bf16_hi(wp[e]));
-            dp[e] = fmaf(s0, zk[8 * cc + 2 * e], dp[e]);
-            dp[e] = fmaf(s1, zk[8 * cc + 2 * e + 1], dp[e]);
-            wp[e] = pack_bf16x2(s0, s1);
+          for (int i = 0; i < 8; ++i) {
+            const float4 za = *reinterpret_cast<const float4*>(zk + 8 * (c8 + i));
+            const float4 zb = *reinterpret_cast<const float4*>(zk + 8 * (c8 + i) + 4);
+            const float zz[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
+            uint32_t* wp = reinterpret_cast<uint32_t*>(&v[i]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float s0 = elu1(bf16_lo(wp[e])), s1 = elu1(bf16_hi(wp[e]));
+              dp[e] = fmaf(s0, zz[2 * e], dp[e]);
+              dp[e] = fmaf(s1, zz[2 * e + 1], dp[e]);
+              wp[e] = pack_bf16x2(s0, s1);
+            }
           }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) sts128(q + swz_chunk(row, c8 + i), v[i]);
         }
         ATTN_TRACE(tr, 1024 * k + 16 * it + 10);
-#pragma unroll
-        for (int cc = 0; cc < 16; ++cc) sts128(q + swz_chunk(row, cc), wq[cc]);
         den = (dp[0] + dp[1]) + (dp[2] + dp[3]);
         fence_proxy_async_smem();
         mbar_arrive(bar(B_SQ0 + k));
@@ -616,31 +625,40 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const float gw = 1.f / (1.f + __expf(-a.beta[w.h]));
       const float wdot = (1.f - gw) / l;
       const float wmem = den != 0.f ? gw / den : 0.f;
-      uint32_t pk[64];
+      const int qrow = (w.tq0 + k) * kTile + row;
+      const bool valid = qrow < w.n_s;
+      uint4* dst = reinterpret_cast<uint4*>(a.out + w.b * a.os[0] + w.h * a.os[1] + (w.seg0 + qrow) * a.os[2]);
+      // two halves of 64 columns: four TMEM loads in flight per wait
+#pragma unroll 1
+      for (int c2 = 0; c2 < 4; c2 += 2) {
+        uint32_t ro[64], rm[64];
+        {
+          uint32_t (&ro0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&ro[0]);
+          uint32_t (&ro1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&ro[32]);
+          uint32_t (&rm0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&rm[0]);
+          uint32_t (&rm1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&rm[32]);
+          tmem_ld32(tO + 32u * c2, ro0);
+          tmem_ld32(tO + 32u * (c2 + 1), ro1);
+          tmem_ld32(tS + 32u * c2, rm0);
+          tmem_ld32(tS + 32u * (c2 + 1), rm1);
+          tmem_ld_wait();
+        }
+        uint32_t pk[32];
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t ro[32], rm[32];
-        tmem_ld32(tO + 32u * cc, ro);
-        tmem_ld32(tS + 32u * cc, rm);
-        tmem_ld_wait();
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
+        for (int e = 0; e < 32; ++e) {
           const float v0 = wmem * __uint_as_float(rm[2 * e]) + wdot * __uint_as_float(ro[2 * e]);
           const float v1 = wmem * __uint_as_float(rm[2 * e + 1]) + wdot * __uint_as_float(ro[2 * e + 1]);
-          pk[16 * cc + e] = pack_bf16x2(v0, v1);
+          pk[e] = pack_bf16x2(v0, v1);
+        }
+        if (valid) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) dst[4 * c2 + e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
         }
       }
       // S_k and O_k are read out: the next item's products may overwrite them
-      // while this row goes to memory.
       tc_fence_before();
       mbar_arrive(bar(B_OF0 + k));
       ATTN_TRACE(tr, 1024 * k + 16 * it + 5);
-      const int qrow = (w.tq0 + k) * kTile + row;
-      if (qrow < w.n_s) {
-        uint4* dst = reinterpret_cast<uint4*>(a.out + w.b * a.os[0] + w.h * a.os[1] + (w.seg0 + qrow) * a.os[2]);
-#pragma unroll
-        for (int e = 0; e < 16; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
-      }
       ATTN_TRACE(tr, 1024 * k + 16 * it + 6);
     }
     }
