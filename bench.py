@@ -340,6 +340,7 @@ def run_ours(args, w: W.Workload, mode: int):
     result = {
         "metric": METRIC, "value": tokens / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "step_ms_min_max": [min(step_ms), max(step_ms)],
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32",
         "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "N": w.N, "dk": w.dk, "dv": w.dv,

@@ -36,7 +36,9 @@ namespace tc {
 // overwrites V in place)),
 // warp 9 issues the MMAs:
 //   dM += sK_hi^T U_hi + sK_lo^T U_hi (+ sK_hi^T U_lo)   (fp32 in TMEM)
-//   dz += sK_hi^T 1 + sK_lo^T 1                        (N = 16 block of ones)
+//   dz += sK_hi^T 1 + sK_lo^T 1                        (N = 16 block of ones; delta:
+//                                                       16 extra columns of the first
+//                                                       two products, B = [U_hi | 1])
 // which keeps the update within ~2^-16 relative of fp32 arithmetic.  The lo
 // parts of the next chunk wait in registers until the MMAs of the previous
 // chunk have released the lo buffers, so the CUDA-core pass overlaps them.
@@ -66,11 +68,14 @@ struct UpdSmem {
   static constexpr int VST = DELTA ? 1 : 2;   // V ring depth
   static constexpr uint32_t K0 = 0;           // K ring (KST x 32 KB); sigma(K)_hi in place
   static constexpr uint32_t V0 = KST * 32768u;  // V ring; U_hi in place (delta)
-  static constexpr uint32_t KLO = V0 + VST * 32768u;
+  // delta: 16 KB of ones right after the single V stage, the third 64-column
+  // block of the B operand [U_hi | 1] (N = 144) whose extra columns gather dz
+  static constexpr uint32_t ONESB = V0 + VST * 32768u;
+  static constexpr uint32_t KLO = ONESB + (DELTA ? 16384u : 0u);
   static constexpr uint32_t ULO = KLO + 32768u;                 // delta
   static constexpr uint32_t MT = ULO + 32768u;                  // delta: M_{s-1} [dk][dv]
-  static constexpr uint32_t ONES = DELTA ? MT + 32768u : KLO + 32768u;
-  static constexpr uint32_t Z = ONES + 4096u;
+  static constexpr uint32_t ONES = KLO + 32768u;                // linear: 16-row K-major block of ones (4 KB)
+  static constexpr uint32_t Z = DELTA ? MT + 32768u : ONES + 4096u;
   static constexpr uint32_t DENP = Z + 512u;  // [2 buffers][2 halves][128]
   static constexpr uint32_t BAR = DENP + 2048u;
   static constexpr uint32_t SLOT = BAR + 256u;
@@ -154,8 +159,8 @@ __global__ void __launch_bounds__(UpdWarps<DELTA>::THREADS, 1)
       fence_barrier_init();
     }
     {
-      uint32_t* ones = reinterpret_cast<uint32_t*>(gbase + SL::ONES);
-      for (int e = threadIdx.x; e < 1024; e += blockDim.x) ones[e] = 0x3f803f80u;  // bf16 1.0 pairs
+      uint32_t* ones = reinterpret_cast<uint32_t*>(gbase + (DELTA ? SL::ONESB : SL::ONES));
+      for (int e = threadIdx.x; e < (DELTA ? 4096 : 1024); e += blockDim.x) ones[e] = 0x3f803f80u;  // bf16 1.0 pairs
     }
     if (threadIdx.x < 128) zs[threadIdx.x] = DELTA ? a.snapz[((long long)bh * a.S + s) * 128 + threadIdx.x] : 0.f;
     if (warp == NCW + 1) {
@@ -199,6 +204,7 @@ __global__ void __launch_bounds__(UpdWarps<DELTA>::THREADS, 1)
         // ---------------------------------------------------------- MMA issuer
         constexpr uint32_t idesc_r = idesc_bf16(128, 128, 0, 1);  // B = M_{s-1} [dk][dv], MN-major
         constexpr uint32_t idesc_m = idesc_bf16(128, 128, 1, 1);
+        constexpr uint32_t idesc_m1 = idesc_bf16(128, 144, 1, 1);  // delta: B = [U_hi | 1]
         constexpr uint32_t idesc_z = idesc_bf16(128, 16, 1, 0);
         for (int c = 0; c < nchunks; ++c) {
           const int kst = c % KST, vst = c % VST;
@@ -220,12 +226,18 @@ __global__ void __launch_bounds__(UpdWarps<DELTA>::THREADS, 1)
             const uint32_t acc = (c > 0 || kk > 0) ? 1u : 0u;
             const uint64_t aH = mnmajor_desc(sK(kst), kk), aL = mnmajor_desc(sKlo, kk);
             const uint64_t bH = mnmajor_desc(sV(vst), kk);
-            mma_ss(tM, aH, bH, idesc_m, acc);
-            mma_ss(tM, aL, bH, idesc_m, 1u);
-            if (DELTA) mma_ss(tM, aH, mnmajor_desc(sUlo, kk), idesc_m, 1u);
-            const uint64_t bO = ones_desc(sOnes, kk);
-            mma_ss(tZ, aH, bO, idesc_z, acc);
-            mma_ss(tZ, aL, bO, idesc_z, 1u);
+            if (DELTA) {
+              // columns 128-143 of [dM | dz] (TMEM tZ) collect sigma(K)^T 1
+              mma_ss(tM, aH, bH, idesc_m1, acc);
+              mma_ss(tM, aL, bH, idesc_m1, 1u);
+              mma_ss(tM, aH, mnmajor_desc(sUlo, kk), idesc_m, 1u);
+            } else {
+              mma_ss(tM, aH, bH, idesc_m, acc);
+              mma_ss(tM, aL, bH, idesc_m, 1u);
+              const uint64_t bO = ones_desc(sOnes, kk);
+              mma_ss(tZ, aH, bO, idesc_z, acc);
+              mma_ss(tZ, aL, bO, idesc_z, 1u);
+            }
           }
           mma_commit(bar(U_MMA));
           UPD_TRACE(c < 64, 3200 + 8 * c + 6);
