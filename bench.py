@@ -291,6 +291,11 @@ def run_ours(args, w: W.Workload, mode: int):
     barrier(dev)
     torch.cuda.synchronize(dev)
     launches0 = api.infini_attn_launch_count()
+    # Hold the stream for a few ms so that the host queues the timed steps
+    # ahead of the device: the events then time device work back to back, not
+    # host launch jitter (the e2e measurement below includes the host).
+    if hasattr(torch.cuda, "_sleep"):
+        torch.cuda._sleep(int(3e6 + 1e5 * args.steps))
     wall0 = time.perf_counter()
     for i in range(args.steps):
         reset_state()

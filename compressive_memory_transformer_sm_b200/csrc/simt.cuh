@@ -170,10 +170,25 @@ __global__ void __launch_bounds__(256) state_kernel(float* __restrict__ M, float
     }
   };
   if (op == 0) {
-    for (int sl = 0; sl < nseg; ++sl) {
-      snap(sl, acc);
-      const float* p = partial + ((long long)bh * nseg + sl) * G * pstride + e;
-      for (int gi = 0; gi < G; ++gi) acc += p[gi * pstride];
+    // eight segments at a time: their partial sums are loaded together, so
+    // the scan waits on memory once per eight segments rather than per segment
+    for (int s8 = 0; s8 < nseg; s8 += 8) {
+      float d[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        d[u] = 0.f;
+        if (s8 + u < nseg) {
+          const float* p = partial + ((long long)bh * nseg + s8 + u) * G * pstride + e;
+          for (int gi = 0; gi < G; ++gi) d[u] += p[gi * pstride];
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (s8 + u < nseg) {
+          snap(s8 + u, acc);
+          acc += d[u];
+        }
+      }
     }
     *st = acc;
   } else if (op == 1) {
