@@ -76,8 +76,8 @@ struct UpdSmem {
   static constexpr uint32_t MT = ULO + 32768u;                  // delta: M_{s-1} [dk][dv]
   static constexpr uint32_t ONES = KLO + 32768u;                // linear: 16-row K-major block of ones (4 KB)
   static constexpr uint32_t Z = DELTA ? MT + 32768u : ONES + 4096u;
-  static constexpr uint32_t DENP = Z + 512u;  // [2 buffers][2 halves][128]
-  static constexpr uint32_t BAR = DENP + 2048u;
+  static constexpr uint32_t DENP = Z + 512u;  // [2 buffers][4 parts of a row][128]
+  static constexpr uint32_t BAR = DENP + 4096u;
   static constexpr uint32_t SLOT = BAR + 256u;
   static constexpr uint32_t BYTES = SLOT + 16u + 1024u;
   static_assert(BYTES <= 232448, "update kernel exceeds 227 KB of shared memory");
@@ -87,13 +87,15 @@ struct UpdSmem {
 };
 
 enum : int {
-  U_KF0 = 0, U_KE0 = 3, U_VF0 = 6, U_VE0 = 8, U_MT = 10, U_SK = 11, U_R = 12, U_U = 13, U_MMA = 14, U_COUNT = 15
+  U_KF0 = 0, U_KE0 = 3, U_VF0 = 6, U_VE0 = 8, U_MT = 10, U_SK = 11, U_R = 12, U_U = 13, U_MMA = 14,
+  U_SKH = 15,  // delta: sigma(K)_hi of the chunk written (the R product may start)
+  U_COUNT = 16
 };
-// Compute warps: 16 for the linear rule (four threads per token row, 32
-// columns each, to hide the latency of the sigma pass), 8 for the delta rule
-// (two per row: its U pass needs the registers).  Plus a TMA and an MMA warp.
+// Compute warps: 16 (four threads per token row, 32 columns each), so that
+// enough warps hide the latency of the sigma and U passes.  Plus a TMA and an
+// MMA warp.
 template <bool DELTA> struct UpdWarps {
-  static constexpr int NCW = DELTA ? 8 : 16;
+  static constexpr int NCW = 16;
   static constexpr int PARTS = NCW / 4;        // threads per token row
   static constexpr int CH = 16 / PARTS;        // 16-byte chunks (8 columns) per thread
   static constexpr int THREADS = 32 * (NCW + 2);
@@ -153,6 +155,7 @@ __global__ void __launch_bounds__(UpdWarps<DELTA>::THREADS, 1)
       }
       mbar_init(bar(U_MT), 1);
       mbar_init(bar(U_SK), 32 * NCW);
+      mbar_init(bar(U_SKH), 32 * NCW);
       mbar_init(bar(U_R), 1);
       mbar_init(bar(U_U), 32 * NCW);
       mbar_init(bar(U_MMA), 1);
@@ -208,16 +211,19 @@ __global__ void __launch_bounds__(UpdWarps<DELTA>::THREADS, 1)
         constexpr uint32_t idesc_z = idesc_bf16(128, 16, 1, 0);
         for (int c = 0; c < nchunks; ++c) {
           const int kst = c % KST, vst = c % VST;
-          mbar_wait(bar(U_SK), c & 1);
           if (DELTA) {
+            // R = sigma(K)_hi M_{s-1} needs only the hi part: it starts while
+            // the compute warps store the lo part and exchange the denominators
+            mbar_wait(bar(U_SKH), c & 1);
             if (c == 0) mbar_wait(bar(U_MT), 0);
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
               mma_ss(tR, kmajor_desc(sK(kst), kk), mnmajor_desc(sMs, kk), idesc_r, kk > 0 ? 1u : 0u);
             mma_commit(bar(U_R));
-            mbar_wait(bar(U_U), c & 1);
+            mbar_wait(bar(U_U), c & 1);  // after the lo part and U: the dM products
           } else {
+            mbar_wait(bar(U_SK), c & 1);
             mbar_wait(bar(U_VF0 + vst), (c / VST) & 1);
           }
           tc_fence_after();
@@ -264,21 +270,40 @@ __global__ void __launch_bounds__(UpdWarps<DELTA>::THREADS, 1)
 #pragma unroll
         for (int i = 0; i < CH; ++i) {
           uint32_t* wp = reinterpret_cast<uint32_t*>(&w[i]);
+          float zz[8];
+          if (DELTA) {
+            const float4 za = *reinterpret_cast<const float4*>(zs + 8 * (CH * hh + i));
+            const float4 zb = *reinterpret_cast<const float4*>(zs + 8 * (CH * hh + i) + 4);
+            zz[0] = za.x; zz[1] = za.y; zz[2] = za.z; zz[3] = za.w;
+            zz[4] = zb.x; zz[5] = zb.y; zz[6] = zb.z; zz[7] = zb.w;
+          }
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float s0 = valid ? elu1(bf16_lo(wp[e])) : 0.f;
-            const float s1 = valid ? elu1(bf16_hi(wp[e])) : 0.f;
+            const float s0 = elu1(bf16_lo(wp[e]));
+            const float s1 = elu1(bf16_hi(wp[e]));
             if (DELTA) {
-              dp[e] = fmaf(s0, zs[8 * (CH * hh + i) + 2 * e], dp[e]);
-              dp[e] = fmaf(s1, zs[8 * (CH * hh + i) + 2 * e + 1], dp[e]);
+              dp[e] = fmaf(s0, zz[2 * e], dp[e]);
+              dp[e] = fmaf(s1, zz[2 * e + 1], dp[e]);
             }
             const uint32_t hi = pack_bf16x2(s0, s1);
             wp[e] = hi;
             lo[4 * i + e] = pack_bf16x2(s0 - bf16_lo(hi), s1 - bf16_hi(hi));
           }
         }
+        if (!valid) {  // a token past the end of the segment (the TMA read zeros) contributes nothing
+#pragma unroll
+          for (int i = 0; i < CH; ++i) w[i] = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+          for (int i = 0; i < 4 * CH; ++i) lo[i] = 0u;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dp[e] = 0.f;
+        }
 #pragma unroll
         for (int i = 0; i < CH; ++i) sts128(sK(kst) + swz_chunk(row, CH * hh + i), w[i]);
+        if (DELTA) {
+          fence_proxy_async_smem();
+          mbar_arrive(bar(U_SKH));
+        }
         const float dpart = (dp[0] + dp[1]) + (dp[2] + dp[3]);
         UPD_TRACE(tr, 3200 + 8 * c + 1);
         if (c > 0) mbar_wait(bar(U_MMA), (c - 1) & 1);  // MMAs of chunk c-1 released the lo buffers
@@ -288,9 +313,11 @@ __global__ void __launch_bounds__(UpdWarps<DELTA>::THREADS, 1)
           sts128(sKlo + swz_chunk(row, CH * hh + i), make_uint4(lo[4 * i], lo[4 * i + 1], lo[4 * i + 2], lo[4 * i + 3]));
         float den = 0.f;
         if (DELTA) {
-          denp[(c & 1) * 256 + hh * 128 + row] = dpart;
+          float* dpb = denp + (c & 1) * (PARTS * 128);
+          dpb[hh * 128 + row] = dpart;
           named_bar_sync(1, 32 * NCW);
-          den = denp[(c & 1) * 256 + row] + denp[(c & 1) * 256 + 128 + row];
+#pragma unroll
+          for (int pp = 0; pp < PARTS; ++pp) den += dpb[pp * 128 + row];  // fixed order
         }
         fence_proxy_async_smem();
         mbar_arrive(bar(U_SK));
@@ -300,25 +327,25 @@ __global__ void __launch_bounds__(UpdWarps<DELTA>::THREADS, 1)
           UPD_TRACE(tr, 3200 + 8 * c + 4);
           tc_fence_after();
           const float rinv = den != 0.f ? 1.f / den : 0.f;
-          uint32_t r0[32], r1[32];
-          tmem_ld32(tR + lrow + 64u * hh, r0);
-          tmem_ld32(tR + lrow + 64u * hh + 32u, r1);
+          constexpr int CPT = 128 / PARTS;  // value columns of this thread
+          uint32_t r[CPT];
+#pragma unroll
+          for (int q2 = 0; q2 < CPT / 32; ++q2)
+            tmem_ld32(tR + lrow + (uint32_t)(CPT * hh + 32 * q2), *reinterpret_cast<uint32_t(*)[32]>(&r[32 * q2]));
           tmem_ld_wait();
           mbar_wait(bar(U_VF0 + vst), (c / VST) & 1);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const uint32_t off = swz_chunk(row, 8 * hh + i);
+          for (int i = 0; i < CH; ++i) {
+            const uint32_t off = swz_chunk(row, CH * hh + i);
             uint4 w = lds128(sV(vst) + off);
             uint4 wl;
             uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
             uint32_t* lp = reinterpret_cast<uint32_t*>(&wl);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const int col = 8 * i + 2 * e;  // within this thread's 64 columns
-              const float rr0 = __uint_as_float(col < 32 ? r0[col] : r1[col - 32]);
-              const float rr1 = __uint_as_float(col + 1 < 32 ? r0[col + 1] : r1[col + 1 - 32]);
-              const float u0 = bf16_lo(wp[e]) - rr0 * rinv;
-              const float u1 = bf16_hi(wp[e]) - rr1 * rinv;
+              const int col = 8 * i + 2 * e;  // within this thread's columns
+              const float u0 = bf16_lo(wp[e]) - __uint_as_float(r[col]) * rinv;
+              const float u1 = bf16_hi(wp[e]) - __uint_as_float(r[col + 1]) * rinv;
               const uint32_t hi = pack_bf16x2(u0, u1);
               wp[e] = hi;
               lp[e] = pack_bf16x2(u0 - bf16_lo(hi), u1 - bf16_hi(hi));
