@@ -261,7 +261,7 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale) {
   });
   const dim3 sgrid((E + 128 + 255) / 256, BH);
   tc::UpdArgs ua;
-  ua.snapz = snapz; ua.partial = part; ua.M = p.M; ua.z = p.z; ua.snapM = snapM16; ua.snapzw = snapz;
+  ua.partial = part; ua.M = p.M; ua.z = p.z; ua.snapM = snapM16; ua.snapzw = snapz;
   ua.B = p.B; ua.H = p.H; ua.S = pl.S; ua.N = p.N; ua.L = p.L;
   ua.G = pl.G; ua.cpb = pl.cpb;
   if (!pl.delta) {
@@ -269,17 +269,12 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale) {
     {
       LaunchScope ls(kPhaseUpdate, p.stream);
       tc::mem_update_tc_kernel<false><<<BH * pl.S * pl.G, tc::UpdWarps<false>::THREADS, tc::UpdSmem<false>::BYTES, p.stream>>>(
-          tm_k, tm_v, tm_mt, ua);
+          tm_k, tm_v, ua);
     }
     LaunchScope ls(kPhaseState, p.stream);
     state_kernel<<<sgrid, 256, 0, p.stream>>>(p.M, p.z, part, 128, 128, pl.S, 0, 0, pl.S, pl.G, nullptr, snapM16,
                                               snapz);
   } else {
-    {
-      LaunchScope ls(kPhaseState, p.stream);
-      state_kernel<<<sgrid, 256, 0, p.stream>>>(p.M, p.z, part, 128, 128, pl.S, 2, 0, 1, pl.G, nullptr, snapM16,
-                                                snapz);
-    }
     ua.nseg = 1;
     // one cluster of G CTAs per head; G <= 8 (plan)
     cudaLaunchConfig_t cfg = {};
@@ -295,11 +290,11 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     for (int s = 0; s < pl.S; ++s) {
-      // partials of segment s, reduced inside each head's cluster into M, z and
-      // the snapshot of M_s for segment s + 1
+      // snapshot of M_{s-1}, z_{s-1} for segment s, then the partials of
+      // segment s, reduced inside each head's cluster into M, z
       ua.seg0 = s;
       LaunchScope ls(kPhaseUpdate, p.stream);
-      if (cudaLaunchKernelEx(&cfg, tc::mem_update_tc_kernel<true>, tm_k, tm_v, tm_mt, ua) != cudaSuccess)
+      if (cudaLaunchKernelEx(&cfg, tc::mem_update_tc_kernel<true>, tm_k, tm_v, ua) != cudaSuccess)
         return INFINI_ERR_LAUNCH;
     }
   }

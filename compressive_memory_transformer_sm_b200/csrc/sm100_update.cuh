@@ -50,12 +50,11 @@ namespace tc {
 // snapshot of M_s for the next segment.  A second cluster barrier keeps every
 // CTA's shared memory alive until its peers have read it.
 struct UpdArgs {
-  const float* snapz;           // [BH][S][128]
   float* partial;               // [BH][nseg][G][128*128 + 128] (linear)
   float* M;                     // running state (delta)
   float* z;
   __nv_bfloat16* snapM;         // [BH][S][128][128] bf16 [dk][dv] (delta: M_s for segment s+1)
-  float* snapzw;                // [BH][S][128] (delta: z_s for segment s+1)
+  float* snapzw;                // [BH][S][128] (delta: z_{s-1} for segment s)
   int B, H, S, N;
   long long L;
   int seg0, nseg, G, cpb;
@@ -104,7 +103,7 @@ template <bool DELTA> struct UpdWarps {
 template <bool DELTA>
 __global__ void __launch_bounds__(UpdWarps<DELTA>::THREADS, 1)
     mem_update_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                         const __grid_constant__ CUtensorMap tm_mt, const UpdArgs a) {
+                         const UpdArgs a) {
   using SL = UpdSmem<DELTA>;
   using WR = UpdWarps<DELTA>;
   constexpr int KST = SL::KST, VST = SL::VST;
@@ -130,6 +129,31 @@ __global__ void __launch_bounds__(UpdWarps<DELTA>::THREADS, 1)
   const int nchunks = t_begin < t_end ? (t_end - t_begin + kTile - 1) / kTile : 0;
 
   float* red = reinterpret_cast<float*>(gbase + SL::RED);
+  if (DELTA) {
+    // M_{s-1}, z_{s-1} of the head: every CTA with tokens converts M to bf16
+    // in its shared memory (the B operand of R, in the layout a 128-byte
+    // swizzled TMA load would give); CTA grp writes slice grp of the bf16
+    // snapshot of segment s that the attention kernel reads, CTA 0 the z
+    // snapshot.  The running M, z change only after the cluster barrier below,
+    // once every CTA of the head has passed this point.
+    const float* Mh = a.M + (long long)bh * 16384;
+    __nv_bfloat16* snap = a.snapM + ((long long)bh * a.S + s) * 16384;
+    const int per = (2048 + a.G - 1) / a.G;  // 16-byte chunks of the snapshot per CTA
+    const int c_lo = grp * per, c_hi = min(2048, c_lo + per);
+    for (int ch = threadIdx.x; ch < 2048; ch += blockDim.x) {
+      const bool mine = ch >= c_lo && ch < c_hi;
+      if (nchunks == 0 && !mine) continue;
+      const int r = ch >> 4, cc = ch & 15;
+      const float4 f0 = *reinterpret_cast<const float4*>(Mh + r * 128 + 8 * cc);
+      const float4 f1 = *reinterpret_cast<const float4*>(Mh + r * 128 + 8 * cc + 4);
+      const uint4 v = make_uint4(pack_bf16x2(f0.x, f0.y), pack_bf16x2(f0.z, f0.w), pack_bf16x2(f1.x, f1.y),
+                                 pack_bf16x2(f1.z, f1.w));
+      if (nchunks > 0) sts128(base + SL::MT + swz_chunk(r, cc), v);
+      if (mine) *reinterpret_cast<uint4*>(snap + r * 128 + 8 * cc) = v;
+    }
+    if (grp == 0 && threadIdx.x < 128)
+      a.snapzw[((long long)bh * a.S + s) * 128 + threadIdx.x] = a.z[(long long)bh * 128 + threadIdx.x];
+  }
   if (nchunks == 0) {  // group past the end of a short segment: contributes nothing
     if (DELTA) {
       for (int e = threadIdx.x; e < 128 * 128 + 128; e += blockDim.x) red[e] = 0.f;
@@ -153,7 +177,6 @@ __global__ void __launch_bounds__(UpdWarps<DELTA>::THREADS, 1)
         mbar_init(bar(U_VF0 + i), 1);
         mbar_init(bar(U_VE0 + i), 1);
       }
-      mbar_init(bar(U_MT), 1);
       mbar_init(bar(U_SK), 32 * NCW);
       mbar_init(bar(U_SKH), 32 * NCW);
       mbar_init(bar(U_R), 1);
@@ -165,7 +188,7 @@ __global__ void __launch_bounds__(UpdWarps<DELTA>::THREADS, 1)
       uint32_t* ones = reinterpret_cast<uint32_t*>(gbase + (DELTA ? SL::ONESB : SL::ONES));
       for (int e = threadIdx.x; e < (DELTA ? 4096 : 1024); e += blockDim.x) ones[e] = 0x3f803f80u;  // bf16 1.0 pairs
     }
-    if (threadIdx.x < 128) zs[threadIdx.x] = DELTA ? a.snapz[((long long)bh * a.S + s) * 128 + threadIdx.x] : 0.f;
+    if (threadIdx.x < 128) zs[threadIdx.x] = DELTA ? a.z[(long long)bh * 128 + threadIdx.x] : 0.f;
     if (warp == NCW + 1) {
       tmem_alloc(smem_u32(tmem_slot), 512);
       tmem_relinquish();
@@ -182,12 +205,6 @@ __global__ void __launch_bounds__(UpdWarps<DELTA>::THREADS, 1)
         // ---------------------------------------------------------- producer
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
-        if (DELTA) {
-          const int row = (bh * a.S + s) * 128;
-          mbar_expect_tx(bar(U_MT), kTileBytes);
-          tma_load_2d(sMs, &tm_mt, bar(U_MT), 0, row);
-          tma_load_2d(sMs + kBox, &tm_mt, bar(U_MT), 64, row);
-        }
         for (int c = 0; c < nchunks; ++c) {
           const int lt = (int)(seg_start + t_begin + (long long)c * kTile);
           const int kst = c % KST;
@@ -215,7 +232,6 @@ __global__ void __launch_bounds__(UpdWarps<DELTA>::THREADS, 1)
             // R = sigma(K)_hi M_{s-1} needs only the hi part: it starts while
             // the compute warps store the lo part and exchange the denominators
             mbar_wait(bar(U_SKH), c & 1);
-            if (c == 0) mbar_wait(bar(U_MT), 0);
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
@@ -258,7 +274,7 @@ __global__ void __launch_bounds__(UpdWarps<DELTA>::THREADS, 1)
       const uint32_t lrow = (uint32_t)((warp & 3) * 32) << 16;
       for (int c = 0; c < nchunks; ++c) {
         const int kst = c % KST, vst = c % VST;
-        const bool tr = threadIdx.x == 0 && c < 64;
+        [[maybe_unused]] const bool tr = threadIdx.x == 0 && c < 64;
         mbar_wait(bar(U_KF0 + kst), (c / KST) & 1);
         UPD_TRACE(tr, 3200 + 8 * c + 0);
         const bool valid = t_begin + c * kTile + row < t_end;
@@ -397,8 +413,6 @@ __global__ void __launch_bounds__(UpdWarps<DELTA>::THREADS, 1)
     const int per = (E4 + a.G - 1) / a.G;
     const int e4_begin = grp * per, e4_end = min(E4, e4_begin + per);
     const uint32_t red_addr = smem_u32(red);
-    const bool snap_next = s + 1 < a.S;
-    const long long sb = (long long)bh * a.S + s + 1;
     for (int e4 = e4_begin + (int)threadIdx.x; e4 < e4_end; e4 += blockDim.x) {
       const int e = 4 * e4;
       float4* st = e < 16384 ? reinterpret_cast<float4*>(&a.M[(long long)bh * 16384 + e])
@@ -412,14 +426,6 @@ __global__ void __launch_bounds__(UpdWarps<DELTA>::THREADS, 1)
         acc.w += v.w;
       }
       *st = acc;
-      if (snap_next) {
-        if (e < 16384) {
-          *reinterpret_cast<uint2*>(a.snapM + sb * 16384 + e) =
-              make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
-        } else {
-          *reinterpret_cast<float4*>(&a.snapzw[sb * 128 + (e - 16384)]) = acc;
-        }
-      }
     }
   }
   cluster_sync();  // peers have finished reading this CTA's shared memory
