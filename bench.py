@@ -29,6 +29,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import gc
 import json
 import os
 import statistics
@@ -295,7 +296,9 @@ def run_ours(args, w: W.Workload, mode: int):
     # ahead of the device: the events then time device work back to back, not
     # host launch jitter (the e2e measurement below includes the host).
     if hasattr(torch.cuda, "_sleep"):
-        torch.cuda._sleep(int(3e6 + 1e5 * args.steps))
+        torch.cuda._sleep(int(2e6 + 1e6 * args.steps))  # ~0.5 ms per step: room for host hiccups
+    gc_was_enabled = gc.isenabled()
+    gc.disable()
     wall0 = time.perf_counter()
     for i in range(args.steps):
         reset_state()
@@ -306,6 +309,8 @@ def run_ours(args, w: W.Workload, mode: int):
     torch.cuda.synchronize(dev)
     barrier(dev)
     wall = time.perf_counter() - wall0
+    if gc_was_enabled:
+        gc.enable()
     launches = api.infini_attn_launch_count() - launches0
     api.infini_attn_profile_enable(0)
     clocks = sampler.stop() if sampler else None

@@ -283,36 +283,49 @@ __global__ void __launch_bounds__(UpdWarps<DELTA>::THREADS, 1)
         uint4 w[CH];
 #pragma unroll
         for (int i = 0; i < CH; ++i) w[i] = lds128(sK(kst) + swz_chunk(row, CH * hh + i));
+        if (!DELTA) {
 #pragma unroll
-        for (int i = 0; i < CH; ++i) {
-          uint32_t* wp = reinterpret_cast<uint32_t*>(&w[i]);
-          float zz[8];
-          if (DELTA) {
-            const float4 za = *reinterpret_cast<const float4*>(zs + 8 * (CH * hh + i));
-            const float4 zb = *reinterpret_cast<const float4*>(zs + 8 * (CH * hh + i) + 4);
-            zz[0] = za.x; zz[1] = za.y; zz[2] = za.z; zz[3] = za.w;
-            zz[4] = zb.x; zz[5] = zb.y; zz[6] = zb.z; zz[7] = zb.w;
+          for (int i = 0; i < CH; ++i) {
+            uint32_t* wp = reinterpret_cast<uint32_t*>(&w[i]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float s0 = valid ? elu1(bf16_lo(wp[e])) : 0.f;
+              const float s1 = valid ? elu1(bf16_hi(wp[e])) : 0.f;
+              const uint32_t hi = pack_bf16x2(s0, s1);
+              wp[e] = hi;
+              lo[4 * i + e] = pack_bf16x2(s0 - bf16_lo(hi), s1 - bf16_hi(hi));
+            }
           }
+        } else {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float s0 = elu1(bf16_lo(wp[e]));
-            const float s1 = elu1(bf16_hi(wp[e]));
-            if (DELTA) {
+          for (int i = 0; i < CH; ++i) {
+            uint32_t* wp = reinterpret_cast<uint32_t*>(&w[i]);
+            float zz[8];
+            {
+              const float4 za = *reinterpret_cast<const float4*>(zs + 8 * (CH * hh + i));
+              const float4 zb = *reinterpret_cast<const float4*>(zs + 8 * (CH * hh + i) + 4);
+              zz[0] = za.x; zz[1] = za.y; zz[2] = za.z; zz[3] = za.w;
+              zz[4] = zb.x; zz[5] = zb.y; zz[6] = zb.z; zz[7] = zb.w;
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float s0 = elu1(bf16_lo(wp[e]));
+              const float s1 = elu1(bf16_hi(wp[e]));
               dp[e] = fmaf(s0, zz[2 * e], dp[e]);
               dp[e] = fmaf(s1, zz[2 * e + 1], dp[e]);
+              const uint32_t hi = pack_bf16x2(s0, s1);
+              wp[e] = hi;
+              lo[4 * i + e] = pack_bf16x2(s0 - bf16_lo(hi), s1 - bf16_hi(hi));
             }
-            const uint32_t hi = pack_bf16x2(s0, s1);
-            wp[e] = hi;
-            lo[4 * i + e] = pack_bf16x2(s0 - bf16_lo(hi), s1 - bf16_hi(hi));
           }
-        }
-        if (!valid) {  // a token past the end of the segment (the TMA read zeros) contributes nothing
+          if (!valid) {  // a token past the end of the segment (the TMA read zeros) contributes nothing
 #pragma unroll
-          for (int i = 0; i < CH; ++i) w[i] = make_uint4(0u, 0u, 0u, 0u);
+            for (int i = 0; i < CH; ++i) w[i] = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-          for (int i = 0; i < 4 * CH; ++i) lo[i] = 0u;
+            for (int i = 0; i < 4 * CH; ++i) lo[i] = 0u;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) dp[e] = 0.f;
+            for (int e = 0; e < 4; ++e) dp[e] = 0.f;
+          }
         }
 #pragma unroll
         for (int i = 0; i < CH; ++i) sts128(sK(kst) + swz_chunk(row, CH * hh + i), w[i]);
