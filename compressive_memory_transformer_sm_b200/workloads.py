@@ -91,3 +91,15 @@ def random_state(w: Workload, device="cpu", seed=None, scale=1.0):
     M = scale * torch.randn(w.B, w.H, w.dk, w.dv, generator=g, device=device) * (w.N ** 0.5)
     z = scale * (1.0 + torch.randn(w.B, w.H, w.dk, generator=g, device=device).abs()) * w.N
     return M.float(), z.float()
+
+
+def make_layer_inputs(B: int, H: int, L: int, d_model: int, seed: int, device="cpu", head: int = 128):
+    """Inputs of the full layer in bf16: x [B,L,D] ~ N(0, 1); w_qkv [D, 3*H*head] ~ N(0, 1/D)
+    and w_o [H*head, D] ~ N(0, 1/(H*head)) (unit-variance projections); beta [H] fp32 ~ N(0, 1)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    x = torch.randn(B, L, d_model, generator=g, device=device).to(torch.bfloat16)
+    w_qkv = (torch.randn(d_model, 3 * H * head, generator=g, device=device) / d_model ** 0.5).to(torch.bfloat16)
+    w_o = (torch.randn(H * head, d_model, generator=g, device=device) / (H * head) ** 0.5).to(torch.bfloat16)
+    beta = torch.randn(H, generator=g, device=device)
+    return x, w_qkv, w_o, beta

@@ -21,6 +21,9 @@ Approach", and uses the paper's equation numbers:
 * Eq. 10 gate ``A = sigmoid(beta) * A_mem + (1 - sigmoid(beta)) * A_dot``
 * section 3 "Training infrastructure": segment chunking of the length-L
   sequence inside each attention layer (the last segment may be shorter).
+* Eq. 5  projections ``Q = X W_Q, K = X W_K, V = X W_V`` per head and
+  Eq. 11 ``O = [A_1; ...; A_H] W_O`` (section 3, "Multi-Head
+  Infini-Attention") for the full layer (``layer_forward``).
 
 Readings taken where the pages are silent or ambiguous (each is also a test):
 
@@ -37,7 +40,11 @@ Readings taken where the pages are silent or ambiguous (each is also a test):
   the update happens after the segment's output;
 * the causal mask is inclusive (a query sees itself) and A_dot never looks
   across a segment boundary;
-* beta is one scalar per head shared by every batch row, token and channel.
+* beta is one scalar per head shared by every batch row, token and channel;
+* full layer: the pages fix no precision for the projections; with
+  ``round_intermediates`` the layer keeps Q, K, V and the concatenated head
+  outputs in bfloat16 between its steps (round to nearest, ties to even), as
+  a bf16 implementation stores them; the arithmetic stays fp64.
 
 Everything is evaluated in float64 with NumPy matrix products; there is no
 blocking, fusion or reordering beyond what the equations state.
@@ -231,3 +238,42 @@ def segment_output(Qs, Ks, Vs, M, z, beta_h, scale=None):
     """Output A of one segment of one head given the memory (M_{s-1}, z_{s-1}) it reads (Eq. 6, 7, 10)."""
     A, _, _, _ = infini_attention_segment(Qs, Ks, Vs, M, z, beta_h, LINEAR, scale)
     return A
+
+
+def bf16_round(a) -> np.ndarray:
+    """Nearest bfloat16 value (ties to even), as float64: the storage of the
+    layer's intermediates in a bf16 implementation (a reading; see the header)."""
+    a32 = np.asarray(a, dtype=np.float32)
+    u = a32.view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000).astype(np.uint32)
+    return r.view(np.float32).astype(np.float64)
+
+
+def layer_forward(x, w_qkv, w_o, beta, H, N, mode=LINEAR, M0=None, z0=None, dk=128, round_intermediates=True,
+                  scale=None):
+    """Multi-head layer around the recurrence: Q, K, V = X W_Q, X W_K, X W_V
+    per head (Eq. 5), the whole-sequence ``forward``, then
+    O = [A_1; ...; A_H] W_O (Eq. 11).
+
+    x: [B, L, D]; w_qkv: [D, 3 H dk], column blocks Q | K | V, head h in the
+    columns h dk .. h dk + dk - 1 of each block; w_o: [H dv, D] with dv = dk,
+    row h dv + j multiplying value column j of head h.  Returns
+    ``y [B, L, D]``, ``M_S``, ``z_S`` in float64.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    w_qkv = np.asarray(w_qkv, dtype=np.float64)
+    w_o = np.asarray(w_o, dtype=np.float64)
+    B, L, D = x.shape
+    qkv = x @ w_qkv  # Eq. 5 for all heads at once: [B, L, 3 H dk]
+    if round_intermediates:
+        qkv = bf16_round(qkv)
+
+    def heads(block):
+        cols = qkv[:, :, block * H * dk:(block + 1) * H * dk]
+        return cols.reshape(B, L, H, dk).transpose(0, 2, 1, 3)  # [B, H, L, dk]
+
+    out, M, z = forward(heads(0), heads(1), heads(2), beta, N, mode=mode, M0=M0, z0=z0, scale=scale)
+    a = out.transpose(0, 2, 1, 3).reshape(B, L, H * dk)  # concatenation along the feature axis (Eq. 11)
+    if round_intermediates:
+        a = bf16_round(a)
+    return a @ w_o, M, z

@@ -348,3 +348,71 @@ def pin_trajectory(ref):
 
 
 ALL_PINS.append(pin_trajectory)
+
+
+# ---------------------------------------------------------------------------
+def pin_layer_identity(ref):
+    """With W_Q = W_K = W_V = I and W_O = I (d_model = H d) the layer reduces to the
+    recurrence on X split into heads (Eq. 5 and Eq. 11 with identity projections)."""
+    fails = []
+    B, H, L, dk, N = 2, 3, 11, 4, 4
+    D = H * dk
+    x = _rand((B, L, D), 50)
+    beta = _rand((H,), 51)
+    eye = np.eye(D)
+    w_qkv = np.concatenate([eye, eye, eye], axis=1)
+    xh = x.reshape(B, L, H, dk).transpose(0, 2, 1, 3)
+    for mode in (ref.LINEAR, ref.DELTA):
+        y, M, z = ref.layer_forward(x, w_qkv, eye, beta, H, N, mode=mode, dk=dk, round_intermediates=False)
+        out, M2, z2 = ref.forward(xh, xh, xh, beta, N, mode=mode)
+        fails += _close(y, out.transpose(0, 2, 1, 3).reshape(B, L, D), 1e-12, f"identity layer output (mode {mode})")
+        fails += _close(M, M2, 1e-12, f"identity layer M (mode {mode})")
+        fails += _close(z, z2, 1e-12, f"identity layer z (mode {mode})")
+    return fails
+
+
+ALL_PINS.append(pin_layer_identity)
+
+
+def pin_layer_loops(ref):
+    """Projections written out as sums over the model dimension, element by element
+    (Eq. 5: q_j = sum_c x_c W_Q[c, j]; Eq. 11: o_c = sum_{h, j} a_{h, j} W_O[h d + j, c]),
+    around the recurrence, on a tiny layer with d_model != H d."""
+    fails = []
+    B, H, L, dk, N, D = 1, 2, 5, 3, 2, 4
+    x = _rand((B, L, D), 60)
+    w_qkv = _rand((D, 3 * H * dk), 61, 0.5)
+    w_o = _rand((H * dk, D), 62, 0.5)
+    beta = _rand((H,), 63)
+    proj = np.zeros((3, B, H, L, dk))
+    for blk in range(3):
+        for b in range(B):
+            for h in range(H):
+                for t in range(L):
+                    for j in range(dk):
+                        proj[blk, b, h, t, j] = sum(x[b, t, c] * w_qkv[c, blk * H * dk + h * dk + j] for c in range(D))
+    for mode in (ref.LINEAR, ref.DELTA):
+        out, _, _ = ref.forward(proj[0], proj[1], proj[2], beta, N, mode=mode)
+        want = np.zeros((B, L, D))
+        for b in range(B):
+            for t in range(L):
+                for c in range(D):
+                    want[b, t, c] = sum(out[b, h, t, j] * w_o[h * dk + j, c] for h in range(H) for j in range(dk))
+        y, _, _ = ref.layer_forward(x, w_qkv, w_o, beta, H, N, mode=mode, dk=dk, round_intermediates=False)
+        fails += _close(y, want, 1e-12, f"layer vs element-wise projections (mode {mode})")
+    return fails
+
+
+ALL_PINS.append(pin_layer_loops)
+
+
+def pin_bf16_rounding(ref):
+    """The layer's bf16 storage equals torch's round-to-nearest-even bfloat16 cast."""
+    a = _rand((4096,), 70, 3.0)
+    a[:4] = [1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, -(1.0 + 2.0 ** -8), 2.0 ** -130]  # ties and a denormal
+    want = torch.from_numpy(a.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+    got = ref.bf16_round(a)
+    return [] if np.array_equal(got, want) else ["bf16_round differs from torch's bfloat16 cast"]
+
+
+ALL_PINS.append(pin_bf16_rounding)

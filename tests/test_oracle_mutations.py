@@ -140,6 +140,42 @@ def m_flops_full_square(ref):
     ref.forward_flops = bad
 
 
+def _bad_layer(ref, swap_kv=False, head_major_cols=True):
+    good_forward = ref.forward
+
+    def layer(x, w_qkv, w_o, beta, H, N, mode=0, M0=None, z0=None, dk=128, round_intermediates=True, scale=None):
+        x, w_qkv, w_o = (np.asarray(t, dtype=np.float64) for t in (x, w_qkv, w_o))
+        B, L, D = x.shape
+        qkv = x @ w_qkv
+
+        def heads(block):
+            cols = qkv[:, :, block * H * dk:(block + 1) * H * dk]
+            if head_major_cols:
+                return cols.reshape(B, L, H, dk).transpose(0, 2, 1, 3)
+            return cols.reshape(B, L, dk, H).transpose(0, 3, 1, 2)
+
+        kb, vb = (2, 1) if swap_kv else (1, 2)
+        out, M, z = good_forward(heads(0), heads(kb), heads(vb), beta, N, mode=mode, M0=M0, z0=z0, scale=scale)
+        return out.transpose(0, 2, 1, 3).reshape(B, L, H * dk) @ w_o, M, z
+
+    return layer
+
+
+def m_layer_k_v_swapped(ref):
+    ref.layer_forward = _bad_layer(ref, swap_kv=True)
+
+
+def m_layer_head_columns_interleaved(ref):
+    ref.layer_forward = _bad_layer(ref, head_major_cols=False)
+
+
+def m_bf16_truncates(ref):
+    def bad(a):
+        u = np.asarray(a, dtype=np.float32).view(np.uint32)
+        return (u & np.uint32(0xFFFF0000)).view(np.float32).astype(np.float64)
+    ref.bf16_round = bad
+
+
 MUTANTS = [v for k, v in sorted(globals().items()) if k.startswith("m_")]
 
 
