@@ -442,6 +442,79 @@ def run_e2e(args, w: W.Workload, mode: int, dev, stream, rank):
 
 
 # ------------------------------------------------------------------ reference arm
+LAYER_METRIC = "Infini-attn layer fwd tokens/s (QKV projection + Infini-attention + output projection)"
+
+
+def run_layer(args, w: W.Workload, mode: int):
+    """``--layer``: the full multi-head layer through ``infini_attn_layer_forward`` on the
+    workload's shape with d_model = H * 128, timed like the default line (device events
+    per step, L2 flushed and the state reset between steps, outside the events)."""
+    from compressive_memory_transformer_sm_b200 import api
+
+    rank, world = init_dist("nccl")
+    _, _, local = dist_env()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    D = w.H * w.dk
+    x, w_qkv, w_o, beta = W.make_layer_inputs(w.B, w.H, w.L, D, seed=rank_seed(w, rank), device=dev)
+    M, z = W.empty_state(w, device=dev)
+    y = torch.empty(w.B, w.L, D, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(api.infini_attn_layer_workspace_size(w.B, w.H, w.L, w.N, D, mode), dtype=torch.uint8,
+                     device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        M.zero_()
+        z.zero_()
+        flush.fill_(1)
+
+    for _ in range(args.warmup):
+        step()
+        api.infini_attn_layer_forward(x, w_qkv, w_o, beta, M, z, y, w.H, w.N, mode, workspace=ws, stream=stream)
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(local)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    launches0 = api.infini_attn_launch_count()
+    if hasattr(torch.cuda, "_sleep"):
+        torch.cuda._sleep(int(2e6 + 1e6 * args.steps))
+    for i in range(args.steps):
+        step()
+        evs[i][0].record(stream)
+        api.infini_attn_layer_forward(x, w_qkv, w_o, beta, M, z, y, w.H, w.N, mode, workspace=ws, stream=stream)
+        evs[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    launches = api.infini_attn_launch_count() - launches0
+    clocks = sampler.stop() if sampler else None
+    if api.infini_attn_device_status() != api.INFINI_OK:
+        raise RuntimeError("a device-side wait timed out during the benchmark")
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    ms = max_over_ranks(sum(step_ms) / len(step_ms), dev)
+    f_attn, f_upd = algorithmic_flops(w, mode)
+    f_proj = 2 * w.B * w.L * D * (3 * w.H * w.dk) + 2 * w.B * w.L * (w.H * w.dv) * D
+    peaks, peak_src = load_peaks()
+    peak = peaks["bf16_tflops_sustained"] if ms > 10.0 else peaks["bf16_tflops"]
+    tflops = (f_attn + f_upd + f_proj) * world / (ms * 1e-3) / 1e12
+    result = {
+        "metric": LAYER_METRIC, "value": w.B * w.L * world / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "step_ms_min_max": [min(step_ms), max(step_ms)], "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "N": w.N, "d_model": D,
+                   "mode": W.MODE_NAMES[mode], "layer": "x W_qkv -> Infini-attention -> A W_o",
+                   "l2": "1 GiB buffer written between timed steps (outside the step events)"},
+        "tflops": tflops, "pct_of_bf16_peak": 100.0 * tflops / world / peak,
+        "peak_source": f"{peak_src} {'bf16_tflops_sustained' if ms > 10.0 else 'bf16_tflops'}",
+        "flops_per_step": {"projections": f_proj, "attention": f_attn, "update": f_upd},
+        "gpu_launches": int(launches), "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
 def run_reference(args, w: W.Workload, mode: int):
     rank, world, _ = dist_env()
     if rank != 0:
@@ -488,6 +561,8 @@ def parse(argv=None):
     ap.add_argument("--mode", choices=("linear", "delta"), default=None)
     ap.add_argument("--force-simt", action="store_true", help="time the CUDA-core kernels instead")
     ap.add_argument("--shape", default=None, help="B,H,L,N override of the workload's sizes (for profiling)")
+    ap.add_argument("--layer", action="store_true",
+                    help="time the full layer (QKV projection + attention + output projection) instead")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
@@ -506,6 +581,8 @@ def main(argv=None):
         raise SystemExit("--warmup must be at least 3")
     if args.impl == "reference":
         run_reference(args, w, mode)
+    elif args.layer:
+        run_layer(args, w, mode)
     else:
         run_ours(args, w, mode)
 

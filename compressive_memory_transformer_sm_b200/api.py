@@ -36,6 +36,7 @@ EXPORTED = (
     "infini_attn_error_string", "infini_attn_device_status", "infini_attn_selftest_timeout",
     "infini_attn_params_size", "infini_attn_path", "infini_attn_profile_enable", "infini_attn_profile_read",
     "infini_attn_launch_count", "infini_attn_forward_noalloc", "infini_attn_selftest_exp2",
+    "infini_attn_layer_forward", "infini_attn_layer_workspace_size",
 )
 
 
@@ -74,6 +75,10 @@ lib.infini_attn_profile_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes
 lib.infini_attn_profile_read.restype = _i
 lib.infini_attn_launch_count.argtypes = []
 lib.infini_attn_launch_count.restype = _ll
+lib.infini_attn_layer_forward.argtypes = [_vp] * 7 + [_i, _i, _l, _i, _i, _i, _vp, ctypes.c_size_t, _vp]
+lib.infini_attn_layer_forward.restype = _i
+lib.infini_attn_layer_workspace_size.argtypes = [_i, _i, _l, _i, _i, _i]
+lib.infini_attn_layer_workspace_size.restype = ctypes.c_size_t
 
 PHASE_UPDATE, PHASE_STATE, PHASE_ATTN = 0, 1, 2
 
@@ -154,6 +159,23 @@ def infini_attn_segment_step(q, k, v, beta, M, z, out, mode: int = LINEAR, strea
                                       z.data_ptr(), out.data_ptr(), B, H, n, dk, dv, _mode(mode, q),
                                       _stream(stream))
     return _check(rc, "infini_attn_segment_step", raise_on_error)
+
+
+def infini_attn_layer_forward(x, w_qkv, w_o, beta, M, z, y, H: int, N: int, mode: int = LINEAR, workspace=None,
+                              stream=None, raise_on_error=True):
+    """Full layer: x [B,L,D] bf16; w_qkv [D, 3*H*128] (Q | K | V column blocks, head-major); w_o [H*128, D];
+    y [B,L,D] bf16 (written); beta [H]; M [B,H,128,128]; z [B,H,128].  workspace: optional uint8 device
+    tensor of at least infini_attn_layer_workspace_size(...) bytes."""
+    B, L, D = x.shape
+    ws, wsb = (workspace.data_ptr(), workspace.numel() * workspace.element_size()) if workspace is not None else (None, 0)
+    rc = lib.infini_attn_layer_forward(x.data_ptr(), w_qkv.data_ptr(), w_o.data_ptr(), beta.data_ptr(), M.data_ptr(),
+                                       z.data_ptr(), y.data_ptr(), B, int(H), L, int(N), D, int(mode), ws, wsb,
+                                       _stream(stream))
+    return _check(rc, "infini_attn_layer_forward", raise_on_error)
+
+
+def infini_attn_layer_workspace_size(B, H, L, N, d_model, mode=LINEAR) -> int:
+    return int(lib.infini_attn_layer_workspace_size(B, H, L, N, d_model, mode))
 
 
 def _bhl_strides(t: torch.Tensor):

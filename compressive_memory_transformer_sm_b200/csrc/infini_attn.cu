@@ -11,6 +11,7 @@
 //     query tile), reading the snapshots.
 // The order "read with M_{s-1}, then update" of the pages holds because the
 // attention kernel reads the snapshot of M_{s-1}, never the running state.
+#include <cublas_v2.h>
 #include <math.h>
 #include <stdio.h>
 #include <string.h>
@@ -454,6 +455,63 @@ int noalloc_scratch(void** out) {
 
 using namespace infini;
 
+// ------------------------------------------------------------------ full layer
+// Q, K, V = X W_{Q,K,V}, the Infini-attention forward, Y = A W_O (multi-head
+// formulation, Eq. 5 and Eq. 11).  The projections are plain cuBLAS GEMMs;
+// the layout keeps them copy-free: the QKV product [B*L, 3*H*128] is read by
+// the attention kernels through strided views, and the attention writes its
+// output as [B, L, H, 128], the A operand of the output projection.
+namespace {
+
+constexpr int kLayerHead = 128;
+
+struct LayerPlan {
+  size_t off_qkv, off_ao, off_attn, attn_bytes, total;
+  long long rows;  // B * L
+};
+
+bool layer_plan(int B, int H, long long L, int N, int d_model, int mode, LayerPlan* lp) {
+  if (B <= 0 || H <= 0 || L <= 0 || N <= 0 || d_model <= 0) return false;
+  if ((mode & ~INFINI_DELTA) != 0) return false;  // bf16 layer: no INFINI_F32
+  const long long rows = (long long)B * L;
+  if (rows > (1LL << 31) - 1 || 3LL * H * kLayerHead > (1LL << 31) - 1) return false;
+  const size_t attn = infini_attn_workspace_size(B, H, (long)L, N, kLayerHead, kLayerHead, mode);
+  if (attn == 0) return false;
+  size_t off = 0;
+  lp->off_qkv = off;
+  off = align_up(off + (size_t)rows * 3 * H * kLayerHead * 2);
+  lp->off_ao = off;
+  off = align_up(off + (size_t)rows * H * kLayerHead * 2);
+  lp->off_attn = off;
+  lp->attn_bytes = attn;
+  lp->total = align_up(off + attn);
+  lp->rows = rows;
+  return true;
+}
+
+std::mutex g_blas_mu;
+std::vector<cublasHandle_t> g_blas;  // one handle per device, created on first use
+
+// Row-major C[m, n] = A[m, k] B[k, n] in bf16 with fp32 accumulation, as the
+// column-major product C^T = B^T A^T.
+int gemm_bf16(int dev, cudaStream_t st, const void* A, const void* Bm, void* C, long long m, int n, int k) {
+  std::lock_guard<std::mutex> lk(g_blas_mu);
+  if ((int)g_blas.size() <= dev) g_blas.resize(dev + 1, nullptr);
+  if (!g_blas[dev] && cublasCreate(&g_blas[dev]) != CUBLAS_STATUS_SUCCESS) {
+    g_blas[dev] = nullptr;
+    return INFINI_ERR_LAUNCH;
+  }
+  cublasHandle_t h = g_blas[dev];
+  if (cublasSetStream(h, st) != CUBLAS_STATUS_SUCCESS) return INFINI_ERR_LAUNCH;
+  const float one = 1.f, zero = 0.f;
+  const cublasStatus_t rc =
+      cublasGemmEx(h, CUBLAS_OP_N, CUBLAS_OP_N, n, (int)m, k, &one, Bm, CUDA_R_16BF, n, A, CUDA_R_16BF, k, &zero, C,
+                   CUDA_R_16BF, n, CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT);
+  return rc == CUBLAS_STATUS_SUCCESS ? INFINI_OK : INFINI_ERR_LAUNCH;
+}
+
+}  // namespace
+
 extern "C" {
 
 int infini_attn_forward(const void* q, const void* k, const void* v, const float* beta, float* M, float* z, void* out,
@@ -506,6 +564,77 @@ size_t infini_attn_workspace_size(int B, int H, long L, int N, int dk, int dv, i
   Plan pl2;  // a layout that falls back to CUDA cores needs the fp32 snapshots
   if (make_plan(B, H, L, N, dk, dv, mode, INFINI_FLAG_FORCE_SIMT, &pl2) != INFINI_OK) return 0;
   return std::max(pl.total, pl2.total);
+}
+
+
+size_t infini_attn_layer_workspace_size(int B, int H, long L, int N, int d_model, int mode) {
+  LayerPlan lp;
+  return layer_plan(B, H, L, N, d_model, mode, &lp) ? lp.total : 0;
+}
+
+int infini_attn_layer_forward(const void* x, const void* w_qkv, const void* w_o, const float* beta, float* M,
+                              float* z, void* y, int B, int H, long L, int N, int d_model, int mode, void* workspace,
+                              size_t workspace_bytes, cudaStream_t stream) {
+  if (!x || !w_qkv || !w_o || !beta || !M || !z || !y) return INFINI_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || L <= 0 || N <= 0 || d_model <= 0) return INFINI_ERR_INVALID_ARG;
+  LayerPlan lp;
+  if (!layer_plan(B, H, L, N, d_model, mode, &lp)) return INFINI_ERR_UNSUPPORTED;
+  const size_t ybytes = (size_t)lp.rows * d_model * 2;
+  if (ranges_overlap(y, ybytes, x, ybytes) || ranges_overlap(y, ybytes, w_qkv, (size_t)d_model * 3 * H * kLayerHead * 2) ||
+      ranges_overlap(y, ybytes, w_o, (size_t)H * kLayerHead * d_model * 2))
+    return INFINI_ERR_INVALID_ARG;
+  if (workspace && (workspace_bytes < lp.total || reinterpret_cast<uintptr_t>(workspace) % kAlign != 0))
+    return INFINI_ERR_WORKSPACE;
+  int rc = check_device(true);
+  if (rc != INFINI_OK) return rc;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return INFINI_ERR_DEVICE;
+  char* ws = static_cast<char*>(workspace);
+  bool own = false;
+  if (!ws) {
+    void* w = nullptr;
+    if (cudaMallocAsync(&w, lp.total, stream) != cudaSuccess) {
+      cudaGetLastError();
+      return INFINI_ERR_WORKSPACE;
+    }
+    ws = static_cast<char*>(w);
+    own = true;
+  }
+  const long long HD = (long long)H * kLayerHead;
+  __nv_bfloat16* qkv = reinterpret_cast<__nv_bfloat16*>(ws + lp.off_qkv);
+  __nv_bfloat16* ao = reinterpret_cast<__nv_bfloat16*>(ws + lp.off_ao);
+  rc = gemm_bf16(dev, stream, x, w_qkv, qkv, lp.rows, (int)(3 * HD), d_model);
+  if (rc == INFINI_OK) {
+    infini_attn_params p;
+    memset(&p, 0, sizeof(p));
+    p.q = qkv;
+    p.k = qkv + HD;
+    p.v = qkv + 2 * HD;
+    p.beta = beta;
+    p.M = M;
+    p.z = z;
+    p.out = ao;
+    p.B = B;
+    p.H = H;
+    p.L = L;
+    p.N = N;
+    p.dk = p.dv = kLayerHead;
+    p.mode = mode;
+    // views of the [B*L, 3*H*128] product: (B, H, L) strides
+    const long long in_st[3] = {(long long)L * 3 * HD, kLayerHead, 3 * HD};
+    const long long out_st[3] = {(long long)L * HD, kLayerHead, HD};
+    for (int i = 0; i < 3; ++i) {
+      p.q_stride[i] = p.k_stride[i] = p.v_stride[i] = in_st[i];
+      p.o_stride[i] = out_st[i];
+    }
+    p.workspace = ws + lp.off_attn;
+    p.workspace_bytes = lp.attn_bytes;
+    p.stream = stream;
+    rc = forward_impl(p);
+  }
+  if (rc == INFINI_OK) rc = gemm_bf16(dev, stream, ao, w_o, y, lp.rows, d_model, (int)HD);
+  if (own && cudaFreeAsync(ws, stream) != cudaSuccess && rc == INFINI_OK) rc = INFINI_ERR_WORKSPACE;
+  return rc;
 }
 
 const char* infini_attn_error_string(int code) {

@@ -172,6 +172,34 @@ INFINI_API int infini_attn_forward_ex(const infini_attn_params* p);
 /* Bytes of workspace a forward of this shape needs (0 if the shape is invalid). */
 INFINI_API size_t infini_attn_workspace_size(int B, int H, long L, int N, int dk, int dv, int mode);
 
+/*
+ * Full multi-head layer around the Infini-attention step (multi-head
+ * formulation, Eq. 5 and Eq. 11 of "Leave No Context Behind"):
+ * Q = X W_Q, K = X W_K, V = X W_V per head, the forward of
+ * infini_attn_forward on them, and Y = [A_1 ... A_H] W_O.  bf16 only,
+ * head size 128 (dk = dv = 128, tensor-core path), d_model = D >= 1.
+ *   x      [B, L, D] bf16, contiguous
+ *   w_qkv  [D, 3*H*128] bf16, row-major: columns [0, H*128) give Q (head h
+ *          in columns h*128 .. h*128 + 127), then K, then V
+ *   w_o    [H*128, D] bf16, row-major (row h*128 + j multiplies value
+ *          column j of head h)
+ *   y      [B, L, D] bf16, written
+ *   beta, M, z, N, mode as in infini_attn_forward (mode without INFINI_F32).
+ * The projections are plain GEMMs (cuBLAS: bf16 operands, fp32
+ * accumulation, bf16 results); Q, K, V and the attention output are stored
+ * in bf16 between the steps, in a workspace of
+ * infini_attn_layer_workspace_size(...) bytes (256-byte aligned) that the
+ * call allocates and frees on `stream` when `workspace` is NULL.  Errors as
+ * infini_attn_forward; a cuBLAS failure returns INFINI_ERR_LAUNCH.  Calls
+ * from several host threads share one cuBLAS handle per device under a lock.
+ */
+INFINI_API int infini_attn_layer_forward(const void* x, const void* w_qkv, const void* w_o, const float* beta,
+                                         float* M, float* z, void* y, int B, int H, long L, int N, int d_model,
+                                         int mode, void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Bytes of workspace infini_attn_layer_forward needs (0 if the shape is invalid). */
+INFINI_API size_t infini_attn_layer_workspace_size(int B, int H, long L, int N, int d_model, int mode);
+
 /* Static English text for a return code; never NULL. */
 INFINI_API const char* infini_attn_error_string(int code);
 

@@ -112,3 +112,37 @@ def test_forward_ex_rejects_null_and_small_workspace():
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU answer")
 def test_wellformed_call_without_gpu_reports_device():
     assert _call() == api.INFINI_ERR_DEVICE
+
+
+# ---------------------------------------------------------------- full layer
+def _layer(**over):
+    a = dict(x=1 << 20, w_qkv=2 << 20, w_o=3 << 20, beta=4 << 20, M=5 << 20, z=6 << 20, y=7 << 20,
+             B=1, H=2, L=256, N=128, D=64, mode=LINEAR, ws=None, wsb=0)
+    a.update(over)
+    return api.lib.infini_attn_layer_forward(a["x"], a["w_qkv"], a["w_o"], a["beta"], a["M"], a["z"], a["y"],
+                                             a["B"], a["H"], a["L"], a["N"], a["D"], a["mode"], a["ws"], a["wsb"],
+                                             None)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(x=None), -1), (dict(w_qkv=None), -1), (dict(w_o=None), -1), (dict(y=None), -1), (dict(M=None), -1),
+    (dict(B=0), -1), (dict(D=0), -1), (dict(N=0), -1),
+    (dict(mode=LINEAR | F32), -2),       # the layer is bf16 only
+    (dict(y=(1 << 20) + 64), -1),        # y aliases x
+    (dict(ws=1 << 30, wsb=16), -3),      # workspace too small
+])
+def test_layer_invalid_arguments_rejected_on_host(over, code):
+    assert _layer(**over) == code
+
+
+def test_layer_workspace_size():
+    s = api.infini_attn_layer_workspace_size(1, 8, 32768, 2048, 1024, LINEAR)
+    # Q, K, V and the attention output in bf16, plus the attention workspace
+    assert s >= 32768 * (3 + 1) * 8 * 128 * 2 + api.infini_attn_workspace_size(1, 8, 32768, 2048, 128, 128, LINEAR)
+    assert api.infini_attn_layer_workspace_size(1, 8, 32768, 2048, 0, LINEAR) == 0
+    assert api.infini_attn_layer_workspace_size(1, 8, 32768, 2048, 1024, LINEAR | F32) == 0
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU answer")
+def test_layer_wellformed_call_without_gpu_reports_device():
+    assert _layer() == api.INFINI_ERR_DEVICE
