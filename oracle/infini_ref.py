@@ -21,6 +21,11 @@ Approach", and uses the paper's equation numbers:
 * Eq. 10 gate ``A = sigmoid(beta) * A_mem + (1 - sigmoid(beta)) * A_dot``
 * section 3 "Training infrastructure": segment chunking of the length-L
   sequence inside each attention layer (the last segment may be shorter).
+* token-level streaming decode (``decode_step``): the abstract's "fast
+  streaming inference" read as one new token at a time inside the current
+  segment, its keys and values kept in a per-segment cache and folded into
+  the memory (Eq. 8 / Eq. 9) once the segment is complete; it must give the
+  same outputs and state as the whole-sequence forward.
 * Eq. 5  projections ``Q = X W_Q, K = X W_K, V = X W_V`` per head and
   Eq. 11 ``O = [A_1; ...; A_H] W_O`` (section 3, "Multi-Head
   Infini-Attention") for the full layer (``layer_forward``).
@@ -277,3 +282,43 @@ def layer_forward(x, w_qkv, w_o, beta, H, N, mode=LINEAR, M0=None, z0=None, dk=1
     if round_intermediates:
         a = bf16_round(a)
     return a @ w_o, M, z
+
+
+def decode_step(q_t, k_t, v_t, k_cache, v_cache, beta, M, z, pos, mode=LINEAR, fold=False, scale=None):
+    """One new token per (batch, head) at position ``pos`` of the current segment.
+
+    q_t, k_t: [B, H, dk]; v_t: [B, H, dv]; k_cache [B, H, N, dk] and v_cache
+    [B, H, N, dv] hold the segment's earlier keys and values (updated in
+    place: row ``pos`` receives k_t, v_t); M [B, H, dk, dv], z [B, H, dk] are
+    the memory entering the segment, M_{s-1} and z_{s-1}.  The token attends
+    causally to the segment's keys 0..pos (Eq. 6 for one query row), reads the
+    memory (Eq. 7) and blends (Eq. 10).  When the segment is complete
+    (pos = N - 1) or ``fold`` is set, the segment's keys and values update the
+    memory (Eq. 8 / Eq. 9).  Returns ``out [B, H, dv]``, M, z.
+    """
+    q_t, k_t, v_t = (np.asarray(t, dtype=np.float64) for t in (q_t, k_t, v_t))
+    B, H, dk = q_t.shape
+    dv = v_t.shape[2]
+    N = k_cache.shape[2]
+    scale = 1.0 / math.sqrt(dk) if scale is None else scale
+    k_cache[:, :, pos] = k_t
+    v_cache[:, :, pos] = v_t
+    out = np.zeros((B, H, dv))
+    M = np.array(M, dtype=np.float64)
+    z = np.array(z, dtype=np.float64)
+    for b in range(B):
+        for h in range(H):
+            keys, vals = k_cache[b, h, :pos + 1], v_cache[b, h, :pos + 1]
+            s = scale * (keys @ q_t[b, h])               # scores of the new query row
+            p = np.exp(s - s.max())
+            a_dot = (p / p.sum()) @ vals
+            a_mem = memory_retrieval(elu_plus_one(q_t[b, h][None, :]), M[b, h], z[b, h])[0]
+            g = gate_weight(beta[h])
+            out[b, h] = g * a_mem + (1.0 - g) * a_dot
+    if fold or pos == N - 1:
+        for b in range(B):
+            for h in range(H):
+                sk = elu_plus_one(k_cache[b, h, :pos + 1])
+                upd = linear_update if mode == LINEAR else delta_update
+                M[b, h], z[b, h] = upd(M[b, h], z[b, h], sk, v_cache[b, h, :pos + 1])
+    return out, M, z

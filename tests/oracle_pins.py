@@ -416,3 +416,28 @@ def pin_bf16_rounding(ref):
 
 
 ALL_PINS.append(pin_bf16_rounding)
+
+
+def pin_decode_matches_forward(ref):
+    """Token-by-token decode (a cache per segment, folded into the memory when the
+    segment completes, and at the last token) reproduces the whole-sequence forward:
+    outputs and final state, both rules, with a short tail segment."""
+    fails = []
+    B, H, L, dk, dv, N = 2, 2, 13, 3, 4, 5
+    q, k, v = _rand((B, H, L, dk), 80), _rand((B, H, L, dk), 81), _rand((B, H, L, dv), 82)
+    beta = _rand((H,), 83)
+    for mode in (ref.LINEAR, ref.DELTA):
+        want, wM, wz = ref.forward(q, k, v, beta, N, mode=mode)
+        M, z = np.zeros((B, H, dk, dv)), np.zeros((B, H, dk))
+        kc, vc = np.zeros((B, H, N, dk)), np.zeros((B, H, N, dv))
+        got = np.zeros_like(want)
+        for t in range(L):
+            got[:, :, t], M, z = ref.decode_step(q[:, :, t], k[:, :, t], v[:, :, t], kc, vc, beta, M, z, t % N,
+                                                 mode=mode, fold=(t == L - 1))
+        fails += _close(got, want, 1e-12, f"decode outputs (mode {mode})")
+        fails += _close(M, wM, 1e-12, f"decode final M (mode {mode})")
+        fails += _close(z, wz, 1e-12, f"decode final z (mode {mode})")
+    return fails
+
+
+ALL_PINS.append(pin_decode_matches_forward)

@@ -176,6 +176,14 @@ def m_bf16_truncates(ref):
     ref.bf16_round = bad
 
 
+def m_decode_folds_every_token(ref):
+    good = ref.decode_step
+
+    def bad(q_t, k_t, v_t, k_cache, v_cache, beta, M, z, pos, mode=0, fold=False, scale=None):
+        return good(q_t, k_t, v_t, k_cache, v_cache, beta, M, z, pos, mode=mode, fold=True, scale=scale)
+    ref.decode_step = bad
+
+
 MUTANTS = [v for k, v in sorted(globals().items()) if k.startswith("m_")]
 
 
