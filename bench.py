@@ -515,6 +515,67 @@ def run_layer(args, w: W.Workload, mode: int):
         print(json.dumps(result), flush=True)
 
 
+DECODE_METRIC = "Infini-attn token-level streaming decode tokens/s (one token per (b, h) per call, fold per segment)"
+
+
+def run_decode(args, w: W.Workload, mode: int):
+    """``--decode``: one step = one segment of N tokens fed through ``infini_attn_decode_step``
+    one token at a time (cache append, attention over the segment so far, memory read, gate;
+    the fold into M, z on the segment's last token).  Device events around each segment."""
+    from compressive_memory_transformer_sm_b200 import api
+
+    rank, world = init_dist("nccl")
+    _, _, local = dist_env()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    seg = w.with_(name=w.name, L=w.N)
+    q, k, v, beta = W.make_inputs(seg, device=dev, seed=rank_seed(w, rank))
+    qs = [q[:, :, t].contiguous() for t in range(w.N)]
+    ks = [k[:, :, t].contiguous() for t in range(w.N)]
+    vs = [v[:, :, t].contiguous() for t in range(w.N)]
+    M, z = W.empty_state(w, device=dev)
+    kc = torch.zeros(w.B, w.H, w.N, w.dk, dtype=w.dtype, device=dev)
+    vc = torch.zeros(w.B, w.H, w.N, w.dv, dtype=w.dtype, device=dev)
+    o = torch.empty(w.B, w.H, w.dv, dtype=w.dtype, device=dev)
+
+    def segment():
+        for t in range(w.N):
+            api.infini_attn_decode_step(qs[t], ks[t], vs[t], kc, vc, beta, M, z, o, t, mode, stream=stream)
+
+    for _ in range(args.warmup):
+        segment()
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(local)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    launches0 = api.infini_attn_launch_count()
+    for i in range(args.steps):
+        evs[i][0].record(stream)
+        segment()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    launches = api.infini_attn_launch_count() - launches0
+    clocks = sampler.stop() if sampler else None
+    if api.infini_attn_device_status() != api.INFINI_OK:
+        raise RuntimeError("a device-side wait timed out during the benchmark")
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    ms = max_over_ranks(sum(step_ms) / len(step_ms), dev)
+    result = {
+        "metric": DECODE_METRIC, "value": w.B * w.N * world / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "us_per_token": 1e3 * ms / w.N,
+        "higher_is_better": True, "step_ms_min_max": [min(step_ms), max(step_ms)], "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "dk": w.dk, "dv": w.dv,
+                   "mode": W.MODE_NAMES[mode], "step": "one segment of N decode calls, fold on the last"},
+        "gpu_launches": int(launches), "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
 def run_reference(args, w: W.Workload, mode: int):
     rank, world, _ = dist_env()
     if rank != 0:
@@ -563,6 +624,8 @@ def parse(argv=None):
     ap.add_argument("--shape", default=None, help="B,H,L,N override of the workload's sizes (for profiling)")
     ap.add_argument("--layer", action="store_true",
                     help="time the full layer (QKV projection + attention + output projection) instead")
+    ap.add_argument("--decode", action="store_true",
+                    help="time token-level streaming decode (one segment of single-token calls per step)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
@@ -583,6 +646,8 @@ def main(argv=None):
         run_reference(args, w, mode)
     elif args.layer:
         run_layer(args, w, mode)
+    elif args.decode:
+        run_decode(args, w, mode)
     else:
         run_ours(args, w, mode)
 

@@ -36,7 +36,7 @@ EXPORTED = (
     "infini_attn_error_string", "infini_attn_device_status", "infini_attn_selftest_timeout",
     "infini_attn_params_size", "infini_attn_path", "infini_attn_profile_enable", "infini_attn_profile_read",
     "infini_attn_launch_count", "infini_attn_forward_noalloc", "infini_attn_selftest_exp2",
-    "infini_attn_layer_forward", "infini_attn_layer_workspace_size",
+    "infini_attn_layer_forward", "infini_attn_layer_workspace_size", "infini_attn_decode_step",
 )
 
 
@@ -75,6 +75,8 @@ lib.infini_attn_profile_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes
 lib.infini_attn_profile_read.restype = _i
 lib.infini_attn_launch_count.argtypes = []
 lib.infini_attn_launch_count.restype = _ll
+lib.infini_attn_decode_step.argtypes = [_vp] * 9 + [_i] * 8 + [_vp]
+lib.infini_attn_decode_step.restype = _i
 lib.infini_attn_layer_forward.argtypes = [_vp] * 7 + [_i, _i, _l, _i, _i, _i, _vp, ctypes.c_size_t, _vp]
 lib.infini_attn_layer_forward.restype = _i
 lib.infini_attn_layer_workspace_size.argtypes = [_i, _i, _l, _i, _i, _i]
@@ -159,6 +161,20 @@ def infini_attn_segment_step(q, k, v, beta, M, z, out, mode: int = LINEAR, strea
                                       z.data_ptr(), out.data_ptr(), B, H, n, dk, dv, _mode(mode, q),
                                       _stream(stream))
     return _check(rc, "infini_attn_segment_step", raise_on_error)
+
+
+def infini_attn_decode_step(q_t, k_t, v_t, k_cache, v_cache, beta, M, z, out, pos: int, mode: int = LINEAR,
+                            fold: bool = False, stream=None, raise_on_error=True):
+    """One token per (b, h) at position ``pos`` of the current segment: q_t, k_t [B,H,dk], v_t, out [B,H,dv];
+    k_cache [B,H,N,dk], v_cache [B,H,N,dv] (same dtype, bf16 or fp32); folds the segment into M, z when
+    pos == N - 1 or ``fold``."""
+    B, H, dk = q_t.shape
+    dv = v_t.shape[2]
+    N = k_cache.shape[2]
+    rc = lib.infini_attn_decode_step(q_t.data_ptr(), k_t.data_ptr(), v_t.data_ptr(), k_cache.data_ptr(),
+                                     v_cache.data_ptr(), beta.data_ptr(), M.data_ptr(), z.data_ptr(), out.data_ptr(),
+                                     B, H, N, int(pos), dk, dv, _mode(mode, q_t), int(bool(fold)), _stream(stream))
+    return _check(rc, "infini_attn_decode_step", raise_on_error)
 
 
 def infini_attn_layer_forward(x, w_qkv, w_o, beta, M, z, y, H: int, N: int, mode: int = LINEAR, workspace=None,

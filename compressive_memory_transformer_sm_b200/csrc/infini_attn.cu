@@ -24,6 +24,7 @@
 #include "../../include/infini_attn.h"
 #include "common.cuh"
 #include "simt.cuh"
+#include "decode.cuh"
 #include "sm100_attn.cuh"
 #include "sm100_update.cuh"
 
@@ -566,6 +567,81 @@ size_t infini_attn_workspace_size(int B, int H, long L, int N, int dk, int dv, i
   return std::max(pl.total, pl2.total);
 }
 
+
+int infini_attn_decode_step(const void* q_t, const void* k_t, const void* v_t, void* k_cache, void* v_cache,
+                            const float* beta, float* M, float* z, void* out, int B, int H, int N, int pos, int dk,
+                            int dv, int mode, int fold, cudaStream_t stream) {
+  if (!q_t || !k_t || !v_t || !k_cache || !v_cache || !beta || !M || !z || !out) return INFINI_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || N <= 0 || dk <= 0 || dv <= 0 || pos < 0 || pos >= N) return INFINI_ERR_INVALID_ARG;
+  if ((mode & ~(INFINI_DELTA | INFINI_F32)) != 0 || dk > 128 || dv > 128) return INFINI_ERR_UNSUPPORTED;
+  const bool f32 = (mode & INFINI_F32) != 0;
+  const size_t es = f32 ? 4 : 2;
+  const long long BH = (long long)B * H;
+  if (BH > (1LL << 31) - 1) return INFINI_ERR_UNSUPPORTED;
+  int rc = check_device(false);
+  if (rc != INFINI_OK) return rc;
+  // 1. the token's key and value into row pos of every (b, h) cache
+  char* kc = static_cast<char*>(k_cache);
+  char* vc = static_cast<char*>(v_cache);
+  if (cudaMemcpy2DAsync(kc + (size_t)pos * dk * es, (size_t)N * dk * es, k_t, (size_t)dk * es, (size_t)dk * es,
+                        (size_t)BH, cudaMemcpyDeviceToDevice, stream) != cudaSuccess ||
+      cudaMemcpy2DAsync(vc + (size_t)pos * dv * es, (size_t)N * dv * es, v_t, (size_t)dv * es, (size_t)dv * es,
+                        (size_t)BH, cudaMemcpyDeviceToDevice, stream) != cudaSuccess)
+    return INFINI_ERR_LAUNCH;
+  // 2. the token's output
+  const float scale = 1.f / sqrtf((float)dk);
+  {
+    LaunchScope ls(kPhaseAttn, stream);
+    if (f32)
+      decode_kernel<float><<<(unsigned)BH, 32 * kDecodeWarps, 0, stream>>>(
+          static_cast<const float*>(q_t), reinterpret_cast<const float*>(kc), reinterpret_cast<const float*>(vc),
+          beta, M, z, static_cast<float*>(out), H, N, pos + 1, dk, dv, scale);
+    else
+      decode_kernel<__nv_bfloat16><<<(unsigned)BH, 32 * kDecodeWarps, 0, stream>>>(
+          static_cast<const __nv_bfloat16*>(q_t), reinterpret_cast<const __nv_bfloat16*>(kc),
+          reinterpret_cast<const __nv_bfloat16*>(vc), beta, M, z, static_cast<__nv_bfloat16*>(out), H, N, pos + 1,
+          dk, dv, scale);
+  }
+  rc = launch_status();
+  if (rc != INFINI_OK || !(fold || pos == N - 1)) return rc;
+  // 3. the segment is complete: fold its keys and values into M, z with the
+  // forward's kernels on the cached segment (their attention output is
+  // scratch; the update reads only K, V, M, z)
+  const int n = pos + 1;
+  void* scratch = nullptr;
+  if (cudaMallocAsync(&scratch, (size_t)BH * n * dv * es, stream) != cudaSuccess) {
+    cudaGetLastError();
+    return INFINI_ERR_WORKSPACE;
+  }
+  infini_attn_params p;
+  memset(&p, 0, sizeof(p));
+  p.q = kc;
+  p.k = kc;
+  p.v = vc;
+  p.beta = beta;
+  p.M = M;
+  p.z = z;
+  p.out = scratch;
+  p.B = B;
+  p.H = H;
+  p.L = n;
+  p.N = n;
+  p.dk = dk;
+  p.dv = dv;
+  p.mode = mode;
+  const long long ks[3] = {(long long)H * N * dk, (long long)N * dk, dk};
+  const long long vs[3] = {(long long)H * N * dv, (long long)N * dv, dv};
+  const long long os[3] = {(long long)H * n * dv, (long long)n * dv, dv};
+  for (int i = 0; i < 3; ++i) {
+    p.q_stride[i] = p.k_stride[i] = ks[i];
+    p.v_stride[i] = vs[i];
+    p.o_stride[i] = os[i];
+  }
+  p.stream = stream;
+  rc = forward_impl(p);
+  if (cudaFreeAsync(scratch, stream) != cudaSuccess && rc == INFINI_OK) rc = INFINI_ERR_WORKSPACE;
+  return rc;
+}
 
 size_t infini_attn_layer_workspace_size(int B, int H, long L, int N, int d_model, int mode) {
   LayerPlan lp;

@@ -173,6 +173,32 @@ INFINI_API int infini_attn_forward_ex(const infini_attn_params* p);
 INFINI_API size_t infini_attn_workspace_size(int B, int H, long L, int N, int dk, int dv, int mode);
 
 /*
+ * Token-level streaming decode (the "fast streaming inference" of the
+ * abstract, taken one token at a time): every (b, h) appends one token at
+ * position pos (0 <= pos < N, the same for all (b, h)) of its current
+ * segment of N tokens.  The call
+ *   1. writes k_t, v_t into row pos of the caller-owned caches,
+ *   2. computes the token's output: causal softmax attention over the
+ *      segment's keys 0..pos (Eq. 6 for one query row), the memory read with
+ *      the live M, z = M_{s-1}, z_{s-1} (Eq. 7, 0 when the denominator is 0)
+ *      and the gate (Eq. 10), into out,
+ *   3. when pos == N - 1 or fold != 0, folds the segment's pos + 1 keys and
+ *      values into M, z with the linear (Eq. 8) or delta (Eq. 9) rule.
+ * Feeding a sequence token by token with pos = t mod N, and fold on its last
+ * token, gives the outputs and final state of infini_attn_forward.
+ *   q_t, k_t, out: [B, H, dk] / [B, H, dv]; v_t [B, H, dv]; contiguous, bf16 or
+ *   fp32 (mode | INFINI_F32); k_cache [B, H, N, dk], v_cache [B, H, N, dv] in
+ *   the same type, contiguous, caller-owned, rows > pos not read.
+ * The fold runs the forward's kernels on the cached segment (its attention
+ * output goes to a scratch buffer allocated on `stream`).  Errors as
+ * infini_attn_forward; pos outside [0, N) is INFINI_ERR_INVALID_ARG.
+ */
+INFINI_API int infini_attn_decode_step(const void* q_t, const void* k_t, const void* v_t, void* k_cache,
+                                       void* v_cache, const float* beta, float* M, float* z, void* out, int B,
+                                       int H, int N, int pos, int dk, int dv, int mode, int fold,
+                                       cudaStream_t stream);
+
+/*
  * Full multi-head layer around the Infini-attention step (multi-head
  * formulation, Eq. 5 and Eq. 11 of "Leave No Context Behind"):
  * Q = X W_Q, K = X W_K, V = X W_V per head, the forward of

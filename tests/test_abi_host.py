@@ -146,3 +146,26 @@ def test_layer_workspace_size():
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU answer")
 def test_layer_wellformed_call_without_gpu_reports_device():
     assert _layer() == api.INFINI_ERR_DEVICE
+
+
+# ---------------------------------------------------------------- streaming decode
+def _decode(**over):
+    a = dict(q=1 << 20, k=2 << 20, v=3 << 20, kc=4 << 20, vc=5 << 20, beta=6 << 20, M=7 << 20, z=8 << 20,
+             out=9 << 20, B=1, H=2, N=64, pos=0, dk=128, dv=128, mode=LINEAR, fold=0)
+    a.update(over)
+    return api.lib.infini_attn_decode_step(a["q"], a["k"], a["v"], a["kc"], a["vc"], a["beta"], a["M"], a["z"],
+                                           a["out"], a["B"], a["H"], a["N"], a["pos"], a["dk"], a["dv"], a["mode"],
+                                           a["fold"], None)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(q=None), -1), (dict(kc=None), -1), (dict(out=None), -1), (dict(B=0), -1), (dict(N=0), -1),
+    (dict(pos=-1), -1), (dict(pos=64), -1), (dict(dk=129), -2), (dict(mode=0x4), -2),
+])
+def test_decode_invalid_arguments_rejected_on_host(over, code):
+    assert _decode(**over) == code
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU answer")
+def test_decode_wellformed_call_without_gpu_reports_device():
+    assert _decode() == api.INFINI_ERR_DEVICE
