@@ -121,6 +121,25 @@ def _mode(mode: int, t: torch.Tensor) -> int:
     return int(mode) | (F32 if t.dtype == torch.float32 else 0)
 
 
+def _args(where: str, shapes: dict, contiguous: bool = True):
+    """Marshalling checks before a pointer leaves Python: every tensor on a CUDA device, with the
+    expected number of dimensions, contiguous unless the call takes strides; raises ValueError."""
+    for name, (t, ndim) in shapes.items():
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{where}: {name} must be a torch.Tensor")
+        if t.dim() != ndim:
+            raise ValueError(f"{where}: {name} must have {ndim} dimensions, got shape {tuple(t.shape)}")
+        if t.device.type != "cuda":
+            raise ValueError(f"{where}: {name} must be on a CUDA device, got {t.device}")
+        if contiguous and not t.is_contiguous():
+            raise ValueError(f"{where}: {name} must be contiguous (use infini_attn_forward_ex for strided views)")
+
+
+def _same(where: str, what: str, *vals):
+    if len(set(vals)) != 1:
+        raise ValueError(f"{where}: {what} disagree: {vals}")
+
+
 def _check(rc: int, where: str, raise_on_error: bool):
     if rc != INFINI_OK and raise_on_error:
         raise InfiniAttnError(rc, where)
@@ -129,8 +148,12 @@ def _check(rc: int, where: str, raise_on_error: bool):
 
 def infini_attn_forward(q, k, v, beta, M, z, out, N: int, mode: int = LINEAR, stream=None, raise_on_error=True):
     """q, k [B,H,L,dk], v, out [B,H,L,dv] (bf16 or fp32, contiguous); beta [H]; M [B,H,dk,dv]; z [B,H,dk]."""
+    _args("infini_attn_forward", dict(q=(q, 4), k=(k, 4), v=(v, 4), out=(out, 4), beta=(beta, 1), M=(M, 4),
+                                      z=(z, 3)))
     B, H, L, dk = q.shape
     dv = v.shape[3]
+    _same("infini_attn_forward", "q / k / v / out (B, H, L)", tuple(q.shape[:3]), tuple(k.shape[:3]),
+          tuple(v.shape[:3]), tuple(out.shape[:3]))
     rc = lib.infini_attn_forward(q.data_ptr(), k.data_ptr(), v.data_ptr(), beta.data_ptr(), M.data_ptr(),
                                  z.data_ptr(), out.data_ptr(), B, H, L, int(N), dk, dv, _mode(mode, q),
                                  _stream(stream))
@@ -145,8 +168,12 @@ def infini_attn_forward_noalloc(q, k, v, beta, M, z, out, N: int, mode: int = LI
     cudaMallocAsync; shapes needing more are refused (INFINI_ERR_SCRATCH_LIMIT).  Calls that
     overlap on the GPU share that buffer and race, so keep them on one stream.
     """
+    _args("infini_attn_forward_noalloc", dict(q=(q, 4), k=(k, 4), v=(v, 4), out=(out, 4), beta=(beta, 1),
+                                              M=(M, 4), z=(z, 3)))
     B, H, L, dk = q.shape
     dv = v.shape[3]
+    _same("infini_attn_forward_noalloc", "q / k / v / out (B, H, L)", tuple(q.shape[:3]), tuple(k.shape[:3]),
+          tuple(v.shape[:3]), tuple(out.shape[:3]))
     rc = lib.infini_attn_forward_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), beta.data_ptr(), M.data_ptr(),
                                          z.data_ptr(), out.data_ptr(), B, H, L, int(N), dk, dv, _mode(mode, q),
                                          _stream(stream))
@@ -155,8 +182,12 @@ def infini_attn_forward_noalloc(q, k, v, beta, M, z, out, N: int, mode: int = LI
 
 def infini_attn_segment_step(q, k, v, beta, M, z, out, mode: int = LINEAR, stream=None, raise_on_error=True):
     """One segment of n tokens per (b, h): q, k [B,H,n,dk], v, out [B,H,n,dv]."""
+    _args("infini_attn_segment_step", dict(q=(q, 4), k=(k, 4), v=(v, 4), out=(out, 4), beta=(beta, 1),
+                                           M=(M, 4), z=(z, 3)))
     B, H, n, dk = q.shape
     dv = v.shape[3]
+    _same("infini_attn_segment_step", "q / k / v / out (B, H, n)", tuple(q.shape[:3]), tuple(k.shape[:3]),
+          tuple(v.shape[:3]), tuple(out.shape[:3]))
     rc = lib.infini_attn_segment_step(q.data_ptr(), k.data_ptr(), v.data_ptr(), beta.data_ptr(), M.data_ptr(),
                                       z.data_ptr(), out.data_ptr(), B, H, n, dk, dv, _mode(mode, q),
                                       _stream(stream))
@@ -168,9 +199,14 @@ def infini_attn_decode_step(q_t, k_t, v_t, k_cache, v_cache, beta, M, z, out, po
     """One token per (b, h) at position ``pos`` of the current segment: q_t, k_t [B,H,dk], v_t, out [B,H,dv];
     k_cache [B,H,N,dk], v_cache [B,H,N,dv] (same dtype, bf16 or fp32); folds the segment into M, z when
     pos == N - 1 or ``fold``."""
+    _args("infini_attn_decode_step", dict(q_t=(q_t, 3), k_t=(k_t, 3), v_t=(v_t, 3), k_cache=(k_cache, 4),
+                                          v_cache=(v_cache, 4), out=(out, 3), beta=(beta, 1), M=(M, 4), z=(z, 3)))
     B, H, dk = q_t.shape
     dv = v_t.shape[2]
     N = k_cache.shape[2]
+    _same("infini_attn_decode_step", "token and cache (B, H)", tuple(q_t.shape[:2]), tuple(k_t.shape[:2]),
+          tuple(v_t.shape[:2]), tuple(out.shape[:2]), tuple(k_cache.shape[:2]), tuple(v_cache.shape[:2]))
+    _same("infini_attn_decode_step", "cache lengths", k_cache.shape[2], v_cache.shape[2])
     rc = lib.infini_attn_decode_step(q_t.data_ptr(), k_t.data_ptr(), v_t.data_ptr(), k_cache.data_ptr(),
                                      v_cache.data_ptr(), beta.data_ptr(), M.data_ptr(), z.data_ptr(), out.data_ptr(),
                                      B, H, N, int(pos), dk, dv, _mode(mode, q_t), int(bool(fold)), _stream(stream))
@@ -182,7 +218,13 @@ def infini_attn_layer_forward(x, w_qkv, w_o, beta, M, z, y, H: int, N: int, mode
     """Full layer: x [B,L,D] bf16; w_qkv [D, 3*H*128] (Q | K | V column blocks, head-major); w_o [H*128, D];
     y [B,L,D] bf16 (written); beta [H]; M [B,H,128,128]; z [B,H,128].  workspace: optional uint8 device
     tensor of at least infini_attn_layer_workspace_size(...) bytes."""
+    _args("infini_attn_layer_forward", dict(x=(x, 3), w_qkv=(w_qkv, 2), w_o=(w_o, 2), y=(y, 3), beta=(beta, 1),
+                                            M=(M, 4), z=(z, 3)))
     B, L, D = x.shape
+    _same("infini_attn_layer_forward", "x / y shapes", tuple(x.shape), tuple(y.shape))
+    if tuple(w_qkv.shape) != (D, 3 * int(H) * 128) or tuple(w_o.shape) != (int(H) * 128, D):
+        raise ValueError(f"infini_attn_layer_forward: w_qkv must be [{D}, {3 * int(H) * 128}] and w_o "
+                         f"[{int(H) * 128}, {D}], got {tuple(w_qkv.shape)} and {tuple(w_o.shape)}")
     ws, wsb = (workspace.data_ptr(), workspace.numel() * workspace.element_size()) if workspace is not None else (None, 0)
     rc = lib.infini_attn_layer_forward(x.data_ptr(), w_qkv.data_ptr(), w_o.data_ptr(), beta.data_ptr(), M.data_ptr(),
                                        z.data_ptr(), y.data_ptr(), B, int(H), L, int(N), D, int(mode), ws, wsb,
@@ -204,6 +246,8 @@ def _bhl_strides(t: torch.Tensor):
 def infini_attn_forward_ex(q, k, v, beta, M, z, out, N: int, mode: int = LINEAR, scale: float = 0.0,
                            workspace=None, flags: int = 0, stream=None, raise_on_error=True):
     """Extended call: [B,H,L,d] views with any (B, H, L) strides, explicit scale, caller workspace, flags."""
+    _args("infini_attn_forward_ex", dict(q=(q, 4), k=(k, 4), v=(v, 4), out=(out, 4)), contiguous=False)
+    _args("infini_attn_forward_ex", dict(beta=(beta, 1), M=(M, 4), z=(z, 3)))
     B, H, L, dk = q.shape
     dv = v.shape[3]
     p = InfiniAttnParams()

@@ -169,3 +169,16 @@ def test_decode_invalid_arguments_rejected_on_host(over, code):
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU answer")
 def test_decode_wellformed_call_without_gpu_reports_device():
     assert _decode() == api.INFINI_ERR_DEVICE
+
+
+# ---------------------------------------------------------------- Python marshalling checks
+def test_binding_rejects_host_and_strided_tensors():
+    q = torch.zeros(1, 2, 8, 16)
+    with pytest.raises(ValueError, match="CUDA device"):
+        api.infini_attn_forward(q, q, q, torch.zeros(2), torch.zeros(1, 2, 16, 16), torch.zeros(1, 2, 16), q, 4)
+    with pytest.raises(ValueError, match="dimensions"):
+        api.infini_attn_segment_step(q[0], q, q, torch.zeros(2), torch.zeros(1, 2, 16, 16), torch.zeros(1, 2, 16), q)
+    with pytest.raises(ValueError):
+        api.infini_attn_layer_forward(torch.zeros(1, 8, 64), torch.zeros(64, 3 * 128), torch.zeros(128, 64),
+                                      torch.zeros(1), torch.zeros(1, 1, 128, 128), torch.zeros(1, 1, 128),
+                                      torch.zeros(1, 8, 64), 1, 4)
