@@ -123,9 +123,12 @@ def delta_update(M: np.ndarray, z: np.ndarray, sig_k: np.ndarray, V: np.ndarray)
     return M + sig_k.T @ (V - retrieved), z + sig_k.sum(axis=0)
 
 
-def infini_attention_segment(Qs, Ks, Vs, M, z, beta_h, mode=LINEAR, scale=None):
+def infini_attention_segment(Qs, Ks, Vs, M, z, beta_h, mode=LINEAR, scale=None, q_local=None, k_local=None):
     """One application of the recurrent layer to one segment of one head (Eq. 4).
 
+    ``q_local`` / ``k_local``: the segment's Q and K with position embeddings,
+    used by the local attention only (section 4.1: no position embeddings for
+    the compressive memory's keys and queries); Q and K themselves otherwise.
     Returns ``(A, M_s, z_s, parts)`` where ``parts`` holds ``A_dot`` and
     ``A_mem`` for tests that check them separately.
     """
@@ -136,7 +139,8 @@ def infini_attention_segment(Qs, Ks, Vs, M, z, beta_h, mode=LINEAR, scale=None):
         scale = 1.0 / math.sqrt(Qs.shape[1])
     sig_q = elu_plus_one(Qs)
     sig_k = elu_plus_one(Ks)
-    a_dot = causal_softmax_attention(Qs, Ks, Vs, scale)
+    a_dot = causal_softmax_attention(Qs if q_local is None else q_local, Ks if k_local is None else k_local, Vs,
+                                     scale)
     a_mem = memory_retrieval(sig_q, M, z)
     g = gate_weight(beta_h)
     A = g * a_mem + (1.0 - g) * a_dot
@@ -149,6 +153,23 @@ def infini_attention_segment(Qs, Ks, Vs, M, z, beta_h, mode=LINEAR, scale=None):
     return A, M_new, z_new, {"A_dot": a_dot, "A_mem": a_mem}
 
 
+def rope(x, positions, base=10000.0) -> np.ndarray:
+    """Rotary position embedding of the rows of x [n, d] (d even) at ``positions`` [n]:
+    the pair (x_2i, x_2i+1) is rotated by the angle p * base^(-2i/d).  A reading: the pages
+    say only that position embeddings act on the local attention's Q and K (section 4.1);
+    rotary embeddings in their original pairwise form are taken as the plainest kind."""
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[1]
+    i = np.arange(d // 2, dtype=np.float64)
+    ang = np.asarray(positions, dtype=np.float64)[:, None] * base ** (-2.0 * i / d)[None, :]
+    c, s = np.cos(ang), np.sin(ang)
+    x0, x1 = x[:, 0::2], x[:, 1::2]
+    out = np.empty_like(x)
+    out[:, 0::2] = x0 * c - x1 * s
+    out[:, 1::2] = x0 * s + x1 * c
+    return out
+
+
 def segment_bounds(L: int, N: int):
     """Segment chunking: S = ceil(L/N) segments of N tokens, the last one possibly shorter."""
     if L <= 0 or N <= 0:
@@ -156,10 +177,13 @@ def segment_bounds(L: int, N: int):
     return [(s0, min(s0 + N, L)) for s0 in range(0, L, N)]
 
 
-def forward(q, k, v, beta, N, mode=LINEAR, M0=None, z0=None, scale=None, return_parts=False):
+def forward(q, k, v, beta, N, mode=LINEAR, M0=None, z0=None, scale=None, return_parts=False, rope_base=None,
+            rope_offset=0):
     """Whole-sequence forward: segment chunking then the recurrence of Eq. 4 per (batch, head).
 
     q, k: [B, H, L, dk]; v: [B, H, L, dv]; beta: [H]; M0: [B, H, dk, dv]; z0: [B, H, dk].
+    ``rope_base``: rotary position embeddings (``rope``) on the local attention's Q and K
+    at token positions ``rope_offset + t``; the memory reads and writes un-rotated Q, K.
     Returns ``out [B, H, L, dv]``, ``M_S``, ``z_S`` in float64 (and the A_dot / A_mem
     planes when ``return_parts``).
     """
@@ -178,8 +202,12 @@ def forward(q, k, v, beta, N, mode=LINEAR, M0=None, z0=None, scale=None, return_
         for h in range(H):
             Mbh, zbh = M[b, h], z[b, h]
             for s0, s1 in segment_bounds(L, N):
+                pe = {}
+                if rope_base is not None:
+                    pos = rope_offset + np.arange(s0, s1, dtype=np.float64)
+                    pe = dict(q_local=rope(q[b, h, s0:s1], pos, rope_base), k_local=rope(k[b, h, s0:s1], pos, rope_base))
                 A, Mbh, zbh, parts = infini_attention_segment(
-                    q[b, h, s0:s1], k[b, h, s0:s1], v[b, h, s0:s1], Mbh, zbh, beta[h], mode, scale)
+                    q[b, h, s0:s1], k[b, h, s0:s1], v[b, h, s0:s1], Mbh, zbh, beta[h], mode, scale, **pe)
                 out[b, h, s0:s1] = A
                 if return_parts:
                     a_dot_all[b, h, s0:s1] = parts["A_dot"]

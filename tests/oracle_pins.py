@@ -441,3 +441,64 @@ def pin_decode_matches_forward(ref):
 
 
 ALL_PINS.append(pin_decode_matches_forward)
+
+
+# ---------------------------------------------------------------------------
+def pin_rope_as_complex_rotation(ref):
+    """The rotary embedding equals multiplying each pair (x_2i + i x_2i+1) by exp(i p base^(-2i/d))."""
+    n, d, base = 7, 8, 10000.0
+    x = _rand((n, d), 90)
+    pos = np.array([0, 1, 2, 5, 11, 100, 2047], dtype=np.float64)
+    zc = (x[:, 0::2] + 1j * x[:, 1::2]) * np.exp(1j * pos[:, None] * base ** (-np.arange(0, d, 2) / d)[None, :])
+    want = np.empty_like(x)
+    want[:, 0::2], want[:, 1::2] = zc.real, zc.imag
+    fails = _close(ref.rope(x, pos, base), want, 1e-12, "rope vs complex rotation")
+    fails += _close(ref.rope(x, np.zeros(n), base), x, 0.0, "rope at position 0")
+    return fails
+
+
+ALL_PINS.append(pin_rope_as_complex_rotation)
+
+
+def pin_rope_split(ref):
+    """Position embeddings on the local branch only (section 4.1): the memory state and the
+    memory read are those of the forward without them; the local branch alone is causal
+    softmax attention on the rotated Q, K (torch SDPA, per segment); and it depends only on
+    relative positions, so shifting every position leaves the output unchanged."""
+    fails = []
+    B, H, L, d, N, base = 1, 2, 23, 6, 8, 500.0
+    q, k, v = _rand((B, H, L, d), 91), _rand((B, H, L, d), 92), _rand((B, H, L, d), 93)
+    beta = _rand((H,), 94)
+    for mode in (ref.LINEAR, ref.DELTA):
+        o0, M0, z0 = ref.forward(q, k, v, beta, N, mode=mode)
+        o1, M1, z1 = ref.forward(q, k, v, beta, N, mode=mode, rope_base=base)
+        fails += _close(M1, M0, 1e-12, f"rope leaves M unchanged (mode {mode})")
+        fails += _close(z1, z0, 1e-12, f"rope leaves z unchanged (mode {mode})")
+        inf = np.full(H, np.inf)
+        fails += _close(ref.forward(q, k, v, inf, N, mode=mode, rope_base=base)[0],
+                        ref.forward(q, k, v, inf, N, mode=mode)[0], 1e-12, f"memory read without PE (mode {mode})")
+        shifted = ref.forward(q, k, v, beta, N, mode=mode, rope_base=base, rope_offset=37)[0]
+        fails += _close(shifted, o1, 1e-9, f"rope output shift-invariant (mode {mode})")
+    # local branch alone against SDPA on rotated Q, K computed with complex numbers
+    ninf = np.full(H, -np.inf)
+    got = ref.forward(q, k, v, ninf, N, rope_base=base)[0]
+    want = np.zeros_like(got)
+    for s0 in range(0, L, N):
+        s1 = min(L, s0 + N)
+        pos = np.arange(s0, s1, dtype=np.float64)
+        rot = np.exp(1j * pos[:, None] * base ** (-np.arange(0, d, 2) / d)[None, :])
+
+        def rc(t):
+            zc = (t[..., 0::2] + 1j * t[..., 1::2]) * rot
+            out = np.empty_like(t)
+            out[..., 0::2], out[..., 1::2] = zc.real, zc.imag
+            return out
+
+        qs, ks = rc(q[:, :, s0:s1]), rc(k[:, :, s0:s1])
+        want[:, :, s0:s1] = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(qs), torch.from_numpy(ks), torch.from_numpy(v[:, :, s0:s1]), is_causal=True).numpy()
+    fails += _close(got, want, 1e-12, "local branch with rope vs SDPA")
+    return fails
+
+
+ALL_PINS.append(pin_rope_split)

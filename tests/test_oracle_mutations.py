@@ -184,6 +184,30 @@ def m_decode_folds_every_token(ref):
     ref.decode_step = bad
 
 
+def m_rope_half_split_pairs(ref):
+    def bad(x, positions, base=10000.0):
+        x = np.asarray(x, dtype=np.float64)
+        d = x.shape[1]
+        h = d // 2
+        ang = np.asarray(positions, dtype=np.float64)[:, None] * base ** (-2.0 * np.arange(h) / d)[None, :]
+        c, s = np.cos(ang), np.sin(ang)
+        out = np.empty_like(x)
+        out[:, :h] = x[:, :h] * c - x[:, h:] * s
+        out[:, h:] = x[:, :h] * s + x[:, h:] * c
+        return out
+    ref.rope = bad
+
+
+def m_rope_applied_to_memory(ref):
+    good_segment = ref.infini_attention_segment
+
+    def bad(Qs, Ks, Vs, M, z, beta_h, mode=0, scale=None, q_local=None, k_local=None):
+        if q_local is not None:
+            Qs, Ks = q_local, k_local
+        return good_segment(Qs, Ks, Vs, M, z, beta_h, mode, scale, q_local, k_local)
+    ref.infini_attention_segment = bad
+
+
 MUTANTS = [v for k, v in sorted(globals().items()) if k.startswith("m_")]
 
 
