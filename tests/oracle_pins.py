@@ -502,3 +502,41 @@ def pin_rope_split(ref):
 
 
 ALL_PINS.append(pin_rope_split)
+
+
+# ---------------------------------------------------------------------------
+def pin_backward_finite_differences(ref):
+    """The back-propagation oracle (``oracle.infini_bwd``) against central finite
+    differences of the forward, every coordinate of q, k, v, beta, M_0, z_0, both rules,
+    three segments with a tail, a non-empty initial memory (z_0 > 0)."""
+    from oracle import infini_bwd
+
+    fails = []
+    B, H, L, dk, dv, N = 1, 2, 7, 3, 2, 3
+    q, k, v = _rand((B, H, L, dk), 100), _rand((B, H, L, dk), 101), _rand((B, H, L, dv), 102)
+    beta = _rand((H,), 103)
+    M0 = _rand((B, H, dk, dv), 104)
+    z0 = 1.0 + np.abs(_rand((B, H, dk), 105))
+    W_out, W_M, w_z = _rand((B, H, L, dv), 106), _rand((B, H, dk, dv), 107), _rand((B, H, dk), 108)
+    for mode in (ref.LINEAR, ref.DELTA):
+        def loss(q_, k_, v_, beta_, M_, z_):
+            out, M_S, z_S = ref.forward(q_, k_, v_, beta_, N, mode=mode, M0=M_, z0=z_)
+            return float(np.sum(W_out * out) + np.sum(W_M * M_S) + np.sum(w_z * z_S))
+
+        grads = infini_bwd.backward(q, k, v, beta, N, W_out, W_M, w_z, mode=mode, M0=M0, z0=z0)
+        args = [q, k, v, beta, M0, z0]
+        for ai, (name, g) in enumerate(zip(("q", "k", "v", "beta", "M0", "z0"), grads)):
+            num = np.zeros_like(args[ai])
+            eps = 1e-6
+            for idx in np.ndindex(args[ai].shape):
+                plus = [a.copy() for a in args]
+                minus = [a.copy() for a in args]
+                plus[ai][idx] += eps
+                minus[ai][idx] -= eps
+                num[idx] = (loss(*plus) - loss(*minus)) / (2 * eps)
+            tol = 1e-6 * max(1.0, float(np.max(np.abs(num))))
+            fails += _close(g, num, tol, f"d loss / d {name} (mode {mode})")
+    return fails
+
+
+ALL_PINS.append(pin_backward_finite_differences)

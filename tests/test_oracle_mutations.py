@@ -218,3 +218,31 @@ def test_pins_catch_mutant(mutate):
     mutate(ref)
     bad = oracle_pins.run_all(ref)
     assert bad, f"no pin caught mutation {mutate.__name__}"
+
+
+@pytest.mark.parametrize("which", ["sigma_prime_one", "no_gate_grad", "every_second_retrieval_grad_dropped"])
+def test_backward_pin_catches_mutant(which, monkeypatch):
+    """Plausible mistakes in the back-propagation oracle fail the finite-difference pin."""
+    from oracle import infini_bwd
+
+    if which == "sigma_prime_one":
+        monkeypatch.setattr(infini_bwd, "_sigma_prime", lambda x: np.ones_like(x))
+    elif which == "no_gate_grad":
+        good = infini_bwd.segment_backward
+
+        def bad(*a, **kw):
+            r = good(*a, **kw)
+            return r[0], r[1], r[2], 0.0, r[4], r[5]
+        monkeypatch.setattr(infini_bwd, "segment_backward", bad)
+    else:
+        good_rb = infini_bwd._retrieval_backward
+        calls = {"n": 0}
+
+        def bad_rb(sig_x, M, z, out, d_out):
+            calls["n"] += 1
+            d_sig, dM, dz = good_rb(sig_x, M, z, out, d_out)
+            # every second retrieval (the delta update's, or every other segment's read) loses its contribution
+            return (d_sig * 0.0, dM * 0.0, dz * 0.0) if calls["n"] % 2 == 0 else (d_sig, dM, dz)
+        monkeypatch.setattr(infini_bwd, "_retrieval_backward", bad_rb)
+    ref = fresh_oracle()
+    assert oracle_pins.pin_backward_finite_differences(ref), f"finite-difference pin missed {which}"
