@@ -253,14 +253,26 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale) {
   if (!encode_bhld(&tm_q, p.q, p.B, p.H, p.L, p.q_stride) || !encode_bhld(&tm_k, p.k, p.B, p.H, p.L, p.k_stride) ||
       !encode_bhld(&tm_v, p.v, p.B, p.H, p.L, p.v_stride) || !encode_rows(&tm_mt, snapM16, (long long)BH * pl.S * 128))
     return INFINI_ERR_LAUNCH;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kAttnSmem);
-    cudaFuncSetAttribute(tc::mem_update_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)tc::UpdSmem<false>::BYTES);
-    cudaFuncSetAttribute(tc::mem_update_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)tc::UpdSmem<true>::BYTES);
-  });
+  {
+    // The dynamic shared-memory limit is an attribute of the function on the
+    // current device: set it once for every device the process uses.
+    static std::mutex mu;
+    static std::vector<char> done;
+    int cur = 0;
+    if (cudaGetDevice(&cur) != cudaSuccess) return INFINI_ERR_DEVICE;
+    std::lock_guard<std::mutex> lk(mu);
+    if ((int)done.size() <= cur) done.resize(cur + 1, 0);
+    if (!done[cur]) {
+      if (cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)tc::kAttnSmem) != cudaSuccess ||
+          cudaFuncSetAttribute(tc::mem_update_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)tc::UpdSmem<false>::BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(tc::mem_update_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)tc::UpdSmem<true>::BYTES) != cudaSuccess)
+        return INFINI_ERR_LAUNCH;
+      done[cur] = 1;
+    }
+  }
   const dim3 sgrid((E + 128 + 255) / 256, BH);
   tc::UpdArgs ua;
   ua.partial = part; ua.M = p.M; ua.z = p.z; ua.snapM = snapM16; ua.snapzw = snapz;
