@@ -29,7 +29,7 @@ from . import LINEAR, DELTA
 def read_trace() -> np.ndarray:
     fn = getattr(api.lib, "infini_attn_debug_trace", None)
     if fn is None:
-        raise SystemExit("this build records no trace: rebuild with INFINI_NVCC_FLAGS=-DINFINI_ATTN_TRACE=<cta>")
+        raise SystemExit("the library was built without a trace: rebuild it with INFINI_NVCC_FLAGS=-DINFINI_ATTN_TRACE=<cta>")
     fn.argtypes = [ctypes.c_void_p, ctypes.c_int]
     buf = (ctypes.c_ulonglong * 4096)()
     if fn(buf, 4096) != 0:
