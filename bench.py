@@ -7,8 +7,10 @@ A step is one pass of the whole forward (segment chunking, memory update,
 local attention, memory read, gate) over one batch of the workload with the
 inputs resident in HBM: one ``infini_attn_forward`` call, or for the
 streaming workload one ``infini_attn_segment_step`` call per segment.  The
-default workload is the 1B-shaped layer (B=1, H=8, d=128, N=2048,
-L=32768, bf16, linear rule).  Under torchrun each rank runs its own copy of
+default workload is the 8B-shaped long input (B=2, H=32, d=128, N=8192,
+L=524288, bf16); both update rules are timed on the same inputs, the linear
+rule gives the headline figures and the delta rule's are under ``modes``.
+``--workload`` / ``--mode`` select another workload or a single rule.  Under torchrun each rank runs its own copy of
 the workload on its own GPU (independent (batch, head) problems, no
 collective on the data path): weak scaling, value = tokens of all ranks /
 max over ranks of the step time.
@@ -246,7 +248,8 @@ def cpu_baseline(w: W.Workload, mode: int, budget_s: float):
 
 
 # ------------------------------------------------------------------ our arm
-def run_ours(args, w: W.Workload, mode: int):
+def run_ours(args, w: W.Workload, modes):
+    """Times every rule in ``modes`` on the same inputs; the first one is the headline line."""
     from compressive_memory_transformer_sm_b200 import api
 
     rank, world = init_dist("nccl")
@@ -269,7 +272,7 @@ def run_ours(args, w: W.Workload, mode: int):
         M.zero_()
         z.zero_()
 
-    def step():
+    def step(mode):
         if w.streaming:
             for s in range(w.segments):
                 api.infini_attn_segment_step(q[s], k[s], v[s], beta, M, z, out[s], mode, stream=stream)
@@ -278,105 +281,119 @@ def run_ours(args, w: W.Workload, mode: int):
         else:
             api.infini_attn_forward(q, k, v, beta, M, z, out, w.N, mode, stream=stream)
 
+    peaks, peak_src = load_peaks()
     sampler = ClockSampler(local)
-    for _ in range(args.warmup):
-        reset_state()
-        flush.fill_(1)
-        step()
-    torch.cuda.synchronize(dev)
-    api.infini_attn_profile_read(reset=True)
+    per_mode = {}
+    for mode in modes:
+        for _ in range(args.warmup):
+            reset_state()
+            flush.fill_(1)
+            step(mode)
+        torch.cuda.synchronize(dev)
+        api.infini_attn_profile_read(reset=True)
 
-    # ---------------------------------------------------------------- timed region
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    api.infini_attn_profile_enable(1 << api.PHASE_ATTN)
-    barrier(dev)
-    torch.cuda.synchronize(dev)
-    launches0 = api.infini_attn_launch_count()
-    # Hold the stream for a few ms so that the host queues the timed steps
-    # ahead of the device: the events then time device work back to back, not
-    # host launch jitter (the e2e measurement below includes the host).
-    if hasattr(torch.cuda, "_sleep"):
-        torch.cuda._sleep(int(2e6 + 1e6 * args.steps))  # ~0.5 ms per step: room for host hiccups
-    gc_was_enabled = gc.isenabled()
-    gc.disable()
-    wall0 = time.perf_counter()
-    for i in range(args.steps):
-        reset_state()
-        flush.fill_(i & 0xff)
-        evs[i][0].record(stream)
-        step()
-        evs[i][1].record(stream)
-    torch.cuda.synchronize(dev)
-    barrier(dev)
-    wall = time.perf_counter() - wall0
-    if gc_was_enabled:
-        gc.enable()
-    launches = api.infini_attn_launch_count() - launches0
-    api.infini_attn_profile_enable(0)
+        # ------------------------------------------------------------ timed region
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        api.infini_attn_profile_enable(1 << api.PHASE_ATTN)
+        barrier(dev)
+        torch.cuda.synchronize(dev)
+        launches0 = api.infini_attn_launch_count()
+        # Hold the stream for a few ms so that the host queues the timed steps
+        # ahead of the device: the events then time device work back to back, not
+        # host launch jitter (the e2e measurement below includes the host).
+        if hasattr(torch.cuda, "_sleep"):
+            torch.cuda._sleep(int(2e6 + 1e6 * args.steps))  # ~0.5 ms per step: room for host hiccups
+        gc_was_enabled = gc.isenabled()
+        gc.disable()
+        wall0 = time.perf_counter()
+        for i in range(args.steps):
+            reset_state()
+            flush.fill_(i & 0xff)
+            evs[i][0].record(stream)
+            step(mode)
+            evs[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(dev)
+        wall = time.perf_counter() - wall0
+        if gc_was_enabled:
+            gc.enable()
+        launches = api.infini_attn_launch_count() - launches0
+        api.infini_attn_profile_enable(0)
+        if api.infini_attn_device_status() != api.INFINI_OK:
+            raise RuntimeError("a device-side wait timed out during the benchmark")
+        step_ms = [a.elapsed_time(b) for a, b in evs]
+        ms_local = sum(step_ms) / len(step_ms)
+        attn_ms, attn_n = api.infini_attn_profile_read(reset=True)
+        attn_ms_per_launch_local = attn_ms[api.PHASE_ATTN] / max(1, attn_n[api.PHASE_ATTN])
+
+        # per-phase breakdown: a second pass of K steps with every launch bracketed
+        api.infini_attn_profile_enable(7)
+        for i in range(args.steps):
+            reset_state()
+            flush.fill_(i & 0xff)
+            step(mode)
+        torch.cuda.synchronize(dev)
+        api.infini_attn_profile_enable(0)
+        phase_ms, phase_n = api.infini_attn_profile_read(reset=True)
+
+        ms = max_over_ranks(ms_local, dev)
+        attn_ms_per_launch = max_over_ranks(attn_ms_per_launch_local, dev)
+        f_attn, f_upd = algorithmic_flops(w, mode)
+        per_launch_attn_flops = f_attn / (w.segments if w.streaming else 1)
+        achieved = per_launch_attn_flops / (attn_ms_per_launch * 1e-3) / 1e12
+        sustained = attn_ms_per_launch > 10.0
+        peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+        per_mode[mode] = {
+            "ms_per_step": ms, "value": w.B * w.L * world / (ms * 1e-3),
+            "step_ms_min_max": [min(step_ms), max(step_ms)],
+            "tflops": (f_attn + f_upd) * world / (ms * 1e-3) / 1e12,
+            "pct_of_bf16_peak": 100.0 * (f_attn + f_upd) / (ms * 1e-3) / 1e12 / peak,
+            "hbm_gbs": algorithmic_bytes(w) * world / (ms * 1e-3) / 1e9,
+            "roofline": {"kernel": "attn_tc_kernel" if not args.force_simt else "simt_attn_kernel",
+                         "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak,
+                         "traffic": measured_traffic(w.name, W.MODE_NAMES[mode]),
+                         "peak_source": f"{peak_src} {'bf16_tflops_sustained' if sustained else 'bf16_tflops'}",
+                         "launch_ms": attn_ms_per_launch, "flops_per_launch": per_launch_attn_flops},
+            "phases_ms_per_step": {name: phase_ms[i] / args.steps
+                                   for i, name in enumerate(("update", "state", "attention"))},
+            "phase_launches_per_step": {name: phase_n[i] / args.steps
+                                        for i, name in enumerate(("update", "state", "attention"))},
+            "gpu_launches": int(launches), "wall_s_timed_region": wall,
+        }
     clocks = sampler.stop() if sampler else None
-    if api.infini_attn_device_status() != api.INFINI_OK:
-        raise RuntimeError("a device-side wait timed out during the benchmark")
-    step_ms = [a.elapsed_time(b) for a, b in evs]
-    ms_local = sum(step_ms) / len(step_ms)
-    attn_ms, attn_n = api.infini_attn_profile_read(reset=True)
-    attn_ms_per_launch_local = attn_ms[api.PHASE_ATTN] / max(1, attn_n[api.PHASE_ATTN])
-
-    # per-phase breakdown: a second pass of K steps with every launch bracketed
-    api.infini_attn_profile_enable(7)
-    for i in range(args.steps):
-        reset_state()
-        flush.fill_(i & 0xff)
-        step()
-    torch.cuda.synchronize(dev)
-    api.infini_attn_profile_enable(0)
-    phase_ms, phase_n = api.infini_attn_profile_read(reset=True)
-
-    ms = max_over_ranks(ms_local, dev)
-    attn_ms_per_launch = max_over_ranks(attn_ms_per_launch_local, dev)
+    head = per_mode[modes[0]]
+    del q, k, v, out, flush
+    torch.cuda.empty_cache()
 
     # ---------------------------------------------------------------- end to end, host buffers
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, w, mode, dev, stream, rank)
+        e2e = run_e2e(args, w, modes[0], dev, stream, rank)
 
-    tokens = w.B * w.L * world
-    f_attn, f_upd = algorithmic_flops(w, mode)
-    peaks, peak_src = load_peaks()
-    per_launch_attn_flops = f_attn / (w.segments if w.streaming else 1)
-    achieved = per_launch_attn_flops / (attn_ms_per_launch * 1e-3) / 1e12
-    sustained = attn_ms_per_launch > 10.0
-    peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
-    traffic = measured_traffic(w.name, W.MODE_NAMES[mode])
     result = {
-        "metric": METRIC, "value": tokens / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-        "step_ms_min_max": [min(step_ms), max(step_ms)],
+        "metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+        "step_ms_min_max": head["step_ms_min_max"],
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32",
         "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "N": w.N, "dk": w.dk, "dv": w.dv,
-                   "mode": W.MODE_NAMES[mode], "path": "simt" if args.force_simt else "tensor",
+                   "mode": W.MODE_NAMES[modes[0]], "modes_timed": [W.MODE_NAMES[m] for m in modes],
+                   "path": "simt" if args.force_simt else "tensor",
                    "streaming_steps": w.segments if w.streaming else 0,
                    "l2": "1 GiB buffer written between timed steps (outside the step events)",
                    "parallelism": f"independent problem per rank x{world}"},
-        "tflops": (f_attn + f_upd) * world / (ms * 1e-3) / 1e12,
-        "pct_of_bf16_peak": 100.0 * (f_attn + f_upd) / (ms * 1e-3) / 1e12 / peak,
-        "hbm_gbs": algorithmic_bytes(w) * world / (ms * 1e-3) / 1e9,
-        "roofline": {"kernel": "attn_tc_kernel" if not args.force_simt else "simt_attn_kernel", "bound": "tensor",
-                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                     "traffic": traffic,
-                     "peak_source": f"{peak_src} {'bf16_tflops_sustained' if sustained else 'bf16_tflops'}",
-                     "launch_ms": attn_ms_per_launch, "flops_per_launch": per_launch_attn_flops},
-        "phases_ms_per_step": {name: phase_ms[i] / args.steps for i, name in enumerate(("update", "state",
-                                                                                          "attention"))},
-        "phase_launches_per_step": {name: phase_n[i] / args.steps for i, name in enumerate(("update", "state",
-                                                                                              "attention"))},
-        "gpu_launches": int(launches),
-        "clocks": clocks, "wall_s_timed_region": wall,
+        "tflops": head["tflops"], "pct_of_bf16_peak": head["pct_of_bf16_peak"], "hbm_gbs": head["hbm_gbs"],
+        "roofline": head["roofline"], "phases_ms_per_step": head["phases_ms_per_step"],
+        "phase_launches_per_step": head["phase_launches_per_step"],
+        "gpu_launches": head["gpu_launches"], "clocks": clocks, "wall_s_timed_region": head["wall_s_timed_region"],
+        "modes": {W.MODE_NAMES[m]: r for m, r in per_mode.items()},
     }
     if e2e is not None:
         result["e2e"] = e2e
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(w, mode, args.cpu_budget)
+        result["cpu_baseline"] = cpu_baseline(w, modes[0], args.cpu_budget)
     if rank == 0:
         print(json.dumps(result), flush=True)
     import torch.distributed as dist
@@ -390,15 +407,17 @@ def run_e2e(args, w: W.Workload, mode: int, dev, stream, rank):
     the forward, D2H of the output and the state, all inside each step's events."""
     from compressive_memory_transformer_sm_b200 import api
 
-    q, k, v, beta = W.make_inputs(w, device=dev, seed=rank_seed(w, rank))
-    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
-    hb = beta.cpu().pin_memory()
-    del q, k, v
+    dq, dk_, dv_, db = W.make_inputs(w, device=dev, seed=rank_seed(w, rank))
+    try:
+        hq, hk, hv = (torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (dq, dk_, dv_))
+        ho = torch.empty(w.B, w.H, w.L, w.dv, dtype=w.dtype, pin_memory=True)
+    except RuntimeError as e:  # not enough pinnable host memory for this workload
+        return {"value": None, "unit": "tokens/s", "unavailable": f"pinned host buffers: {str(e).splitlines()[0]}"}
+    for h, d in ((hq, dq), (hk, dk_), (hv, dv_)):
+        h.copy_(d)
+    hb = db.cpu().pin_memory()
     hM = torch.zeros(w.B, w.H, w.dk, w.dv).pin_memory()
     hz = torch.zeros(w.B, w.H, w.dk).pin_memory()
-    ho = torch.empty(w.B, w.H, w.L, w.dv, dtype=w.dtype).pin_memory()
-    dq, dk_, dv_ = (torch.empty(t.shape, dtype=t.dtype, device=dev) for t in (hq, hk, hv))
-    db = torch.empty(w.H, device=dev)
     dM = torch.empty(hM.shape, device=dev)
     dz = torch.empty(hz.shape, device=dev)
     do = torch.empty(ho.shape, dtype=w.dtype, device=dev)
@@ -420,11 +439,11 @@ def run_e2e(args, w: W.Workload, mode: int, dev, stream, rank):
         for h, d in ((ho, do), (hM, dM), (hz, dz)):
             h.copy_(d, non_blocking=True)
 
-    for _ in range(max(1, min(args.warmup, 3))):
+    for _ in range(max(1, min(args.warmup, args.e2e_steps))):
         flush.fill_(1)
         step()
     torch.cuda.synchronize(dev)
-    n = max(1, min(args.steps, 10))
+    n = max(1, min(args.steps, args.e2e_steps))
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
     barrier(dev)
     for i in range(n):
@@ -437,7 +456,7 @@ def run_e2e(args, w: W.Workload, mode: int, dev, stream, rank):
     ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / n, dev)
     world = int(os.environ.get("WORLD_SIZE", 1))
     return {"value": w.B * w.L * world / (ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": n,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": n, "mode": W.MODE_NAMES[mode],
             "path": "pinned host -> device, forward, device -> pinned host, per step"}
 
 
@@ -618,7 +637,7 @@ def parse(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", choices=sorted(W.WORKLOADS), default=W.LAYER_1B.name)
+    ap.add_argument("--workload", choices=sorted(W.WORKLOADS), default=W.LONG_8B.name)
     ap.add_argument("--mode", choices=("linear", "delta"), default=None)
     ap.add_argument("--force-simt", action="store_true", help="time the CUDA-core kernels instead")
     ap.add_argument("--shape", default=None, help="B,H,L,N override of the workload's sizes (for profiling)")
@@ -627,6 +646,7 @@ def parse(argv=None):
     ap.add_argument("--decode", action="store_true",
                     help="time token-level streaming decode (one segment of single-token calls per step)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=3, help="timed steps of the host-buffer measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--ref-step-budget", type=float, default=5.0)
@@ -639,7 +659,8 @@ def main(argv=None):
     if args.shape:
         B, H, L, N = (int(x) for x in args.shape.split(","))
         w = w.with_(name=f"{w.name}@{B}x{H}x{L}x{N}", B=B, H=H, L=L, N=N)
-    mode = {"linear": LINEAR, "delta": DELTA}[args.mode] if args.mode else w.modes[0]
+    modes = ({"linear": LINEAR, "delta": DELTA}[args.mode],) if args.mode else tuple(w.modes)
+    mode = modes[0]
     if args.warmup < 3 and args.impl == "ours":
         raise SystemExit("--warmup must be at least 3")
     if args.impl == "reference":
@@ -649,7 +670,7 @@ def main(argv=None):
     elif args.decode:
         run_decode(args, w, mode)
     else:
-        run_ours(args, w, mode)
+        run_ours(args, w, modes)
 
 
 if __name__ == "__main__":

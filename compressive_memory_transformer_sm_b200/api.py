@@ -35,7 +35,7 @@ EXPORTED = (
     "infini_attn_forward", "infini_attn_segment_step", "infini_attn_forward_ex", "infini_attn_workspace_size",
     "infini_attn_error_string", "infini_attn_device_status", "infini_attn_selftest_timeout",
     "infini_attn_params_size", "infini_attn_path", "infini_attn_profile_enable", "infini_attn_profile_read",
-    "infini_attn_launch_count", "infini_attn_forward_noalloc", "infini_attn_selftest_exp2",
+    "infini_attn_launch_count", "infini_attn_forward_noalloc",
     "infini_attn_layer_forward", "infini_attn_layer_workspace_size", "infini_attn_decode_step",
 )
 
@@ -65,8 +65,6 @@ lib.infini_attn_selftest_timeout.argtypes = [ctypes.c_uint, _vp]
 lib.infini_attn_selftest_timeout.restype = _i
 lib.infini_attn_params_size.argtypes = []
 lib.infini_attn_params_size.restype = ctypes.c_size_t
-lib.infini_attn_selftest_exp2.argtypes = [_vp, _vp, _i, _vp]
-lib.infini_attn_selftest_exp2.restype = _i
 lib.infini_attn_path.argtypes = [_i, _i, _i, _i]
 lib.infini_attn_path.restype = _i
 lib.infini_attn_profile_enable.argtypes = [_i]
@@ -277,11 +275,6 @@ def infini_attn_device_status(reset: bool = False) -> int:
 
 def infini_attn_selftest_timeout(limit_us: int, stream=None) -> int:
     return int(lib.infini_attn_selftest_timeout(int(limit_us), _stream(stream)))
-
-
-def infini_attn_selftest_exp2(x, y, stream=None) -> int:
-    """y = 2^x with the attention kernel's polynomial exponential (float32 device tensors)."""
-    return int(lib.infini_attn_selftest_exp2(x.data_ptr(), y.data_ptr(), x.numel(), _stream(stream)))
 
 
 def infini_attn_path(dk: int, dv: int, mode: int, flags: int = 0) -> int:

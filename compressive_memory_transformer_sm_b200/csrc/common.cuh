@@ -40,22 +40,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// 2^x on the FMA and ALU pipes, to offload the exponential unit: x = n + f
-// with n the nearest integer (rounding by adding 1.5 * 2^23) and f in
-// [-1/2, 1/2] (Cody-Waite style range reduction); 2^f by the cubic that
-// minimises the maximum relative error on that interval (coefficients from
-// csrc/fit_exp2_poly.py: max relative error 7.5e-5); n is added to the
-// exponent field.  For x in [-125, 125]; smaller x (and -inf) give ~2^-125.
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -125.f);
-  const float t = x + 12582912.f;  // low mantissa bits of t hold round(x)
-  const float n = t - 12582912.f;
-  const float f = x - n;
-  const float p =
-      fmaf(fmaf(fmaf(5.517221987e-02f, f, 2.426111549e-01f), f, 6.932608485e-01f), f, 9.999280572e-01f);
-  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
-}
-
 // Packed fp32 pairs (sm_100): d = a * b + c and d = a + b on two lanes at once.
 __device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0, float c1) {
   asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
@@ -70,12 +54,6 @@ __device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1, f
       "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
       : "=f"(d0), "=f"(d1)
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
-}
-
-// Two finite non-negative floats to packed bf16 on the integer pipe (round
-// half up): add half an ulp of bf16, keep the upper halves.
-__device__ __forceinline__ uint32_t pack_bf16x2_alu(float lo, float hi) {
-  return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -4,9 +4,12 @@
 //   linear rule (Eq. 8): update partials for every (b, h, segment, group) in
 //     one launch, then one state launch that scans the segments in order,
 //     writing the snapshots (M_{s-1}, z_{s-1}) and the final (M_S, z_S);
-//   delta rule (Eq. 9): a snapshot of (M_0, z_0), then per segment one
-//     update launch (reads M_{s-1}) and one state launch (adds the partials
-//     and snapshots M_s);
+//   delta rule (Eq. 9), tensor cores: one update launch per segment, which
+//     snapshots (M_{s-1}, z_{s-1}), computes the segment's partials and
+//     reduces them into M, z inside each head's thread-block cluster;
+//   delta rule, CUDA cores: a snapshot launch of (M_0, z_0), then per segment
+//     one update launch (reads M_{s-1}) and one state launch (adds the
+//     partials and snapshots M_s);
 //   then one attention launch (Eq. 6, 7, 10) over every (b, h, segment,
 //     query tile), reading the snapshots.
 // The order "read with M_{s-1}, then update" of the pages holds because the
@@ -19,6 +22,7 @@
 #include <algorithm>
 #include <atomic>
 #include <mutex>
+#include <utility>
 #include <vector>
 
 #include "../../include/infini_attn.h"
@@ -145,6 +149,33 @@ EncodeTiledFn get_encode() {
   return fn;
 }
 
+// Unique id of the CUDA context current on this thread (0 if none or on
+// failure).  Per-context caches key on it rather than on the device ordinal:
+// a context that is destroyed and recreated (cudaDeviceReset, a primary
+// context reset) gets a new id, so nothing cached for the old one is reused.
+unsigned long long current_context_id() {
+  typedef CUresult (*GetCurrentFn)(CUcontext*);
+  typedef CUresult (*GetIdFn)(CUcontext, unsigned long long*);
+  static GetCurrentFn get_current = nullptr;
+  static GetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrentFn>(f);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetIdFn>(f);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
 // 4-D map over a [B, H, L, 128] bf16 tensor with element strides st[0..2]
 // (d contiguous); box 64 x 128 tokens, 128-byte swizzle.
 bool encode_bhld(CUtensorMap* m, const void* ptr, int B, int H, long long L, const long long st[3]) {
@@ -254,15 +285,14 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale) {
       !encode_bhld(&tm_v, p.v, p.B, p.H, p.L, p.v_stride) || !encode_rows(&tm_mt, snapM16, (long long)BH * pl.S * 128))
     return INFINI_ERR_LAUNCH;
   {
-    // The dynamic shared-memory limit is an attribute of the function on the
-    // current device: set it once for every device the process uses.
+    // The dynamic shared-memory limit is an attribute of the function in the
+    // current context: set it once for every context the process uses (an
+    // unknown context id, 0, sets it on every call).
     static std::mutex mu;
-    static std::vector<char> done;
-    int cur = 0;
-    if (cudaGetDevice(&cur) != cudaSuccess) return INFINI_ERR_DEVICE;
+    static std::vector<unsigned long long> done;
+    const unsigned long long ctx = current_context_id();
     std::lock_guard<std::mutex> lk(mu);
-    if ((int)done.size() <= cur) done.resize(cur + 1, 0);
-    if (!done[cur]) {
+    if (ctx == 0 || std::find(done.begin(), done.end(), ctx) == done.end()) {
       if (cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)tc::kAttnSmem) != cudaSuccess ||
           cudaFuncSetAttribute(tc::mem_update_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -270,7 +300,7 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale) {
           cudaFuncSetAttribute(tc::mem_update_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)tc::UpdSmem<true>::BYTES) != cudaSuccess)
         return INFINI_ERR_LAUNCH;
-      done[cur] = 1;
+      if (ctx != 0) done.push_back(ctx);
     }
   }
   const dim3 sgrid((E + 128 + 255) / 256, BH);
@@ -419,11 +449,6 @@ int forward_impl(infini_attn_params p) {
   return rc;
 }
 
-__global__ void selftest_exp2_kernel(const float* x, float* y, int n) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) y[i] = exp2_poly(x[i]);
-}
-
 __global__ void selftest_wait_kernel(unsigned long long limit_ns) {
   __shared__ __align__(8) unsigned long long bar;
   const uint32_t b = smem_u32(&bar);
@@ -439,27 +464,30 @@ __global__ void selftest_wait_kernel(unsigned long long limit_ns) {
 constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-// Device address of the buffer on the current device.  The symbol's name is
+// Device address of the buffer in the current context.  The symbol's name is
 // only a host-side handle; the address comes from cudaGetSymbolAddress, once
-// per device, with that device current.
+// per context (so once per device while its context lives), with that
+// device current.  Keyed by context id: after a device reset the address is
+// looked up again instead of reusing one from the destroyed context.
 int noalloc_scratch(void** out) {
   static std::mutex mu;
-  static void* addr[256] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) {
-    cudaGetLastError();
-    return INFINI_ERR_DEVICE;
-  }
+  static std::vector<std::pair<unsigned long long, void*>> addr;
   std::lock_guard<std::mutex> lk(mu);
-  if (!addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
-      cudaGetLastError();
-      return INFINI_ERR_LAUNCH;
+  unsigned long long ctx = current_context_id();
+  for (const auto& e : addr)
+    if (ctx != 0 && e.first == ctx) {
+      *out = e.second;
+      return INFINI_OK;
     }
-    addr[dev] = p;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+    cudaGetLastError();
+    return INFINI_ERR_LAUNCH;
   }
-  *out = addr[dev];
+  // the lookup made the device's primary context current if none was
+  ctx = current_context_id();
+  if (ctx != 0) addr.emplace_back(ctx, p);
+  *out = p;
   return INFINI_OK;
 }
 
@@ -759,15 +787,6 @@ int infini_attn_selftest_timeout(unsigned limit_us, cudaStream_t stream) {
   if (cudaGetLastError() != cudaSuccess) return INFINI_ERR_LAUNCH;
   if (cudaStreamSynchronize(stream) != cudaSuccess) return INFINI_ERR_LAUNCH;
   return infini_attn_device_status(0);
-}
-
-int infini_attn_selftest_exp2(const float* x, float* y, int n, cudaStream_t stream) {
-  if (!x || !y || n < 0) return INFINI_ERR_INVALID_ARG;
-  if (n == 0) return INFINI_OK;
-  int rc = check_device(false);
-  if (rc != INFINI_OK) return rc;
-  selftest_exp2_kernel<<<(n + 255) / 256, 256, 0, stream>>>(x, y, n);
-  return launch_status();
 }
 
 int infini_attn_path(int dk, int dv, int mode, int flags) {

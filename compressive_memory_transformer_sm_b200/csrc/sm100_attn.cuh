@@ -5,20 +5,6 @@
 
 #include "sm100_common.cuh"
 
-// Softmax tuning knobs (compile time): every INFINI_POLY_EVERY-th pair of
-// exponentials runs on the FMA pipe (0 = none), and P is packed to bf16 on the
-// integer pipe when INFINI_PACK_ALU is 1.
-#ifndef INFINI_POLY_EVERY
-#define INFINI_POLY_EVERY 0
-#endif
-#ifndef INFINI_PACK_ALU
-#define INFINI_PACK_ALU 0
-#endif
-// 1: scale-and-subtract and the row sum use packed fp32x2 instructions.
-#ifndef INFINI_F32X2
-#define INFINI_F32X2 1
-#endif
-
 namespace infini {
 namespace tc {
 
@@ -526,31 +512,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int e = 0; e < 64; ++e) {
+          // scale-and-subtract and the row sum in packed fp32x2 instructions
           float a0, a1;
-          if (INFINI_F32X2) {
-            fma2(a0, a1, __uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1]), c, c, nm, nm);
+          fma2(a0, a1, __uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1]), c, c, nm, nm);
+          const float p0 = ex2_approx(a0), p1 = ex2_approx(a1);
+          if ((e & 1) == 0) {
+            add2(ls[0], ls[1], ls[0], ls[1], p0, p1);
           } else {
-            a0 = fmaf(__uint_as_float(x[2 * e]), c, nm);
-            a1 = fmaf(__uint_as_float(x[2 * e + 1]), c, nm);
+            add2(ls[2], ls[3], ls[2], ls[3], p0, p1);
           }
-          float p0, p1;
-          if (INFINI_POLY_EVERY > 0 && (e % (INFINI_POLY_EVERY > 0 ? INFINI_POLY_EVERY : 1)) == INFINI_POLY_EVERY - 1) {
-            p0 = exp2_poly(a0);
-            p1 = exp2_poly(a1);
-          } else {
-            p0 = ex2_approx(a0);
-            p1 = ex2_approx(a1);
-          }
-          if (INFINI_F32X2) {
-            if ((e & 1) == 0) {
-              add2(ls[0], ls[1], ls[0], ls[1], p0, p1);
-            } else {
-              add2(ls[2], ls[3], ls[2], ls[3], p0, p1);
-            }
-          } else {
-            ls[e & 3] += p0 + p1;
-          }
-          x[e] = INFINI_PACK_ALU ? pack_bf16x2_alu(p0, p1) : pack_bf16x2(p0, p1);
+          x[e] = pack_bf16x2(p0, p1);
           if (e == 31) {  // keys 0-63 done: their P goes to TMEM while the rest is computed
             uint32_t (&ph)[32] = *reinterpret_cast<uint32_t(*)[32]>(&x[0]);
             tmem_st32(tS, ph);

@@ -125,8 +125,9 @@ INFINI_API int infini_attn_segment_step(const void* q, const void* k, const void
  *   - Shapes whose workspace (infini_attn_workspace_size) exceeds 32 MiB are
  *     rejected with INFINI_ERR_SCRATCH_LIMIT before anything is launched.
  *   - The first call on a device looks up that device's address of the
- *     buffer (with the device current); make that first call before any
- *     stream capture.  Nothing else is set up, and no call allocates.
+ *     buffer (with the device current), and so does the first call after the
+ *     device's context was reset; make that first call before any stream
+ *     capture.  Nothing else is set up, and no call allocates.
  *   - All calls on a device share the one buffer and it keeps the previous
  *     call's contents; nothing in it has to start at zero, since a call reads
  *     only what it wrote earlier in the same call.  Calls whose work overlaps
@@ -262,14 +263,6 @@ INFINI_API int infini_attn_profile_enable(int phase_mask);
 INFINI_API int infini_attn_profile_read(double* ms, long long* launches, int reset);
 /* Number of kernels this library has launched in this process (all phases). */
 INFINI_API long long infini_attn_launch_count(void);
-
-/*
- * Self-test of the polynomial 2^x used inside the attention kernel to take
- * part of the exponentials off the exponential unit: y[i] = 2^x[i] for n
- * device floats, asynchronously on `stream`.  Relative error <= 1e-4 for
- * x in [-125, 125]; smaller x give about 2^-125.
- */
-INFINI_API int infini_attn_selftest_exp2(const float* x, float* y, int n, cudaStream_t stream);
 
 /* sizeof(infini_attn_params), for bindings that build the struct themselves. */
 INFINI_API size_t infini_attn_params_size(void);

@@ -281,16 +281,54 @@ def test_workload_8b_long_both_rules():
         del out
 
 
-def test_polynomial_exp2_error_bound():
-    """The FMA-pipe 2^x used for part of the softmax stays within its fitted error bound."""
-    x = torch.cat([torch.linspace(-125.0, 125.0, 1_000_001), torch.tensor([-126.5, -300.0, -float("inf")])])
-    xd = x.to(DEV)
-    y = torch.empty_like(xd)
-    assert api.infini_attn_selftest_exp2(xd, y) == api.INFINI_OK
+# ----------------------------------------------------------------- memory read alone, full size
+def _check_amem_head(q, k, v, out, b, h, N, mode, segments, what):
+    """Gate forced to 1 (out = A_mem): relative L2 of sampled segments against the oracle's
+    sigma(Q) M_{s-1} / (sigma(Q) z_{s-1}), with M_{s-1}, z_{s-1} from the oracle's own trajectory."""
+    K, V, Q = np64(k[b, h]), np64(v[b, h]), np64(q[b, h])
+    states, _ = R.memory_trajectory(K, V, N, mode)
+    bounds = R.segment_bounds(K.shape[0], N)
+    got = np64(out[b, h])
+    worst = 0.0
+    for si in segments:
+        s0, s1 = bounds[si]
+        want = R.memory_retrieval(R.elu_plus_one(Q[s0:s1]), *states[si])
+        rl = rel_l2(got[s0:s1], want)
+        print(f"A_mem alone {what} (b={b}, h={h}) segment {si}: rel-L2 {rl:.3e} "
+              f"(tolerance 5e-3, margin {5e-3 / rl:.1f}x)")
+        assert np.all(np.isfinite(got[s0:s1]))
+        assert rl <= 5e-3, f"A_mem {what} segment {si}: rel-L2 {rl:.3e}"
+        worst = max(worst, rl)
+    return worst
+
+
+def test_memory_read_alone_full_size():
+    """A_mem at full size on every workload (both rules on the 8B shape): its magnitude,
+    about 1/sqrt(tokens), would hide under the output's absolute tolerance, so the gate is
+    forced to 1 and the relative tolerance applies to A_mem itself."""
+    cases = [(W.LONG_8B, LINEAR, [(W.LONG_8B.B - 1, W.LONG_8B.H - 1)], [1, 2, 63]),
+             (W.LONG_8B, DELTA, [(W.LONG_8B.B - 1, W.LONG_8B.H - 1)], [1, 2, 63]),
+             (W.BATCH_1B, DELTA, [(0, 0), (7, 7)], [1, 7, 15])]
+    for w, mode, heads, segs in cases:
+        q, k, v, _ = W.make_inputs(w, device=DEV)
+        beta = torch.full((w.H,), float("inf"), device=DEV)
+        out, _, _ = run(q, k, v, beta, w.N, mode)
+        for b, h in heads:
+            _check_amem_head(q, k, v, out, b, h, w.N, mode, segs, f"{w.name} mode={mode}")
+        del q, k, v, out
+        torch.cuda.empty_cache()
+    # the passkey stream, one segment_step call per segment
+    w = W.PASSKEY_1M
+    q, k, v, _ = W.make_inputs(w, device=DEV)
+    beta = torch.full((w.H,), float("inf"), device=DEV)
+    S = w.segments
+    seg = lambda t: t.view(w.B, w.H, S, w.N, t.shape[3]).permute(2, 0, 1, 3, 4).contiguous()  # noqa: E731
+    qs, ks, vs = seg(q), seg(k), seg(v)
+    M, z = W.empty_state(w, device=DEV)
+    outs = torch.empty_like(vs)
+    for s in range(S):
+        api.infini_attn_segment_step(qs[s], ks[s], vs[s], beta, M, z, outs[s], DELTA)
     torch.cuda.synchronize()
-    got = y.double().cpu().numpy()
-    want = np.exp2(x.double().numpy())
-    inner = slice(0, 1_000_001)
-    rel = np.abs(got[inner] / want[inner] - 1.0)
-    assert float(rel.max()) <= 1e-4, float(rel.max())
-    assert np.all(got[-3:] <= 2.0 ** -124) and np.all(got[-3:] >= 0.0)
+    assert api.infini_attn_device_status() == api.INFINI_OK
+    out = outs.permute(1, 2, 0, 3, 4).reshape(w.B, w.H, w.L, w.dv)
+    _check_amem_head(q, k, v, out, 0, 3, w.N, DELTA, [1, 255, S - 1], "passkey_1m_stream")

@@ -3,11 +3,13 @@
 The no-allocation variant serves callers that may not allocate device memory
 while they run (a serving loop that forbids allocation after start-up, a
 fixed memory budget).  It takes its workspace from the library's fixed
-32 MiB device buffer, so it must give the same results as the ordinary call,
-on consecutive calls that reuse the buffer, and refuse shapes that need more.
+32 MiB device buffer, so it must give exactly the results of the ordinary
+call -- the kernels and their order of summation are the same, only the
+workspace differs -- on consecutive calls that reuse the buffer, including
+calls that find it dirty from a larger shape, and refuse shapes that need
+more.
 """
 
-import numpy as np
 import pytest
 import torch
 
@@ -31,26 +33,25 @@ def _run(fn, q, k, v, beta, N, mode):
     fn(q, k, v, beta, M, z, out, N, mode)
     torch.cuda.synchronize()
     assert api.infini_attn_device_status() == api.INFINI_OK
-    return [t.double().cpu().numpy() for t in (out, M, z)]
+    return out, M, z
 
 
-def _close(a, b, what):
-    err = float(np.max(np.abs(a - b)))
-    rel = float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
-    assert np.all(np.isfinite(a)), what
-    assert err <= 2e-2 and rel <= 5e-3, f"{what}: max-abs {err:.3e} rel-L2 {rel:.3e}"
-
-
-def test_noalloc_matches_forward_on_two_calls_in_a_row():
+@pytest.mark.parametrize("mode", [DELTA, LINEAR])
+def test_noalloc_matches_forward_on_two_calls_in_a_row(mode):
     N = 256
-    for call, (seed, mode) in enumerate(((31, DELTA), (32, LINEAR))):
-        q, k, v, beta = _inputs(seed)
-        B, H, L, d = q.shape
-        assert api.infini_attn_workspace_size(B, H, L, N, d, d, mode) <= api.NOALLOC_SCRATCH_BYTES
+    # a larger call of the same rule first, so the checked calls find the
+    # shared buffer full of another shape's snapshots and partials
+    big = _inputs(30, H=8)
+    assert api.infini_attn_workspace_size(1, 8, 640, N, 128, 128, mode) <= api.NOALLOC_SCRATCH_BYTES
+    _run(api.infini_attn_forward_noalloc, *big, N, mode)
+    q, k, v, beta = _inputs(31 + mode)
+    B, H, L, d = q.shape
+    want = _run(api.infini_attn_forward, q, k, v, beta, N, mode)
+    for call in range(2):
         got = _run(api.infini_attn_forward_noalloc, q, k, v, beta, N, mode)
-        want = _run(api.infini_attn_forward, q, k, v, beta, N, mode)
         for g, w_, name in zip(got, want, ("out", "M", "z")):
-            _close(g, w_, f"call {call} {name}")
+            assert torch.isfinite(g).all(), f"call {call} {name}: non-finite"
+            assert torch.equal(g, w_), f"call {call} {name}: max-abs {(g.float() - w_.float()).abs().max().item():.3e}"
 
 
 def test_noalloc_refuses_shapes_beyond_its_scratch():
