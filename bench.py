@@ -52,6 +52,7 @@ from compressive_memory_transformer_sm_b200 import workloads as W  # noqa: E402
 METRIC = "Infini-attn fwd tokens/s per layer; TFLOP/s and % of B200 bf16 tensor peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FLUSH_BYTES = 1 << 30
+PHASE_NAMES = ("update", "state", "attention", "rope", "projections")
 
 
 # ------------------------------------------------------------------ work model
@@ -276,8 +277,9 @@ def run_ours(args, w: W.Workload, modes):
         if w.streaming:
             for s in range(w.segments):
                 api.infini_attn_segment_step(q[s], k[s], v[s], beta, M, z, out[s], mode, stream=stream)
-        elif flags:
-            api.infini_attn_forward_ex(q, k, v, beta, M, z, out, w.N, mode, flags=flags, stream=stream)
+        elif flags or args.rope:
+            api.infini_attn_forward_ex(q, k, v, beta, M, z, out, w.N, mode, flags=flags, stream=stream,
+                                       rope_base=args.rope)
         else:
             api.infini_attn_forward(q, k, v, beta, M, z, out, w.N, mode, stream=stream)
 
@@ -328,7 +330,7 @@ def run_ours(args, w: W.Workload, modes):
         attn_ms_per_launch_local = attn_ms[api.PHASE_ATTN] / max(1, attn_n[api.PHASE_ATTN])
 
         # per-phase breakdown: a second pass of K steps with every launch bracketed
-        api.infini_attn_profile_enable(7)
+        api.infini_attn_profile_enable((1 << api.PHASES) - 1)
         for i in range(args.steps):
             reset_state()
             flush.fill_(i & 0xff)
@@ -356,10 +358,8 @@ def run_ours(args, w: W.Workload, modes):
                          "traffic": measured_traffic(w.name, W.MODE_NAMES[mode]),
                          "peak_source": f"{peak_src} {'bf16_tflops_sustained' if sustained else 'bf16_tflops'}",
                          "launch_ms": attn_ms_per_launch, "flops_per_launch": per_launch_attn_flops},
-            "phases_ms_per_step": {name: phase_ms[i] / args.steps
-                                   for i, name in enumerate(("update", "state", "attention"))},
-            "phase_launches_per_step": {name: phase_n[i] / args.steps
-                                        for i, name in enumerate(("update", "state", "attention"))},
+            "phases_ms_per_step": {name: phase_ms[i] / args.steps for i, name in enumerate(PHASE_NAMES)},
+            "phase_launches_per_step": {name: phase_n[i] / args.steps for i, name in enumerate(PHASE_NAMES)},
             "gpu_launches": int(launches), "wall_s_timed_region": wall,
         }
     clocks = sampler.stop() if sampler else None
@@ -381,6 +381,7 @@ def run_ours(args, w: W.Workload, modes):
         "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "N": w.N, "dk": w.dk, "dv": w.dv,
                    "mode": W.MODE_NAMES[modes[0]], "modes_timed": [W.MODE_NAMES[m] for m in modes],
                    "path": "simt" if args.force_simt else "tensor",
+                   "rope_base": args.rope or None,
                    "streaming_steps": w.segments if w.streaming else 0,
                    "l2": "1 GiB buffer written between timed steps (outside the step events)",
                    "parallelism": f"independent problem per rank x{world}"},
@@ -512,8 +513,18 @@ def run_layer(args, w: W.Workload, mode: int):
         raise RuntimeError("a device-side wait timed out during the benchmark")
     step_ms = [a.elapsed_time(b) for a, b in evs]
     ms = max_over_ranks(sum(step_ms) / len(step_ms), dev)
+    # per-phase breakdown: a second pass with every launch bracketed
+    api.infini_attn_profile_read(reset=True)
+    api.infini_attn_profile_enable((1 << api.PHASES) - 1)
+    for _ in range(args.steps):
+        step()
+        api.infini_attn_layer_forward(x, w_qkv, w_o, beta, M, z, y, w.H, w.N, mode, workspace=ws, stream=stream)
+    torch.cuda.synchronize(dev)
+    api.infini_attn_profile_enable(0)
+    phase_ms, phase_n = api.infini_attn_profile_read(reset=True)
     f_attn, f_upd = algorithmic_flops(w, mode)
     f_proj = 2 * w.B * w.L * D * (3 * w.H * w.dk) + 2 * w.B * w.L * (w.H * w.dv) * D
+    proj_ms = phase_ms[api.PHASE_PROJ] / args.steps
     peaks, peak_src = load_peaks()
     peak = peaks["bf16_tflops_sustained"] if ms > 10.0 else peaks["bf16_tflops"]
     tflops = (f_attn + f_upd + f_proj) * world / (ms * 1e-3) / 1e12
@@ -528,6 +539,10 @@ def run_layer(args, w: W.Workload, mode: int):
         "tflops": tflops, "pct_of_bf16_peak": 100.0 * tflops / world / peak,
         "peak_source": f"{peak_src} {'bf16_tflops_sustained' if ms > 10.0 else 'bf16_tflops'}",
         "flops_per_step": {"projections": f_proj, "attention": f_attn, "update": f_upd},
+        "phases_ms_per_step": {name: phase_ms[i] / args.steps for i, name in enumerate(PHASE_NAMES)},
+        "projection_gemm": {"kernel": "gemm_tc_kernel", "ms_per_step": proj_ms, "launches_per_step":
+                            phase_n[api.PHASE_PROJ] / args.steps,
+                            "tflops": f_proj / (proj_ms * 1e-3) / 1e12 if proj_ms > 0 else None},
         "gpu_launches": int(launches), "clocks": clocks,
     }
     if rank == 0:
@@ -641,6 +656,8 @@ def parse(argv=None):
     ap.add_argument("--mode", choices=("linear", "delta"), default=None)
     ap.add_argument("--force-simt", action="store_true", help="time the CUDA-core kernels instead")
     ap.add_argument("--shape", default=None, help="B,H,L,N override of the workload's sizes (for profiling)")
+    ap.add_argument("--rope", type=float, default=0.0,
+                    help="rotary position embeddings with this base on the local attention (0: none)")
     ap.add_argument("--layer", action="store_true",
                     help="time the full layer (QKV projection + attention + output projection) instead")
     ap.add_argument("--decode", action="store_true",
@@ -661,6 +678,8 @@ def main(argv=None):
         w = w.with_(name=f"{w.name}@{B}x{H}x{L}x{N}", B=B, H=H, L=L, N=N)
     modes = ({"linear": LINEAR, "delta": DELTA}[args.mode],) if args.mode else tuple(w.modes)
     mode = modes[0]
+    if args.rope and (w.streaming or args.layer or args.decode):
+        raise SystemExit("--rope applies to the whole-sequence forward (infini_attn_forward_ex) only")
     if args.warmup < 3 and args.impl == "ours":
         raise SystemExit("--warmup must be at least 3")
     if args.impl == "reference":

@@ -37,6 +37,7 @@ EXPORTED = (
     "infini_attn_params_size", "infini_attn_path", "infini_attn_profile_enable", "infini_attn_profile_read",
     "infini_attn_launch_count", "infini_attn_forward_noalloc",
     "infini_attn_layer_forward", "infini_attn_layer_workspace_size", "infini_attn_decode_step",
+    "infini_attn_workspace_size_ex", "infini_attn_gemm_bf16",
 )
 
 
@@ -79,8 +80,11 @@ lib.infini_attn_layer_forward.argtypes = [_vp] * 7 + [_i, _i, _l, _i, _i, _i, _v
 lib.infini_attn_layer_forward.restype = _i
 lib.infini_attn_layer_workspace_size.argtypes = [_i, _i, _l, _i, _i, _i]
 lib.infini_attn_layer_workspace_size.restype = ctypes.c_size_t
+lib.infini_attn_gemm_bf16.argtypes = [_vp, _vp, _vp, _l, _i, _i, _vp]
+lib.infini_attn_gemm_bf16.restype = _i
 
-PHASE_UPDATE, PHASE_STATE, PHASE_ATTN = 0, 1, 2
+PHASE_UPDATE, PHASE_STATE, PHASE_ATTN, PHASE_PRE, PHASE_PROJ = 0, 1, 2, 3, 4
+PHASES = 5
 
 
 class InfiniAttnParams(ctypes.Structure):
@@ -92,11 +96,14 @@ class InfiniAttnParams(ctypes.Structure):
         ("scale", ctypes.c_float),
         ("q_stride", _ll * 3), ("k_stride", _ll * 3), ("v_stride", _ll * 3), ("o_stride", _ll * 3),
         ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t), ("flags", _i), ("stream", _vp),
+        ("rope_base", ctypes.c_double), ("rope_offset", _ll),
     ]
 
 
 lib.infini_attn_forward_ex.argtypes = [ctypes.POINTER(InfiniAttnParams)]
 lib.infini_attn_forward_ex.restype = _i
+lib.infini_attn_workspace_size_ex.argtypes = [ctypes.POINTER(InfiniAttnParams)]
+lib.infini_attn_workspace_size_ex.restype = ctypes.c_size_t
 
 
 class InfiniAttnError(RuntimeError):
@@ -230,6 +237,20 @@ def infini_attn_layer_forward(x, w_qkv, w_o, beta, M, z, y, H: int, N: int, mode
     return _check(rc, "infini_attn_layer_forward", raise_on_error)
 
 
+def infini_attn_gemm_bf16(a, b, c, stream=None, raise_on_error=True):
+    """c[M, N] = a[M, K] @ b[K, N]: contiguous bf16 device matrices, fp32 accumulation (the layer's projection)."""
+    _args("infini_attn_gemm_bf16", dict(a=(a, 2), b=(b, 2), c=(c, 2)))
+    M, K = a.shape
+    N = b.shape[1]
+    if b.shape[0] != K or tuple(c.shape) != (M, N):
+        raise ValueError(f"infini_attn_gemm_bf16: shapes {tuple(a.shape)} @ {tuple(b.shape)} -> {tuple(c.shape)}")
+    for name, t in (("a", a), ("b", b), ("c", c)):
+        if t.dtype != torch.bfloat16:
+            raise ValueError(f"infini_attn_gemm_bf16: {name} must be bfloat16")
+    rc = lib.infini_attn_gemm_bf16(a.data_ptr(), b.data_ptr(), c.data_ptr(), M, N, K, _stream(stream))
+    return _check(rc, "infini_attn_gemm_bf16", raise_on_error)
+
+
 def infini_attn_layer_workspace_size(B, H, L, N, d_model, mode=LINEAR) -> int:
     return int(lib.infini_attn_layer_workspace_size(B, H, L, N, d_model, mode))
 
@@ -242,8 +263,11 @@ def _bhl_strides(t: torch.Tensor):
 
 
 def infini_attn_forward_ex(q, k, v, beta, M, z, out, N: int, mode: int = LINEAR, scale: float = 0.0,
-                           workspace=None, flags: int = 0, stream=None, raise_on_error=True):
-    """Extended call: [B,H,L,d] views with any (B, H, L) strides, explicit scale, caller workspace, flags."""
+                           workspace=None, flags: int = 0, stream=None, raise_on_error=True, rope_base: float = 0.0,
+                           rope_offset: int = 0):
+    """Extended call: [B,H,L,d] views with any (B, H, L) strides, explicit scale, caller workspace, flags, and
+    rotary position embeddings on the local attention only (``rope_base`` > 0, token t at position
+    ``rope_offset + t``)."""
     _args("infini_attn_forward_ex", dict(q=(q, 4), k=(k, 4), v=(v, 4), out=(out, 4)), contiguous=False)
     _args("infini_attn_forward_ex", dict(beta=(beta, 1), M=(M, 4), z=(z, 3)))
     B, H, L, dk = q.shape
@@ -261,12 +285,22 @@ def infini_attn_forward_ex(q, k, v, beta, M, z, out, N: int, mode: int = LINEAR,
         p.workspace_bytes = workspace.numel() * workspace.element_size()
     p.flags = int(flags)
     p.stream = _stream(stream)
+    p.rope_base = float(rope_base)
+    p.rope_offset = int(rope_offset)
     rc = lib.infini_attn_forward_ex(ctypes.byref(p))
     return _check(rc, "infini_attn_forward_ex", raise_on_error)
 
 
 def infini_attn_workspace_size(B, H, L, N, dk, dv, mode=LINEAR) -> int:
     return int(lib.infini_attn_workspace_size(B, H, L, N, dk, dv, mode))
+
+
+def infini_attn_workspace_size_ex(B, H, L, N, dk, dv, mode=LINEAR, rope_base: float = 0.0) -> int:
+    """Workspace of infini_attn_forward_ex for this shape, including the rotated q, k when rope_base > 0."""
+    p = InfiniAttnParams()
+    p.B, p.H, p.L, p.N, p.dk, p.dv, p.mode = int(B), int(H), int(L), int(N), int(dk), int(dv), int(mode)
+    p.rope_base = float(rope_base)
+    return int(lib.infini_attn_workspace_size_ex(ctypes.byref(p)))
 
 
 def infini_attn_device_status(reset: bool = False) -> int:
@@ -286,9 +320,10 @@ def infini_attn_profile_enable(phase_mask: int) -> int:
 
 
 def infini_attn_profile_read(reset: bool = True):
-    """Returns ([ms per phase], [timed launches per phase]) for phases update, state, attention."""
-    ms = (ctypes.c_double * 3)(0.0, 0.0, 0.0)
-    n = (_ll * 3)(0, 0, 0)
+    """Returns ([ms per phase], [timed launches per phase]) for phases update, state, attention and the
+    position-embedding pre-pass."""
+    ms = (ctypes.c_double * PHASES)()
+    n = (_ll * PHASES)()
     rc = lib.infini_attn_profile_read(ms, n, 1 if reset else 0)
     if rc != INFINI_OK:
         raise InfiniAttnError(rc, "infini_attn_profile_read")

@@ -46,7 +46,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     tmp = LIB + ".tmp"
     cmd = [nvcc_path(), ARCH, "-O3", "-std=c++17", "-lineinfo", "-shared", "-Xcompiler", "-fPIC",
            "-Xcompiler", "-fvisibility=hidden", "-I", os.path.join(ROOT, "include"),
-           "-o", tmp, os.path.join(CSRC, "infini_attn.cu"), "-lcublas"]
+           "-o", tmp, os.path.join(CSRC, "infini_attn.cu")]
     extra = os.environ.get("INFINI_NVCC_FLAGS", "").split()
     cmd[1:1] = extra + ["-Xptxas=-v"]
     if verbose:

@@ -14,12 +14,12 @@
 //     query tile), reading the snapshots.
 // The order "read with M_{s-1}, then update" of the pages holds because the
 // attention kernel reads the snapshot of M_{s-1}, never the running state.
-#include <cublas_v2.h>
 #include <math.h>
 #include <stdio.h>
 #include <string.h>
 
 #include <algorithm>
+#include <cmath>
 #include <atomic>
 #include <mutex>
 #include <utility>
@@ -29,8 +29,10 @@
 #include "common.cuh"
 #include "simt.cuh"
 #include "decode.cuh"
+#include "rope.cuh"
 #include "sm100_attn.cuh"
 #include "sm100_update.cuh"
+#include "sm100_gemm.cuh"
 
 namespace infini {
 namespace {
@@ -43,7 +45,7 @@ constexpr size_t kAlign = 256;
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 // ------------------------------------------------------------ launch accounting
-enum Phase { kPhaseUpdate = 0, kPhaseState = 1, kPhaseAttn = 2 };
+enum Phase { kPhaseUpdate = 0, kPhaseState = 1, kPhaseAttn = 2, kPhasePre = 3, kPhaseProj = 4, kPhases = 5 };
 std::atomic<long long> g_launches{0};
 std::atomic<int> g_profile_mask{0};
 struct EventPair {
@@ -222,8 +224,63 @@ int check_device(bool need_tc) {
 
 int launch_status() { return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_LAUNCH; }
 
+// What the local attention (Eq. 6) reads: q, k themselves, or their rotated
+// copies in the workspace when position embeddings are on (then qm is the
+// un-rotated q that sigma(Q) of the memory read takes).
+struct LocalQK {
+  const void* q;
+  const void* k;
+  long long qs[3], ks[3];
+  const void* qm;  // nullptr: no position embeddings
+};
+
+size_t rope_bytes(const infini_attn_params& p) {
+  if (p.rope_base == 0.0) return 0;
+  const size_t es = (p.mode & INFINI_F32) ? 4 : 2;
+  return 2 * align_up((size_t)p.B * p.H * (size_t)p.L * p.dk * es);
+}
+
+// Rotated copies of q and k (contiguous [B, H, L, dk]) at `dst`.
+int run_rope(const infini_attn_params& p, char* dst, LocalQK* loc) {
+  const bool f32 = (p.mode & INFINI_F32) != 0;
+  const size_t es = f32 ? 4 : 2;
+  const size_t one = align_up((size_t)p.B * p.H * (size_t)p.L * p.dk * es);
+  RopeArgs ra;
+  memset(&ra, 0, sizeof(ra));
+  ra.q = p.q; ra.k = p.k; ra.qr = dst; ra.kr = dst + one;
+  for (int i = 0; i < 3; ++i) {
+    ra.qs[i] = p.q_stride[i];
+    ra.ks[i] = p.k_stride[i];
+  }
+  ra.L = p.L; ra.offset = p.rope_offset; ra.B = p.B; ra.H = p.H; ra.dk = p.dk;
+  for (int i = 0; i < p.dk / 2; ++i) ra.inv_freq[i] = pow(p.rope_base, -2.0 * i / p.dk);
+  // 16-byte vectors need dk % 8 == 0 and rows that start on 16 bytes
+  bool vec = p.dk % 8 == 0 && reinterpret_cast<uintptr_t>(p.q) % 16 == 0 && reinterpret_cast<uintptr_t>(p.k) % 16 == 0;
+  for (int i = 0; i < 3; ++i)
+    vec = vec && (p.q_stride[i] * (long long)es) % 16 == 0 && (p.k_stride[i] * (long long)es) % 16 == 0;
+  const int E = vec ? 8 : 2;
+  const long long work = (long long)p.B * p.H * p.L * (p.dk / E);
+  const unsigned blocks = (unsigned)std::max<long long>(1, std::min<long long>((work + 255) / 256, 8LL * kSms));
+  {
+    LaunchScope ls(kPhasePre, p.stream);
+    if (f32) {
+      if (vec) rope_kernel<float, 8><<<blocks, 256, 0, p.stream>>>(ra);
+      else rope_kernel<float, 2><<<blocks, 256, 0, p.stream>>>(ra);
+    } else {
+      if (vec) rope_kernel<__nv_bfloat16, 8><<<blocks, 256, 0, p.stream>>>(ra);
+      else rope_kernel<__nv_bfloat16, 2><<<blocks, 256, 0, p.stream>>>(ra);
+    }
+  }
+  loc->q = ra.qr;
+  loc->k = ra.kr;
+  const long long st[3] = {(long long)p.H * p.L * p.dk, p.L * p.dk, p.dk};
+  for (int i = 0; i < 3; ++i) loc->qs[i] = loc->ks[i] = st[i];
+  loc->qm = p.q;
+  return launch_status();
+}
+
 template <typename T>
-int run_simt(const infini_attn_params& p, const Plan& pl, char* ws, float scale) {
+int run_simt(const infini_attn_params& p, const Plan& pl, char* ws, float scale, const LocalQK& loc) {
   Geo g;
   g.B = p.B; g.H = p.H; g.L = p.L; g.N = p.N; g.dk = p.dk; g.dv = p.dv; g.S = pl.S;
   for (int i = 0; i < 3; ++i) {
@@ -269,40 +326,103 @@ int run_simt(const infini_attn_params& p, const Plan& pl, char* ws, float scale)
   const int QT = (p.N + 31) / 32;
   const size_t attn_smem = (size_t)(32 * (p.dk + 1) + 32 * p.dv + 32 * p.dk) * 4;
   cudaFuncSetAttribute(simt_attn_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)attn_smem);
+  Geo ga = g;  // the local attention's q, k (rotated copies under position embeddings)
+  for (int i = 0; i < 3; ++i) {
+    ga.qs[i] = loc.qs[i];
+    ga.ks[i] = loc.ks[i];
+    ga.qms[i] = p.q_stride[i];
+  }
   LaunchScope ls(kPhaseAttn, p.stream);
   simt_attn_kernel<T><<<(unsigned)((long long)QT * BH * pl.S), 256, attn_smem, p.stream>>>(
-      static_cast<const T*>(p.q), k, v, p.beta, static_cast<T*>(p.out), g, scale, QT, snapM, snapz);
+      static_cast<const T*>(loc.q), static_cast<const T*>(loc.k), v, p.beta, static_cast<T*>(p.out), ga, scale, QT,
+      snapM, snapz, static_cast<const T*>(loc.qm));
   return launch_status();
 }
 
-int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale) {
-  CUtensorMap tm_q, tm_k, tm_v, tm_mt;
+// The dynamic shared-memory limit is an attribute of a function in the
+// current context: set it for the tensor-core kernels once for every context
+// the process uses (an unknown context id, 0, sets it on every call).
+int set_tc_smem_limits() {
+  static std::mutex mu;
+  static std::vector<unsigned long long> done;
+  const unsigned long long ctx = current_context_id();
+  std::lock_guard<std::mutex> lk(mu);
+  if (ctx != 0 && std::find(done.begin(), done.end(), ctx) != done.end()) return INFINI_OK;
+  if (cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kAttnSmem) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(tc::mem_update_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)tc::UpdSmem<false>::BYTES) != cudaSuccess ||
+      cudaFuncSetAttribute(tc::mem_update_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)tc::UpdSmem<true>::BYTES) != cudaSuccess ||
+      cudaFuncSetAttribute(tc::gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kGemmSmem) !=
+          cudaSuccess)
+    return INFINI_ERR_LAUNCH;
+  if (ctx != 0) done.push_back(ctx);
+  return INFINI_OK;
+}
+
+// 2-D map over a row-major bf16 matrix [rows, cols] with a row stride of ld
+// elements; box box_c x box_r, 128-byte swizzle (box_c = 64).
+bool encode_mat(CUtensorMap* m, const void* ptr, long long rows, long long cols, long long ld, uint32_t box_c,
+                uint32_t box_r) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {box_c, box_r};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// C[M, N] = A[M, K] B[K, N], row-major bf16 with row strides lda, ldb, ldc
+// (elements), fp32 accumulation: the tcgen05 GEMM.  Needs N, K, lda, ldb, ldc
+// multiples of 8 and 16-byte aligned bases (TMA rows start on 16 bytes).
+int gemm_tc(const void* A, long long lda, const void* Bm, long long ldb, void* C, long long ldc, long long M, long long N,
+            long long K, cudaStream_t st) {
+  if (M <= 0 || N <= 0 || K <= 0) return INFINI_ERR_INVALID_ARG;
+  if (N % 8 || K % 8 || lda % 8 || ldb % 8 || ldc % 8 || lda < K || ldb < N || ldc < N) return INFINI_ERR_UNSUPPORTED;
+  if (reinterpret_cast<uintptr_t>(A) % 16 || reinterpret_cast<uintptr_t>(Bm) % 16 || reinterpret_cast<uintptr_t>(C) % 16)
+    return INFINI_ERR_UNSUPPORTED;
+  if (M >= (1LL << 31) || N >= (1LL << 31) || K >= (1LL << 31)) return INFINI_ERR_UNSUPPORTED;
+  const long long tiles_m = (M + tc::kGemmBM - 1) / tc::kGemmBM, tiles_n = (N + tc::kGemmBN - 1) / tc::kGemmBN;
+  if (tiles_m * tiles_n >= (1LL << 31)) return INFINI_ERR_UNSUPPORTED;
+  if (!get_encode()) return INFINI_ERR_DEVICE;
+  CUtensorMap tm_a, tm_b;
+  if (!encode_mat(&tm_a, A, M, K, lda, 64, tc::kGemmBM) || !encode_mat(&tm_b, Bm, K, N, ldb, 64, tc::kGemmBK))
+    return INFINI_ERR_LAUNCH;
+  if (set_tc_smem_limits() != INFINI_OK) return INFINI_ERR_LAUNCH;
+  tc::GemmArgs ga;
+  ga.C = static_cast<__nv_bfloat16*>(C);
+  ga.ldc = ldc;
+  ga.M = (int)M;
+  ga.N = (int)N;
+  ga.K = (int)K;
+  ga.tiles_m = (int)tiles_m;
+  ga.tiles_n = (int)tiles_n;
+  int dev = 0, sms = kSms;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    sms = kSms;
+  LaunchScope ls(kPhaseProj, st);
+  tc::gemm_tc_kernel<<<(unsigned)std::min<long long>(tiles_m * tiles_n, sms), tc::kGemmThreads, tc::kGemmSmem, st>>>(
+      tm_a, tm_b, ga);
+  return launch_status();
+}
+
+int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale, const LocalQK& loc) {
+  // tm_k: the keys of the memory update (un-rotated); tm_qa / tm_ka: the
+  // local attention's queries and keys
+  CUtensorMap tm_qa, tm_k, tm_ka, tm_v, tm_mt;
   __nv_bfloat16* snapM16 = reinterpret_cast<__nv_bfloat16*>(ws + pl.off_snapM);
   float* snapz = reinterpret_cast<float*>(ws + pl.off_snapz);
   float* part = reinterpret_cast<float*>(ws + pl.off_part);
   const int BH = p.B * p.H, E = 128 * 128;
-  if (!encode_bhld(&tm_q, p.q, p.B, p.H, p.L, p.q_stride) || !encode_bhld(&tm_k, p.k, p.B, p.H, p.L, p.k_stride) ||
-      !encode_bhld(&tm_v, p.v, p.B, p.H, p.L, p.v_stride) || !encode_rows(&tm_mt, snapM16, (long long)BH * pl.S * 128))
+  if (!encode_bhld(&tm_qa, loc.q, p.B, p.H, p.L, loc.qs) || !encode_bhld(&tm_k, p.k, p.B, p.H, p.L, p.k_stride) ||
+      !encode_bhld(&tm_ka, loc.k, p.B, p.H, p.L, loc.ks) || !encode_bhld(&tm_v, p.v, p.B, p.H, p.L, p.v_stride) ||
+      !encode_rows(&tm_mt, snapM16, (long long)BH * pl.S * 128))
     return INFINI_ERR_LAUNCH;
-  {
-    // The dynamic shared-memory limit is an attribute of the function in the
-    // current context: set it once for every context the process uses (an
-    // unknown context id, 0, sets it on every call).
-    static std::mutex mu;
-    static std::vector<unsigned long long> done;
-    const unsigned long long ctx = current_context_id();
-    std::lock_guard<std::mutex> lk(mu);
-    if (ctx == 0 || std::find(done.begin(), done.end(), ctx) == done.end()) {
-      if (cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)tc::kAttnSmem) != cudaSuccess ||
-          cudaFuncSetAttribute(tc::mem_update_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)tc::UpdSmem<false>::BYTES) != cudaSuccess ||
-          cudaFuncSetAttribute(tc::mem_update_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)tc::UpdSmem<true>::BYTES) != cudaSuccess)
-        return INFINI_ERR_LAUNCH;
-      if (ctx != 0) done.push_back(ctx);
-    }
-  }
+  if (set_tc_smem_limits() != INFINI_OK) return INFINI_ERR_LAUNCH;
   const dim3 sgrid((E + 128 + 255) / 256, BH);
   tc::UpdArgs ua;
   ua.partial = part; ua.M = p.M; ua.z = p.z; ua.snapM = snapM16; ua.snapzw = snapz;
@@ -346,7 +466,11 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale) {
   aa.beta = p.beta; aa.snapz = snapz; aa.out = static_cast<__nv_bfloat16*>(p.out);
   aa.B = p.B; aa.H = p.H; aa.S = pl.S; aa.T = (p.N + 127) / 128; aa.L = p.L; aa.N = p.N;
   aa.scale_log2 = scale * 1.4426950408889634f;
-  for (int i = 0; i < 3; ++i) aa.os[i] = p.o_stride[i];
+  for (int i = 0; i < 3; ++i) {
+    aa.os[i] = p.o_stride[i];
+    aa.qms[i] = p.q_stride[i];
+  }
+  aa.qm = static_cast<const __nv_bfloat16*>(loc.qm);
   // Scheduling groups of GS segments: about one wave of CTAs per group.
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
@@ -368,7 +492,7 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale) {
     return INFINI_ERR_LAUNCH;
   LaunchScope ls(kPhaseAttn, p.stream);
   tc::attn_tc_kernel<<<(unsigned)std::min<long long>(items, sms), tc::kAttnThreads, tc::kAttnSmem, p.stream>>>(
-      tm_q, tm_k, tm_v, tm_mt, aa);
+      tm_qa, tm_ka, tm_v, tm_mt, aa);
   return launch_status();
 }
 
@@ -415,13 +539,18 @@ int forward_impl(infini_attn_params p) {
       ranges_overlap(p.out, out_ext, p.beta, (size_t)p.H * 4) ||
       ranges_overlap(p.M, (size_t)p.B * p.H * p.dk * p.dv * 4, p.z, (size_t)p.B * p.H * p.dk * 4))
     return INFINI_ERR_INVALID_ARG;
+  const bool rope = p.rope_base != 0.0;
+  if (rope && !(p.rope_base > 0.0 && std::isfinite(p.rope_base))) return INFINI_ERR_INVALID_ARG;
+  if (rope && p.dk % 2 != 0) return INFINI_ERR_UNSUPPORTED;
   if (pl.tc && !tc_layout_ok(p)) {
     // The tensor-core kernels need TMA-compatible strides; other layouts run on CUDA cores.
     rc = make_plan(p.B, p.H, p.L, p.N, p.dk, p.dv, p.mode, p.flags | INFINI_FLAG_FORCE_SIMT, &pl);
     if (rc != INFINI_OK) return rc;
   }
+  // workspace: the plan's buffers, then the rotated q, k under position embeddings
+  const size_t need = pl.total + rope_bytes(p);
   if (p.workspace) {
-    if (p.workspace_bytes < pl.total || reinterpret_cast<uintptr_t>(p.workspace) % kAlign != 0)
+    if (p.workspace_bytes < need || reinterpret_cast<uintptr_t>(p.workspace) % kAlign != 0)
       return INFINI_ERR_WORKSPACE;
   }
   rc = check_device(pl.tc);
@@ -432,19 +561,29 @@ int forward_impl(infini_attn_params p) {
   bool own = false;
   if (!ws) {
     void* w = nullptr;
-    if (cudaMallocAsync(&w, pl.total, p.stream) != cudaSuccess) {
+    if (cudaMallocAsync(&w, need, p.stream) != cudaSuccess) {
       cudaGetLastError();
       return INFINI_ERR_WORKSPACE;
     }
     ws = static_cast<char*>(w);
     own = true;
   }
-  if (pl.tc)
-    rc = run_tc(p, pl, ws, scale);
+  LocalQK loc;
+  memset(&loc, 0, sizeof(loc));
+  loc.q = p.q;
+  loc.k = p.k;
+  for (int i = 0; i < 3; ++i) {
+    loc.qs[i] = p.q_stride[i];
+    loc.ks[i] = p.k_stride[i];
+  }
+  rc = rope ? run_rope(p, ws + pl.total, &loc) : INFINI_OK;
+  if (rc != INFINI_OK) {
+  } else if (pl.tc)
+    rc = run_tc(p, pl, ws, scale, loc);
   else if (pl.f32)
-    rc = run_simt<float>(p, pl, ws, scale);
+    rc = run_simt<float>(p, pl, ws, scale, loc);
   else
-    rc = run_simt<__nv_bfloat16>(p, pl, ws, scale);
+    rc = run_simt<__nv_bfloat16>(p, pl, ws, scale, loc);
   if (own && cudaFreeAsync(ws, p.stream) != cudaSuccess && rc == INFINI_OK) rc = INFINI_ERR_WORKSPACE;
   return rc;
 }
@@ -530,27 +669,6 @@ bool layer_plan(int B, int H, long long L, int N, int d_model, int mode, LayerPl
   return true;
 }
 
-std::mutex g_blas_mu;
-std::vector<cublasHandle_t> g_blas;  // one handle per device, created on first use
-
-// Row-major C[m, n] = A[m, k] B[k, n] in bf16 with fp32 accumulation, as the
-// column-major product C^T = B^T A^T.
-int gemm_bf16(int dev, cudaStream_t st, const void* A, const void* Bm, void* C, long long m, int n, int k) {
-  std::lock_guard<std::mutex> lk(g_blas_mu);
-  if ((int)g_blas.size() <= dev) g_blas.resize(dev + 1, nullptr);
-  if (!g_blas[dev] && cublasCreate(&g_blas[dev]) != CUBLAS_STATUS_SUCCESS) {
-    g_blas[dev] = nullptr;
-    return INFINI_ERR_LAUNCH;
-  }
-  cublasHandle_t h = g_blas[dev];
-  if (cublasSetStream(h, st) != CUBLAS_STATUS_SUCCESS) return INFINI_ERR_LAUNCH;
-  const float one = 1.f, zero = 0.f;
-  const cublasStatus_t rc =
-      cublasGemmEx(h, CUBLAS_OP_N, CUBLAS_OP_N, n, (int)m, k, &one, Bm, CUDA_R_16BF, n, A, CUDA_R_16BF, k, &zero, C,
-                   CUDA_R_16BF, n, CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT);
-  return rc == CUBLAS_STATUS_SUCCESS ? INFINI_OK : INFINI_ERR_LAUNCH;
-}
-
 }  // namespace
 
 extern "C" {
@@ -607,6 +725,13 @@ size_t infini_attn_workspace_size(int B, int H, long L, int N, int dk, int dv, i
   return std::max(pl.total, pl2.total);
 }
 
+
+size_t infini_attn_workspace_size_ex(const infini_attn_params* p) {
+  if (!p) return 0;
+  if (p->rope_base != 0.0 && !(p->rope_base > 0.0 && std::isfinite(p->rope_base) && p->dk % 2 == 0)) return 0;
+  const size_t base = infini_attn_workspace_size(p->B, p->H, (long)p->L, p->N, p->dk, p->dv, p->mode);
+  return base == 0 ? 0 : base + rope_bytes(*p);
+}
 
 int infini_attn_decode_step(const void* q_t, const void* k_t, const void* v_t, void* k_cache, void* v_cache,
                             const float* beta, float* M, float* z, void* out, int B, int H, int N, int pos, int dk,
@@ -683,6 +808,17 @@ int infini_attn_decode_step(const void* q_t, const void* k_t, const void* v_t, v
   return rc;
 }
 
+int infini_attn_gemm_bf16(const void* A, const void* Bm, void* C, long M, int N, int K, cudaStream_t stream) {
+  if (!A || !Bm || !C) return INFINI_ERR_INVALID_ARG;
+  if (M <= 0 || N <= 0 || K <= 0) return INFINI_ERR_INVALID_ARG;
+  if (ranges_overlap(C, (size_t)M * N * 2, A, (size_t)M * K * 2) || ranges_overlap(C, (size_t)M * N * 2, Bm, (size_t)K * N * 2))
+    return INFINI_ERR_INVALID_ARG;
+  if (N % 8 || K % 8) return INFINI_ERR_UNSUPPORTED;
+  const int rc = check_device(true);
+  if (rc != INFINI_OK) return rc;
+  return gemm_tc(A, K, Bm, N, C, N, M, N, K, stream);
+}
+
 size_t infini_attn_layer_workspace_size(int B, int H, long L, int N, int d_model, int mode) {
   LayerPlan lp;
   return layer_plan(B, H, L, N, d_model, mode, &lp) ? lp.total : 0;
@@ -701,10 +837,11 @@ int infini_attn_layer_forward(const void* x, const void* w_qkv, const void* w_o,
     return INFINI_ERR_INVALID_ARG;
   if (workspace && (workspace_bytes < lp.total || reinterpret_cast<uintptr_t>(workspace) % kAlign != 0))
     return INFINI_ERR_WORKSPACE;
+  if (d_model % 8 != 0 || reinterpret_cast<uintptr_t>(x) % 16 || reinterpret_cast<uintptr_t>(w_qkv) % 16 ||
+      reinterpret_cast<uintptr_t>(w_o) % 16 || reinterpret_cast<uintptr_t>(y) % 16)
+    return INFINI_ERR_UNSUPPORTED;
   int rc = check_device(true);
   if (rc != INFINI_OK) return rc;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return INFINI_ERR_DEVICE;
   char* ws = static_cast<char*>(workspace);
   bool own = false;
   if (!ws) {
@@ -719,7 +856,7 @@ int infini_attn_layer_forward(const void* x, const void* w_qkv, const void* w_o,
   const long long HD = (long long)H * kLayerHead;
   __nv_bfloat16* qkv = reinterpret_cast<__nv_bfloat16*>(ws + lp.off_qkv);
   __nv_bfloat16* ao = reinterpret_cast<__nv_bfloat16*>(ws + lp.off_ao);
-  rc = gemm_bf16(dev, stream, x, w_qkv, qkv, lp.rows, (int)(3 * HD), d_model);
+  rc = gemm_tc(x, d_model, w_qkv, 3 * HD, qkv, 3 * HD, lp.rows, 3 * HD, d_model, stream);
   if (rc == INFINI_OK) {
     infini_attn_params p;
     memset(&p, 0, sizeof(p));
@@ -748,7 +885,7 @@ int infini_attn_layer_forward(const void* x, const void* w_qkv, const void* w_o,
     p.stream = stream;
     rc = forward_impl(p);
   }
-  if (rc == INFINI_OK) rc = gemm_bf16(dev, stream, ao, w_o, y, lp.rows, d_model, (int)HD);
+  if (rc == INFINI_OK) rc = gemm_tc(ao, HD, w_o, d_model, y, d_model, lp.rows, d_model, HD, stream);
   if (own && cudaFreeAsync(ws, stream) != cudaSuccess && rc == INFINI_OK) rc = INFINI_ERR_WORKSPACE;
   return rc;
 }
@@ -809,7 +946,7 @@ INFINI_API int infini_attn_debug_trace(unsigned long long* host, int n) {
 #endif
 
 int infini_attn_profile_enable(int phase_mask) {
-  if (phase_mask < 0 || phase_mask > 7) return INFINI_ERR_INVALID_ARG;
+  if (phase_mask < 0 || phase_mask >= (1 << kPhases)) return INFINI_ERR_INVALID_ARG;
   g_profile_mask.store(phase_mask);
   return INFINI_OK;
 }
@@ -817,8 +954,8 @@ int infini_attn_profile_enable(int phase_mask) {
 int infini_attn_profile_read(double* ms, long long* launches, int reset) {
   std::lock_guard<std::mutex> lk(g_prof_mu);
   int rc = INFINI_OK;
-  double acc[3] = {0, 0, 0};
-  long long cnt[3] = {0, 0, 0};
+  double acc[kPhases] = {};
+  long long cnt[kPhases] = {};
   for (const EventPair& e : g_prof) {
     float t = 0.f;
     if (cudaEventSynchronize(e.b) != cudaSuccess || cudaEventElapsedTime(&t, e.a, e.b) != cudaSuccess) {
@@ -828,7 +965,7 @@ int infini_attn_profile_read(double* ms, long long* launches, int reset) {
     acc[e.phase] += t;
     cnt[e.phase] += 1;
   }
-  for (int i = 0; i < 3; ++i) {
+  for (int i = 0; i < kPhases; ++i) {
     if (ms) ms[i] += acc[i];
     if (launches) launches[i] += cnt[i];
   }

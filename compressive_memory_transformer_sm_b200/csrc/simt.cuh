@@ -23,6 +23,7 @@ struct Geo {
   long long L;
   int N, dk, dv, S;
   long long qs[3], ks[3], vs[3], os[3];  // element strides of (B, H, L)
+  long long qms[3];                       // strides of the attention kernel's un-rotated q (qm)
 };
 
 __device__ __forceinline__ long long off3(const long long (&st)[3], int b, int h, long long l) {
@@ -207,11 +208,12 @@ __global__ void __launch_bounds__(256) state_kernel(float* __restrict__ M, float
 // keeps a running max and sum per row; the memory read uses the fp32
 // snapshot M_{s-1}, z_{s-1} of the segment.
 template <typename T>
-__global__ void __launch_bounds__(256) simt_attn_kernel(const T* __restrict__ q, const T* __restrict__ k,
+__global__ void __launch_bounds__(256, 2) simt_attn_kernel(const T* __restrict__ q, const T* __restrict__ k,
                                                         const T* __restrict__ v, const float* __restrict__ beta,
                                                         T* __restrict__ out, Geo g, float scale, int QT,
                                                         const float* __restrict__ snapM,
-                                                        const float* __restrict__ snapz) {
+                                                        const float* __restrict__ snapz,
+                                                        const T* __restrict__ qm) {
   extern __shared__ float sm[];
   const int dk = g.dk, dv = g.dv, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int BHS = g.B * g.H * g.S;
@@ -288,6 +290,16 @@ __global__ void __launch_bounds__(256) simt_attn_kernel(const T* __restrict__ q,
     }
   }
 
+  if (qm != nullptr) {
+    // q and k carry rotary position embeddings for the scores above; the
+    // memory read takes sigma of the un-rotated rows
+    __syncthreads();
+    for (int e = tid; e < 32 * dk; e += 256) {
+      const int r = e / dk, i = e - r * dk;
+      Qs[e] = (q0 + r < n_s) ? to_f32(qm[off3(g.qms, b, h, seg_start + q0 + r) + i]) : 0.f;
+    }
+    __syncthreads();
+  }
   const float gw = 1.f / (1.f + expf(-beta[h]));
   const float* Mp = snapM + ((long long)bh * g.S + s) * dk * dv;
   const float* zp = snapz + ((long long)bh * g.S + s) * dk;

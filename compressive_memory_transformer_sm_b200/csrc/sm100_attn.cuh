@@ -39,6 +39,11 @@ struct AttnArgs {
   int N;
   float scale_log2;       // softmax scale * log2(e)
   long long os[3];        // element strides of out
+  // Un-rotated q for sigma(Q) when the Q tiles loaded by TMA carry rotary
+  // position embeddings (local attention only); nullptr: sigma(Q) from the
+  // Q tiles themselves.  qms: element strides of its (B, H, L) dimensions.
+  const __nv_bfloat16* qm;
+  long long qms[3];
 };
 
 // Shared memory of the attention kernel (offsets from a 1024-aligned base).
@@ -558,14 +563,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         ATTN_TRACE(tr, 1024 * k + 16 * it + 9);
         const uint32_t q = sQ(k);
         float dp[4] = {0.f, 0.f, 0.f, 0.f};
+        // With position embeddings the Q tile holds rotated rows: sigma(Q) is
+        // formed from the un-rotated row in global memory instead (a row past
+        // the segment's end reads zeros; it is never stored).
+        const int grow = (w.tq0 + k) * kTile + row;
+        const uint4* gq = a.qm == nullptr || grow >= w.n_s
+                              ? nullptr
+                              : reinterpret_cast<const uint4*>(a.qm + w.b * a.qms[0] + w.h * a.qms[1] +
+                                                               (w.seg0 + grow) * a.qms[2]);
         // Two batches of 8 chunks: the loads of a batch are in flight
         // together and its 64 elements are independent, while the code stays
         // small enough for the instruction cache (this runs once per item).
 #pragma unroll 1
         for (int c8 = 0; c8 < 16; c8 += 8) {
           uint4 v[8];
+          if (a.qm == nullptr) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) v[i] = lds128(q + swz_chunk(row, c8 + i));
+            for (int i = 0; i < 8; ++i) v[i] = lds128(q + swz_chunk(row, c8 + i));
+          } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = gq ? __ldg(gq + c8 + i) : make_uint4(0u, 0u, 0u, 0u);
+          }
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const float4 za = *reinterpret_cast<const float4*>(zk + 8 * (c8 + i));

@@ -166,12 +166,29 @@ typedef struct infini_attn_params {
   size_t workspace_bytes;
   int flags; /* INFINI_FLAG_* */
   cudaStream_t stream;
+  /* Rotary position embeddings on the local attention only (section 4.1 of
+   * the paper, quoted on the explainer page: position embeddings act on the
+   * Q, K of the dot-product attention and not on the compressive memory's).
+   * rope_base > 0 turns them on: A_dot (Eq. 6) is computed from rotated
+   * Q, K, where the pair (x_2i, x_2i+1) of a row at position p is rotated by
+   * the angle p * rope_base^(-2i/dk), and p = rope_offset + t for token t of
+   * the call (0 <= t < L).  sigma(Q) of the memory read (Eq. 7) and the
+   * update (Eq. 8 / 9) use the un-rotated q, k.  dk must be even.  The
+   * rotated copies of q and k live in the workspace
+   * (infini_attn_workspace_size_ex).  rope_base = 0: no position embedding. */
+  double rope_base;
+  long long rope_offset;
 } infini_attn_params;
 
 INFINI_API int infini_attn_forward_ex(const infini_attn_params* p);
 
 /* Bytes of workspace a forward of this shape needs (0 if the shape is invalid). */
 INFINI_API size_t infini_attn_workspace_size(int B, int H, long L, int N, int dk, int dv, int mode);
+
+/* Bytes of workspace infini_attn_forward_ex(p) needs (0 if p is invalid):
+ * infini_attn_workspace_size of the shape, plus the rotated q and k when
+ * p->rope_base > 0.  Only the shape, mode and rope_base fields are read. */
+INFINI_API size_t infini_attn_workspace_size_ex(const infini_attn_params* p);
 
 /*
  * Token-level streaming decode (the "fast streaming inference" of the
@@ -212,13 +229,14 @@ INFINI_API int infini_attn_decode_step(const void* q_t, const void* k_t, const v
  *          column j of head h)
  *   y      [B, L, D] bf16, written
  *   beta, M, z, N, mode as in infini_attn_forward (mode without INFINI_F32).
- * The projections are plain GEMMs (cuBLAS: bf16 operands, fp32
- * accumulation, bf16 results); Q, K, V and the attention output are stored
- * in bf16 between the steps, in a workspace of
- * infini_attn_layer_workspace_size(...) bytes (256-byte aligned) that the
- * call allocates and frees on `stream` when `workspace` is NULL.  Errors as
- * infini_attn_forward; a cuBLAS failure returns INFINI_ERR_LAUNCH.  Calls
- * from several host threads share one cuBLAS handle per device under a lock.
+ * The projections run on this library's tensor-core GEMM
+ * (infini_attn_gemm_bf16: bf16 operands, fp32 accumulation, bf16 results);
+ * Q, K, V and the attention output are stored in bf16 between the steps, in
+ * a workspace of infini_attn_layer_workspace_size(...) bytes (256-byte
+ * aligned) that the call allocates and frees on `stream` when `workspace` is
+ * NULL.  d_model must be a multiple of 8 and x, w_qkv, w_o, y 16-byte
+ * aligned (rows of the GEMM operands are loaded by TMA), else
+ * INFINI_ERR_UNSUPPORTED.  Errors otherwise as infini_attn_forward.
  */
 INFINI_API int infini_attn_layer_forward(const void* x, const void* w_qkv, const void* w_o, const float* beta,
                                          float* M, float* z, void* y, int B, int H, long L, int N, int d_model,
@@ -226,6 +244,19 @@ INFINI_API int infini_attn_layer_forward(const void* x, const void* w_qkv, const
 
 /* Bytes of workspace infini_attn_layer_forward needs (0 if the shape is invalid). */
 INFINI_API size_t infini_attn_layer_workspace_size(int B, int H, long L, int N, int d_model, int mode);
+
+/*
+ * The projection product of the full layer (Eq. 5, Q K V = X W; Eq. 11,
+ * Y = [A_1 ... A_H] W_O) on its own: C[M, N] = A[M, K] B[K, N] for row-major
+ * contiguous bf16 matrices, fp32 accumulation, C rounded to bf16 (nearest
+ * even).  A tcgen05 kernel: 128 x 256 output tiles over a persistent grid,
+ * operands staged by TMA, accumulators in tensor memory.  N and K must be
+ * multiples of 8 and the pointers 16-byte aligned (INFINI_ERR_UNSUPPORTED
+ * otherwise); C must not overlap A or B.  Device pointers, asynchronous on
+ * `stream`; no workspace.
+ */
+INFINI_API int infini_attn_gemm_bf16(const void* A, const void* B, void* C, long M, int N, int K,
+                                     cudaStream_t stream);
 
 /* Static English text for a return code; never NULL. */
 INFINI_API const char* infini_attn_error_string(int code);
@@ -250,12 +281,14 @@ INFINI_API int infini_attn_selftest_timeout(unsigned limit_us, cudaStream_t stre
 /*
  * Kernel timing for benchmarks.  phase_mask selects phases (bit 0 = memory
  * update kernels, bit 1 = state/snapshot kernels, bit 2 = attention
- * kernel); while a bit is set, every launch of that phase is bracketed by
- * two CUDA events recorded on the launch's stream.  0 turns timing off.
+ * kernel, bit 3 = position-embedding pre-pass, bit 4 = projection GEMMs of
+ * the full layer); while a bit is set, every
+ * launch of that phase is bracketed by two CUDA events recorded on the
+ * launch's stream.  0 turns timing off.
  */
 INFINI_API int infini_attn_profile_enable(int phase_mask);
 /*
- * Synchronises the recorded events and adds, per phase p in 0..2, the
+ * Synchronises the recorded events and adds, per phase p in 0..4, the
  * elapsed milliseconds to ms[p] and the number of timed launches to
  * launches[p], for everything recorded since the last reset; reset != 0
  * then drops the records.  Either array may be NULL.

@@ -182,3 +182,31 @@ def test_binding_rejects_host_and_strided_tensors():
         api.infini_attn_layer_forward(torch.zeros(1, 8, 64), torch.zeros(64, 3 * 128), torch.zeros(128, 64),
                                       torch.zeros(1), torch.zeros(1, 1, 128, 128), torch.zeros(1, 1, 128),
                                       torch.zeros(1, 8, 64), 1, 4)
+
+
+def _call_ex(**over):
+    p = api.InfiniAttnParams()
+    vals = dict(q=1 << 20, k=2 << 20, v=3 << 20, beta=4 << 20, M=5 << 20, z=6 << 20, out=7 << 20,
+                B=1, H=2, L=64, N=16, dk=16, dv=16, mode=LINEAR | F32, rope_base=10000.0, rope_offset=0)
+    vals.update(over)
+    for key, val in vals.items():
+        setattr(p, key, val)
+    return api.lib.infini_attn_forward_ex(ctypes.byref(p))
+
+
+def test_rope_arguments_are_validated_before_any_cuda_call():
+    assert _call_ex(rope_base=-1.0) == api.INFINI_ERR_INVALID_ARG
+    assert _call_ex(rope_base=float("nan")) == api.INFINI_ERR_INVALID_ARG
+    assert _call_ex(rope_base=float("inf")) == api.INFINI_ERR_INVALID_ARG
+    assert _call_ex(dk=15) == api.INFINI_ERR_UNSUPPORTED  # pairs need an even head size
+    # a valid call reaches the device check (no GPU here) or runs
+    assert _call_ex() in (api.INFINI_ERR_DEVICE, api.INFINI_OK) or torch.cuda.is_available()
+
+
+def test_workspace_size_ex_counts_the_rotated_copies():
+    base = api.infini_attn_workspace_size(1, 8, 32768, 2048, 128, 128, LINEAR)
+    assert api.infini_attn_workspace_size_ex(1, 8, 32768, 2048, 128, 128, LINEAR) == base
+    with_rope = api.infini_attn_workspace_size_ex(1, 8, 32768, 2048, 128, 128, LINEAR, rope_base=10000.0)
+    assert with_rope >= base + 2 * 8 * 32768 * 128 * 2  # rotated q and k in bf16
+    assert api.infini_attn_workspace_size_ex(1, 8, 32768, 2048, 127, 128, LINEAR, rope_base=10000.0) == 0
+    assert api.infini_attn_workspace_size_ex(1, 8, 32768, 2048, 128, 128, LINEAR, rope_base=-5.0) == 0
