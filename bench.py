@@ -52,7 +52,7 @@ from compressive_memory_transformer_sm_b200 import workloads as W  # noqa: E402
 METRIC = "Infini-attn fwd tokens/s per layer; TFLOP/s and % of B200 bf16 tensor peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FLUSH_BYTES = 1 << 30
-PHASE_NAMES = ("update", "state", "attention", "rope", "projections")
+PHASE_NAMES = ("update", "state", "attention", "rope", "projections", "backward")
 
 
 # ------------------------------------------------------------------ work model
@@ -610,6 +610,90 @@ def run_decode(args, w: W.Workload, mode: int):
         print(json.dumps(result), flush=True)
 
 
+BACKWARD_METRIC = "Infini-attn bwd tokens/s per layer (gradients of q, k, v, beta, M_0, z_0 through the forward)"
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965  # SMs x fp32 lanes x FMA x max SM clock (GHz): 74.4 TFLOP/s
+
+
+def run_backward(args, w: W.Workload, mode: int):
+    """``--backward``: one step = one ``infini_attn_backward`` call (forward recomputation
+    included) on the workload's shape, timed like the default line."""
+    from compressive_memory_transformer_sm_b200 import api
+
+    rank, world = init_dist("nccl")
+    _, _, local = dist_env()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    q, k, v, beta = W.make_inputs(w, device=dev, seed=rank_seed(w, rank))
+    g = torch.Generator(device=dev)
+    g.manual_seed(rank_seed(w, rank) + 1)
+    d_out = torch.randn(v.shape, generator=g, device=dev).to(w.dtype)
+    ws = torch.empty(api.infini_attn_backward_workspace_size(w.B, w.H, w.L, w.N, w.dk, w.dv, mode), dtype=torch.uint8,
+                     device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        return api.infini_attn_backward(q, k, v, beta, d_out, w.N, mode, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(local)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    launches0 = api.infini_attn_launch_count()
+    for i in range(args.steps):
+        flush.fill_(i & 0xff)
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    launches = api.infini_attn_launch_count() - launches0
+    clocks = sampler.stop() if sampler else None
+    if api.infini_attn_device_status() != api.INFINI_OK:
+        raise RuntimeError("a device-side wait timed out during the benchmark")
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    ms = max_over_ranks(sum(step_ms) / len(step_ms), dev)
+    api.infini_attn_profile_read(reset=True)
+    api.infini_attn_profile_enable((1 << api.PHASES) - 1)
+    for _ in range(args.steps):
+        step()
+    torch.cuda.synchronize(dev)
+    api.infini_attn_profile_enable(0)
+    phase_ms, phase_n = api.infini_attn_profile_read(reset=True)
+    # algorithmic work: the forward recomputation plus the backward's products (local
+    # attention: S, dP, dV, dK, dQ = 5 causal n(n+1)d/2-pair products per segment; memory
+    # read and update: about 12 n dk dv for the linear rule, 18 for the delta rule)
+    f_fwd_attn, f_fwd_upd = algorithmic_flops(w, mode)
+    f_bwd = 0
+    for s0 in range(0, w.L, w.N):
+        n = min(w.N, w.L - s0)
+        f_bwd += 5 * n * (n + 1) * w.dk // 2 * 2 + (12 if mode == LINEAR else 18) * n * w.dk * w.dv
+    f_bwd *= w.B * w.H
+    total = f_fwd_attn + f_fwd_upd + f_bwd
+    tflops = total * world / (ms * 1e-3) / 1e12
+    result = {
+        "metric": BACKWARD_METRIC, "value": w.B * w.L * world / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "step_ms_min_max": [min(step_ms), max(step_ms)], "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "N": w.N, "dk": w.dk, "dv": w.dv,
+                   "mode": W.MODE_NAMES[mode], "step": "infini_attn_backward (forward recomputed inside)",
+                   "l2": "1 GiB buffer written between timed steps (outside the step events)"},
+        "tflops": tflops, "flops_per_step": total,
+        "roofline": {"kernel": "backward (CUDA cores, fp32)", "bound": "alu", "achieved": tflops / world,
+                     "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s", "frac": tflops / world / FP32_ALU_TFLOPS,
+                     "peak_source": "148 SMs x 128 fp32 lanes x 2 (FMA) x 1.965 GHz"},
+        "phases_ms_per_step": {name: phase_ms[i] / args.steps for i, name in enumerate(PHASE_NAMES)},
+        "gpu_launches": int(launches), "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
 def run_reference(args, w: W.Workload, mode: int):
     rank, world, _ = dist_env()
     if rank != 0:
@@ -662,6 +746,8 @@ def parse(argv=None):
                     help="time the full layer (QKV projection + attention + output projection) instead")
     ap.add_argument("--decode", action="store_true",
                     help="time token-level streaming decode (one segment of single-token calls per step)")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward pass (infini_attn_backward, forward recomputed inside)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3, help="timed steps of the host-buffer measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -678,7 +764,7 @@ def main(argv=None):
         w = w.with_(name=f"{w.name}@{B}x{H}x{L}x{N}", B=B, H=H, L=L, N=N)
     modes = ({"linear": LINEAR, "delta": DELTA}[args.mode],) if args.mode else tuple(w.modes)
     mode = modes[0]
-    if args.rope and (w.streaming or args.layer or args.decode):
+    if args.rope and (w.streaming or args.layer or args.decode or args.backward):
         raise SystemExit("--rope applies to the whole-sequence forward (infini_attn_forward_ex) only")
     if args.warmup < 3 and args.impl == "ours":
         raise SystemExit("--warmup must be at least 3")
@@ -688,6 +774,8 @@ def main(argv=None):
         run_layer(args, w, mode)
     elif args.decode:
         run_decode(args, w, mode)
+    elif args.backward:
+        run_backward(args, w, mode)
     else:
         run_ours(args, w, modes)
 

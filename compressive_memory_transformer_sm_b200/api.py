@@ -37,7 +37,8 @@ EXPORTED = (
     "infini_attn_params_size", "infini_attn_path", "infini_attn_profile_enable", "infini_attn_profile_read",
     "infini_attn_launch_count", "infini_attn_forward_noalloc",
     "infini_attn_layer_forward", "infini_attn_layer_workspace_size", "infini_attn_decode_step",
-    "infini_attn_workspace_size_ex", "infini_attn_gemm_bf16",
+    "infini_attn_workspace_size_ex", "infini_attn_gemm_bf16", "infini_attn_backward",
+    "infini_attn_backward_workspace_size",
 )
 
 
@@ -83,8 +84,8 @@ lib.infini_attn_layer_workspace_size.restype = ctypes.c_size_t
 lib.infini_attn_gemm_bf16.argtypes = [_vp, _vp, _vp, _l, _i, _i, _vp]
 lib.infini_attn_gemm_bf16.restype = _i
 
-PHASE_UPDATE, PHASE_STATE, PHASE_ATTN, PHASE_PRE, PHASE_PROJ = 0, 1, 2, 3, 4
-PHASES = 5
+PHASE_UPDATE, PHASE_STATE, PHASE_ATTN, PHASE_PRE, PHASE_PROJ, PHASE_BWD = 0, 1, 2, 3, 4, 5
+PHASES = 6
 
 
 class InfiniAttnParams(ctypes.Structure):
@@ -104,6 +105,23 @@ lib.infini_attn_forward_ex.argtypes = [ctypes.POINTER(InfiniAttnParams)]
 lib.infini_attn_forward_ex.restype = _i
 lib.infini_attn_workspace_size_ex.argtypes = [ctypes.POINTER(InfiniAttnParams)]
 lib.infini_attn_workspace_size_ex.restype = ctypes.c_size_t
+
+
+class InfiniAttnBwdParams(ctypes.Structure):
+    """Mirror of ``infini_attn_bwd_params`` (include/infini_attn.h)."""
+
+    _fields_ = [
+        ("q", _vp), ("k", _vp), ("v", _vp), ("beta", _vp), ("M0", _vp), ("z0", _vp), ("d_out", _vp),
+        ("dM_S", _vp), ("dz_S", _vp), ("dq", _vp), ("dk", _vp), ("dv", _vp), ("dbeta", _vp), ("dM0", _vp),
+        ("dz0", _vp), ("B", _i), ("H", _i), ("L", _ll), ("N", _i), ("d_k", _i), ("d_v", _i), ("mode", _i),
+        ("scale", ctypes.c_float), ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t), ("stream", _vp),
+    ]
+
+
+lib.infini_attn_backward.argtypes = [ctypes.POINTER(InfiniAttnBwdParams)]
+lib.infini_attn_backward.restype = _i
+lib.infini_attn_backward_workspace_size.argtypes = [ctypes.POINTER(InfiniAttnBwdParams)]
+lib.infini_attn_backward_workspace_size.restype = ctypes.c_size_t
 
 
 class InfiniAttnError(RuntimeError):
@@ -289,6 +307,51 @@ def infini_attn_forward_ex(q, k, v, beta, M, z, out, N: int, mode: int = LINEAR,
     p.rope_offset = int(rope_offset)
     rc = lib.infini_attn_forward_ex(ctypes.byref(p))
     return _check(rc, "infini_attn_forward_ex", raise_on_error)
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def infini_attn_backward(q, k, v, beta, d_out, N: int, mode: int = LINEAR, M0=None, z0=None, dM_S=None, dz_S=None,
+                         want_state_grad: bool = True, scale: float = 0.0, workspace=None, stream=None,
+                         raise_on_error=True):
+    """Gradients through the forward: returns (dq, dk, dv, dbeta, dM0, dz0) as new device tensors
+    (dM0, dz0 are None unless ``want_state_grad``).  q, k [B,H,L,dk], v, d_out [B,H,L,dv] contiguous,
+    one dtype (bf16 or fp32); beta [H]; M0, dM_S [B,H,dk,dv], z0, dz_S [B,H,dk] fp32 or None."""
+    _args("infini_attn_backward", dict(q=(q, 4), k=(k, 4), v=(v, 4), d_out=(d_out, 4), beta=(beta, 1)))
+    for name, t, nd in (("M0", M0, 4), ("z0", z0, 3), ("dM_S", dM_S, 4), ("dz_S", dz_S, 3)):
+        if t is not None:
+            _args("infini_attn_backward", {name: (t, nd)})
+    B, H, L, dk = q.shape
+    dv = v.shape[3]
+    _same("infini_attn_backward", "q / k / v / d_out (B, H, L)", tuple(q.shape[:3]), tuple(k.shape[:3]),
+          tuple(v.shape[:3]), tuple(d_out.shape[:3]))
+    dq, dk_, dv_ = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dbeta = torch.empty(H, dtype=torch.float32, device=q.device)
+    dM0 = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device) if want_state_grad else None
+    dz0 = torch.empty(B, H, dk, dtype=torch.float32, device=q.device) if want_state_grad else None
+    p = InfiniAttnBwdParams()
+    p.q, p.k, p.v, p.beta, p.d_out = q.data_ptr(), k.data_ptr(), v.data_ptr(), beta.data_ptr(), d_out.data_ptr()
+    p.M0, p.z0, p.dM_S, p.dz_S = _ptr(M0), _ptr(z0), _ptr(dM_S), _ptr(dz_S)
+    p.dq, p.dk, p.dv, p.dbeta, p.dM0, p.dz0 = dq.data_ptr(), dk_.data_ptr(), dv_.data_ptr(), dbeta.data_ptr(), \
+        _ptr(dM0), _ptr(dz0)
+    p.B, p.H, p.L, p.N, p.d_k, p.d_v = B, H, L, int(N), dk, dv
+    p.mode = _mode(mode, q)
+    p.scale = float(scale)
+    if workspace is not None:
+        p.workspace = workspace.data_ptr()
+        p.workspace_bytes = workspace.numel() * workspace.element_size()
+    p.stream = _stream(stream)
+    rc = lib.infini_attn_backward(ctypes.byref(p))
+    _check(rc, "infini_attn_backward", raise_on_error)
+    return dq, dk_, dv_, dbeta, dM0, dz0
+
+
+def infini_attn_backward_workspace_size(B, H, L, N, dk, dv, mode=LINEAR) -> int:
+    p = InfiniAttnBwdParams()
+    p.B, p.H, p.L, p.N, p.d_k, p.d_v, p.mode = int(B), int(H), int(L), int(N), int(dk), int(dv), int(mode)
+    return int(lib.infini_attn_backward_workspace_size(ctypes.byref(p)))
 
 
 def infini_attn_workspace_size(B, H, L, N, dk, dv, mode=LINEAR) -> int:

@@ -28,6 +28,7 @@
 #include "../../include/infini_attn.h"
 #include "common.cuh"
 #include "simt.cuh"
+#include "bwd_simt.cuh"
 #include "decode.cuh"
 #include "rope.cuh"
 #include "sm100_attn.cuh"
@@ -45,7 +46,7 @@ constexpr size_t kAlign = 256;
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 // ------------------------------------------------------------ launch accounting
-enum Phase { kPhaseUpdate = 0, kPhaseState = 1, kPhaseAttn = 2, kPhasePre = 3, kPhaseProj = 4, kPhases = 5 };
+enum Phase { kPhaseUpdate = 0, kPhaseState = 1, kPhaseAttn = 2, kPhasePre = 3, kPhaseProj = 4, kPhaseBwd = 5, kPhases = 6 };
 std::atomic<long long> g_launches{0};
 std::atomic<int> g_profile_mask{0};
 struct EventPair {
@@ -280,7 +281,8 @@ int run_rope(const infini_attn_params& p, char* dst, LocalQK* loc) {
 }
 
 template <typename T>
-int run_simt(const infini_attn_params& p, const Plan& pl, char* ws, float scale, const LocalQK& loc) {
+int run_simt(const infini_attn_params& p, const Plan& pl, char* ws, float scale, const LocalQK& loc,
+             float* adot = nullptr, float* lse = nullptr) {
   Geo g;
   g.B = p.B; g.H = p.H; g.L = p.L; g.N = p.N; g.dk = p.dk; g.dv = p.dv; g.S = pl.S;
   for (int i = 0; i < 3; ++i) {
@@ -335,7 +337,7 @@ int run_simt(const infini_attn_params& p, const Plan& pl, char* ws, float scale,
   LaunchScope ls(kPhaseAttn, p.stream);
   simt_attn_kernel<T><<<(unsigned)((long long)QT * BH * pl.S), 256, attn_smem, p.stream>>>(
       static_cast<const T*>(loc.q), static_cast<const T*>(loc.k), v, p.beta, static_cast<T*>(p.out), ga, scale, QT,
-      snapM, snapz, static_cast<const T*>(loc.qm));
+      snapM, snapz, static_cast<const T*>(loc.qm), adot, lse);
   return launch_status();
 }
 
@@ -597,6 +599,224 @@ __global__ void selftest_wait_kernel(unsigned long long limit_ns) {
   mbar_wait(b, 0, limit_ns);
 }
 
+// ------------------------------------------------------------ backward
+// Workspace of the backward: the forward's CUDA-core plan (fp32 snapshots of
+// M^(s), z^(s)), a copy of the running state, the forward's output, A_dot and
+// lse, the per-row terms, the partials of the memory-gradient chain, its
+// snapshots (linear) or running value (delta), and the update's dk, dv terms.
+struct BwdPlan {
+  Plan fwd;
+  int Gc, cpbc, Gu, cpbu;
+  size_t off_fwd, off_state, off_out, off_adot, off_lse, off_D, off_brow, off_dden, off_ddenr, off_dnum, off_dnumr,
+      off_cpart, off_upart, off_g, off_dkupd, off_dvupd, total;
+};
+
+int bwd_plan(const infini_attn_bwd_params& p, BwdPlan* bp) {
+  if (p.B <= 0 || p.H <= 0 || p.L <= 0 || p.N <= 0 || p.d_k <= 0 || p.d_v <= 0) return INFINI_ERR_INVALID_ARG;
+  int rc = make_plan(p.B, p.H, p.L, p.N, p.d_k, p.d_v, p.mode, INFINI_FLAG_FORCE_SIMT, &bp->fwd);
+  if (rc != INFINI_OK) return rc;
+  const Plan& f = bp->fwd;
+  const long long BH = (long long)p.B * p.H, rows = BH * p.L;
+  if (rows >= (1LL << 40)) return INFINI_ERR_UNSUPPORTED;
+  const size_t E = (size_t)p.d_k * p.d_v, es = f.f32 ? 4 : 2;
+  const int chunks = (int)((std::min<long long>(p.N, p.L) + kChunk - 1) / kChunk);
+  auto groups = [&](long long units, int* cpb) {
+    long long c = (units * chunks + kTargetCtas - 1) / kTargetCtas;
+    c = std::max<long long>(1, std::min<long long>(c, chunks));
+    *cpb = (int)c;
+    return (int)((chunks + c - 1) / c);
+  };
+  bp->Gc = groups(BH * f.S, &bp->cpbc);
+  bp->Gu = groups(BH, &bp->cpbu);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes);
+    return o;
+  };
+  bp->off_fwd = take(f.total);
+  bp->off_state = take((size_t)BH * (E + p.d_k) * 4);
+  bp->off_out = take((size_t)rows * p.d_v * es);
+  bp->off_adot = take((size_t)rows * p.d_v * 4);
+  bp->off_lse = take((size_t)rows * 4);
+  bp->off_D = take((size_t)rows * 4);
+  bp->off_brow = take((size_t)rows * 4);
+  bp->off_dden = take((size_t)rows * 4);
+  bp->off_ddenr = take(f.delta ? (size_t)rows * 4 : 0);
+  bp->off_dnum = take((size_t)rows * p.d_v * 4);
+  bp->off_dnumr = take(f.delta ? (size_t)rows * p.d_v * 4 : 0);
+  bp->off_cpart = take((size_t)BH * f.S * bp->Gc * (E + p.d_k) * 4);
+  bp->off_upart = take(f.delta ? (size_t)BH * bp->Gu * (E + p.d_k) * 4 : 0);
+  bp->off_g = take((size_t)BH * (f.delta ? 1 : f.S) * (E + p.d_k) * 4);
+  bp->off_dkupd = take((size_t)rows * p.d_k * 4);
+  bp->off_dvupd = take((size_t)rows * p.d_v * 4);
+  bp->total = off;
+  return INFINI_OK;
+}
+
+template <typename T>
+int run_backward(const infini_attn_bwd_params& p, const BwdPlan& bp, char* ws) {
+  const Plan& f = bp.fwd;
+  const int dk = p.d_k, dv = p.d_v, BH = p.B * p.H;
+  const size_t E = (size_t)dk * dv;
+  const float scale = p.scale != 0.f ? p.scale : 1.f / sqrtf((float)dk);
+  cudaStream_t st = p.stream;
+  float* Mst = reinterpret_cast<float*>(ws + bp.off_state);
+  float* zst = Mst + (size_t)BH * E;
+  // 1. forward again from (M_0, z_0): snapshots of M^(s), z^(s), A_dot, lse
+  if ((p.M0 ? cudaMemcpyAsync(Mst, p.M0, (size_t)BH * E * 4, cudaMemcpyDeviceToDevice, st)
+            : cudaMemsetAsync(Mst, 0, (size_t)BH * E * 4, st)) != cudaSuccess ||
+      (p.z0 ? cudaMemcpyAsync(zst, p.z0, (size_t)BH * dk * 4, cudaMemcpyDeviceToDevice, st)
+            : cudaMemsetAsync(zst, 0, (size_t)BH * dk * 4, st)) != cudaSuccess)
+    return INFINI_ERR_LAUNCH;
+  infini_attn_params fp;
+  memset(&fp, 0, sizeof(fp));
+  fp.q = p.q; fp.k = p.k; fp.v = p.v; fp.beta = p.beta; fp.M = Mst; fp.z = zst; fp.out = ws + bp.off_out;
+  fp.B = p.B; fp.H = p.H; fp.L = p.L; fp.N = p.N; fp.dk = dk; fp.dv = dv; fp.mode = p.mode; fp.stream = st;
+  const long long cst[2][3] = {{(long long)p.H * p.L * dk, p.L * dk, dk}, {(long long)p.H * p.L * dv, p.L * dv, dv}};
+  for (int i = 0; i < 3; ++i) {
+    fp.q_stride[i] = fp.k_stride[i] = cst[0][i];
+    fp.v_stride[i] = fp.o_stride[i] = cst[1][i];
+  }
+  LocalQK loc;
+  memset(&loc, 0, sizeof(loc));
+  loc.q = p.q; loc.k = p.k;
+  for (int i = 0; i < 3; ++i) loc.qs[i] = loc.ks[i] = cst[0][i];
+  float* adot = reinterpret_cast<float*>(ws + bp.off_adot);
+  float* lse = reinterpret_cast<float*>(ws + bp.off_lse);
+  char* fws = ws + bp.off_fwd;
+  int rc = run_simt<T>(fp, f, fws, scale, loc, adot, lse);
+  if (rc != INFINI_OK) return rc;
+  const float* snapM = reinterpret_cast<const float*>(fws + f.off_snapM);
+  const float* snapz = reinterpret_cast<const float*>(fws + f.off_snapz);
+  BwdGeo g;
+  g.B = p.B; g.H = p.H; g.S = f.S; g.N = p.N; g.dk = dk; g.dv = dv; g.L = p.L;
+  const T* q = static_cast<const T*>(p.q);
+  const T* k = static_cast<const T*>(p.k);
+  const T* v = static_cast<const T*>(p.v);
+  const T* dout = static_cast<const T*>(p.d_out);
+  float* Drow = reinterpret_cast<float*>(ws + bp.off_D);
+  float* brow = reinterpret_cast<float*>(ws + bp.off_brow);
+  float* dden = reinterpret_cast<float*>(ws + bp.off_dden);
+  float* dnum = reinterpret_cast<float*>(ws + bp.off_dnum);
+  float* ddenr = reinterpret_cast<float*>(ws + bp.off_ddenr);
+  float* dnumr = reinterpret_cast<float*>(ws + bp.off_dnumr);
+  float* cpart = reinterpret_cast<float*>(ws + bp.off_cpart);
+  float* upart = reinterpret_cast<float*>(ws + bp.off_upart);
+  float* gst = reinterpret_cast<float*>(ws + bp.off_g);
+  float* dkupd = reinterpret_cast<float*>(ws + bp.off_dkupd);
+  float* dvupd = reinterpret_cast<float*>(ws + bp.off_dvupd);
+  // 2. dq, D, the dbeta row terms, d_num and d_den rows
+  const int QT = (p.N + 31) / 32;
+  const size_t q_smem = (size_t)(32 * (dk + 1) + 32 * dv + 32 * dk + 2 * 32 * dv) * 4;
+  cudaFuncSetAttribute(bwd_q_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)q_smem);
+  {
+    LaunchScope ls(kPhaseBwd, st);
+    bwd_q_kernel<T><<<(unsigned)((long long)QT * BH * f.S), 256, q_smem, st>>>(
+        q, k, v, dout, p.beta, adot, lse, snapM, snapz, g, scale, QT, static_cast<T*>(p.dq), Drow, brow, dnum, dden);
+  }
+  // 3. the memory read's partials sigma(Q)^T [d_num | d_den] of every segment
+  const size_t outer_smem = (size_t)(32 * dk + 32 * (dv + 1)) * 4;
+  cudaFuncSetAttribute(bwd_outer_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)outer_smem);
+  {
+    LaunchScope ls(kPhaseBwd, st);
+    bwd_outer_kernel<T><<<(unsigned)((long long)BH * f.S * bp.Gc), 256, outer_smem, st>>>(q, dnum, dden, g, dv, 0, f.S,
+                                                                                          bp.Gc, bp.cpbc, cpart);
+  }
+  const dim3 sgrid((unsigned)((E + dk + 255) / 256), BH);
+  const size_t pst = E + dk;
+  const int bps = (std::min(p.N, (int)std::min<long long>(p.N, p.L)) + 127) / 128;
+  const size_t upd_smem = (size_t)((f.delta ? 2 : 1) * dk * (dv + 1) + 2 * dk + 32 * dk + 2 * 32 * dv) * 4;
+  cudaFuncSetAttribute(bwd_upd_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)upd_smem);
+  // 4. the memory-gradient chain and the update's dk, dv terms
+  if (!f.delta) {
+    {
+      LaunchScope ls(kPhaseBwd, st);
+      bwd_state_kernel<<<sgrid, 256, 0, st>>>(nullptr, p.dM_S, p.dz_S, cpart, nullptr, dk, dv, f.S, 0, 0, bp.Gc, 0, gst,
+                                              p.dM0, p.dz0);
+    }
+    LaunchScope ls(kPhaseBwd, st);
+    bwd_upd_kernel<T><<<(unsigned)((long long)BH * f.S * bps), 256, upd_smem, st>>>(
+        k, v, g, 0, gst, (long long)pst, (long long)f.S * pst, nullptr, nullptr, dkupd, dvupd, nullptr, nullptr, bps);
+  } else {
+    {
+      LaunchScope ls(kPhaseBwd, st);
+      bwd_state_kernel<<<sgrid, 256, 0, st>>>(gst, p.dM_S, p.dz_S, nullptr, nullptr, dk, dv, f.S, 2, 0, bp.Gc, 0,
+                                              nullptr, nullptr, nullptr);
+    }
+    for (int s = f.S - 1; s >= 0; --s) {
+      {
+        LaunchScope ls(kPhaseBwd, st);
+        bwd_upd_kernel<T><<<(unsigned)((long long)BH * bps), 256, upd_smem, st>>>(
+            k, v, g, s, gst, 0, (long long)pst, snapM, snapz, dkupd, dvupd, dnumr, ddenr, bps);
+      }
+      {
+        LaunchScope ls(kPhaseBwd, st);
+        bwd_outer_kernel<T><<<(unsigned)((long long)BH * bp.Gu), 256, outer_smem, st>>>(k, dnumr, ddenr, g, dv, s, 1,
+                                                                                       bp.Gu, bp.cpbu, upart);
+      }
+      LaunchScope ls(kPhaseBwd, st);
+      bwd_state_kernel<<<sgrid, 256, 0, st>>>(gst, nullptr, nullptr, cpart, upart, dk, dv, f.S, 1, s, bp.Gc, bp.Gu,
+                                              nullptr, nullptr, nullptr);
+    }
+    LaunchScope ls(kPhaseBwd, st);
+    bwd_state_kernel<<<sgrid, 256, 0, st>>>(gst, nullptr, nullptr, nullptr, nullptr, dk, dv, f.S, 3, 0, 0, 0, nullptr,
+                                            p.dM0, p.dz0);
+  }
+  // 5. dk, dv of the local attention plus the update's terms
+  const size_t kv_smem = (size_t)(32 * dk + 32 * dv + 32 * (dk + 1) + 32 * (dv + 1) + 64) * 4;
+  cudaFuncSetAttribute(bwd_kv_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kv_smem);
+  {
+    LaunchScope ls(kPhaseBwd, st);
+    bwd_kv_kernel<T><<<(unsigned)((long long)QT * BH * f.S), 256, kv_smem, st>>>(
+        q, k, v, dout, p.beta, lse, Drow, dkupd, dvupd, g, scale, QT, static_cast<T*>(p.dk), static_cast<T*>(p.dv));
+  }
+  // 6. dbeta
+  LaunchScope ls(kPhaseBwd, st);
+  bwd_beta_kernel<<<p.H, 256, 0, st>>>(brow, p.beta, p.B, p.H, p.L, p.dbeta);
+  return launch_status();
+}
+
+int backward_impl(const infini_attn_bwd_params& p) {
+  if (!p.q || !p.k || !p.v || !p.beta || !p.d_out || !p.dq || !p.dk || !p.dv || !p.dbeta) return INFINI_ERR_INVALID_ARG;
+  BwdPlan bp;
+  int rc = bwd_plan(p, &bp);
+  if (rc != INFINI_OK) return rc;
+  const bool f32 = bp.fwd.f32;
+  const size_t es = f32 ? 4 : 2;
+  const long long BH = (long long)p.B * p.H;
+  const size_t nq = (size_t)BH * p.L * p.d_k * es, nv = (size_t)BH * p.L * p.d_v * es;
+  // outputs must not overlap the inputs or one another
+  const void* outs[3] = {p.dq, p.dk, p.dv};
+  const size_t outn[3] = {nq, nq, nv};
+  const void* ins[4] = {p.q, p.k, p.v, p.d_out};
+  const size_t inn[4] = {nq, nq, nv, nv};
+  for (int a = 0; a < 3; ++a) {
+    for (int b = 0; b < 4; ++b)
+      if (ranges_overlap(outs[a], outn[a], ins[b], inn[b])) return INFINI_ERR_INVALID_ARG;
+    for (int b = a + 1; b < 3; ++b)
+      if (ranges_overlap(outs[a], outn[a], outs[b], outn[b])) return INFINI_ERR_INVALID_ARG;
+  }
+  if (p.workspace && (p.workspace_bytes < bp.total || reinterpret_cast<uintptr_t>(p.workspace) % kAlign != 0))
+    return INFINI_ERR_WORKSPACE;
+  rc = check_device(false);
+  if (rc != INFINI_OK) return rc;
+  char* ws = static_cast<char*>(p.workspace);
+  bool own = false;
+  if (!ws) {
+    void* w = nullptr;
+    if (cudaMallocAsync(&w, bp.total, p.stream) != cudaSuccess) {
+      cudaGetLastError();
+      return INFINI_ERR_WORKSPACE;
+    }
+    ws = static_cast<char*>(w);
+    own = true;
+  }
+  rc = f32 ? run_backward<float>(p, bp, ws) : run_backward<__nv_bfloat16>(p, bp, ws);
+  if (own && cudaFreeAsync(ws, p.stream) != cudaSuccess && rc == INFINI_OK) rc = INFINI_ERR_WORKSPACE;
+  return rc;
+}
+
 // ------------------------------------------------------------ fixed scratch
 // Workspace of infini_attn_forward_noalloc: one buffer per device, part of
 // the module image, so it exists from load to exit and no call allocates.
@@ -725,6 +945,17 @@ size_t infini_attn_workspace_size(int B, int H, long L, int N, int dk, int dv, i
   return std::max(pl.total, pl2.total);
 }
 
+
+int infini_attn_backward(const infini_attn_bwd_params* p) {
+  if (!p) return INFINI_ERR_INVALID_ARG;
+  return backward_impl(*p);
+}
+
+size_t infini_attn_backward_workspace_size(const infini_attn_bwd_params* p) {
+  if (!p) return 0;
+  BwdPlan bp;
+  return bwd_plan(*p, &bp) == INFINI_OK ? bp.total : 0;
+}
 
 size_t infini_attn_workspace_size_ex(const infini_attn_params* p) {
   if (!p) return 0;

@@ -213,7 +213,8 @@ __global__ void __launch_bounds__(256, 2) simt_attn_kernel(const T* __restrict__
                                                         T* __restrict__ out, Geo g, float scale, int QT,
                                                         const float* __restrict__ snapM,
                                                         const float* __restrict__ snapz,
-                                                        const T* __restrict__ qm) {
+                                                        const T* __restrict__ qm, float* __restrict__ adot_out,
+                                                        float* __restrict__ lse_out) {
   extern __shared__ float sm[];
   const int dk = g.dk, dv = g.dv, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int BHS = g.B * g.H * g.S;
@@ -321,12 +322,17 @@ __global__ void __launch_bounds__(256, 2) simt_attn_kernel(const T* __restrict__
     }
     const float inv_l = 1.f / l_i[rr];
     T* orow = out + off3(g.os, b, h, seg_start + qi);
+    // for the backward's recomputation: A_dot and log-sum-exp of the row,
+    // [B*H*L][dv] and [B*H*L] (contiguous), when asked for
+    const long long xrow = (long long)bh * g.L + seg_start + qi;
+    if (lse_out != nullptr && lane == 0) lse_out[xrow] = m_i[rr] + logf(l_i[rr]);
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       const int col = lane + 32 * c;
       if (col < dv) {
         const float a_mem = den != 0.f ? num[c] / den : 0.f;
         orow[col] = from_f32<T>(gw * a_mem + (1.f - gw) * (o[rr][c] * inv_l));
+        if (adot_out != nullptr) adot_out[xrow * dv + col] = o[rr][c] * inv_l;
       }
     }
   }

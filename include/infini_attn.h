@@ -258,6 +258,61 @@ INFINI_API size_t infini_attn_layer_workspace_size(int B, int H, long L, int N, 
 INFINI_API int infini_attn_gemm_bf16(const void* A, const void* B, void* C, long M, int N, int K,
                                      cudaStream_t stream);
 
+/*
+ * Backward pass: gradients of a scalar loss through infini_attn_forward, by
+ * back-propagation through time over the compressive memory (explainer page
+ * "Leave No Context Behind", section 3, "Training infrastructure"; the chain
+ * rule through Eq. 6-10 segment by segment in reverse, the forward's
+ * conventions kept: zero retrieval rows where a denominator is 0, sigma'(x) =
+ * 1 above zero and e^x at or below).  Given dLoss/d out and, optionally,
+ * dLoss/d M_S and dLoss/d z_S, returns dLoss/d q, k, v, beta and, optionally,
+ * dLoss/d M_0 and dLoss/d z_0.  The forward quantities it needs (the memory
+ * entering every segment, the local attention's output and row
+ * log-sum-exp) are recomputed from q, k, v, beta, M_0, z_0 inside the call.
+ *
+ * Layouts: q, k, dq, dk [B, H, L, dk]; v, d_out, dv [B, H, L, dv], all
+ * contiguous, bf16 or fp32 (mode | INFINI_F32, one type for all); beta,
+ * dbeta [H] fp32 (dbeta sums over the batch); M0, dM_S, dM0 [B, H, dk, dv]
+ * and z0, dz_S, dz0 [B, H, dk] fp32.  M0 / z0 NULL: the empty memory;
+ * dM_S / dz_S NULL: zero; dM0 / dz0 NULL: not returned.  Every pointer is
+ * caller-owned device memory; the inputs are read only, the outputs written.
+ * Arithmetic in fp32 (CUDA cores); no position embeddings.  Workspace as for
+ * the forward: taken on `stream` unless given
+ * (infini_attn_backward_workspace_size bytes, 256-byte aligned).  Errors as
+ * infini_attn_forward.
+ */
+typedef struct infini_attn_bwd_params {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* beta;
+  const float* M0;
+  const float* z0;
+  const void* d_out;
+  const float* dM_S;
+  const float* dz_S;
+  void* dq;
+  void* dk;
+  void* dv;
+  float* dbeta;
+  float* dM0;
+  float* dz0;
+  int B, H;
+  long long L;
+  int N;
+  int d_k, d_v;
+  int mode;    /* INFINI_LINEAR | INFINI_DELTA, optionally | INFINI_F32 */
+  float scale; /* softmax scale; 0 selects 1/sqrt(dk) */
+  void* workspace;
+  size_t workspace_bytes;
+  cudaStream_t stream;
+} infini_attn_bwd_params;
+
+INFINI_API int infini_attn_backward(const infini_attn_bwd_params* p);
+
+/* Bytes of workspace infini_attn_backward needs for p's shape and mode (0 if invalid). */
+INFINI_API size_t infini_attn_backward_workspace_size(const infini_attn_bwd_params* p);
+
 /* Static English text for a return code; never NULL. */
 INFINI_API const char* infini_attn_error_string(int code);
 
@@ -282,13 +337,13 @@ INFINI_API int infini_attn_selftest_timeout(unsigned limit_us, cudaStream_t stre
  * Kernel timing for benchmarks.  phase_mask selects phases (bit 0 = memory
  * update kernels, bit 1 = state/snapshot kernels, bit 2 = attention
  * kernel, bit 3 = position-embedding pre-pass, bit 4 = projection GEMMs of
- * the full layer); while a bit is set, every
+ * the full layer, bit 5 = backward kernels); while a bit is set, every
  * launch of that phase is bracketed by two CUDA events recorded on the
  * launch's stream.  0 turns timing off.
  */
 INFINI_API int infini_attn_profile_enable(int phase_mask);
 /*
- * Synchronises the recorded events and adds, per phase p in 0..4, the
+ * Synchronises the recorded events and adds, per phase p in 0..5, the
  * elapsed milliseconds to ms[p] and the number of timed launches to
  * launches[p], for everything recorded since the last reset; reset != 0
  * then drops the records.  Either array may be NULL.
