@@ -473,6 +473,8 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale, c
     aa.qms[i] = p.q_stride[i];
   }
   aa.qm = static_cast<const __nv_bfloat16*>(loc.qm);
+  aa.adot = nullptr;
+  aa.lse2 = nullptr;
   // Scheduling groups of GS segments: about one wave of CTAs per group.
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)

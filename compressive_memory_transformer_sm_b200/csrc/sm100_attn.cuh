@@ -44,6 +44,11 @@ struct AttnArgs {
   // Q tiles themselves.  qms: element strides of its (B, H, L) dimensions.
   const __nv_bfloat16* qm;
   long long qms[3];
+  // For the backward's recomputation (nullptr otherwise): A_dot of every row
+  // in bf16, contiguous [B*H*L][128], and the row's log2-sum-exp2 of the
+  // scaled scores (P = 2^(s * scale_log2 - lse2)), [B*H*L] fp32.
+  __nv_bfloat16* adot;
+  float* lse2;
 };
 
 // Shared memory of the attention kernel (offsets from a 1024-aligned base).
@@ -643,7 +648,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
           for (int e = 0; e < 8; ++e) dst[4 * c2 + e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
         }
+        if (a.adot != nullptr && valid) {
+          const float inv_l = 1.f / l;
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            pk[e] = pack_bf16x2(__uint_as_float(ro[2 * e]) * inv_l, __uint_as_float(ro[2 * e + 1]) * inv_l);
+          uint4* ad = reinterpret_cast<uint4*>(a.adot + (((long long)w.b * a.H + w.h) * a.L + w.seg0 + qrow) * 128);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) ad[4 * c2 + e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+        }
       }
+      if (a.lse2 != nullptr && valid) a.lse2[((long long)w.b * a.H + w.h) * a.L + w.seg0 + qrow] = m_ref + __log2f(l);
       // S_k and O_k are read out: the next item's products may overwrite them
       tc_fence_before();
       mbar_arrive(bar(B_OF0 + k));
