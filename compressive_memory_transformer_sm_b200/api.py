@@ -115,6 +115,7 @@ class InfiniAttnBwdParams(ctypes.Structure):
         ("dM_S", _vp), ("dz_S", _vp), ("dq", _vp), ("dk", _vp), ("dv", _vp), ("dbeta", _vp), ("dM0", _vp),
         ("dz0", _vp), ("B", _i), ("H", _i), ("L", _ll), ("N", _i), ("d_k", _i), ("d_v", _i), ("mode", _i),
         ("scale", ctypes.c_float), ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t), ("stream", _vp),
+        ("flags", _i),
     ]
 
 
@@ -314,8 +315,8 @@ def _ptr(t):
 
 
 def infini_attn_backward(q, k, v, beta, d_out, N: int, mode: int = LINEAR, M0=None, z0=None, dM_S=None, dz_S=None,
-                         want_state_grad: bool = True, scale: float = 0.0, workspace=None, stream=None,
-                         raise_on_error=True):
+                         want_state_grad: bool = True, scale: float = 0.0, workspace=None, flags: int = 0,
+                         stream=None, raise_on_error=True):
     """Gradients through the forward: returns (dq, dk, dv, dbeta, dM0, dz0) as new device tensors
     (dM0, dz0 are None unless ``want_state_grad``).  q, k [B,H,L,dk], v, d_out [B,H,L,dv] contiguous,
     one dtype (bf16 or fp32); beta [H]; M0, dM_S [B,H,dk,dv], z0, dz_S [B,H,dk] fp32 or None."""
@@ -343,14 +344,16 @@ def infini_attn_backward(q, k, v, beta, d_out, N: int, mode: int = LINEAR, M0=No
         p.workspace = workspace.data_ptr()
         p.workspace_bytes = workspace.numel() * workspace.element_size()
     p.stream = _stream(stream)
+    p.flags = int(flags)
     rc = lib.infini_attn_backward(ctypes.byref(p))
     _check(rc, "infini_attn_backward", raise_on_error)
     return dq, dk_, dv_, dbeta, dM0, dz0
 
 
-def infini_attn_backward_workspace_size(B, H, L, N, dk, dv, mode=LINEAR) -> int:
+def infini_attn_backward_workspace_size(B, H, L, N, dk, dv, mode=LINEAR, flags: int = 0) -> int:
     p = InfiniAttnBwdParams()
     p.B, p.H, p.L, p.N, p.d_k, p.d_v, p.mode = int(B), int(H), int(L), int(N), int(dk), int(dv), int(mode)
+    p.flags = int(flags)
     return int(lib.infini_attn_backward_workspace_size(ctypes.byref(p)))
 
 

@@ -208,6 +208,113 @@ __global__ void __launch_bounds__(256, 2)
   }
 }
 
+// The memory read's backward (Eq. 7) and the per-row terms for the tensor-core
+// path, where the local attention's gradients come from the tcgen05 kernels:
+// for 128 query rows of one (b, h, segment) (four passes of 32; warp w: rows
+// 4w .. 4w+3 of a pass, lane = column), D'_i = dO_i . A_dot_i (A_dot bf16
+// from the forward), the dbeta row term dO_i . (A_mem_i - A_dot_i), and
+// dq_mem = sigma'(q) (d_num M^T + d_den z) with d_num, d_den rows written for
+// the memory chain.  M^(s) is staged in shared memory once per block.
+template <typename T>
+__global__ void __launch_bounds__(256, 2) bwd_qmem_kernel(const T* __restrict__ q, const T* __restrict__ dout,
+                                                       const __nv_bfloat16* __restrict__ adot,
+                                                       const float* __restrict__ beta,
+                                                       const float* __restrict__ snapM,
+                                                       const float* __restrict__ snapz, BwdGeo g,
+                                                       int blocks_per_seg, float* __restrict__ dq_mem,
+                                                       float* __restrict__ Dp, float* __restrict__ brow,
+                                                       float* __restrict__ dnum, float* __restrict__ dden) {
+  extern __shared__ float sm[];
+  const int dk = g.dk, dv = g.dv, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  int idx = blockIdx.x;
+  const int blk = idx % blocks_per_seg;
+  idx /= blocks_per_seg;
+  const int s = idx % g.S;
+  const int bh = idx / g.S;
+  const int h = bh % g.H;
+  const long long seg_start = (long long)s * g.N;
+  const int n_s = (int)min((long long)g.N, g.L - seg_start);
+  const int r0 = blk * 128;
+  if (r0 >= n_s) return;
+  const int rend = min(n_s, r0 + 128);
+  const float gw = 1.f / (1.f + expf(-beta[h]));
+  float* Ms = sm;                  // [dk][dv + 1]
+  float* zs = Ms + dk * (dv + 1);  // [dk]
+  float* sq = zs + dk;             // [8 warps][dk] sigma(q) of the warp's current row
+  float* wn = sq + 8 * dk;         // [8 warps][dv] d_num of the warp's current row
+  const float* Mp = snapM + ((long long)bh * g.S + s) * dk * dv;
+  for (int e = tid; e < dk * dv; e += 256) Ms[(e / dv) * (dv + 1) + e % dv] = Mp[e];
+  for (int e = tid; e < dk; e += 256) zs[e] = snapz[((long long)bh * g.S + s) * dk + e];
+  __syncthreads();
+  float* sqw = sq + warp * dk;
+  float* wnw = wn + warp * dv;
+  for (int t = r0 + warp; t < rend; t += 8) {  // one row per warp at a time
+    const long long row = bwd_row(g, bh, seg_start + t);
+    float xq[4];
+    float dpart = 0.f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int i = lane + 32 * c;
+      xq[c] = i < dk ? to_f32(q[row * dk + i]) : 0.f;
+      if (i < dk) {
+        const float sg = elu1_accurate(xq[c]);
+        sqw[i] = sg;
+        dpart = fmaf(sg, zs[i], dpart);
+      }
+    }
+    const float den = warp_sum(dpart);
+    __syncwarp();
+    float num[4] = {0.f, 0.f, 0.f, 0.f};
+    if (den != 0.f) {
+      for (int i = 0; i < dk; ++i) {
+        const float si = sqw[i];
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          if (lane + 32 * c < dv) num[c] = fmaf(si, Ms[i * (dv + 1) + lane + 32 * c], num[c]);
+      }
+    }
+    float dd = 0.f, bterm = 0.f, dpr = 0.f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int j = lane + 32 * c;
+      if (j < dv) {
+        const float dA = to_f32(dout[row * dv + j]);
+        const float ad = __bfloat162float(adot[row * dv + j]);
+        const float am = den != 0.f ? num[c] / den : 0.f;
+        dpr = fmaf(dA, ad, dpr);
+        bterm = fmaf(dA, am - ad, bterm);
+        float w = 0.f;
+        if (den != 0.f) {
+          w = gw * dA / den;
+          dd = fmaf(gw * dA, am, dd);
+        }
+        wnw[j] = w;
+        dnum[row * dv + j] = w;
+      }
+    }
+    const float d_den = den != 0.f ? -warp_sum(dd) / den : 0.f;
+    dpr = warp_sum(dpr);
+    bterm = warp_sum(bterm);
+    if (lane == 0) {
+      Dp[row] = dpr;
+      brow[row] = bterm;
+      dden[row] = d_den;
+    }
+    __syncwarp();
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int i = lane + 32 * c;
+      if (i < dk) {
+        float a = d_den * zs[i];
+        if (den != 0.f)
+          for (int j = 0; j < dv; ++j) a = fmaf(wnw[j], Ms[i * (dv + 1) + j], a);
+        dq_mem[row * dk + i] = sigma_prime(xq[c]) * a;
+      }
+    }
+    __syncwarp();
+  }
+}
+
 // Partials of sigma(X)^T Y (dk x dy) and sigma(X)^T y0 (dk) for the rows of
 // one (b, h, segment, token group); layout [BH][nseg][G][dk*dy + dk] like the
 // forward's update partials.  Rows of X: element strides given by rows of

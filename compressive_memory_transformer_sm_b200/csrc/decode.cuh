@@ -1,9 +1,9 @@
-// decode_kernel: token-level streaming decode of the Infini-attention layer.
-// One new query row per (b, h) against the cached keys 0..n-1 of its current
-// segment (local causal attention, Eq. 6, for one row), the memory read with
-// the live M, z = M_{s-1}, z_{s-1} (Eq. 7) and the gate (Eq. 10), in fp32 on
-// CUDA cores.  The work is one matrix-vector product per (b, h): bound by
-// reading the n (dk + dv) cached elements, and by latency at small B * H.
+// Token-level streaming decode of the Infini-attention layer: one new query
+// row per (b, h) against the cached keys 0..n-1 of its current segment (local
+// causal attention, Eq. 6, for one row), the memory read with the live
+// M, z = M_{s-1}, z_{s-1} (Eq. 7) and the gate (Eq. 10), in fp32 on CUDA
+// cores.  The work is one matrix-vector product per (b, h): bound by reading
+// the n (dk + dv) cached elements, and by latency at small B * H.
 #pragma once
 
 #include "common.cuh"
@@ -11,43 +11,63 @@
 
 namespace infini {
 
-constexpr int kDecodeWarps = 8;
 
-// Block = 8 warps per (b, h): warp w takes keys w, w + 8, ...; lanes split the
-// head dimensions (lane + 32 c); each warp keeps its own running max, sum and
-// output row, merged in a fixed order at the end (deterministic).
+// ------------------------------------------------------------------ split decode
+// The same step spread over many CTAs: the keys 0..n-1 of a (b, h) are cut
+// into `splits` ranges, one CTA each (grid B*H x splits), so a short batch
+// still fills the GPU.  Each range yields a partial softmax state -- running
+// max m, sum l and unnormalised output o -- that decode_merge_kernel combines
+// in a fixed order (deterministic), adding the memory read and the gate.
+// Key n - 1 is the new token: read from k_t, v_t, which CTA 0 of the (b, h)
+// also appends to the caches (row n - 1); no CTA of the launch reads that row.
 template <typename T>
-__global__ void __launch_bounds__(32 * kDecodeWarps)
-    decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* __restrict__ vc,
-                  const float* __restrict__ beta, const float* __restrict__ M, const float* __restrict__ z,
-                  T* __restrict__ out, int H, int N, int n, int dk, int dv, float scale) {
-  __shared__ float qs[128], sq[128];
-  __shared__ float wm[kDecodeWarps], wl[kDecodeWarps], wacc[kDecodeWarps][128];
-  __shared__ float den_s;
-  const int bh = blockIdx.x, h = bh % H;
+__global__ void __launch_bounds__(256)
+    decode_part_kernel(const T* __restrict__ q, const T* __restrict__ k_t, const T* __restrict__ v_t,
+                       T* __restrict__ kc, T* __restrict__ vc, int N, int n, int dk, int dv, float scale, int per,
+                       float* __restrict__ part) {
+  __shared__ float qs[128];
+  __shared__ float wm[8], wl[8], wacc[8][128];
+  const int bh = blockIdx.x, split = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const T* qrow = q + (long long)bh * dk;
-  for (int i = tid; i < dk; i += blockDim.x) {
-    const float x = to_f32(qrow[i]);
-    qs[i] = x;
-    sq[i] = elu1_accurate(x);
+  const long long BH = gridDim.x;
+  if (split == 0) {  // append the token to the caches
+    for (int i = tid; i < dk; i += 256) kc[((long long)bh * N + n - 1) * dk + i] = k_t[(long long)bh * dk + i];
+    for (int i = tid; i < dv; i += 256) vc[((long long)bh * N + n - 1) * dv + i] = v_t[(long long)bh * dv + i];
   }
+  for (int i = tid; i < dk; i += 256) qs[i] = to_f32(q[(long long)bh * dk + i]);
   __syncthreads();
+  const int j0 = split * per, j1 = min(n, j0 + per);
   const T* kb = kc + (long long)bh * N * dk;
   const T* vb = vc + (long long)bh * N * dv;
+  // warp w: keys j0 + 32 w' + lane for w' = w, w + 8, ... (a lane per key for the
+  // scores, then a lane per column for the weighted sum of the 32 value rows)
   float m = -INFINITY, l = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int j = warp; j < n; j += kDecodeWarps) {
-    float s = 0.f;
-    for (int i = lane; i < dk; i += 32) s = fmaf(qs[i], to_f32(kb[(long long)j * dk + i]), s);
-    s = warp_sum(s) * scale;
-    const float mn = fmaxf(m, s);
-    const float alpha = expf(m - mn);  // 0 for the first key (m = -inf)
-    const float p = expf(s - mn);
-    l = l * alpha + p;
+  for (int jb = j0 + 32 * warp; jb < j1; jb += 256) {
+    const int j = jb + lane;
+    float s = -INFINITY;
+    if (j < j1) {
+      const T* kr = j == n - 1 ? k_t + (long long)bh * dk : kb + (long long)j * dk;
+      float d = 0.f;
+      for (int i = 0; i < dk; ++i) d = fmaf(qs[i], to_f32(kr[i]), d);
+      s = d * scale;
+    }
+    const float mx = warp_max(s);
+    const float mn = fmaxf(m, mx);
+    const float alpha = expf(m - mn);  // 0 while m = -inf
+    const float p = j < j1 ? expf(s - mn) : 0.f;
+    l = l * alpha + warp_sum(p);
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int d = lane + 32 * c;
-      if (d < dv) acc[c] = fmaf(p, to_f32(vb[(long long)j * dv + d]), acc[c] * alpha);
+    for (int c = 0; c < 4; ++c) acc[c] *= alpha;
+    const int cnt = min(32, j1 - jb);
+    for (int jj = 0; jj < cnt; ++jj) {
+      const float pj = __shfl_sync(0xffffffffu, p, jj);
+      const int key = jb + jj;
+      const T* vr = key == n - 1 ? v_t + (long long)bh * dv : vb + (long long)key * dv;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int d = lane + 32 * c;
+        if (d < dv) acc[c] = fmaf(pj, to_f32(vr[d]), acc[c]);
+      }
     }
     m = mn;
   }
@@ -56,30 +76,64 @@ __global__ void __launch_bounds__(32 * kDecodeWarps)
     wl[warp] = l;
   }
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    const int d = lane + 32 * c;
-    if (d < dv) wacc[warp][d] = acc[c];
-  }
-  const float* Mh = M + (long long)bh * dk * dv;
-  const float* zh = z + (long long)bh * dk;
-  if (warp == 0) {
-    float d = 0.f;
-    for (int i = lane; i < dk; i += 32) d = fmaf(sq[i], zh[i], d);
-    d = warp_sum(d);
-    if (lane == 0) den_s = d;
-  }
+  for (int c = 0; c < 4; ++c)
+    if (lane + 32 * c < dv) wacc[warp][lane + 32 * c] = acc[c];
   __syncthreads();
+  // the block's state: merge the eight warps in order
   float gm = -INFINITY;
-  for (int w = 0; w < kDecodeWarps; ++w) gm = fmaxf(gm, wm[w]);
+  for (int w = 0; w < 8; ++w) gm = fmaxf(gm, wm[w]);
+  float* out = part + ((long long)split * BH + bh) * (dv + 2);
+  if (tid == 0) {
+    float gl = 0.f;
+    for (int w = 0; w < 8; ++w) gl += gm == -INFINITY ? 0.f : wl[w] * expf(wm[w] - gm);
+    out[0] = gm;
+    out[1] = gl;
+  }
+  for (int c = tid; c < dv; c += 256) {
+    float o = 0.f;
+    for (int w = 0; w < 8; ++w) o += gm == -INFINITY ? 0.f : wacc[w][c] * expf(wm[w] - gm);
+    out[2 + c] = o;
+  }
+}
+
+// One block per (b, h), a thread per output column: the ranges' states merged
+// in split order, the memory read sigma(q) M / sigma(q) z (Eq. 7, 0 when the
+// denominator is 0) and the gate (Eq. 10).
+template <typename T>
+__global__ void __launch_bounds__(128)
+    decode_merge_kernel(const T* __restrict__ q, const float* __restrict__ beta, const float* __restrict__ M,
+                        const float* __restrict__ z, const float* __restrict__ part, int splits, int H, int dk, int dv,
+                        T* __restrict__ out) {
+  __shared__ float sq[128];
+  __shared__ float red[4];
+  const int bh = blockIdx.x, h = bh % H, tid = threadIdx.x;
+  const long long BH = gridDim.x;
+  for (int i = tid; i < dk; i += 128) sq[i] = elu1_accurate(to_f32(q[(long long)bh * dk + i]));
+  __syncthreads();
+  const float* zh = z + (long long)bh * dk;
+  float d = 0.f;
+  for (int i = tid; i < dk; i += 128) d = fmaf(sq[i], zh[i], d);
+  d = warp_sum(d);
+  if ((tid & 31) == 0) red[tid >> 5] = d;
+  __syncthreads();
+  const float den = (red[0] + red[1]) + (red[2] + red[3]);
+  float gm = -INFINITY;
+  for (int sp = 0; sp < splits; ++sp) gm = fmaxf(gm, part[((long long)sp * BH + bh) * (dv + 2)]);
   float gl = 0.f;
-  for (int w = 0; w < kDecodeWarps; ++w) gl += wl[w] * expf(wm[w] - gm);  // a warp without keys adds 0
+  for (int sp = 0; sp < splits; ++sp) {
+    const float* ps = part + ((long long)sp * BH + bh) * (dv + 2);
+    gl += ps[0] == -INFINITY ? 0.f : ps[1] * expf(ps[0] - gm);
+  }
   const float g = 1.f / (1.f + expf(-beta[h]));
-  const float den = den_s;
-  for (int c = tid; c < dv; c += blockDim.x) {
+  const float* Mh = M + (long long)bh * dk * dv;
+  for (int c = tid; c < dv; c += 128) {
+    float o = 0.f;
+    for (int sp = 0; sp < splits; ++sp) {
+      const float* ps = part + ((long long)sp * BH + bh) * (dv + 2);
+      o += ps[0] == -INFINITY ? 0.f : ps[2 + c] * expf(ps[0] - gm);
+    }
     float num = 0.f;
     for (int i = 0; i < dk; ++i) num = fmaf(sq[i], Mh[(long long)i * dv + c], num);
-    float o = 0.f;
-    for (int w = 0; w < kDecodeWarps; ++w) o = fmaf(wacc[w][c], expf(wm[w] - gm), o);
     const float a_mem = den != 0.f ? num / den : 0.f;
     out[(long long)bh * dv + c] = from_f32<T>(g * a_mem + (1.f - g) * (o / gl));
   }

@@ -34,6 +34,7 @@
 #include "sm100_attn.cuh"
 #include "sm100_update.cuh"
 #include "sm100_gemm.cuh"
+#include "sm100_bwd.cuh"
 
 namespace infini {
 namespace {
@@ -42,6 +43,9 @@ constexpr int kChunk = 128;        // tokens per update chunk
 constexpr int kSms = 148;          // B200 SM count: grid sizing (device independent, so plans are too)
 constexpr int kTargetCtas = 4 * kSms;  // CUDA-core update grid size aim
 constexpr size_t kAlign = 256;
+// Internal flag of forward_impl (not in the header): run the memory update
+// only -- no attention launch, no output -- for the decode step's fold.
+constexpr int kFlagUpdateOnly = 0x1000;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
@@ -260,16 +264,21 @@ int run_rope(const infini_attn_params& p, char* dst, LocalQK* loc) {
   for (int i = 0; i < 3; ++i)
     vec = vec && (p.q_stride[i] * (long long)es) % 16 == 0 && (p.k_stride[i] * (long long)es) % 16 == 0;
   const int E = vec ? 8 : 2;
-  const long long work = (long long)p.B * p.H * p.L * (p.dk / E);
-  const unsigned blocks = (unsigned)std::max<long long>(1, std::min<long long>((work + 255) / 256, 8LL * kSms));
+  // block: the dk / E element groups of rows_per tokens; grid: tokens x heads
+  const int groups = p.dk / E;
+  const int rows_per = std::max(1, 256 / groups);
+  const long long bx = (p.L + rows_per - 1) / rows_per;
+  if (bx >= (1LL << 31)) return INFINI_ERR_UNSUPPORTED;
+  const dim3 block((unsigned)groups, (unsigned)rows_per);
+  const dim3 grid((unsigned)bx, (unsigned)std::min<long long>((long long)p.B * p.H, 65535));
   {
     LaunchScope ls(kPhasePre, p.stream);
     if (f32) {
-      if (vec) rope_kernel<float, 8><<<blocks, 256, 0, p.stream>>>(ra);
-      else rope_kernel<float, 2><<<blocks, 256, 0, p.stream>>>(ra);
+      if (vec) rope_kernel<float, 8><<<grid, block, 0, p.stream>>>(ra);
+      else rope_kernel<float, 2><<<grid, block, 0, p.stream>>>(ra);
     } else {
-      if (vec) rope_kernel<__nv_bfloat16, 8><<<blocks, 256, 0, p.stream>>>(ra);
-      else rope_kernel<__nv_bfloat16, 2><<<blocks, 256, 0, p.stream>>>(ra);
+      if (vec) rope_kernel<__nv_bfloat16, 8><<<grid, block, 0, p.stream>>>(ra);
+      else rope_kernel<__nv_bfloat16, 2><<<grid, block, 0, p.stream>>>(ra);
     }
   }
   loc->q = ra.qr;
@@ -325,6 +334,7 @@ int run_simt(const infini_attn_params& p, const Plan& pl, char* ws, float scale,
                                                 snapz);
     }
   }
+  if (p.flags & kFlagUpdateOnly) return launch_status();
   const int QT = (p.N + 31) / 32;
   const size_t attn_smem = (size_t)(32 * (p.dk + 1) + 32 * p.dv + 32 * p.dk) * 4;
   cudaFuncSetAttribute(simt_attn_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)attn_smem);
@@ -357,6 +367,10 @@ int set_tc_smem_limits() {
       cudaFuncSetAttribute(tc::mem_update_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)tc::UpdSmem<true>::BYTES) != cudaSuccess ||
       cudaFuncSetAttribute(tc::gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kGemmSmem) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(tc::bwd_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kDQSmem) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(tc::bwd_dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kKVSmem) !=
           cudaSuccess)
     return INFINI_ERR_LAUNCH;
   if (ctx != 0) done.push_back(ctx);
@@ -412,7 +426,15 @@ int gemm_tc(const void* A, long long lda, const void* Bm, long long ldb, void* C
   return launch_status();
 }
 
-int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale, const LocalQK& loc) {
+// Extra outputs of a forward run for the backward's recomputation.
+struct FwdExtra {
+  float* snapM32;       // fp32 [BH][S][dk][dv] snapshots of M^(s)
+  __nv_bfloat16* adot;  // [B*H*L][128] A_dot
+  float* lse2;          // [B*H*L] row log2-sum-exp2 of the scaled scores
+};
+
+int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale, const LocalQK& loc,
+           const FwdExtra* extra = nullptr) {
   // tm_k: the keys of the memory update (un-rotated); tm_qa / tm_ka: the
   // local attention's queries and keys
   CUtensorMap tm_qa, tm_k, tm_ka, tm_v, tm_mt;
@@ -428,6 +450,7 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale, c
   const dim3 sgrid((E + 128 + 255) / 256, BH);
   tc::UpdArgs ua;
   ua.partial = part; ua.M = p.M; ua.z = p.z; ua.snapM = snapM16; ua.snapzw = snapz;
+  ua.snapM32 = extra ? extra->snapM32 : nullptr;
   ua.B = p.B; ua.H = p.H; ua.S = pl.S; ua.N = p.N; ua.L = p.L;
   ua.G = pl.G; ua.cpb = pl.cpb;
   if (!pl.delta) {
@@ -438,8 +461,8 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale, c
           tm_k, tm_v, ua);
     }
     LaunchScope ls(kPhaseState, p.stream);
-    state_kernel<<<sgrid, 256, 0, p.stream>>>(p.M, p.z, part, 128, 128, pl.S, 0, 0, pl.S, pl.G, nullptr, snapM16,
-                                              snapz);
+    state_kernel<<<sgrid, 256, 0, p.stream>>>(p.M, p.z, part, 128, 128, pl.S, 0, 0, pl.S, pl.G,
+                                              extra ? extra->snapM32 : nullptr, snapM16, snapz);
   } else {
     ua.nseg = 1;
     // one cluster of G CTAs per head; G <= 8 (plan)
@@ -464,6 +487,7 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale, c
         return INFINI_ERR_LAUNCH;
     }
   }
+  if (p.flags & kFlagUpdateOnly) return launch_status();
   tc::AttnArgs aa;
   aa.beta = p.beta; aa.snapz = snapz; aa.out = static_cast<__nv_bfloat16*>(p.out);
   aa.B = p.B; aa.H = p.H; aa.S = pl.S; aa.T = (p.N + 127) / 128; aa.L = p.L; aa.N = p.N;
@@ -473,8 +497,8 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale, c
     aa.qms[i] = p.q_stride[i];
   }
   aa.qm = static_cast<const __nv_bfloat16*>(loc.qm);
-  aa.adot = nullptr;
-  aa.lse2 = nullptr;
+  aa.adot = extra ? extra->adot : nullptr;
+  aa.lse2 = extra ? extra->lse2 : nullptr;
   // Scheduling groups of GS segments: about one wave of CTAs per group.
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
@@ -514,7 +538,8 @@ bool tc_layout_ok(const infini_attn_params& p) {
 }
 
 int forward_impl(infini_attn_params p) {
-  if (!p.q || !p.k || !p.v || !p.beta || !p.M || !p.z || !p.out) return INFINI_ERR_INVALID_ARG;
+  const bool update_only = (p.flags & kFlagUpdateOnly) != 0;
+  if (!p.q || !p.k || !p.v || !p.beta || !p.M || !p.z || (!p.out && !update_only)) return INFINI_ERR_INVALID_ARG;
   Plan pl;
   int rc = make_plan(p.B, p.H, p.L, p.N, p.dk, p.dv, p.mode, p.flags, &pl);
   if (rc != INFINI_OK) return rc;
@@ -534,7 +559,7 @@ int forward_impl(infini_attn_params p) {
     if (p.q_stride[i] < 0 || p.k_stride[i] < 0 || p.v_stride[i] < 0 || p.o_stride[i] <= 0)
       return INFINI_ERR_INVALID_ARG;
   const size_t es = pl.f32 ? 4 : 2;
-  const size_t out_ext = extent_bytes(p.o_stride, p.B, p.H, p.L, p.dv, es);
+  const size_t out_ext = update_only ? 0 : extent_bytes(p.o_stride, p.B, p.H, p.L, p.dv, es);
   if (ranges_overlap(p.out, out_ext, p.q, extent_bytes(p.q_stride, p.B, p.H, p.L, p.dk, es)) ||
       ranges_overlap(p.out, out_ext, p.k, extent_bytes(p.k_stride, p.B, p.H, p.L, p.dk, es)) ||
       ranges_overlap(p.out, out_ext, p.v, extent_bytes(p.v_stride, p.B, p.H, p.L, p.dv, es)) ||
@@ -608,15 +633,21 @@ __global__ void selftest_wait_kernel(unsigned long long limit_ns) {
 // snapshots (linear) or running value (delta), and the update's dk, dv terms.
 struct BwdPlan {
   Plan fwd;
+  bool tc;  // tensor-core local-attention gradients (bf16, dk = dv = 128)
   int Gc, cpbc, Gu, cpbu;
   size_t off_fwd, off_state, off_out, off_adot, off_lse, off_D, off_brow, off_dden, off_ddenr, off_dnum, off_dnumr,
-      off_cpart, off_upart, off_g, off_dkupd, off_dvupd, total;
+      off_cpart, off_upart, off_g, off_dkupd, off_dvupd, off_snap32, off_dqmem, total;
 };
 
 int bwd_plan(const infini_attn_bwd_params& p, BwdPlan* bp) {
   if (p.B <= 0 || p.H <= 0 || p.L <= 0 || p.N <= 0 || p.d_k <= 0 || p.d_v <= 0) return INFINI_ERR_INVALID_ARG;
-  int rc = make_plan(p.B, p.H, p.L, p.N, p.d_k, p.d_v, p.mode, INFINI_FLAG_FORCE_SIMT, &bp->fwd);
+  int rc = make_plan(p.B, p.H, p.L, p.N, p.d_k, p.d_v, p.mode, p.flags & INFINI_FLAG_FORCE_SIMT, &bp->fwd);
   if (rc != INFINI_OK) return rc;
+  bp->tc = bp->fwd.tc;
+  if (!bp->tc && !(p.flags & INFINI_FLAG_FORCE_SIMT)) {
+    rc = make_plan(p.B, p.H, p.L, p.N, p.d_k, p.d_v, p.mode, INFINI_FLAG_FORCE_SIMT, &bp->fwd);
+    if (rc != INFINI_OK) return rc;
+  }
   const Plan& f = bp->fwd;
   const long long BH = (long long)p.B * p.H, rows = BH * p.L;
   if (rows >= (1LL << 40)) return INFINI_ERR_UNSUPPORTED;
@@ -639,7 +670,7 @@ int bwd_plan(const infini_attn_bwd_params& p, BwdPlan* bp) {
   bp->off_fwd = take(f.total);
   bp->off_state = take((size_t)BH * (E + p.d_k) * 4);
   bp->off_out = take((size_t)rows * p.d_v * es);
-  bp->off_adot = take((size_t)rows * p.d_v * 4);
+  bp->off_adot = take((size_t)rows * p.d_v * (bp->tc ? 2 : 4));
   bp->off_lse = take((size_t)rows * 4);
   bp->off_D = take((size_t)rows * 4);
   bp->off_brow = take((size_t)rows * 4);
@@ -652,6 +683,8 @@ int bwd_plan(const infini_attn_bwd_params& p, BwdPlan* bp) {
   bp->off_g = take((size_t)BH * (f.delta ? 1 : f.S) * (E + p.d_k) * 4);
   bp->off_dkupd = take((size_t)rows * p.d_k * 4);
   bp->off_dvupd = take((size_t)rows * p.d_v * 4);
+  bp->off_snap32 = take(bp->tc ? (size_t)BH * f.S * E * 4 : 0);
+  bp->off_dqmem = take(bp->tc ? (size_t)rows * p.d_k * 4 : 0);
   bp->total = off;
   return INFINI_OK;
 }
@@ -687,9 +720,21 @@ int run_backward(const infini_attn_bwd_params& p, const BwdPlan& bp, char* ws) {
   float* adot = reinterpret_cast<float*>(ws + bp.off_adot);
   float* lse = reinterpret_cast<float*>(ws + bp.off_lse);
   char* fws = ws + bp.off_fwd;
-  int rc = run_simt<T>(fp, f, fws, scale, loc, adot, lse);
+  int rc;
+  const float* snapM;
+  if (bp.tc) {
+    // tensor-core forward: A_dot in bf16, lse in log2 units, fp32 snapshots of M^(s)
+    FwdExtra ex;
+    ex.snapM32 = reinterpret_cast<float*>(ws + bp.off_snap32);
+    ex.adot = reinterpret_cast<__nv_bfloat16*>(ws + bp.off_adot);
+    ex.lse2 = lse;
+    rc = run_tc(fp, f, fws, scale, loc, &ex);
+    snapM = ex.snapM32;
+  } else {
+    rc = run_simt<T>(fp, f, fws, scale, loc, adot, lse);
+    snapM = reinterpret_cast<const float*>(fws + f.off_snapM);
+  }
   if (rc != INFINI_OK) return rc;
-  const float* snapM = reinterpret_cast<const float*>(fws + f.off_snapM);
   const float* snapz = reinterpret_cast<const float*>(fws + f.off_snapz);
   BwdGeo g;
   g.B = p.B; g.H = p.H; g.S = f.S; g.N = p.N; g.dk = dk; g.dv = dv; g.L = p.L;
@@ -710,9 +755,37 @@ int run_backward(const infini_attn_bwd_params& p, const BwdPlan& bp, char* ws) {
   float* dvupd = reinterpret_cast<float*>(ws + bp.off_dvupd);
   // 2. dq, D, the dbeta row terms, d_num and d_den rows
   const int QT = (p.N + 31) / 32;
-  const size_t q_smem = (size_t)(32 * (dk + 1) + 32 * dv + 32 * dk + 2 * 32 * dv) * 4;
-  cudaFuncSetAttribute(bwd_q_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)q_smem);
-  {
+  const int bps = (int)((std::min<long long>(p.N, p.L) + 127) / 128);
+  CUtensorMap tm_q, tm_k, tm_v, tm_do;
+  tc::BwdTcArgs ta;
+  float* dqmem = reinterpret_cast<float*>(ws + bp.off_dqmem);
+  if (bp.tc) {
+    if (!encode_bhld(&tm_q, p.q, p.B, p.H, p.L, cst[0]) || !encode_bhld(&tm_k, p.k, p.B, p.H, p.L, cst[0]) ||
+        !encode_bhld(&tm_v, p.v, p.B, p.H, p.L, cst[1]) || !encode_bhld(&tm_do, p.d_out, p.B, p.H, p.L, cst[1]))
+      return INFINI_ERR_LAUNCH;
+    if (set_tc_smem_limits() != INFINI_OK) return INFINI_ERR_LAUNCH;
+    // the memory read's backward and D' = dO . A_dot on CUDA cores
+    const size_t qm_smem = (size_t)(dk * (dv + 1) + dk + 8 * dk + 8 * dv) * 4;
+    cudaFuncSetAttribute(bwd_qmem_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qm_smem);
+    {
+      LaunchScope ls(kPhaseBwd, st);
+      bwd_qmem_kernel<T><<<(unsigned)((long long)BH * f.S * bps), 256, qm_smem, st>>>(
+          q, dout, reinterpret_cast<const __nv_bfloat16*>(ws + bp.off_adot), p.beta, snapM, snapz, g, bps, dqmem,
+          Drow, brow, dnum, dden);
+    }
+    memset(&ta, 0, sizeof(ta));
+    ta.lse2 = lse; ta.Dp = Drow; ta.beta = p.beta; ta.mem_q = dqmem;
+    ta.mem_k = reinterpret_cast<float*>(ws + bp.off_dkupd);
+    ta.mem_v = reinterpret_cast<float*>(ws + bp.off_dvupd);
+    ta.B = p.B; ta.H = p.H; ta.S = f.S; ta.T = (p.N + 127) / 128; ta.L = p.L; ta.N = p.N;
+    ta.scale = scale; ta.scale_log2 = scale * 1.4426950408889634f;
+    ta.out0 = static_cast<__nv_bfloat16*>(p.dq);
+    LaunchScope ls(kPhaseBwd, st);
+    tc::bwd_dq_tc_kernel<<<(unsigned)((long long)ta.T * BH * f.S), tc::kBwdThreads, tc::kDQSmem, st>>>(tm_q, tm_k, tm_v,
+                                                                                                    tm_do, ta);
+  } else {
+    const size_t q_smem = (size_t)(32 * (dk + 1) + 32 * dv + 32 * dk + 2 * 32 * dv) * 4;
+    cudaFuncSetAttribute(bwd_q_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)q_smem);
     LaunchScope ls(kPhaseBwd, st);
     bwd_q_kernel<T><<<(unsigned)((long long)QT * BH * f.S), 256, q_smem, st>>>(
         q, k, v, dout, p.beta, adot, lse, snapM, snapz, g, scale, QT, static_cast<T*>(p.dq), Drow, brow, dnum, dden);
@@ -727,7 +800,6 @@ int run_backward(const infini_attn_bwd_params& p, const BwdPlan& bp, char* ws) {
   }
   const dim3 sgrid((unsigned)((E + dk + 255) / 256), BH);
   const size_t pst = E + dk;
-  const int bps = (std::min(p.N, (int)std::min<long long>(p.N, p.L)) + 127) / 128;
   const size_t upd_smem = (size_t)((f.delta ? 2 : 1) * dk * (dv + 1) + 2 * dk + 32 * dk + 2 * 32 * dv) * 4;
   cudaFuncSetAttribute(bwd_upd_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)upd_smem);
   // 4. the memory-gradient chain and the update's dk, dv terms
@@ -766,9 +838,15 @@ int run_backward(const infini_attn_bwd_params& p, const BwdPlan& bp, char* ws) {
                                             p.dM0, p.dz0);
   }
   // 5. dk, dv of the local attention plus the update's terms
-  const size_t kv_smem = (size_t)(32 * dk + 32 * dv + 32 * (dk + 1) + 32 * (dv + 1) + 64) * 4;
-  cudaFuncSetAttribute(bwd_kv_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kv_smem);
-  {
+  if (bp.tc) {
+    ta.out0 = static_cast<__nv_bfloat16*>(p.dk);
+    ta.out1 = static_cast<__nv_bfloat16*>(p.dv);
+    LaunchScope ls(kPhaseBwd, st);
+    tc::bwd_dkdv_tc_kernel<<<(unsigned)((long long)ta.T * BH * f.S), tc::kBwdThreads, tc::kKVSmem, st>>>(
+        tm_q, tm_k, tm_v, tm_do, ta);
+  } else {
+    const size_t kv_smem = (size_t)(32 * dk + 32 * dv + 32 * (dk + 1) + 32 * (dv + 1) + 64) * 4;
+    cudaFuncSetAttribute(bwd_kv_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kv_smem);
     LaunchScope ls(kPhaseBwd, st);
     bwd_kv_kernel<T><<<(unsigned)((long long)QT * BH * f.S), 256, kv_smem, st>>>(
         q, k, v, dout, p.beta, lse, Drow, dkupd, dvupd, g, scale, QT, static_cast<T*>(p.dk), static_cast<T*>(p.dv));
@@ -798,6 +876,16 @@ int backward_impl(const infini_attn_bwd_params& p) {
       if (ranges_overlap(outs[a], outn[a], ins[b], inn[b])) return INFINI_ERR_INVALID_ARG;
     for (int b = a + 1; b < 3; ++b)
       if (ranges_overlap(outs[a], outn[a], outs[b], outn[b])) return INFINI_ERR_INVALID_ARG;
+  }
+  if (bp.tc) {
+    const void* ptrs[7] = {p.q, p.k, p.v, p.d_out, p.dq, p.dk, p.dv};
+    bool aligned = true;
+    for (const void* x : ptrs) aligned = aligned && reinterpret_cast<uintptr_t>(x) % 16 == 0;
+    if (!aligned) {  // TMA needs 16-byte aligned rows: the CUDA-core kernels take the call
+      infini_attn_bwd_params q2 = p;
+      q2.flags |= INFINI_FLAG_FORCE_SIMT;
+      return backward_impl(q2);
+    }
   }
   if (p.workspace && (p.workspace_bytes < bp.total || reinterpret_cast<uintptr_t>(p.workspace) % kAlign != 0))
     return INFINI_ERR_WORKSPACE;
@@ -955,8 +1043,13 @@ int infini_attn_backward(const infini_attn_bwd_params* p) {
 
 size_t infini_attn_backward_workspace_size(const infini_attn_bwd_params* p) {
   if (!p) return 0;
-  BwdPlan bp;
-  return bwd_plan(*p, &bp) == INFINI_OK ? bp.total : 0;
+  BwdPlan bp, bs;
+  if (bwd_plan(*p, &bp) != INFINI_OK) return 0;
+  // a call whose tensors are not 16-byte aligned runs on the CUDA cores, whose plan may be larger
+  infini_attn_bwd_params q = *p;
+  q.flags |= INFINI_FLAG_FORCE_SIMT;
+  if (bwd_plan(q, &bs) != INFINI_OK) return 0;
+  return std::max(bp.total, bs.total);
 }
 
 size_t infini_attn_workspace_size_ex(const infini_attn_params* p) {
@@ -978,48 +1071,57 @@ int infini_attn_decode_step(const void* q_t, const void* k_t, const void* v_t, v
   if (BH > (1LL << 31) - 1) return INFINI_ERR_UNSUPPORTED;
   int rc = check_device(false);
   if (rc != INFINI_OK) return rc;
-  // 1. the token's key and value into row pos of every (b, h) cache
-  char* kc = static_cast<char*>(k_cache);
-  char* vc = static_cast<char*>(v_cache);
-  if (cudaMemcpy2DAsync(kc + (size_t)pos * dk * es, (size_t)N * dk * es, k_t, (size_t)dk * es, (size_t)dk * es,
-                        (size_t)BH, cudaMemcpyDeviceToDevice, stream) != cudaSuccess ||
-      cudaMemcpy2DAsync(vc + (size_t)pos * dv * es, (size_t)N * dv * es, v_t, (size_t)dv * es, (size_t)dv * es,
-                        (size_t)BH, cudaMemcpyDeviceToDevice, stream) != cudaSuccess)
-    return INFINI_ERR_LAUNCH;
-  // 2. the token's output
-  const float scale = 1.f / sqrtf((float)dk);
-  {
-    LaunchScope ls(kPhaseAttn, stream);
-    if (f32)
-      decode_kernel<float><<<(unsigned)BH, 32 * kDecodeWarps, 0, stream>>>(
-          static_cast<const float*>(q_t), reinterpret_cast<const float*>(kc), reinterpret_cast<const float*>(vc),
-          beta, M, z, static_cast<float*>(out), H, N, pos + 1, dk, dv, scale);
-    else
-      decode_kernel<__nv_bfloat16><<<(unsigned)BH, 32 * kDecodeWarps, 0, stream>>>(
-          static_cast<const __nv_bfloat16*>(q_t), reinterpret_cast<const __nv_bfloat16*>(kc),
-          reinterpret_cast<const __nv_bfloat16*>(vc), beta, M, z, static_cast<__nv_bfloat16*>(out), H, N, pos + 1,
-          dk, dv, scale);
-  }
-  rc = launch_status();
-  if (rc != INFINI_OK || !(fold || pos == N - 1)) return rc;
-  // 3. the segment is complete: fold its keys and values into M, z with the
-  // forward's kernels on the cached segment (their attention output is
-  // scratch; the update reads only K, V, M, z)
   const int n = pos + 1;
+  // 1 + 2. the token's output, its key and value appended to the caches by the
+  // same launch: keys split over enough CTAs to fill the GPU (ranges of at
+  // least 64 keys), then one merge per (b, h)
+  const long long want = std::max<long long>(1, (2LL * kSms + BH - 1) / BH);
+  int per = (int)std::max<long long>(64, (n + want - 1) / want);
+  const int splits = (n + per - 1) / per;
+  const float scale = 1.f / sqrtf((float)dk);
   void* scratch = nullptr;
-  if (cudaMallocAsync(&scratch, (size_t)BH * n * dv * es, stream) != cudaSuccess) {
+  if (cudaMallocAsync(&scratch, (size_t)splits * BH * (dv + 2) * 4, stream) != cudaSuccess) {
     cudaGetLastError();
     return INFINI_ERR_WORKSPACE;
   }
+  float* part = static_cast<float*>(scratch);
+  {
+    LaunchScope ls(kPhaseAttn, stream);
+    const dim3 grid((unsigned)BH, (unsigned)splits);
+    if (f32)
+      decode_part_kernel<float><<<grid, 256, 0, stream>>>(
+          static_cast<const float*>(q_t), static_cast<const float*>(k_t), static_cast<const float*>(v_t),
+          static_cast<float*>(k_cache), static_cast<float*>(v_cache), N, n, dk, dv, scale, per, part);
+    else
+      decode_part_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
+          static_cast<const __nv_bfloat16*>(q_t), static_cast<const __nv_bfloat16*>(k_t),
+          static_cast<const __nv_bfloat16*>(v_t), static_cast<__nv_bfloat16*>(k_cache),
+          static_cast<__nv_bfloat16*>(v_cache), N, n, dk, dv, scale, per, part);
+  }
+  {
+    LaunchScope ls(kPhaseAttn, stream);
+    if (f32)
+      decode_merge_kernel<float><<<(unsigned)BH, 128, 0, stream>>>(static_cast<const float*>(q_t), beta, M, z, part,
+                                                                    splits, H, dk, dv, static_cast<float*>(out));
+    else
+      decode_merge_kernel<__nv_bfloat16><<<(unsigned)BH, 128, 0, stream>>>(
+          static_cast<const __nv_bfloat16*>(q_t), beta, M, z, part, splits, H, dk, dv,
+          static_cast<__nv_bfloat16*>(out));
+  }
+  rc = launch_status();
+  if (cudaFreeAsync(scratch, stream) != cudaSuccess && rc == INFINI_OK) rc = INFINI_ERR_WORKSPACE;
+  if (rc != INFINI_OK || !(fold || pos == N - 1)) return rc;
+  // 3. the segment is complete: fold its keys and values into M, z with the
+  // forward's update kernels alone (no attention, no output)
   infini_attn_params p;
   memset(&p, 0, sizeof(p));
-  p.q = kc;
-  p.k = kc;
-  p.v = vc;
+  p.q = k_cache;
+  p.k = k_cache;
+  p.v = v_cache;
   p.beta = beta;
   p.M = M;
   p.z = z;
-  p.out = scratch;
+  p.out = nullptr;
   p.B = B;
   p.H = H;
   p.L = n;
@@ -1027,29 +1129,17 @@ int infini_attn_decode_step(const void* q_t, const void* k_t, const void* v_t, v
   p.dk = dk;
   p.dv = dv;
   p.mode = mode;
+  p.flags = kFlagUpdateOnly;
   const long long ks[3] = {(long long)H * N * dk, (long long)N * dk, dk};
   const long long vs[3] = {(long long)H * N * dv, (long long)N * dv, dv};
-  const long long os[3] = {(long long)H * n * dv, (long long)n * dv, dv};
   for (int i = 0; i < 3; ++i) {
     p.q_stride[i] = p.k_stride[i] = ks[i];
     p.v_stride[i] = vs[i];
-    p.o_stride[i] = os[i];
+    p.o_stride[i] = vs[i];
   }
   p.stream = stream;
-  rc = forward_impl(p);
-  if (cudaFreeAsync(scratch, stream) != cudaSuccess && rc == INFINI_OK) rc = INFINI_ERR_WORKSPACE;
-  return rc;
-}
-
-int infini_attn_gemm_bf16(const void* A, const void* Bm, void* C, long M, int N, int K, cudaStream_t stream) {
-  if (!A || !Bm || !C) return INFINI_ERR_INVALID_ARG;
-  if (M <= 0 || N <= 0 || K <= 0) return INFINI_ERR_INVALID_ARG;
-  if (ranges_overlap(C, (size_t)M * N * 2, A, (size_t)M * K * 2) || ranges_overlap(C, (size_t)M * N * 2, Bm, (size_t)K * N * 2))
-    return INFINI_ERR_INVALID_ARG;
-  if (N % 8 || K % 8) return INFINI_ERR_UNSUPPORTED;
-  const int rc = check_device(true);
-  if (rc != INFINI_OK) return rc;
-  return gemm_tc(A, K, Bm, N, C, N, M, N, K, stream);
+  (void)es;
+  return forward_impl(p);
 }
 
 size_t infini_attn_layer_workspace_size(int B, int H, long L, int N, int d_model, int mode) {

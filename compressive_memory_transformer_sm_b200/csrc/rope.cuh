@@ -13,7 +13,8 @@
 //
 // HBM-bound: one read and one write of q and k.  Each thread handles E
 // consecutive elements (E / 2 pairs) of the same position in q and in k, so a
-// cosine / sine pair serves both tensors.
+// cosine / sine pair serves both tensors (and every head, when the grid has
+// fewer rows than B * H).
 #pragma once
 
 #include "common.cuh"
@@ -78,36 +79,39 @@ __device__ __forceinline__ void rope_angle(long long pos, double f, float& c, fl
   __sincosf((float)r, &s, &c);
 }
 
-// Grid-stride over (b, h, t, group of E elements); E = 8 needs dk % 8 == 0 and
-// vector-aligned rows, E = 2 (one pair) only an even dk.
+// Thread (x, y) of block (bx, by): element group x (E elements) of token
+// t = bx * blockDim.y + y of head by (then by + gridDim.y, ... when B * H
+// exceeds the grid), so that no index needs a division.  E = 8 needs
+// dk % 8 == 0 and vector-aligned rows, E = 2 (one pair) only an even dk.
 template <typename T, int E>
 __global__ void __launch_bounds__(256) rope_kernel(const __grid_constant__ RopeArgs a) {
-  const int groups = a.dk / E;
-  const long long total = (long long)a.B * a.H * a.L * groups;
+  const int j = threadIdx.x;
+  const long long t = (long long)blockIdx.x * blockDim.y + threadIdx.y;
+  if (t >= a.L) return;
+  const long long pos = a.offset + t;
+  // the rotation of this thread's pairs, shared by q and k
+  float cs[E / 2], sn[E / 2];
+#pragma unroll
+  for (int e = 0; e < E / 2; ++e) rope_angle(pos, a.inv_freq[j * (E / 2) + e], cs[e], sn[e]);
   const T* q = static_cast<const T*>(a.q);
   const T* k = static_cast<const T*>(a.k);
   T* qr = static_cast<T*>(a.qr);
   T* kr = static_cast<T*>(a.kr);
-  for (long long c = (long long)blockIdx.x * blockDim.x + threadIdx.x; c < total;
-       c += (long long)gridDim.x * blockDim.x) {
-    const long long row = c / groups;
-    const int j = (int)(c - row * groups);
-    const long long t = row % a.L;
-    const long long bh = row / a.L;
-    const int b = (int)(bh / a.H), h = (int)(bh % a.H);
-    const long long pos = a.offset + t;
+  const int BH = a.B * a.H;
+  for (int bh = blockIdx.y; bh < BH; bh += gridDim.y) {
+    const int b = bh / a.H, h = bh - b * a.H;
+    const long long row = (long long)bh * a.L + t;
     float xq[E], xk[E];
     rope_load<T, E>(q + b * a.qs[0] + h * a.qs[1] + t * a.qs[2] + j * E, xq);
     rope_load<T, E>(k + b * a.ks[0] + h * a.ks[1] + t * a.ks[2] + j * E, xk);
 #pragma unroll
     for (int e = 0; e < E; e += 2) {
-      float cs, sn;
-      rope_angle(pos, a.inv_freq[(j * E + e) >> 1], cs, sn);
+      const float c = cs[e / 2], s = sn[e / 2];
       const float q0 = xq[e], q1 = xq[e + 1], k0 = xk[e], k1 = xk[e + 1];
-      xq[e] = q0 * cs - q1 * sn;
-      xq[e + 1] = q0 * sn + q1 * cs;
-      xk[e] = k0 * cs - k1 * sn;
-      xk[e + 1] = k0 * sn + k1 * cs;
+      xq[e] = q0 * c - q1 * s;
+      xq[e + 1] = q0 * s + q1 * c;
+      xk[e] = k0 * c - k1 * s;
+      xk[e + 1] = k0 * s + k1 * c;
     }
     rope_store<T, E>(qr + row * a.dk + j * E, xq);
     rope_store<T, E>(kr + row * a.dk + j * E, xk);

@@ -208,7 +208,7 @@ __global__ void __launch_bounds__(256) state_kernel(float* __restrict__ M, float
 // keeps a running max and sum per row; the memory read uses the fp32
 // snapshot M_{s-1}, z_{s-1} of the segment.
 template <typename T>
-__global__ void __launch_bounds__(256, 2) simt_attn_kernel(const T* __restrict__ q, const T* __restrict__ k,
+__global__ void __launch_bounds__(256, 3) simt_attn_kernel(const T* __restrict__ q, const T* __restrict__ k,
                                                         const T* __restrict__ v, const float* __restrict__ beta,
                                                         T* __restrict__ out, Geo g, float scale, int QT,
                                                         const float* __restrict__ snapM,

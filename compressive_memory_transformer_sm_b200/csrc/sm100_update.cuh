@@ -55,6 +55,7 @@ struct UpdArgs {
   float* z;
   __nv_bfloat16* snapM;         // [BH][S][128][128] bf16 [dk][dv] (delta: M_s for segment s+1)
   float* snapzw;                // [BH][S][128] (delta: z_{s-1} for segment s)
+  float* snapM32;               // delta, optional: fp32 copy of the snapshot (the backward's recomputation)
   int B, H, S, N;
   long long L;
   int seg0, nseg, G, cpb;
@@ -150,6 +151,11 @@ __global__ void __launch_bounds__(UpdWarps<DELTA>::THREADS, 1)
                                  pack_bf16x2(f1.z, f1.w));
       if (nchunks > 0) sts128(base + SL::MT + swz_chunk(r, cc), v);
       if (mine) *reinterpret_cast<uint4*>(snap + r * 128 + 8 * cc) = v;
+      if (mine && a.snapM32 != nullptr) {
+        float4* s32 = reinterpret_cast<float4*>(a.snapM32 + ((long long)bh * a.S + s) * 16384 + r * 128 + 8 * cc);
+        s32[0] = f0;
+        s32[1] = f1;
+      }
     }
     if (grp == 0 && threadIdx.x < 128)
       a.snapzw[((long long)bh * a.S + s) * 128 + threadIdx.x] = a.z[(long long)bh * 128 + threadIdx.x];

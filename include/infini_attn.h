@@ -207,8 +207,10 @@ INFINI_API size_t infini_attn_workspace_size_ex(const infini_attn_params* p);
  *   q_t, k_t, out: [B, H, dk] / [B, H, dv]; v_t [B, H, dv]; contiguous, bf16 or
  *   fp32 (mode | INFINI_F32); k_cache [B, H, N, dk], v_cache [B, H, N, dv] in
  *   the same type, contiguous, caller-owned, rows > pos not read.
- * The fold runs the forward's kernels on the cached segment (its attention
- * output goes to a scratch buffer allocated on `stream`).  Errors as
+ * Steps 1 and 2 are one launch with the keys split over enough CTAs to fill
+ * the GPU, plus a merge launch (a small scratch buffer of partial softmax
+ * states is taken and released on `stream`); the fold runs the forward's
+ * memory-update kernels alone on the cached segment.  Errors as
  * infini_attn_forward; pos outside [0, N) is INFINI_ERR_INVALID_ARG.
  */
 INFINI_API int infini_attn_decode_step(const void* q_t, const void* k_t, const void* v_t, void* k_cache,
@@ -276,10 +278,13 @@ INFINI_API int infini_attn_gemm_bf16(const void* A, const void* B, void* C, long
  * and z0, dz_S, dz0 [B, H, dk] fp32.  M0 / z0 NULL: the empty memory;
  * dM_S / dz_S NULL: zero; dM0 / dz0 NULL: not returned.  Every pointer is
  * caller-owned device memory; the inputs are read only, the outputs written.
- * Arithmetic in fp32 (CUDA cores); no position embeddings.  Workspace as for
- * the forward: taken on `stream` unless given
- * (infini_attn_backward_workspace_size bytes, 256-byte aligned).  Errors as
- * infini_attn_forward.
+ * bf16 with dk = dv = 128 (16-byte aligned tensors): the local attention's
+ * gradients run on the tensor cores (tcgen05; P and dS rounded to bf16 as
+ * operands, fp32 accumulation), everything else in fp32 on CUDA cores;
+ * other shapes, fp32 tensors and INFINI_FLAG_FORCE_SIMT: all in fp32 on CUDA
+ * cores.  No position embeddings.  Workspace as for the forward: taken on
+ * `stream` unless given (infini_attn_backward_workspace_size bytes, 256-byte
+ * aligned).  Errors as infini_attn_forward.
  */
 typedef struct infini_attn_bwd_params {
   const void* q;
@@ -306,6 +311,7 @@ typedef struct infini_attn_bwd_params {
   void* workspace;
   size_t workspace_bytes;
   cudaStream_t stream;
+  int flags; /* INFINI_FLAG_FORCE_SIMT: CUDA-core kernels even where the tensor-core ones apply */
 } infini_attn_bwd_params;
 
 INFINI_API int infini_attn_backward(const infini_attn_bwd_params* p);
