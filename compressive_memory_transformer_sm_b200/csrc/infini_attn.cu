@@ -351,6 +351,25 @@ int run_simt(const infini_attn_params& p, const Plan& pl, char* ws, float scale,
   return launch_status();
 }
 
+// A second stream of this library in the current context (non-blocking,
+// created on first use), for work that may overlap the caller's stream.
+cudaStream_t side_stream() {
+  static std::mutex mu;
+  static std::vector<std::pair<unsigned long long, cudaStream_t>> streams;
+  const unsigned long long ctx = current_context_id();
+  if (ctx == 0) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
+  for (const auto& e : streams)
+    if (e.first == ctx) return e.second;
+  cudaStream_t st = nullptr;
+  if (cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  streams.emplace_back(ctx, st);
+  return st;
+}
+
 // The dynamic shared-memory limit is an attribute of a function in the
 // current context: set it for the tensor-core kernels once for every context
 // the process uses (an unknown context id, 0, sets it on every call).
@@ -453,6 +472,38 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale, c
   ua.snapM32 = extra ? extra->snapM32 : nullptr;
   ua.B = p.B; ua.H = p.H; ua.S = pl.S; ua.N = p.N; ua.L = p.L;
   ua.G = pl.G; ua.cpb = pl.cpb;
+  // One segment (a streaming step): the attention reads only the snapshot of
+  // (M_0, z_0), which the update never writes after its start, so once the
+  // snapshot is taken the attention runs on a second stream alongside the
+  // update; the caller's stream then waits for both (event fork and join).
+  cudaStream_t as = p.stream;  // the attention's stream
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+  const bool fork = pl.S == 1 && !(p.flags & kFlagUpdateOnly) && extra == nullptr;
+  if (fork) {
+    {
+      LaunchScope ls(kPhaseState, p.stream);
+      state_kernel<<<sgrid, 256, 0, p.stream>>>(p.M, p.z, part, 128, 128, 1, 2, 0, 1, pl.G, nullptr, snapM16, snapz);
+    }
+    cudaStream_t side = side_stream();
+    if (side != nullptr && cudaEventCreateWithFlags(&ev_fork, cudaEventDisableTiming) == cudaSuccess &&
+        cudaEventCreateWithFlags(&ev_join, cudaEventDisableTiming) == cudaSuccess &&
+        cudaEventRecord(ev_fork, p.stream) == cudaSuccess && cudaStreamWaitEvent(side, ev_fork, 0) == cudaSuccess) {
+      as = side;
+    } else {
+      cudaGetLastError();
+    }
+    ua.snapM = nullptr;  // taken above: the update kernels skip it
+    ua.snapzw = nullptr;
+  }
+  // the caller's stream waits for the attention's stream; the events are released
+  auto join = [&]() {
+    if (ev_join != nullptr && as != p.stream) {
+      if (cudaEventRecord(ev_join, as) != cudaSuccess || cudaStreamWaitEvent(p.stream, ev_join, 0) != cudaSuccess)
+        cudaGetLastError();
+    }
+    if (ev_fork) cudaEventDestroy(ev_fork);
+    if (ev_join) cudaEventDestroy(ev_join);
+  };
   if (!pl.delta) {
     ua.seg0 = 0; ua.nseg = pl.S;
     {
@@ -462,7 +513,8 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale, c
     }
     LaunchScope ls(kPhaseState, p.stream);
     state_kernel<<<sgrid, 256, 0, p.stream>>>(p.M, p.z, part, 128, 128, pl.S, 0, 0, pl.S, pl.G,
-                                              extra ? extra->snapM32 : nullptr, snapM16, snapz);
+                                              extra ? extra->snapM32 : nullptr, fork ? nullptr : snapM16,
+                                              fork ? nullptr : snapz);
   } else {
     ua.nseg = 1;
     // one cluster of G CTAs per head; G <= 8 (plan)
@@ -483,8 +535,10 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale, c
       // segment s, reduced inside each head's cluster into M, z
       ua.seg0 = s;
       LaunchScope ls(kPhaseUpdate, p.stream);
-      if (cudaLaunchKernelEx(&cfg, tc::mem_update_tc_kernel<true>, tm_k, tm_v, ua) != cudaSuccess)
+      if (cudaLaunchKernelEx(&cfg, tc::mem_update_tc_kernel<true>, tm_k, tm_v, ua) != cudaSuccess) {
+        join();
         return INFINI_ERR_LAUNCH;
+      }
     }
   }
   if (p.flags & kFlagUpdateOnly) return launch_status();
@@ -514,14 +568,19 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale, c
   const long long groups = (NS + aa.GS - 1) / aa.GS;
   // persistent: one CTA per SM, or one per work item when there are fewer
   const long long items = groups * aa.GS * aa.P;
-  if (items >= (1LL << 31)) return INFINI_ERR_UNSUPPORTED;
   aa.work_counter = reinterpret_cast<unsigned int*>(ws + pl.off_ctr);
-  if (cudaMemsetAsync(aa.work_counter, 0, sizeof(unsigned int), p.stream) != cudaSuccess)
-    return INFINI_ERR_LAUNCH;
-  LaunchScope ls(kPhaseAttn, p.stream);
-  tc::attn_tc_kernel<<<(unsigned)std::min<long long>(items, sms), tc::kAttnThreads, tc::kAttnSmem, p.stream>>>(
-      tm_qa, tm_ka, tm_v, tm_mt, aa);
-  return launch_status();
+  if (items >= (1LL << 31) || cudaMemsetAsync(aa.work_counter, 0, sizeof(unsigned int), as) != cudaSuccess) {
+    join();
+    return items >= (1LL << 31) ? INFINI_ERR_UNSUPPORTED : INFINI_ERR_LAUNCH;
+  }
+  {
+    LaunchScope ls(kPhaseAttn, as);
+    tc::attn_tc_kernel<<<(unsigned)std::min<long long>(items, sms), tc::kAttnThreads, tc::kAttnSmem, as>>>(
+        tm_qa, tm_ka, tm_v, tm_mt, aa);
+  }
+  const int rc = launch_status();
+  join();
+  return rc;
 }
 
 bool tc_layout_ok(const infini_attn_params& p) {
@@ -1140,6 +1199,17 @@ int infini_attn_decode_step(const void* q_t, const void* k_t, const void* v_t, v
   p.stream = stream;
   (void)es;
   return forward_impl(p);
+}
+
+int infini_attn_gemm_bf16(const void* A, const void* Bm, void* C, long M, int N, int K, cudaStream_t stream) {
+  if (!A || !Bm || !C) return INFINI_ERR_INVALID_ARG;
+  if (M <= 0 || N <= 0 || K <= 0) return INFINI_ERR_INVALID_ARG;
+  if (ranges_overlap(C, (size_t)M * N * 2, A, (size_t)M * K * 2) || ranges_overlap(C, (size_t)M * N * 2, Bm, (size_t)K * N * 2))
+    return INFINI_ERR_INVALID_ARG;
+  if (N % 8 || K % 8) return INFINI_ERR_UNSUPPORTED;
+  const int rc = check_device(true);
+  if (rc != INFINI_OK) return rc;
+  return gemm_tc(A, K, Bm, N, C, N, M, N, K, stream);
 }
 
 size_t infini_attn_layer_workspace_size(int B, int H, long L, int N, int d_model, int mode) {

@@ -166,7 +166,7 @@ __global__ void __launch_bounds__(256) state_kernel(float* __restrict__ M, float
     if (e < E) {
       if (snapM32) snapM32[base * E + e] = val;
       if (snapM16) snapM16[base * E + e] = __float2bfloat16_rn(val);
-    } else {
+    } else if (snapz) {
       snapz[base * dk + (e - E)] = val;
     }
   };

@@ -53,8 +53,8 @@ struct UpdArgs {
   float* partial;               // [BH][nseg][G][128*128 + 128] (linear)
   float* M;                     // running state (delta)
   float* z;
-  __nv_bfloat16* snapM;         // [BH][S][128][128] bf16 [dk][dv] (delta: M_s for segment s+1)
-  float* snapzw;                // [BH][S][128] (delta: z_{s-1} for segment s)
+  __nv_bfloat16* snapM;         // [BH][S][128][128] bf16 [dk][dv] (delta: M_{s-1} for segment s); nullptr: not written
+  float* snapzw;                // [BH][S][128] (delta: z_{s-1} for segment s); nullptr: not written
   float* snapM32;               // delta, optional: fp32 copy of the snapshot (the backward's recomputation)
   int B, H, S, N;
   long long L;
@@ -150,14 +150,14 @@ __global__ void __launch_bounds__(UpdWarps<DELTA>::THREADS, 1)
       const uint4 v = make_uint4(pack_bf16x2(f0.x, f0.y), pack_bf16x2(f0.z, f0.w), pack_bf16x2(f1.x, f1.y),
                                  pack_bf16x2(f1.z, f1.w));
       if (nchunks > 0) sts128(base + SL::MT + swz_chunk(r, cc), v);
-      if (mine) *reinterpret_cast<uint4*>(snap + r * 128 + 8 * cc) = v;
+      if (mine && a.snapM != nullptr) *reinterpret_cast<uint4*>(snap + r * 128 + 8 * cc) = v;
       if (mine && a.snapM32 != nullptr) {
         float4* s32 = reinterpret_cast<float4*>(a.snapM32 + ((long long)bh * a.S + s) * 16384 + r * 128 + 8 * cc);
         s32[0] = f0;
         s32[1] = f1;
       }
     }
-    if (grp == 0 && threadIdx.x < 128)
+    if (grp == 0 && threadIdx.x < 128 && a.snapzw != nullptr)
       a.snapzw[((long long)bh * a.S + s) * 128 + threadIdx.x] = a.z[(long long)bh * 128 + threadIdx.x];
   }
   if (nchunks == 0) {  // group past the end of a short segment: contributes nothing

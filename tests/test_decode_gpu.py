@@ -1,6 +1,7 @@
 """Token-level streaming decode through the C ABI: a sequence fed one token at a time
 (pos = t mod N, fold on the last token) against the fp64 oracle's whole-sequence forward
-(the oracle's decode step is pinned to that forward).  Tolerances as for the forward:
+(the oracle's decode step is pinned to that forward).  The segment of 1024 spreads a
+token's keys over up to 16 ranges (CTAs) per (b, h), merged by a second launch.  Tolerances as for the forward:
 bf16 max-abs 2e-2 / relative L2 5e-3 on the outputs, relative L2 5e-3 on the state;
 fp32 max-abs 1e-4 and 1e-5."""
 
@@ -26,7 +27,8 @@ def rel_l2(a, b):
 
 @pytest.mark.parametrize("mode", [LINEAR, DELTA], ids=["linear", "delta"])
 @pytest.mark.parametrize("B,H,L,N,d,dtype", [(1, 2, 160, 64, 128, torch.bfloat16), (2, 1, 40, 16, 32, torch.float32),
-                                             (1, 3, 130, 128, 128, torch.bfloat16)])
+                                             (1, 3, 130, 128, 128, torch.bfloat16),
+                                             (1, 2, 1100, 1024, 128, torch.bfloat16)])
 def test_decode_matches_forward(B, H, L, N, d, dtype, mode):
     w = W.Workload("decode", B=B, H=H, L=L, N=N, dk=d, dv=d, dtype=dtype, modes=(mode,), seed=4242 + L)
     q, k, v, beta = (t.to(DEV) for t in W.make_inputs(w, device="cpu"))
