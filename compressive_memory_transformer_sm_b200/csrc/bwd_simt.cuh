@@ -211,13 +211,13 @@ __global__ void __launch_bounds__(256, 2)
 // The memory read's backward (Eq. 7) and the per-row terms for the tensor-core
 // path, where the local attention's gradients come from the tcgen05 kernels:
 // for 128 query rows of one (b, h, segment) (four passes of 32; warp w: rows
-// 4w .. 4w+3 of a pass, lane = column), D'_i = dO_i . A_dot_i (A_dot bf16
-// from the forward), the dbeta row term dO_i . (A_mem_i - A_dot_i), and
+// 4w .. 4w+3 of a pass, lane = column), D'_i = dO_i . A_dot_i (A_dot from the
+// forward's recomputation), the dbeta row term dO_i . (A_mem_i - A_dot_i), and
 // dq_mem = sigma'(q) (d_num M^T + d_den z) with d_num, d_den rows written for
 // the memory chain.  M^(s) is staged in shared memory once per block.
 template <typename T>
 __global__ void __launch_bounds__(256, 2) bwd_qmem_kernel(const T* __restrict__ q, const T* __restrict__ dout,
-                                                       const __nv_bfloat16* __restrict__ adot,
+                                                       const float* __restrict__ adot,
                                                        const float* __restrict__ beta,
                                                        const float* __restrict__ snapM,
                                                        const float* __restrict__ snapz, BwdGeo g,
@@ -279,7 +279,7 @@ __global__ void __launch_bounds__(256, 2) bwd_qmem_kernel(const T* __restrict__ 
       const int j = lane + 32 * c;
       if (j < dv) {
         const float dA = to_f32(dout[row * dv + j]);
-        const float ad = __bfloat162float(adot[row * dv + j]);
+        const float ad = adot[row * dv + j];
         const float am = den != 0.f ? num[c] / den : 0.f;
         dpr = fmaf(dA, ad, dpr);
         bterm = fmaf(dA, am - ad, bterm);

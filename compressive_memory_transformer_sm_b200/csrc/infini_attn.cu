@@ -448,7 +448,7 @@ int gemm_tc(const void* A, long long lda, const void* Bm, long long ldb, void* C
 // Extra outputs of a forward run for the backward's recomputation.
 struct FwdExtra {
   float* snapM32;       // fp32 [BH][S][dk][dv] snapshots of M^(s)
-  __nv_bfloat16* adot;  // [B*H*L][128] A_dot
+  float* adot;          // [B*H*L][128] A_dot
   float* lse2;          // [B*H*L] row log2-sum-exp2 of the scaled scores
 };
 
@@ -729,7 +729,7 @@ int bwd_plan(const infini_attn_bwd_params& p, BwdPlan* bp) {
   bp->off_fwd = take(f.total);
   bp->off_state = take((size_t)BH * (E + p.d_k) * 4);
   bp->off_out = take((size_t)rows * p.d_v * es);
-  bp->off_adot = take((size_t)rows * p.d_v * (bp->tc ? 2 : 4));
+  bp->off_adot = take((size_t)rows * p.d_v * 4);
   bp->off_lse = take((size_t)rows * 4);
   bp->off_D = take((size_t)rows * 4);
   bp->off_brow = take((size_t)rows * 4);
@@ -785,7 +785,7 @@ int run_backward(const infini_attn_bwd_params& p, const BwdPlan& bp, char* ws) {
     // tensor-core forward: A_dot in bf16, lse in log2 units, fp32 snapshots of M^(s)
     FwdExtra ex;
     ex.snapM32 = reinterpret_cast<float*>(ws + bp.off_snap32);
-    ex.adot = reinterpret_cast<__nv_bfloat16*>(ws + bp.off_adot);
+    ex.adot = adot;
     ex.lse2 = lse;
     rc = run_tc(fp, f, fws, scale, loc, &ex);
     snapM = ex.snapM32;
@@ -829,7 +829,7 @@ int run_backward(const infini_attn_bwd_params& p, const BwdPlan& bp, char* ws) {
     {
       LaunchScope ls(kPhaseBwd, st);
       bwd_qmem_kernel<T><<<(unsigned)((long long)BH * f.S * bps), 256, qm_smem, st>>>(
-          q, dout, reinterpret_cast<const __nv_bfloat16*>(ws + bp.off_adot), p.beta, snapM, snapz, g, bps, dqmem,
+          q, dout, adot, p.beta, snapM, snapz, g, bps, dqmem,
           Drow, brow, dnum, dden);
     }
     memset(&ta, 0, sizeof(ta));

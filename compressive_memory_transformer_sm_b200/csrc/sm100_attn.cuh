@@ -45,9 +45,9 @@ struct AttnArgs {
   const __nv_bfloat16* qm;
   long long qms[3];
   // For the backward's recomputation (nullptr otherwise): A_dot of every row
-  // in bf16, contiguous [B*H*L][128], and the row's log2-sum-exp2 of the
+  // in fp32, contiguous [B*H*L][128], and the row's log2-sum-exp2 of the
   // scaled scores (P = 2^(s * scale_log2 - lse2)), [B*H*L] fp32.
-  __nv_bfloat16* adot;
+  float* adot;
   float* lse2;
 };
 
@@ -650,12 +650,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         if (a.adot != nullptr && valid) {
           const float inv_l = 1.f / l;
+          float4* ad = reinterpret_cast<float4*>(a.adot + (((long long)w.b * a.H + w.h) * a.L + w.seg0 + qrow) * 128);
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            pk[e] = pack_bf16x2(__uint_as_float(ro[2 * e]) * inv_l, __uint_as_float(ro[2 * e + 1]) * inv_l);
-          uint4* ad = reinterpret_cast<uint4*>(a.adot + (((long long)w.b * a.H + w.h) * a.L + w.seg0 + qrow) * 128);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) ad[4 * c2 + e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+          for (int e = 0; e < 16; ++e)
+            ad[16 * (c2 / 2) + e] =
+                make_float4(__uint_as_float(ro[4 * e]) * inv_l, __uint_as_float(ro[4 * e + 1]) * inv_l,
+                            __uint_as_float(ro[4 * e + 2]) * inv_l, __uint_as_float(ro[4 * e + 3]) * inv_l);
         }
       }
       if (a.lse2 != nullptr && valid) a.lse2[((long long)w.b * a.H + w.h) * a.L + w.seg0 + qrow] = m_ref + __log2f(l);

@@ -10,8 +10,13 @@ mixed sign, about the size of the output rounding.  Tolerances (reasoned from th
 arithmetic, the forward's in kind): fp32 tensors relative L2 1e-5 on every gradient; bf16
 tensors relative L2 5e-3 on dq, dk, dv (output rounding alone gives about 1.7e-3, the
 operand roundings of the tensor-core path about as much again) and 1e-4 on the fp32 outputs
-dbeta, dM0, dz0 of the CUDA-core path, 1e-3 of the tensor-core path (their row terms use the
-bf16 A_dot).
+dM0, dz0 (1e-3 on the tensor-core path).
+
+dbeta = g (1 - g) sum dA . (A_mem - A_dot) is a sum of terms of both signs, so its error is
+judged against the sum of their magnitudes, g (1 - g) sum |dA| (|A_mem| + |A_dot|) per head:
+at most 1e-5 of it for fp32 tensors, 1e-4 for bf16 on CUDA cores, and 5e-3 on the tensor-core
+path, whose recomputed A_dot carries the forward's bf16 rounding of P -- about 2^-9 relative
+per element, not averaged away because V has random signs.
 """
 
 import numpy as np
@@ -21,6 +26,7 @@ import torch
 from compressive_memory_transformer_sm_b200 import DELTA, LINEAR, api
 from compressive_memory_transformer_sm_b200 import workloads as W
 from oracle import infini_bwd as RB
+from oracle import infini_ref as R
 from tests.test_parity_gpu import DEV, inputs, np64, rel_l2
 
 pytestmark = pytest.mark.gpu
@@ -53,6 +59,17 @@ def _compare(case, N, mode, f32, what, flags=0):
     for name, gt, wt in zip(NAMES, got, want):
         gt = np64(gt)
         assert np.all(np.isfinite(gt)), f"{what} {name}: non-finite"
+        if name == "dbeta":
+            _, _, _, parts = R.forward(np64(q), np64(k), np64(v), np64(beta), N, mode=mode, M0=n(M0), z0=n(z0),
+                                       return_parts=True)
+            gw = 1.0 / (1.0 + np.exp(-np64(beta)))
+            scale = gw * (1.0 - gw) * (np.abs(np64(d_out)) * (np.abs(parts["A_mem"]) + np.abs(parts["A_dot"]))).sum(
+                axis=(0, 2, 3))
+            rel = float(np.max(np.abs(gt - wt) / scale))
+            tol = 1e-5 if f32 else (5e-3 if tensor else 1e-4)
+            print(f"backward {what} dbeta: error / sum of |terms| {rel:.3e} (tolerance {tol:.0e})")
+            assert rel <= tol, f"{what} dbeta: error {rel:.3e} of the sum of |terms| > {tol}"
+            continue
         rl = rel_l2(gt, wt)
         tol = 1e-5 if f32 else (5e-3 if name in ("dq", "dk", "dv") else (1e-3 if tensor else 1e-4))
         print(f"backward {what} {name}: rel-L2 {rl:.3e} (tolerance {tol:.0e})")
