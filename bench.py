@@ -52,7 +52,7 @@ from compressive_memory_transformer_sm_b200 import workloads as W  # noqa: E402
 METRIC = "Infini-attn fwd tokens/s per layer; TFLOP/s and % of B200 bf16 tensor peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FLUSH_BYTES = 1 << 30
-PHASE_NAMES = ("update", "state", "attention", "rope", "projections", "backward")
+PHASE_NAMES = ("update", "state", "attention", "rope", "projections", "backward_cuda_cores", "backward_tensor")
 
 
 # ------------------------------------------------------------------ work model
@@ -665,16 +665,32 @@ def run_backward(args, w: W.Workload, mode: int):
     api.infini_attn_profile_enable(0)
     phase_ms, phase_n = api.infini_attn_profile_read(reset=True)
     # algorithmic work: the forward recomputation plus the backward's products (local
-    # attention: S, dP, dV, dK, dQ = 5 causal n(n+1)d/2-pair products per segment; memory
-    # read and update: about 12 n dk dv for the linear rule, 18 for the delta rule)
+    # attention: S, dP, dV, dK, dQ = 5 causal products of n(n+1)/2 pairs x d x 2 FLOP per
+    # segment; memory read and update: about 12 n dk dv for the linear rule, 18 for delta)
     f_fwd_attn, f_fwd_upd = algorithmic_flops(w, mode)
-    f_bwd = 0
+    f_local = f_mem = 0
     for s0 in range(0, w.L, w.N):
         n = min(w.N, w.L - s0)
-        f_bwd += 5 * n * (n + 1) * w.dk // 2 * 2 + (12 if mode == LINEAR else 18) * n * w.dk * w.dv
-    f_bwd *= w.B * w.H
-    total = f_fwd_attn + f_fwd_upd + f_bwd
+        f_local += 5 * n * (n + 1) * w.dk
+        f_mem += (12 if mode == LINEAR else 18) * n * w.dk * w.dv
+    f_local *= w.B * w.H
+    f_mem *= w.B * w.H
+    total = f_fwd_attn + f_fwd_upd + f_local + f_mem
     tflops = total * world / (ms * 1e-3) / 1e12
+    tc_ms = phase_ms[api.PHASE_BWD_TC] / args.steps
+    peaks, peak_src = load_peaks()
+    if tc_ms > 0:  # the local attention's gradients on the tensor cores (bf16, head size 128)
+        sustained = tc_ms > 10.0
+        peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+        achieved = f_local / (tc_ms * 1e-3) / 1e12
+        roofline = {"kernel": "bwd_dq_tc_kernel + bwd_dkdv_tc_kernel", "bound": "tensor", "achieved": achieved,
+                    "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                    "peak_source": f"{peak_src} {'bf16_tflops_sustained' if sustained else 'bf16_tflops'}",
+                    "launch_ms": tc_ms, "flops_per_step": f_local}
+    else:
+        roofline = {"kernel": "backward (CUDA cores, fp32)", "bound": "alu", "achieved": tflops / world,
+                    "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s", "frac": tflops / world / FP32_ALU_TFLOPS,
+                    "peak_source": "148 SMs x 128 fp32 lanes x 2 (FMA) x 1.965 GHz"}
     result = {
         "metric": BACKWARD_METRIC, "value": w.B * w.L * world / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
@@ -683,10 +699,7 @@ def run_backward(args, w: W.Workload, mode: int):
         "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "N": w.N, "dk": w.dk, "dv": w.dv,
                    "mode": W.MODE_NAMES[mode], "step": "infini_attn_backward (forward recomputed inside)",
                    "l2": "1 GiB buffer written between timed steps (outside the step events)"},
-        "tflops": tflops, "flops_per_step": total,
-        "roofline": {"kernel": "backward (CUDA cores, fp32)", "bound": "alu", "achieved": tflops / world,
-                     "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s", "frac": tflops / world / FP32_ALU_TFLOPS,
-                     "peak_source": "148 SMs x 128 fp32 lanes x 2 (FMA) x 1.965 GHz"},
+        "tflops": tflops, "flops_per_step": total, "roofline": roofline,
         "phases_ms_per_step": {name: phase_ms[i] / args.steps for i, name in enumerate(PHASE_NAMES)},
         "gpu_launches": int(launches), "clocks": clocks,
     }

@@ -84,8 +84,8 @@ lib.infini_attn_layer_workspace_size.restype = ctypes.c_size_t
 lib.infini_attn_gemm_bf16.argtypes = [_vp, _vp, _vp, _l, _i, _i, _vp]
 lib.infini_attn_gemm_bf16.restype = _i
 
-PHASE_UPDATE, PHASE_STATE, PHASE_ATTN, PHASE_PRE, PHASE_PROJ, PHASE_BWD = 0, 1, 2, 3, 4, 5
-PHASES = 6
+PHASE_UPDATE, PHASE_STATE, PHASE_ATTN, PHASE_PRE, PHASE_PROJ, PHASE_BWD, PHASE_BWD_TC = 0, 1, 2, 3, 4, 5, 6
+PHASES = 7
 
 
 class InfiniAttnParams(ctypes.Structure):

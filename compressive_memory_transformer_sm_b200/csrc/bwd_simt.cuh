@@ -30,16 +30,13 @@
 //                       dz^(s) likewise; dM^(S), dz^(S) are given.
 //   sigma'(x) = 1 above zero, e^x at or below.
 //
-// Kernels (all deterministic: fixed summation orders, no atomics):
+// Kernels (all deterministic: fixed summation orders, no atomics; the memory
+// branch's register-tiled products -- bwd_qmem_kernel, bwd_outer_kernel,
+// bwd_upd_kernel -- are in bwd_mem.cuh):
 //   bwd_q_kernel     per (b, h, segment, 32 query rows): dq (local + memory
 //                    read), D, the dbeta row terms, d_num and d_den rows
-//   bwd_outer_kernel per (b, h, segment, token group): sigma(X)^T [Y | y0]
-//                    partials (X = Q with d_num / d_den, or K with the delta
-//                    rule's d_num_r / d_den_r)
 //   bwd_state_kernel the memory-gradient chain: a reverse scan of the
 //                    partials (linear rule) or one reverse step (delta rule)
-//   bwd_upd_kernel   per (b, h, segment, 128 key rows): the update's dk, dv
-//                    terms (and the delta rule's d_num_r, d_den_r rows)
 //   bwd_kv_kernel    per (b, h, segment, 32 key rows): dk, dv of the local
 //                    attention plus the update terms, one write
 //   bwd_beta_kernel  dbeta per head in a fixed order
@@ -208,175 +205,6 @@ __global__ void __launch_bounds__(256, 2)
   }
 }
 
-// The memory read's backward (Eq. 7) and the per-row terms for the tensor-core
-// path, where the local attention's gradients come from the tcgen05 kernels:
-// for 128 query rows of one (b, h, segment) (four passes of 32; warp w: rows
-// 4w .. 4w+3 of a pass, lane = column), D'_i = dO_i . A_dot_i (A_dot from the
-// forward's recomputation), the dbeta row term dO_i . (A_mem_i - A_dot_i), and
-// dq_mem = sigma'(q) (d_num M^T + d_den z) with d_num, d_den rows written for
-// the memory chain.  M^(s) is staged in shared memory once per block.
-template <typename T>
-__global__ void __launch_bounds__(256, 2) bwd_qmem_kernel(const T* __restrict__ q, const T* __restrict__ dout,
-                                                       const float* __restrict__ adot,
-                                                       const float* __restrict__ beta,
-                                                       const float* __restrict__ snapM,
-                                                       const float* __restrict__ snapz, BwdGeo g,
-                                                       int blocks_per_seg, float* __restrict__ dq_mem,
-                                                       float* __restrict__ Dp, float* __restrict__ brow,
-                                                       float* __restrict__ dnum, float* __restrict__ dden) {
-  extern __shared__ float sm[];
-  const int dk = g.dk, dv = g.dv, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  int idx = blockIdx.x;
-  const int blk = idx % blocks_per_seg;
-  idx /= blocks_per_seg;
-  const int s = idx % g.S;
-  const int bh = idx / g.S;
-  const int h = bh % g.H;
-  const long long seg_start = (long long)s * g.N;
-  const int n_s = (int)min((long long)g.N, g.L - seg_start);
-  const int r0 = blk * 128;
-  if (r0 >= n_s) return;
-  const int rend = min(n_s, r0 + 128);
-  const float gw = 1.f / (1.f + expf(-beta[h]));
-  float* Ms = sm;                  // [dk][dv + 1]
-  float* zs = Ms + dk * (dv + 1);  // [dk]
-  float* sq = zs + dk;             // [8 warps][dk] sigma(q) of the warp's current row
-  float* wn = sq + 8 * dk;         // [8 warps][dv] d_num of the warp's current row
-  const float* Mp = snapM + ((long long)bh * g.S + s) * dk * dv;
-  for (int e = tid; e < dk * dv; e += 256) Ms[(e / dv) * (dv + 1) + e % dv] = Mp[e];
-  for (int e = tid; e < dk; e += 256) zs[e] = snapz[((long long)bh * g.S + s) * dk + e];
-  __syncthreads();
-  float* sqw = sq + warp * dk;
-  float* wnw = wn + warp * dv;
-  for (int t = r0 + warp; t < rend; t += 8) {  // one row per warp at a time
-    const long long row = bwd_row(g, bh, seg_start + t);
-    float xq[4];
-    float dpart = 0.f;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int i = lane + 32 * c;
-      xq[c] = i < dk ? to_f32(q[row * dk + i]) : 0.f;
-      if (i < dk) {
-        const float sg = elu1_accurate(xq[c]);
-        sqw[i] = sg;
-        dpart = fmaf(sg, zs[i], dpart);
-      }
-    }
-    const float den = warp_sum(dpart);
-    __syncwarp();
-    float num[4] = {0.f, 0.f, 0.f, 0.f};
-    if (den != 0.f) {
-      for (int i = 0; i < dk; ++i) {
-        const float si = sqw[i];
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          if (lane + 32 * c < dv) num[c] = fmaf(si, Ms[i * (dv + 1) + lane + 32 * c], num[c]);
-      }
-    }
-    float dd = 0.f, bterm = 0.f, dpr = 0.f;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int j = lane + 32 * c;
-      if (j < dv) {
-        const float dA = to_f32(dout[row * dv + j]);
-        const float ad = adot[row * dv + j];
-        const float am = den != 0.f ? num[c] / den : 0.f;
-        dpr = fmaf(dA, ad, dpr);
-        bterm = fmaf(dA, am - ad, bterm);
-        float w = 0.f;
-        if (den != 0.f) {
-          w = gw * dA / den;
-          dd = fmaf(gw * dA, am, dd);
-        }
-        wnw[j] = w;
-        dnum[row * dv + j] = w;
-      }
-    }
-    const float d_den = den != 0.f ? -warp_sum(dd) / den : 0.f;
-    dpr = warp_sum(dpr);
-    bterm = warp_sum(bterm);
-    if (lane == 0) {
-      Dp[row] = dpr;
-      brow[row] = bterm;
-      dden[row] = d_den;
-    }
-    __syncwarp();
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int i = lane + 32 * c;
-      if (i < dk) {
-        float a = d_den * zs[i];
-        if (den != 0.f)
-          for (int j = 0; j < dv; ++j) a = fmaf(wnw[j], Ms[i * (dv + 1) + j], a);
-        dq_mem[row * dk + i] = sigma_prime(xq[c]) * a;
-      }
-    }
-    __syncwarp();
-  }
-}
-
-// Partials of sigma(X)^T Y (dk x dy) and sigma(X)^T y0 (dk) for the rows of
-// one (b, h, segment, token group); layout [BH][nseg][G][dk*dy + dk] like the
-// forward's update partials.  Rows of X: element strides given by rows of
-// length dk (contiguous [B, H, L, dk]); Y: fp32 [BH*L][dy]; y0: fp32 [BH*L].
-template <typename T>
-__global__ void __launch_bounds__(256) bwd_outer_kernel(const T* __restrict__ x, const float* __restrict__ Y,
-                                                        const float* __restrict__ y0, BwdGeo g, int dy, int seg0,
-                                                        int nseg, int G, int cpb, float* __restrict__ partial) {
-  extern __shared__ float sm[];
-  const int dk = g.dk, tid = threadIdx.x;
-  int idx = blockIdx.x;
-  const int grp = idx % G;
-  idx /= G;
-  const int sl = idx % nseg;
-  const int bh = idx / nseg;
-  const int s = seg0 + sl;
-  const long long seg_start = (long long)s * g.N;
-  const int n_s = (int)min((long long)g.N, g.L - seg_start);
-  const int t_begin = grp * cpb * 128;
-  const int t_end = min(n_s, t_begin + cpb * 128);
-  float* sx = sm;            // [32][dk]
-  float* sy = sx + 32 * dk;  // [32][dy + 1]: Y then y0
-  const int E = dk * dy;
-  float acc[64];
-#pragma unroll
-  for (int r = 0; r < 64; ++r) acc[r] = 0.f;
-  float accz = 0.f;
-  for (int t0 = t_begin; t0 < t_end; t0 += 32) {
-    const int nt = min(32, t_end - t0);
-    __syncthreads();
-    for (int e = tid; e < 32 * dk; e += 256) {
-      const int tt = e / dk, i = e - tt * dk;
-      sx[e] = tt < nt ? elu1_accurate(to_f32(x[bwd_row(g, bh, seg_start + t0 + tt) * dk + i])) : 0.f;
-    }
-    for (int e = tid; e < 32 * (dy + 1); e += 256) {
-      const int tt = e / (dy + 1), j = e - tt * (dy + 1);
-      const long long row = bwd_row(g, bh, seg_start + t0 + tt);
-      sy[e] = tt < nt ? (j < dy ? Y[row * dy + j] : y0[row]) : 0.f;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int r = 0; r < 64; ++r) {
-      const int e = tid + 256 * r;
-      if (e < E) {
-        const int i = e / dy, j = e - i * dy;
-        float a = acc[r];
-        for (int tt = 0; tt < nt; ++tt) a = fmaf(sx[tt * dk + i], sy[tt * (dy + 1) + j], a);
-        acc[r] = a;
-      }
-    }
-    if (tid < dk)
-      for (int tt = 0; tt < nt; ++tt) accz = fmaf(sx[tt * dk + tid], sy[tt * (dy + 1) + dy], accz);
-  }
-  float* out = partial + (((long long)bh * nseg + sl) * G + grp) * (long long)(E + dk);
-#pragma unroll
-  for (int r = 0; r < 64; ++r) {
-    const int e = tid + 256 * r;
-    if (e < E) out[e] = acc[r];
-  }
-  if (tid < dk) out[E + tid] = accz;
-}
-
 // The memory-gradient chain.  Thread e of block (x, bh) owns element e of
 // [dM (dk*dv) | dz (dk)] of head bh.
 //   op 0 (linear, all segments): from the given dM^(S), dz^(S) (or zeros),
@@ -428,131 +256,6 @@ __global__ void __launch_bounds__(256) bwd_state_kernel(float* __restrict__ runn
     running[(long long)bh * pst + e] = initial();
   } else {
     store0(running[(long long)bh * pst + e]);
-  }
-}
-
-// The update's gradient terms for 128 key rows of one (b, h, segment), in
-// four passes of 32 (warp w: rows 4w .. 4w+3 of a pass, lane = column).
-// gst: [dM | dz] gradient after the segment (G, gz), fp32, dk*dv + dk.
-// Writes dk_upd = sigma'(k) dsigma(K) and dv_upd (fp32 [BH*L][d]) and, for
-// the delta rule (snapM != nullptr), the rows d_num_r, d_den_r.
-template <typename T>
-__global__ void __launch_bounds__(256) bwd_upd_kernel(const T* __restrict__ k, const T* __restrict__ v, BwdGeo g,
-                                                      int seg0, const float* __restrict__ gstate, long long gstride_s,
-                                                      long long gstride_bh, const float* __restrict__ snapM,
-                                                      const float* __restrict__ snapz, float* __restrict__ dk_upd,
-                                                      float* __restrict__ dv_upd, float* __restrict__ dnum_r,
-                                                      float* __restrict__ dden_r, int blocks_per_seg) {
-  extern __shared__ float sm[];
-  const int dk = g.dk, dv = g.dv, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool delta = snapM != nullptr;
-  int idx = blockIdx.x;
-  const int blk = idx % blocks_per_seg;
-  idx /= blocks_per_seg;
-  const int sl = idx % (delta ? 1 : g.S);
-  const int bh = idx / (delta ? 1 : g.S);
-  const int s = seg0 + sl;
-  const long long seg_start = (long long)s * g.N;
-  const int n_s = (int)min((long long)g.N, g.L - seg_start);
-  const int r0 = blk * 128;
-  if (r0 >= n_s) return;
-  float* Gs = sm;                     // [dk][dv + 1]
-  float* Ms = Gs + dk * (dv + 1);     // [dk][dv + 1] (delta)
-  float* gz = Ms + (delta ? dk * (dv + 1) : 0);  // [dk]
-  float* zs = gz + dk;                // [dk] (delta)
-  float* sk = zs + dk;                // [32][dk]
-  float* U = sk + 32 * dk;            // [32][dv]
-  float* W = U + 32 * dv;             // [32][dv]  dR / den (delta)
-  const float* gp = gstate + (long long)bh * gstride_bh + (long long)s * gstride_s;
-  for (int e = tid; e < dk * dv; e += 256) Gs[(e / dv) * (dv + 1) + e % dv] = gp[e];
-  for (int e = tid; e < dk; e += 256) gz[e] = gp[dk * dv + e];
-  const float* Mp = delta ? snapM + ((long long)bh * g.S + s) * dk * dv : nullptr;
-  if (delta) {
-    for (int e = tid; e < dk * dv; e += 256) Ms[(e / dv) * (dv + 1) + e % dv] = Mp[e];
-    for (int e = tid; e < dk; e += 256) zs[e] = snapz[((long long)bh * g.S + s) * dk + e];
-  }
-  const int rend = min(n_s, r0 + 128);
-  for (int t0 = r0; t0 < rend; t0 += 32) {
-    __syncthreads();
-    for (int e = tid; e < 32 * dk; e += 256) {
-      const int tt = e / dk, i = e - tt * dk;
-      sk[e] = t0 + tt < rend ? to_f32(k[bwd_row(g, bh, seg_start + t0 + tt) * dk + i]) : 0.f;
-    }
-    for (int e = tid; e < 32 * dv; e += 256) {
-      const int tt = e / dv, j = e - tt * dv;
-      U[e] = t0 + tt < rend ? to_f32(v[bwd_row(g, bh, seg_start + t0 + tt) * dv + j]) : 0.f;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int rr = 0; rr < 4; ++rr) {
-      const int r = warp * 4 + rr;
-      const int t = t0 + r;
-      if (t >= rend) continue;  // warp-uniform
-      const long long row = bwd_row(g, bh, seg_start + t);
-      float* kr = sk + r * dk;  // raw k, then sigma(k) below
-      float* ur = U + r * dv;
-      float* wr = W + r * dv;
-      float xk[4];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) xk[c] = lane + 32 * c < dk ? kr[lane + 32 * c] : 0.f;
-      __syncwarp();
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-        if (lane + 32 * c < dk) kr[lane + 32 * c] = elu1_accurate(xk[c]);
-      __syncwarp();
-      float den = 0.f;
-      if (delta) {
-        float d = 0.f;
-        for (int i = lane; i < dk; i += 32) d = fmaf(kr[i], zs[i], d);
-        den = warp_sum(d);
-      }
-      // dU = sigma(k) G (the dv_upd row), and R = sigma(k) M^(s) / den (delta)
-      float du[4] = {0.f, 0.f, 0.f, 0.f}, rv[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int i = 0; i < dk; ++i) {
-        const float ski = kr[i];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int col = lane + 32 * c;
-          if (col < dv) {
-            du[c] = fmaf(ski, Gs[i * (dv + 1) + col], du[c]);
-            if (delta) rv[c] = fmaf(ski, Ms[i * (dv + 1) + col], rv[c]);
-          }
-        }
-      }
-      float dd = 0.f;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int col = lane + 32 * c;
-        if (col < dv) {
-          dv_upd[row * dv + col] = du[c];
-          if (delta) {
-            const float R = den != 0.f ? rv[c] / den : 0.f;
-            ur[col] -= R;  // U = V - R
-            const float w = den != 0.f ? -du[c] / den : 0.f;  // d_num_r = dR / den, dR = -dU
-            wr[col] = w;
-            dnum_r[row * dv + col] = w;
-            dd = fmaf(-du[c], R, dd);
-          }
-        }
-      }
-      const float d_den = delta && den != 0.f ? -warp_sum(dd) / den : 0.f;
-      if (delta && lane == 0) dden_r[row] = d_den;
-      __syncwarp();
-      // dsigma(k)_i = sum_j U_j G_ij + gz_i (+ sum_j d_num_r_j M_ij + d_den_r z_i)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int col = lane + 32 * c;
-        if (col < dk) {
-          float a = gz[col];
-          for (int j = 0; j < dv; ++j) a = fmaf(ur[j], Gs[col * (dv + 1) + j], a);
-          if (delta) {
-            for (int j = 0; j < dv; ++j) a = fmaf(wr[j], Ms[col * (dv + 1) + j], a);
-            a = fmaf(d_den, zs[col], a);
-          }
-          dk_upd[row * dk + col] = sigma_prime(xk[c]) * a;
-        }
-      }
-    }
   }
 }
 

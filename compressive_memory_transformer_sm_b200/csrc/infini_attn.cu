@@ -29,6 +29,7 @@
 #include "common.cuh"
 #include "simt.cuh"
 #include "bwd_simt.cuh"
+#include "bwd_mem.cuh"
 #include "decode.cuh"
 #include "rope.cuh"
 #include "sm100_attn.cuh"
@@ -50,7 +51,8 @@ constexpr int kFlagUpdateOnly = 0x1000;
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 // ------------------------------------------------------------ launch accounting
-enum Phase { kPhaseUpdate = 0, kPhaseState = 1, kPhaseAttn = 2, kPhasePre = 3, kPhaseProj = 4, kPhaseBwd = 5, kPhases = 6 };
+enum Phase { kPhaseUpdate = 0, kPhaseState = 1, kPhaseAttn = 2, kPhasePre = 3, kPhaseProj = 4, kPhaseBwd = 5, kPhaseBwdTc = 6,
+             kPhases = 7 };
 std::atomic<long long> g_launches{0};
 std::atomic<int> g_profile_mask{0};
 struct EventPair {
@@ -824,7 +826,7 @@ int run_backward(const infini_attn_bwd_params& p, const BwdPlan& bp, char* ws) {
       return INFINI_ERR_LAUNCH;
     if (set_tc_smem_limits() != INFINI_OK) return INFINI_ERR_LAUNCH;
     // the memory read's backward and D' = dO . A_dot on CUDA cores
-    const size_t qm_smem = (size_t)(dk * (dv + 1) + dk + 8 * dk + 8 * dv) * 4;
+    const size_t qm_smem = (size_t)(3 * 128 * kMP + 3 * 128) * 4;
     cudaFuncSetAttribute(bwd_qmem_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qm_smem);
     {
       LaunchScope ls(kPhaseBwd, st);
@@ -839,7 +841,7 @@ int run_backward(const infini_attn_bwd_params& p, const BwdPlan& bp, char* ws) {
     ta.B = p.B; ta.H = p.H; ta.S = f.S; ta.T = (p.N + 127) / 128; ta.L = p.L; ta.N = p.N;
     ta.scale = scale; ta.scale_log2 = scale * 1.4426950408889634f;
     ta.out0 = static_cast<__nv_bfloat16*>(p.dq);
-    LaunchScope ls(kPhaseBwd, st);
+    LaunchScope ls(kPhaseBwdTc, st);
     tc::bwd_dq_tc_kernel<<<(unsigned)((long long)ta.T * BH * f.S), tc::kBwdThreads, tc::kDQSmem, st>>>(tm_q, tm_k, tm_v,
                                                                                                     tm_do, ta);
   } else {
@@ -850,7 +852,7 @@ int run_backward(const infini_attn_bwd_params& p, const BwdPlan& bp, char* ws) {
         q, k, v, dout, p.beta, adot, lse, snapM, snapz, g, scale, QT, static_cast<T*>(p.dq), Drow, brow, dnum, dden);
   }
   // 3. the memory read's partials sigma(Q)^T [d_num | d_den] of every segment
-  const size_t outer_smem = (size_t)(32 * dk + 32 * (dv + 1)) * 4;
+  const size_t outer_smem = (size_t)(64 * kMP + 64 * 130) * 4;
   cudaFuncSetAttribute(bwd_outer_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)outer_smem);
   {
     LaunchScope ls(kPhaseBwd, st);
@@ -859,7 +861,8 @@ int run_backward(const infini_attn_bwd_params& p, const BwdPlan& bp, char* ws) {
   }
   const dim3 sgrid((unsigned)((E + dk + 255) / 256), BH);
   const size_t pst = E + dk;
-  const size_t upd_smem = (size_t)((f.delta ? 2 : 1) * dk * (dv + 1) + 2 * dk + 32 * dk + 2 * 32 * dv) * 4;
+  const size_t upd_smem = (size_t)((f.delta ? 2 : 1) * (128 + 64) * kMP + 2 * 128 + 2 * 64) * 4;
+  const int bps64 = (int)((std::min<long long>(p.N, p.L) + 63) / 64);  // update terms: 64 rows per block
   cudaFuncSetAttribute(bwd_upd_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)upd_smem);
   // 4. the memory-gradient chain and the update's dk, dv terms
   if (!f.delta) {
@@ -869,8 +872,8 @@ int run_backward(const infini_attn_bwd_params& p, const BwdPlan& bp, char* ws) {
                                               p.dM0, p.dz0);
     }
     LaunchScope ls(kPhaseBwd, st);
-    bwd_upd_kernel<T><<<(unsigned)((long long)BH * f.S * bps), 256, upd_smem, st>>>(
-        k, v, g, 0, gst, (long long)pst, (long long)f.S * pst, nullptr, nullptr, dkupd, dvupd, nullptr, nullptr, bps);
+    bwd_upd_kernel<T><<<(unsigned)((long long)BH * f.S * bps64), 256, upd_smem, st>>>(
+        k, v, g, 0, gst, (long long)pst, (long long)f.S * pst, nullptr, nullptr, dkupd, dvupd, nullptr, nullptr, bps64);
   } else {
     {
       LaunchScope ls(kPhaseBwd, st);
@@ -880,8 +883,8 @@ int run_backward(const infini_attn_bwd_params& p, const BwdPlan& bp, char* ws) {
     for (int s = f.S - 1; s >= 0; --s) {
       {
         LaunchScope ls(kPhaseBwd, st);
-        bwd_upd_kernel<T><<<(unsigned)((long long)BH * bps), 256, upd_smem, st>>>(
-            k, v, g, s, gst, 0, (long long)pst, snapM, snapz, dkupd, dvupd, dnumr, ddenr, bps);
+        bwd_upd_kernel<T><<<(unsigned)((long long)BH * bps64), 256, upd_smem, st>>>(
+            k, v, g, s, gst, 0, (long long)pst, snapM, snapz, dkupd, dvupd, dnumr, ddenr, bps64);
       }
       {
         LaunchScope ls(kPhaseBwd, st);
@@ -900,7 +903,7 @@ int run_backward(const infini_attn_bwd_params& p, const BwdPlan& bp, char* ws) {
   if (bp.tc) {
     ta.out0 = static_cast<__nv_bfloat16*>(p.dk);
     ta.out1 = static_cast<__nv_bfloat16*>(p.dv);
-    LaunchScope ls(kPhaseBwd, st);
+    LaunchScope ls(kPhaseBwdTc, st);
     tc::bwd_dkdv_tc_kernel<<<(unsigned)((long long)ta.T * BH * f.S), tc::kBwdThreads, tc::kKVSmem, st>>>(
         tm_q, tm_k, tm_v, tm_do, ta);
   } else {

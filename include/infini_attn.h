@@ -343,13 +343,14 @@ INFINI_API int infini_attn_selftest_timeout(unsigned limit_us, cudaStream_t stre
  * Kernel timing for benchmarks.  phase_mask selects phases (bit 0 = memory
  * update kernels, bit 1 = state/snapshot kernels, bit 2 = attention
  * kernel, bit 3 = position-embedding pre-pass, bit 4 = projection GEMMs of
- * the full layer, bit 5 = backward kernels); while a bit is set, every
+ * the full layer, bit 5 = backward kernels on CUDA cores, bit 6 = backward
+ * kernels on the tensor cores); while a bit is set, every
  * launch of that phase is bracketed by two CUDA events recorded on the
  * launch's stream.  0 turns timing off.
  */
 INFINI_API int infini_attn_profile_enable(int phase_mask);
 /*
- * Synchronises the recorded events and adds, per phase p in 0..5, the
+ * Synchronises the recorded events and adds, per phase p in 0..6, the
  * elapsed milliseconds to ms[p] and the number of timed launches to
  * launches[p], for everything recorded since the last reset; reset != 0
  * then drops the records.  Either array may be NULL.
