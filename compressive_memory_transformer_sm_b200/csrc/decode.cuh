@@ -140,3 +140,133 @@ __global__ void __launch_bounds__(128)
 }
 
 }  // namespace infini
+
+namespace infini {
+
+// ------------------------------------------------------------------ fused decode
+// The split decode in one launch: the CTAs of the key ranges of one (b, h)
+// form a thread-block cluster (grid splits x B*H, cluster splits x 1); each
+// computes its range's softmax state into its own shared memory, and after a
+// cluster barrier rank 0 reads the others' states through distributed shared
+// memory, merges them in rank order (deterministic), adds the memory read
+// (Eq. 7) and the gate (Eq. 10) and writes the row; a second barrier keeps
+// every CTA's shared memory alive until rank 0 is done.  No global scratch.
+// CTA 0 also appends k_t, v_t to row n - 1 of the caches (no CTA reads it).
+constexpr int kDecodeMaxSplits = 16;
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+    decode_fused_kernel(const T* __restrict__ q, const T* __restrict__ k_t, const T* __restrict__ v_t,
+                        T* __restrict__ kc, T* __restrict__ vc, const float* __restrict__ beta,
+                        const float* __restrict__ M, const float* __restrict__ z, T* __restrict__ out, int H, int N,
+                        int n, int dk, int dv, float scale, int per) {
+  __shared__ float qs[128];
+  __shared__ float wm[8], wl[8], wacc[8][128];
+  __shared__ __align__(16) float st[2 + 128];  // this range's state: m, l, o[dv]
+  __shared__ float sq[128];
+  __shared__ float red[8];
+  const int split = blockIdx.x, bh = blockIdx.y, splits = gridDim.x;
+  const int h = bh % H;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (split == 0) {
+    for (int i = tid; i < dk; i += 256) kc[((long long)bh * N + n - 1) * dk + i] = k_t[(long long)bh * dk + i];
+    for (int i = tid; i < dv; i += 256) vc[((long long)bh * N + n - 1) * dv + i] = v_t[(long long)bh * dv + i];
+  }
+  for (int i = tid; i < dk; i += 256) qs[i] = to_f32(q[(long long)bh * dk + i]);
+  __syncthreads();
+  const int j0 = split * per, j1 = min(n, j0 + per);
+  const T* kb = kc + (long long)bh * N * dk;
+  const T* vb = vc + (long long)bh * N * dv;
+  float m = -INFINITY, l = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int jb = j0 + 32 * warp; jb < j1; jb += 256) {
+    const int j = jb + lane;
+    float s = -INFINITY;
+    if (j < j1) {
+      const T* kr = j == n - 1 ? k_t + (long long)bh * dk : kb + (long long)j * dk;
+      float d = 0.f;
+      for (int i = 0; i < dk; ++i) d = fmaf(qs[i], to_f32(kr[i]), d);
+      s = d * scale;
+    }
+    const float mn = fmaxf(m, warp_max(s));
+    const float alpha = expf(m - mn);  // 0 while m = -inf
+    const float p = j < j1 ? expf(s - mn) : 0.f;
+    l = l * alpha + warp_sum(p);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[c] *= alpha;
+    const int cnt = min(32, j1 - jb);
+    for (int jj = 0; jj < cnt; ++jj) {
+      const float pj = __shfl_sync(0xffffffffu, p, jj);
+      const int key = jb + jj;
+      const T* vr = key == n - 1 ? v_t + (long long)bh * dv : vb + (long long)key * dv;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int d = lane + 32 * c;
+        if (d < dv) acc[c] = fmaf(pj, to_f32(vr[d]), acc[c]);
+      }
+    }
+    m = mn;
+  }
+  if (lane == 0) {
+    wm[warp] = m;
+    wl[warp] = l;
+  }
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+    if (lane + 32 * c < dv) wacc[warp][lane + 32 * c] = acc[c];
+  __syncthreads();
+  {
+    float gm = -INFINITY;
+    for (int w = 0; w < 8; ++w) gm = fmaxf(gm, wm[w]);
+    if (tid == 0) {
+      float gl = 0.f;
+      for (int w = 0; w < 8; ++w) gl += gm == -INFINITY ? 0.f : wl[w] * expf(wm[w] - gm);
+      st[0] = gm;
+      st[1] = gl;
+    }
+    for (int c = tid; c < dv; c += 256) {
+      float o = 0.f;
+      for (int w = 0; w < 8; ++w) o += gm == -INFINITY ? 0.f : wacc[w][c] * expf(wm[w] - gm);
+      st[2 + c] = o;
+    }
+  }
+  cluster_sync();  // every range's state is in its CTA's shared memory
+  if (split == 0) {
+    // memory read: sigma(q), den = sigma(q) . z
+    const float* zh = z + (long long)bh * dk;
+    for (int i = tid; i < dk; i += 256) sq[i] = elu1_accurate(qs[i]);
+    __syncthreads();
+    float d = 0.f;
+    for (int i = tid; i < dk; i += 256) d = fmaf(sq[i], zh[i], d);
+    d = warp_sum(d);
+    if (lane == 0) red[warp] = d;
+    __syncthreads();
+    float den = 0.f;
+    for (int w = 0; w < 8; ++w) den += red[w];
+    const uint32_t sbase = smem_u32(st);
+    float gm = -INFINITY;
+    for (int r = 0; r < splits; ++r) gm = fmaxf(gm, ld_dsmem_f32(mapa_shared(sbase, (uint32_t)r)));
+    float gl = 0.f;
+    for (int r = 0; r < splits; ++r) {
+      const uint32_t a = mapa_shared(sbase, (uint32_t)r);
+      const float mr = ld_dsmem_f32(a);
+      gl += mr == -INFINITY ? 0.f : ld_dsmem_f32(a + 4u) * expf(mr - gm);
+    }
+    const float g = 1.f / (1.f + expf(-beta[h]));
+    const float* Mh = M + (long long)bh * dk * dv;
+    for (int c = tid; c < dv; c += 256) {
+      float o = 0.f;
+      for (int r = 0; r < splits; ++r) {
+        const uint32_t a = mapa_shared(sbase, (uint32_t)r);
+        const float mr = ld_dsmem_f32(a);
+        o += mr == -INFINITY ? 0.f : ld_dsmem_f32(a + 4u * (uint32_t)(2 + c)) * expf(mr - gm);
+      }
+      float num = 0.f;
+      for (int i = 0; i < dk; ++i) num = fmaf(sq[i], Mh[(long long)i * dv + c], num);
+      const float a_mem = den != 0.f ? num / den : 0.f;
+      out[(long long)bh * dv + c] = from_f32<T>(g * a_mem + (1.f - g) * (o / gl));
+    }
+  }
+  cluster_sync();  // rank 0 has read every state
+}
+
+}  // namespace infini

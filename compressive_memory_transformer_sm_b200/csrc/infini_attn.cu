@@ -1041,6 +1041,9 @@ bool layer_plan(int B, int H, long long L, int N, int d_model, int mode, LayerPl
   return true;
 }
 
+int decode_fold(void* k_cache, void* v_cache, const float* beta, float* M, float* z, int B, int H, int N, int n,
+                int dk, int dv, int mode, cudaStream_t stream);
+
 }  // namespace
 
 extern "C" {
@@ -1128,19 +1131,57 @@ int infini_attn_decode_step(const void* q_t, const void* k_t, const void* v_t, v
   if (B <= 0 || H <= 0 || N <= 0 || dk <= 0 || dv <= 0 || pos < 0 || pos >= N) return INFINI_ERR_INVALID_ARG;
   if ((mode & ~(INFINI_DELTA | INFINI_F32)) != 0 || dk > 128 || dv > 128) return INFINI_ERR_UNSUPPORTED;
   const bool f32 = (mode & INFINI_F32) != 0;
-  const size_t es = f32 ? 4 : 2;
   const long long BH = (long long)B * H;
   if (BH > (1LL << 31) - 1) return INFINI_ERR_UNSUPPORTED;
   int rc = check_device(false);
   if (rc != INFINI_OK) return rc;
   const int n = pos + 1;
+  const float scale = 1.f / sqrtf((float)dk);
   // 1 + 2. the token's output, its key and value appended to the caches by the
-  // same launch: keys split over enough CTAs to fill the GPU (ranges of at
-  // least 64 keys), then one merge per (b, h)
+  // same launch: one thread-block cluster per (b, h) over up to 8 key ranges
+  // of at least 64 keys, merged through distributed shared memory
+  if (BH <= 65535) {
+    const long long want = std::max<long long>(1, std::min<long long>(8, (2LL * kSms + BH - 1) / BH));
+    const int per = (int)std::max<long long>(64, (n + want - 1) / want);
+    const int splits = (n + per - 1) / per;  // <= 8
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)splits;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3((unsigned)splits, (unsigned)BH);
+    cfg.blockDim = dim3(256);
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e;
+    {
+      LaunchScope ls(kPhaseAttn, stream);
+      if (f32)
+        e = cudaLaunchKernelEx(&cfg, decode_fused_kernel<float>, static_cast<const float*>(q_t),
+                               static_cast<const float*>(k_t), static_cast<const float*>(v_t),
+                               static_cast<float*>(k_cache), static_cast<float*>(v_cache), beta, (const float*)M,
+                               (const float*)z, static_cast<float*>(out), H, N, n, dk, dv, scale, per);
+      else
+        e = cudaLaunchKernelEx(&cfg, decode_fused_kernel<__nv_bfloat16>, static_cast<const __nv_bfloat16*>(q_t),
+                               static_cast<const __nv_bfloat16*>(k_t), static_cast<const __nv_bfloat16*>(v_t),
+                               static_cast<__nv_bfloat16*>(k_cache), static_cast<__nv_bfloat16*>(v_cache), beta,
+                               (const float*)M, (const float*)z, static_cast<__nv_bfloat16*>(out), H, N, n, dk, dv,
+                               scale, per);
+    }
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return INFINI_ERR_LAUNCH;
+    }
+    if (!(fold || pos == N - 1)) return INFINI_OK;
+    return decode_fold(k_cache, v_cache, beta, M, z, B, H, N, n, dk, dv, mode, stream);
+  }
+  // more (b, h) than a grid's second dimension holds: ranges on the second
+  // dimension, partial states in a scratch buffer, a second launch merges
   const long long want = std::max<long long>(1, (2LL * kSms + BH - 1) / BH);
   int per = (int)std::max<long long>(64, (n + want - 1) / want);
   const int splits = (n + per - 1) / per;
-  const float scale = 1.f / sqrtf((float)dk);
   void* scratch = nullptr;
   if (cudaMallocAsync(&scratch, (size_t)splits * BH * (dv + 2) * 4, stream) != cudaSuccess) {
     cudaGetLastError();
@@ -1173,8 +1214,16 @@ int infini_attn_decode_step(const void* q_t, const void* k_t, const void* v_t, v
   rc = launch_status();
   if (cudaFreeAsync(scratch, stream) != cudaSuccess && rc == INFINI_OK) rc = INFINI_ERR_WORKSPACE;
   if (rc != INFINI_OK || !(fold || pos == N - 1)) return rc;
-  // 3. the segment is complete: fold its keys and values into M, z with the
-  // forward's update kernels alone (no attention, no output)
+  return decode_fold(k_cache, v_cache, beta, M, z, B, H, N, n, dk, dv, mode, stream);
+}
+
+}  // extern "C"
+
+namespace {
+// 3. the segment is complete: fold its n keys and values into M, z with the
+// forward's update kernels alone (no attention, no output).
+int decode_fold(void* k_cache, void* v_cache, const float* beta, float* M, float* z, int B, int H, int N, int n,
+                int dk, int dv, int mode, cudaStream_t stream) {
   infini_attn_params p;
   memset(&p, 0, sizeof(p));
   p.q = k_cache;
@@ -1200,9 +1249,11 @@ int infini_attn_decode_step(const void* q_t, const void* k_t, const void* v_t, v
     p.o_stride[i] = vs[i];
   }
   p.stream = stream;
-  (void)es;
   return forward_impl(p);
 }
+}  // namespace
+
+extern "C" {
 
 int infini_attn_gemm_bf16(const void* A, const void* Bm, void* C, long M, int N, int K, cudaStream_t stream) {
   if (!A || !Bm || !C) return INFINI_ERR_INVALID_ARG;
