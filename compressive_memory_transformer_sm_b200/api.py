@@ -153,7 +153,7 @@ def _args(where: str, shapes: dict, contiguous: bool = True):
             raise TypeError(f"{where}: {name} must be a torch.Tensor")
         if t.dim() != ndim:
             raise ValueError(f"{where}: {name} must have {ndim} dimensions, got shape {tuple(t.shape)}")
-        if t.device.type != "cuda":
+        if not t.is_cuda:
             raise ValueError(f"{where}: {name} must be on a CUDA device, got {t.device}")
         if contiguous and not t.is_contiguous():
             raise ValueError(f"{where}: {name} must be contiguous (use infini_attn_forward_ex for strided views)")

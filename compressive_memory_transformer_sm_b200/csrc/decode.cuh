@@ -154,12 +154,45 @@ namespace infini {
 // CTA 0 also appends k_t, v_t to row n - 1 of the caches (no CTA reads it).
 constexpr int kDecodeMaxSplits = 16;
 
+// q . k for one cached key row of dk elements: 16-byte vector loads when
+// `vec` (dk a multiple of 8 for bf16 / 4 for fp32 and 16-byte aligned rows),
+// scalar loads otherwise.
+template <typename T>
+__device__ __forceinline__ float decode_dot(const float* qs, const T* kr, int dk, bool vec) {
+  float d = 0.f;
+  if (vec) {
+    const uint4* k4 = reinterpret_cast<const uint4*>(kr);
+    if constexpr (sizeof(T) == 2) {
+      for (int c = 0; c < dk / 8; ++c) {
+        const uint4 w = __ldg(k4 + c);
+        const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          d = fmaf(qs[8 * c + 2 * e], bf16_lo(u[e]), d);
+          d = fmaf(qs[8 * c + 2 * e + 1], bf16_hi(u[e]), d);
+        }
+      }
+    } else {
+      for (int c = 0; c < dk / 4; ++c) {
+        const float4 w = __ldg(reinterpret_cast<const float4*>(k4 + c));
+        d = fmaf(qs[4 * c], w.x, d);
+        d = fmaf(qs[4 * c + 1], w.y, d);
+        d = fmaf(qs[4 * c + 2], w.z, d);
+        d = fmaf(qs[4 * c + 3], w.w, d);
+      }
+    }
+  } else {
+    for (int i = 0; i < dk; ++i) d = fmaf(qs[i], to_f32(kr[i]), d);
+  }
+  return d;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256)
     decode_fused_kernel(const T* __restrict__ q, const T* __restrict__ k_t, const T* __restrict__ v_t,
                         T* __restrict__ kc, T* __restrict__ vc, const float* __restrict__ beta,
                         const float* __restrict__ M, const float* __restrict__ z, T* __restrict__ out, int H, int N,
-                        int n, int dk, int dv, float scale, int per) {
+                        int n, int dk, int dv, float scale, int per, int vec) {
   __shared__ float qs[128];
   __shared__ float wm[8], wl[8], wacc[8][128];
   __shared__ __align__(16) float st[2 + 128];  // this range's state: m, l, o[dv]
@@ -183,9 +216,7 @@ __global__ void __launch_bounds__(256)
     float s = -INFINITY;
     if (j < j1) {
       const T* kr = j == n - 1 ? k_t + (long long)bh * dk : kb + (long long)j * dk;
-      float d = 0.f;
-      for (int i = 0; i < dk; ++i) d = fmaf(qs[i], to_f32(kr[i]), d);
-      s = d * scale;
+      s = decode_dot<T>(qs, kr, dk, vec != 0) * scale;
     }
     const float mn = fmaxf(m, warp_max(s));
     const float alpha = expf(m - mn);  // 0 while m = -inf

@@ -1141,9 +1141,30 @@ int infini_attn_decode_step(const void* q_t, const void* k_t, const void* v_t, v
   // same launch: one thread-block cluster per (b, h) over up to 8 key ranges
   // of at least 64 keys, merged through distributed shared memory
   if (BH <= 65535) {
-    const long long want = std::max<long long>(1, std::min<long long>(8, (2LL * kSms + BH - 1) / BH));
-    const int per = (int)std::max<long long>(64, (n + want - 1) / want);
-    const int splits = (n + per - 1) / per;  // <= 8
+    const long long want =
+        std::max<long long>(1, std::min<long long>(kDecodeMaxSplits, (2LL * kSms + BH - 1) / BH));
+    int per = (int)std::max<long long>(64, (n + want - 1) / want);
+    int splits = (n + per - 1) / per;  // <= 16: a non-portable cluster size beyond 8
+    // 16-byte row loads: rows of a multiple of 16 bytes, 16-byte aligned bases
+    const size_t es = f32 ? 4 : 2;
+    const int vec = ((size_t)dk * es) % 16 == 0 && reinterpret_cast<uintptr_t>(k_cache) % 16 == 0 &&
+                    reinterpret_cast<uintptr_t>(k_t) % 16 == 0;
+    {
+      static std::mutex mu;
+      static std::vector<unsigned long long> done;  // contexts with the cluster-size attribute set
+      const unsigned long long ctx = current_context_id();
+      std::lock_guard<std::mutex> lk(mu);
+      if (ctx == 0 || std::find(done.begin(), done.end(), ctx) == done.end()) {
+        if (cudaFuncSetAttribute(decode_fused_kernel<float>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(decode_fused_kernel<__nv_bfloat16>,
+                                 cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+          cudaGetLastError();
+          return INFINI_ERR_LAUNCH;
+        }
+        if (ctx != 0) done.push_back(ctx);
+      }
+    }
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1155,20 +1176,30 @@ int infini_attn_decode_step(const void* q_t, const void* k_t, const void* v_t, v
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e;
-    {
+    cudaError_t e = cudaSuccess;
+    for (int attempt = 0; attempt < 2; ++attempt) {
+      if (attempt == 1) {
+        // a 16-CTA cluster could not be placed: ranges for clusters of at most 8
+        if (splits <= 8) break;
+        cudaGetLastError();
+        per = std::max(64, (n + 7) / 8);
+        splits = (n + per - 1) / per;
+        attr[0].val.clusterDim.x = (unsigned)splits;
+        cfg.gridDim = dim3((unsigned)splits, (unsigned)BH);
+      }
       LaunchScope ls(kPhaseAttn, stream);
       if (f32)
         e = cudaLaunchKernelEx(&cfg, decode_fused_kernel<float>, static_cast<const float*>(q_t),
                                static_cast<const float*>(k_t), static_cast<const float*>(v_t),
                                static_cast<float*>(k_cache), static_cast<float*>(v_cache), beta, (const float*)M,
-                               (const float*)z, static_cast<float*>(out), H, N, n, dk, dv, scale, per);
+                               (const float*)z, static_cast<float*>(out), H, N, n, dk, dv, scale, per, vec);
       else
         e = cudaLaunchKernelEx(&cfg, decode_fused_kernel<__nv_bfloat16>, static_cast<const __nv_bfloat16*>(q_t),
                                static_cast<const __nv_bfloat16*>(k_t), static_cast<const __nv_bfloat16*>(v_t),
                                static_cast<__nv_bfloat16*>(k_cache), static_cast<__nv_bfloat16*>(v_cache), beta,
                                (const float*)M, (const float*)z, static_cast<__nv_bfloat16*>(out), H, N, n, dk, dv,
-                               scale, per);
+                               scale, per, vec);
+      if (e == cudaSuccess) break;
     }
     if (e != cudaSuccess) {
       cudaGetLastError();
