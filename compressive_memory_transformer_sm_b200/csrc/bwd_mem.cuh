@@ -45,6 +45,74 @@ __device__ __forceinline__ float row16_sum(float x) {
 // sigma'(x) from sigma(x): 1 above zero (sigma > 1), e^x = sigma at or below.
 __device__ __forceinline__ float sigma_prime_of(float sg) { return sg > 1.f ? 1.f : sg; }
 
+// Stage rows x cols of a row-major fp32 matrix (row stride `cols`) into a
+// [rows_tile][kMP] shared tile, zero beyond nrows x cols (the tile is
+// rows_tile x 128).  float4 loads when cols % 4 == 0 and src is 16-byte aligned.
+__device__ __forceinline__ void stage_f32(float* __restrict__ dst, const float* __restrict__ src, int rows_tile,
+                                          int nrows, int cols) {
+  const bool vec = (cols & 3) == 0 && (reinterpret_cast<uintptr_t>(src) & 15) == 0;
+  if (vec) {
+    for (int e = threadIdx.x; e < rows_tile * 32; e += blockDim.x) {
+      const int r = e >> 5, c = (e & 31) * 4;
+      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (r < nrows && c < cols) x = __ldg(reinterpret_cast<const float4*>(src + (long long)r * cols + c));
+      float* d = dst + r * kMP + c;
+      d[0] = x.x;
+      d[1] = x.y;
+      d[2] = x.z;
+      d[3] = x.w;
+    }
+  } else {
+    for (int e = threadIdx.x; e < rows_tile * 128; e += blockDim.x) {
+      const int r = e >> 7, c = e & 127;
+      dst[r * kMP + c] = (r < nrows && c < cols) ? src[(long long)r * cols + c] : 0.f;
+    }
+  }
+}
+
+// Stage sigma(x) of rows x cols elements of a row-major T matrix (row stride
+// `cols`) into a [rows_tile][kMP] shared tile, zero elsewhere; 16-byte loads
+// when a row is a whole number of 16-byte chunks and src is aligned.
+template <typename T>
+__device__ __forceinline__ void stage_sigma(float* __restrict__ dst, const T* __restrict__ src, int rows_tile,
+                                            int nrows, int cols) {
+  constexpr int PER = 16 / (int)sizeof(T);  // elements per 16 bytes
+  const bool vec = cols % PER == 0 && (reinterpret_cast<uintptr_t>(src) & 15) == 0;
+  if (vec) {
+    constexpr int CH = 128 / PER;  // 16-byte chunks per 128 columns
+    for (int e = threadIdx.x; e < rows_tile * CH; e += blockDim.x) {
+      const int r = e / CH, c = (e % CH) * PER;
+      float x[PER];
+      if (r < nrows && c < cols) {
+        const uint4 w = __ldg(reinterpret_cast<const uint4*>(src + (long long)r * cols + c));
+        if constexpr (sizeof(T) == 2) {
+          const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            x[2 * i] = elu1_accurate(bf16_lo(u[i]));
+            x[2 * i + 1] = elu1_accurate(bf16_hi(u[i]));
+          }
+        } else {
+          x[0] = elu1_accurate(__uint_as_float(w.x));
+          x[1] = elu1_accurate(__uint_as_float(w.y));
+          x[2] = elu1_accurate(__uint_as_float(w.z));
+          x[3] = elu1_accurate(__uint_as_float(w.w));
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < PER; ++i) x[i] = 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < PER; ++i) dst[r * kMP + c + i] = x[i];
+    }
+  } else {
+    for (int e = threadIdx.x; e < rows_tile * 128; e += blockDim.x) {
+      const int r = e >> 7, c = e & 127;
+      dst[r * kMP + c] = (r < nrows && c < cols) ? elu1_accurate(to_f32(src[(long long)r * cols + c])) : 0.f;
+    }
+  }
+}
+
 // Memory read's backward for 128 query rows of one (b, h, segment):
 //   den = sigma(q) z, A_mem = sigma(q) M / den (product 1), the row terms
 //   D'_i = dO_i . A_dot_i and dO_i . (A_mem_i - A_dot_i) (for dbeta),
@@ -78,11 +146,8 @@ __global__ void __launch_bounds__(256, 1)
   float* dens = zs + 128;         // [128]
   float* ddens = dens + 128;      // [128]
   const float* Mp = snapM + ((long long)bh * g.S + s) * dk * dv;
-  for (int e = tid; e < 128 * 128; e += 256) {
-    const int i = e >> 7, j = e & 127;
-    Ms[i * kMP + j] = (i < dk && j < dv) ? Mp[i * dv + j] : 0.f;
-    Sq[i * kMP + j] = (i < nr && j < dk) ? elu1_accurate(to_f32(q[(row0 + i) * dk + j])) : 0.f;
-  }
+  stage_f32(Ms, Mp, 128, dk, dv);
+  stage_sigma<T>(Sq, q + row0 * dk, 128, nr, dk);
   if (tid < 128) zs[tid] = tid < dk ? snapz[((long long)bh * g.S + s) * dk + tid] : 0.f;
   __syncthreads();
   if (tid < 128) {
@@ -186,9 +251,9 @@ __global__ void __launch_bounds__(256, 1) bwd_outer_kernel(const T* __restrict__
     const int nt = min(64, t_end - t0);
     const long long rb = (long long)bh * g.L + seg_start + t0;
     __syncthreads();
+    stage_sigma<T>(Sx, x + rb * dk, 64, nt, dk);
     for (int e = tid; e < 64 * 128; e += 256) {
       const int t = e >> 7, c = e & 127;
-      Sx[t * kMP + c] = (t < nt && c < dk) ? elu1_accurate(to_f32(x[(rb + t) * dk + c])) : 0.f;
       Sy[t * LY + c] = (t < nt && c < dy) ? Y[(rb + t) * dy + c] : 0.f;
     }
     if (tid < 64) Sy[tid * LY + 128] = tid < nt ? y0[rb + tid] : 0.f;
@@ -250,16 +315,9 @@ __global__ void __launch_bounds__(256, 1)
   float* ddr = dens + 64;                           // [64]
   const float* gp = gstate + (long long)bh * gstride_bh + (long long)s * gstride_s;
   const float* Mp = delta ? snapM + ((long long)bh * g.S + s) * dk * dv : nullptr;
-  for (int e = tid; e < 128 * 128; e += 256) {
-    const int i = e >> 7, j = e & 127;
-    const bool in = i < dk && j < dv;
-    Gs[i * kMP + j] = in ? gp[i * dv + j] : 0.f;
-    if (delta) Ms[i * kMP + j] = in ? Mp[i * dv + j] : 0.f;
-  }
-  for (int e = tid; e < 64 * 128; e += 256) {
-    const int t = e >> 7, c = e & 127;
-    Sk[t * kMP + c] = (t < nr && c < dk) ? elu1_accurate(to_f32(k[(row0 + t) * dk + c])) : 0.f;
-  }
+  stage_f32(Gs, gp, 128, dk, dv);
+  if (delta) stage_f32(Ms, Mp, 128, dk, dv);
+  stage_sigma<T>(Sk, k + row0 * dk, 64, nr, dk);
   if (tid < 128) {
     gz[tid] = tid < dk ? gp[dk * dv + tid] : 0.f;
     zs[tid] = (delta && tid < dk) ? snapz[((long long)bh * g.S + s) * dk + tid] : 0.f;
