@@ -163,6 +163,7 @@ __device__ __forceinline__ float decode_dot(const float* qs, const T* kr, int dk
   if (vec) {
     const uint4* k4 = reinterpret_cast<const uint4*>(kr);
     if constexpr (sizeof(T) == 2) {
+#pragma unroll 4
       for (int c = 0; c < dk / 8; ++c) {
         const uint4 w = __ldg(k4 + c);
         const uint32_t u[4] = {w.x, w.y, w.z, w.w};
@@ -173,6 +174,7 @@ __device__ __forceinline__ float decode_dot(const float* qs, const T* kr, int dk
         }
       }
     } else {
+#pragma unroll 4
       for (int c = 0; c < dk / 4; ++c) {
         const float4 w = __ldg(reinterpret_cast<const float4*>(k4 + c));
         d = fmaf(qs[4 * c], w.x, d);
@@ -225,6 +227,7 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
     for (int c = 0; c < 4; ++c) acc[c] *= alpha;
     const int cnt = min(32, j1 - jb);
+#pragma unroll 4
     for (int jj = 0; jj < cnt; ++jj) {
       const float pj = __shfl_sync(0xffffffffu, p, jj);
       const int key = jb + jj;
@@ -291,8 +294,15 @@ __global__ void __launch_bounds__(256)
         const float mr = ld_dsmem_f32(a);
         o += mr == -INFINITY ? 0.f : ld_dsmem_f32(a + 4u * (uint32_t)(2 + c)) * expf(mr - gm);
       }
-      float num = 0.f;
-      for (int i = 0; i < dk; ++i) num = fmaf(sq[i], Mh[(long long)i * dv + c], num);
+      // sigma(q) M column c: eight independent partial sums keep eight loads in flight
+      float nm[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      int i = 0;
+      for (; i + 8 <= dk; i += 8) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) nm[u] = fmaf(sq[i + u], Mh[(long long)(i + u) * dv + c], nm[u]);
+      }
+      for (; i < dk; ++i) nm[0] = fmaf(sq[i], Mh[(long long)i * dv + c], nm[0]);
+      const float num = ((nm[0] + nm[1]) + (nm[2] + nm[3])) + ((nm[4] + nm[5]) + (nm[6] + nm[7]));
       const float a_mem = den != 0.f ? num / den : 0.f;
       out[(long long)bh * dv + c] = from_f32<T>(g * a_mem + (1.f - g) * (o / gl));
     }

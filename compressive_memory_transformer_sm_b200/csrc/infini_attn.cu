@@ -272,7 +272,8 @@ int run_rope(const infini_attn_params& p, char* dst, LocalQK* loc) {
   const long long bx = (p.L + rows_per - 1) / rows_per;
   if (bx >= (1LL << 31)) return INFINI_ERR_UNSUPPORTED;
   const dim3 block((unsigned)groups, (unsigned)rows_per);
-  const dim3 grid((unsigned)bx, (unsigned)std::min<long long>((long long)p.B * p.H, 65535));
+  // up to 8 heads per thread: the sine/cosine of a token's pairs serve them all
+  const dim3 grid((unsigned)bx, (unsigned)std::min<long long>(((long long)p.B * p.H + 7) / 8, 65535));
   {
     LaunchScope ls(kPhasePre, p.stream);
     if (f32) {

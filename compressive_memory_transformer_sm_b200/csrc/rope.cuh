@@ -85,14 +85,20 @@ __device__ __forceinline__ void rope_angle(long long pos, double f, float& c, fl
 // dk % 8 == 0 and vector-aligned rows, E = 2 (one pair) only an even dk.
 template <typename T, int E>
 __global__ void __launch_bounds__(256) rope_kernel(const __grid_constant__ RopeArgs a) {
+  // the frequencies in shared memory: lanes of a warp index different pairs,
+  // which a constant-bank read would serialise
+  __shared__ double fr[kRopeMaxPairs];
+  const int tid = threadIdx.y * blockDim.x + threadIdx.x;
+  if (tid < a.dk / 2) fr[tid] = a.inv_freq[tid];
+  __syncthreads();
   const int j = threadIdx.x;
   const long long t = (long long)blockIdx.x * blockDim.y + threadIdx.y;
   if (t >= a.L) return;
   const long long pos = a.offset + t;
-  // the rotation of this thread's pairs, shared by q and k
+  // the rotation of this thread's pairs, shared by q and k of every head it serves
   float cs[E / 2], sn[E / 2];
 #pragma unroll
-  for (int e = 0; e < E / 2; ++e) rope_angle(pos, a.inv_freq[j * (E / 2) + e], cs[e], sn[e]);
+  for (int e = 0; e < E / 2; ++e) rope_angle(pos, fr[j * (E / 2) + e], cs[e], sn[e]);
   const T* q = static_cast<const T*>(a.q);
   const T* k = static_cast<const T*>(a.k);
   T* qr = static_cast<T*>(a.qr);
