@@ -38,7 +38,7 @@ EXPORTED = (
     "infini_attn_launch_count", "infini_attn_forward_noalloc",
     "infini_attn_layer_forward", "infini_attn_layer_workspace_size", "infini_attn_decode_step",
     "infini_attn_workspace_size_ex", "infini_attn_gemm_bf16", "infini_attn_backward",
-    "infini_attn_backward_workspace_size",
+    "infini_attn_backward_workspace_size", "infini_attn_trim_workspace",
 )
 
 
@@ -123,6 +123,8 @@ lib.infini_attn_backward.argtypes = [ctypes.POINTER(InfiniAttnBwdParams)]
 lib.infini_attn_backward.restype = _i
 lib.infini_attn_backward_workspace_size.argtypes = [ctypes.POINTER(InfiniAttnBwdParams)]
 lib.infini_attn_backward_workspace_size.restype = ctypes.c_size_t
+lib.infini_attn_trim_workspace.argtypes = []
+lib.infini_attn_trim_workspace.restype = _i
 
 
 class InfiniAttnError(RuntimeError):
@@ -133,6 +135,13 @@ class InfiniAttnError(RuntimeError):
 
 def infini_attn_error_string(code: int) -> str:
     return lib.infini_attn_error_string(int(code)).decode()
+
+
+def infini_attn_trim_workspace() -> None:
+    """Return the unused device memory of the library's own workspace pool (current context) to the driver."""
+    rc = lib.infini_attn_trim_workspace()
+    if rc != 0:
+        raise InfiniAttnError(rc, "infini_attn_trim_workspace")
 
 
 def _stream(stream):

@@ -34,6 +34,7 @@
 #include "rope.cuh"
 #include "sm100_attn.cuh"
 #include "sm100_update.cuh"
+#include "sm100_delta.cuh"
 #include "sm100_gemm.cuh"
 #include "sm100_bwd.cuh"
 
@@ -187,12 +188,13 @@ unsigned long long current_context_id() {
 
 // 4-D map over a [B, H, L, 128] bf16 tensor with element strides st[0..2]
 // (d contiguous); box 64 x 128 tokens, 128-byte swizzle.
-bool encode_bhld(CUtensorMap* m, const void* ptr, int B, int H, long long L, const long long st[3]) {
+bool encode_bhld(CUtensorMap* m, const void* ptr, int B, int H, long long L, const long long st[3],
+                 uint32_t box_rows = 128) {
   EncodeTiledFn enc = get_encode();
   if (!enc) return false;
   cuuint64_t dims[4] = {128, (cuuint64_t)L, (cuuint64_t)H, (cuuint64_t)B};
   cuuint64_t strides[3] = {(cuuint64_t)st[2] * 2, (cuuint64_t)st[1] * 2, (cuuint64_t)st[0] * 2};
-  cuuint32_t box[4] = {64, 128, 1, 1};
+  cuuint32_t box[4] = {64, box_rows, 1, 1};
   cuuint32_t es[4] = {1, 1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -373,6 +375,54 @@ cudaStream_t side_stream() {
   return st;
 }
 
+// Workspace the library allocates itself comes from a stream-ordered memory
+// pool of its own, one per context, whose release threshold keeps freed
+// blocks for the next call: repeated calls of one shape take nothing from the
+// driver after the first (the device's default pool, with its threshold of 0,
+// hands memory back at every synchronization, and mapping gigabytes again
+// costs milliseconds).  infini_attn_trim_workspace() returns what is unused.
+std::mutex g_pool_mu;
+std::vector<std::pair<unsigned long long, cudaMemPool_t>> g_pools;
+
+cudaMemPool_t workspace_pool() {
+  const unsigned long long ctx = current_context_id();
+  if (ctx == 0) return nullptr;
+  std::lock_guard<std::mutex> lk(g_pool_mu);
+  for (const auto& e : g_pools)
+    if (e.first == ctx) return e.second;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  cudaMemPoolProps props;
+  memset(&props, 0, sizeof(props));
+  props.allocType = cudaMemAllocationTypePinned;
+  props.location.type = cudaMemLocationTypeDevice;
+  props.location.id = dev;
+  cudaMemPool_t pool = nullptr;
+  if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  uint64_t keep = ~0ull;
+  if (cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep) != cudaSuccess) cudaGetLastError();
+  g_pools.emplace_back(ctx, pool);
+  return pool;
+}
+
+// Stream-ordered workspace allocation (released with cudaFreeAsync).
+bool ws_alloc(void** ptr, size_t bytes, cudaStream_t stream) {
+  cudaMemPool_t pool = workspace_pool();
+  const cudaError_t e =
+      pool != nullptr ? cudaMallocFromPoolAsync(ptr, bytes, pool, stream) : cudaMallocAsync(ptr, bytes, stream);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return true;
+}
+
 // The dynamic shared-memory limit is an attribute of a function in the
 // current context: set it for the tensor-core kernels once for every context
 // the process uses (an unknown context id, 0, sets it on every call).
@@ -386,8 +436,8 @@ int set_tc_smem_limits() {
           cudaSuccess ||
       cudaFuncSetAttribute(tc::mem_update_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)tc::UpdSmem<false>::BYTES) != cudaSuccess ||
-      cudaFuncSetAttribute(tc::mem_update_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)tc::UpdSmem<true>::BYTES) != cudaSuccess ||
+      cudaFuncSetAttribute(tc::delta_update_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)tc::DeltaSmem::BYTES) != cudaSuccess ||
       cudaFuncSetAttribute(tc::gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kGemmSmem) !=
           cudaSuccess ||
       cudaFuncSetAttribute(tc::bwd_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kDQSmem) !=
@@ -520,6 +570,13 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale, c
                                               fork ? nullptr : snapz);
   } else {
     ua.nseg = 1;
+    // 64-token chunks: K and V maps with 64-row boxes
+    CUtensorMap tm_k64, tm_v64;
+    if (!encode_bhld(&tm_k64, p.k, p.B, p.H, p.L, p.k_stride, tc::kDChunk) ||
+        !encode_bhld(&tm_v64, p.v, p.B, p.H, p.L, p.v_stride, tc::kDChunk)) {
+      join();
+      return INFINI_ERR_LAUNCH;
+    }
     // one cluster of G CTAs per head; G <= 8 (plan)
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
@@ -528,8 +585,8 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale, c
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.gridDim = dim3(BH * pl.G);
-    cfg.blockDim = dim3(tc::UpdWarps<true>::THREADS);
-    cfg.dynamicSmemBytes = tc::UpdSmem<true>::BYTES;
+    cfg.blockDim = dim3(tc::kDeltaThreads);
+    cfg.dynamicSmemBytes = tc::DeltaSmem::BYTES;
     cfg.stream = p.stream;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
@@ -538,7 +595,7 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale, c
       // segment s, reduced inside each head's cluster into M, z
       ua.seg0 = s;
       LaunchScope ls(kPhaseUpdate, p.stream);
-      if (cudaLaunchKernelEx(&cfg, tc::mem_update_tc_kernel<true>, tm_k, tm_v, ua) != cudaSuccess) {
+      if (cudaLaunchKernelEx(&cfg, tc::delta_update_tc_kernel, tm_k64, tm_v64, ua) != cudaSuccess) {
         join();
         return INFINI_ERR_LAUNCH;
       }
@@ -652,10 +709,7 @@ int forward_impl(infini_attn_params p) {
   bool own = false;
   if (!ws) {
     void* w = nullptr;
-    if (cudaMallocAsync(&w, need, p.stream) != cudaSuccess) {
-      cudaGetLastError();
-      return INFINI_ERR_WORKSPACE;
-    }
+    if (!ws_alloc(&w, need, p.stream)) return INFINI_ERR_WORKSPACE;
     ws = static_cast<char*>(w);
     own = true;
   }
@@ -958,10 +1012,7 @@ int backward_impl(const infini_attn_bwd_params& p) {
   bool own = false;
   if (!ws) {
     void* w = nullptr;
-    if (cudaMallocAsync(&w, bp.total, p.stream) != cudaSuccess) {
-      cudaGetLastError();
-      return INFINI_ERR_WORKSPACE;
-    }
+    if (!ws_alloc(&w, bp.total, p.stream)) return INFINI_ERR_WORKSPACE;
     ws = static_cast<char*>(w);
     own = true;
   }
@@ -1010,8 +1061,8 @@ using namespace infini;
 
 // ------------------------------------------------------------------ full layer
 // Q, K, V = X W_{Q,K,V}, the Infini-attention forward, Y = A W_O (multi-head
-// formulation, Eq. 5 and Eq. 11).  The projections are plain cuBLAS GEMMs;
-// the layout keeps them copy-free: the QKV product [B*L, 3*H*128] is read by
+// formulation, Eq. 5 and Eq. 11).  The projections run on the library's own
+// tcgen05 GEMM (gemm_tc_kernel); the layout keeps them copy-free: the QKV product [B*L, 3*H*128] is read by
 // the attention kernels through strided views, and the attention writes its
 // output as [B, L, H, 128], the A operand of the output projection.
 namespace {
@@ -1215,10 +1266,7 @@ int infini_attn_decode_step(const void* q_t, const void* k_t, const void* v_t, v
   int per = (int)std::max<long long>(64, (n + want - 1) / want);
   const int splits = (n + per - 1) / per;
   void* scratch = nullptr;
-  if (cudaMallocAsync(&scratch, (size_t)splits * BH * (dv + 2) * 4, stream) != cudaSuccess) {
-    cudaGetLastError();
-    return INFINI_ERR_WORKSPACE;
-  }
+  if (!ws_alloc(&scratch, (size_t)splits * BH * (dv + 2) * 4, stream)) return INFINI_ERR_WORKSPACE;
   float* part = static_cast<float*>(scratch);
   {
     LaunchScope ls(kPhaseAttn, stream);
@@ -1325,10 +1373,7 @@ int infini_attn_layer_forward(const void* x, const void* w_qkv, const void* w_o,
   bool own = false;
   if (!ws) {
     void* w = nullptr;
-    if (cudaMallocAsync(&w, lp.total, stream) != cudaSuccess) {
-      cudaGetLastError();
-      return INFINI_ERR_WORKSPACE;
-    }
+    if (!ws_alloc(&w, lp.total, stream)) return INFINI_ERR_WORKSPACE;
     ws = static_cast<char*>(w);
     own = true;
   }
@@ -1369,6 +1414,16 @@ int infini_attn_layer_forward(const void* x, const void* w_qkv, const void* w_o,
   return rc;
 }
 
+int infini_attn_trim_workspace(void) {
+  const unsigned long long ctx = current_context_id();
+  std::lock_guard<std::mutex> lk(g_pool_mu);
+  for (const auto& e : g_pools)
+    if (e.first == ctx && cudaMemPoolTrimTo(e.second, 0) != cudaSuccess) {
+      cudaGetLastError();
+      return INFINI_ERR_DEVICE;
+    }
+  return INFINI_OK;
+}
 const char* infini_attn_error_string(int code) {
   switch (code) {
     case INFINI_OK: return "ok";

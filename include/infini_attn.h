@@ -319,6 +319,15 @@ INFINI_API int infini_attn_backward(const infini_attn_bwd_params* p);
 /* Bytes of workspace infini_attn_backward needs for p's shape and mode (0 if invalid). */
 INFINI_API size_t infini_attn_backward_workspace_size(const infini_attn_bwd_params* p);
 
+/*
+ * Workspace that the library allocates itself (calls given no workspace)
+ * comes from a stream-ordered pool of its own, one per CUDA context, that
+ * keeps freed blocks for the next call.  This returns the pool's unused
+ * device memory (of the current context) to the driver; blocks still in use
+ * by queued work stay.  INFINI_OK, or INFINI_ERR_DEVICE if the trim failed.
+ */
+INFINI_API int infini_attn_trim_workspace(void);
+
 /* Static English text for a return code; never NULL. */
 INFINI_API const char* infini_attn_error_string(int code);
 
