@@ -577,13 +577,17 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale, c
       join();
       return INFINI_ERR_LAUNCH;
     }
-    // one cluster of G CTAs per head; G <= 8 (plan)
+    // one cluster of G CTAs per head; G <= 8 (plan).  Segments after the
+    // first launch as programmatic dependents of the previous segment's
+    // update (their K, V loads start while it finishes; M, z wait for it).
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = pl.G;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.gridDim = dim3(BH * pl.G);
     cfg.blockDim = dim3(tc::kDeltaThreads);
     cfg.dynamicSmemBytes = tc::DeltaSmem::BYTES;
@@ -594,6 +598,7 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale, c
       // snapshot of M_{s-1}, z_{s-1} for segment s, then the partials of
       // segment s, reduced inside each head's cluster into M, z
       ua.seg0 = s;
+      cfg.numAttrs = s > 0 ? 2 : 1;
       LaunchScope ls(kPhaseUpdate, p.stream);
       if (cudaLaunchKernelEx(&cfg, tc::delta_update_tc_kernel, tm_k64, tm_v64, ua) != cudaSuccess) {
         join();

@@ -4,31 +4,37 @@
 //   M_s = M_{s-1} + sigma(K)^T (V - sigma(K) M_{s-1} / (sigma(K) z_{s-1}))
 //   z_s = z_{s-1} + sum_t sigma(K_t)
 //
-// The products run transposed, so that M_{s-1} and U = V - R / den live in
-// tensor memory as the A operand and only K, sigma(K)_lo and V tiles occupy
-// shared memory (48 KB per 64-token chunk): deep enough rings that the
-// chunks of a CTA overlap.  Per chunk c of 64 tokens:
-//   sigma pass (CUDA cores, thread = a quarter-row of 16 columns):
-//     sigma(K) = ELU + 1, split into bf16 hi (in place of K) + lo parts;
-//     den_t = sigma(K_t) . z_{s-1} in fp32; dz += sigma(K) in fp32 registers
-//   R^T  = M_{s-1}^T sigma(K)_hi^T                   (A: M^T bf16 in TMEM, B: K-major)
-//   U pass (CUDA cores, thread = one value column d = one TMEM lane, 16 tokens):
-//     U = V - R / den in fp32, split into bf16 hi + lo, written to TMEM as U^T
-//   dM^T += U_hi^T sigma(K)_hi + U_hi^T sigma(K)_lo + U_lo^T sigma(K)_hi
-//                                                    (A: U^T in TMEM, B: MN-major)
-// The lo parts keep the accumulated update within ~2^-16 relative of fp32
-// arithmetic; R uses bf16 M_{s-1}, as the memory read does.
+// M_{s-1} is fixed for the whole segment, so the retrieval term factors out
+// of the sum over tokens:
+//   sum_t sigma(K_t)^T sigma(K_t) M_{s-1} / den_t = G M_{s-1},
+//   G = sum_t sigma(K_t)^T sigma(K_t) / den_t      ([dk][dk]),
+// and dM = sigma(K)^T V - G M_{s-1}: every chunk's work is products that
+// read only shared memory, with no retrieval product and no round trip
+// through the CUDA cores between products, plus one G M_{s-1} product per
+// CTA at the end.  (The sums of Eq. 9, reassociated; with the hi + lo splits
+// below the result is closer to fp64 than a retrieval through a bf16 M_{s-1}.)
 //
-// Software pipeline: the compute warps run sigma(c + 1) before U(c), and the
-// MMA warp issues R(c + 1) before dM(c), so the R product of the next chunk
-// runs under the U pass of this one and the dM products under the next
-// sigma pass.  Double-buffered R and U in TMEM (448 of 512 columns).
+// Per chunk c of 64 tokens:
+//   sigma pass (CUDA cores; thread = row rr of the chunk, 16 of its columns):
+//     sigma(K) = ELU + 1 in fp32, split into bf16 hi (in place of K) + lo;
+//     den_t = sigma(K_t) . z_{s-1} (fp32); S_t = sigma(K_t) / den_t (0 where
+//     den_t = 0) in bf16; dz += sigma(K) in fp32 registers
+//   tensor cores (transposed, fp32 accumulators in TMEM):
+//     VM^T += V^T sigma_hi + V^T sigma_lo           (V exact in bf16)
+//     G    += S^T sigma_hi
+// After the last chunk: dM^T = VM^T + M^T (-G^T), with M^T in TMEM (hi + lo
+// parts, the A operand) and -G^T written to shared memory as bf16 hi + lo.
+// sigma^T V and the final product keep ~2^-16 relative accuracy; G's bf16
+// roundings are independent across tokens and average out in the sum, so
+// that the state stays within ~2e-5 relative of fp64 over many segments,
+// closer than a retrieval through a bf16 M_{s-1} (fp32 accumulation).
 //
-// The G CTAs of a head (token ranges of the segment) form one cluster: each
-// stages its partial [dM | dz] in shared memory; after a cluster barrier CTA g
-// adds slice g of every partial, in rank order (deterministic), to the
-// running M, z.  Every CTA first writes its slice of the snapshot of M_{s-1}
-// that the attention kernel reads.
+// The G CTAs of a head (token ranges of the segment) form one cluster.  Once
+// every CTA of the cluster is past its chunks (a cluster barrier), each
+// stores slice g of its partial [dM | dz] into CTA g's shared memory; after a
+// second barrier CTA g adds the G partials of slice g, in rank order
+// (deterministic), to the running M, z.  Every CTA first writes its slice of
+// the snapshot of M_{s-1} that the attention kernel reads.
 #pragma once
 
 #include "sm100_common.cuh"
@@ -37,62 +43,109 @@
 namespace infini {
 namespace tc {
 
-constexpr int kDChunk = 64;           // tokens per chunk
-constexpr uint32_t kDBox = 8192;      // 64 rows x 128 B
-constexpr uint32_t kDTile = 16384;    // 64 tokens x 128 bf16: two boxes
-constexpr int kDeltaThreads = 576;    // 16 compute warps, a TMA warp, an MMA warp
+// Phase timestamps of one CTA (block INFINI_DELTA_TRACE) for tuning builds;
+// shares the attention kernel's trace array (slots 3200 and up): 3200-3209
+// phases of thread 0, 3210 + c its sigma pass of chunk c, 3280 + c the MMA
+// warp's chunk c, 3350 + c the producer's chunk c, 3420-3421 the reduction.
+#if defined(INFINI_DELTA_TRACE) && defined(INFINI_ATTN_TRACE)
+#define DELTA_TRACE(cond, slot)                                                                         \
+  do {                                                                                                  \
+    if ((cond) && blockIdx.x == INFINI_DELTA_TRACE && (slot) < 4096) g_attn_trace[(slot)] = clock64(); \
+  } while (0)
+#else
+#define DELTA_TRACE(cond, slot) \
+  do {                          \
+  } while (0)
+#endif
+
+constexpr int kDChunk = 64;         // tokens per chunk
+constexpr uint32_t kDBox = 8192;    // 64 rows x 128 B
+constexpr uint32_t kDTile = 16384;  // 64 tokens x 128 bf16: two boxes
+constexpr int kDeltaThreads = 608;  // 16 compute warps, a K-load warp, an MMA warp, a V-load warp
 
 struct DeltaSmem {
-  static constexpr int KST = 6;  // K ring (sigma(K)_hi in place): loaded -> dM done
-  static constexpr int LST = 3;  // sigma(K)_lo ring: sigma pass -> dM done
-  static constexpr int VST = 4;  // V ring: loaded -> U pass done
+  static constexpr int KST = 5;  // K ring (sigma(K)_hi in place): loaded -> chunk products done
+  static constexpr int VST = 4;  // V ring: loaded -> chunk products done
+  static constexpr int LST = 2;  // sigma_lo, S: sigma pass -> chunk products done
   static constexpr uint32_t K0 = 0;
-  static constexpr uint32_t KL0 = K0 + KST * kDTile;
-  static constexpr uint32_t V0 = KL0 + LST * kDTile;
-  static constexpr uint32_t Z = V0 + VST * kDTile;  // z_{s-1}, 128 floats
-  // [LST][64] 1 / den of a chunk's tokens: sigma(c + LST) rewrites buffer c % LST
-  // only after its lo-buffer wait (dM(c) done, so every warp's U(c) has read it)
-  static constexpr uint32_t RINV = Z + 512u;
-  static constexpr uint32_t BAR = RINV + 1024u;
-  static_assert(LST * 64 * 4 <= 1024, "1 / den buffers");
-  static constexpr uint32_t SLOT = BAR + 512u;
+  static constexpr uint32_t V0 = K0 + KST * kDTile;
+  static constexpr uint32_t W0 = V0 + VST * kDTile;  // LST x [sigma_lo | S]
+  static constexpr uint32_t END = W0 + LST * 2 * kDTile;  // end of the rings
+  static constexpr uint32_t BAR = END;
+  static constexpr uint32_t SLOT = BAR + 256u;
   static constexpr uint32_t BYTES = SLOT + 16u + 1024u;
   static_assert(BYTES <= 232448, "delta update kernel exceeds 227 KB of shared memory");
-  // after the last chunk, over the rings: the partial [dM (128 x 128) | dz (128)]
-  // (66,048 B from 0) and the 16 warps' dz sums (8 KB)
-  static constexpr uint32_t RED = 0;
-  static constexpr uint32_t DZS = 69632u;
-  static_assert(DZS + 16u * 128u * 4u <= V0, "epilogue scratch must lie in the K / lo rings");
+  // after the last chunk, over the rings: -G^T as bf16 hi and lo K-major
+  // tiles (128 x 128, two 16 KB boxes each), the landing area of this CTA's
+  // slice of the G partials (G x slice <= 4135 float4), the 16 warps' dz sums
+  // (8 KB) and this CTA's partial [dM | dz] staged for sending (66,048 B),
+  // before it M_{s-1} as bf16 hi and lo MN-major tiles (the A operand M^T of
+  // the final product) in the same place
+  static constexpr uint32_t GH = 0;
+  static constexpr uint32_t GL = 32768u;
+  static constexpr uint32_t LAND = 65536u;
+  static constexpr uint32_t DZS = LAND + 66560u;
+  static constexpr uint32_t RED = DZS + 16u * 128u * 4u;
+  static constexpr uint32_t MH = RED;
+  static constexpr uint32_t ML = RED + 32768u;
+  static_assert(RED % 1024u == 0 && ML + 32768u <= RED + 66048u, "M tiles");
+  static_assert(RED + 66048u <= END, "epilogue scratch must lie in the rings");
 };
 
 enum : int {
-  D_KF = 0, D_KE = 6, D_LE = 12, D_VF = 15, D_VE = 19, D_SK = 23, D_RF = 25, D_UR = 27, D_UE = 29, D_MT = 31,
-  D_DONE = 32, D_COUNT = 33
+  D_KF = 0, D_KE = 5, D_VF = 10, D_VE = 14, D_LE = 18, D_SK = 20, D_ACC = 22, D_GR = 23, D_FIN = 24, D_RX = 25,
+  D_COUNT = 26
 };
+constexpr int kDeltaE4 = (128 * 128 + 128) / 4;  // float4 elements of [M | z]
 
 // 16-byte chunk c (0..15) of row r of a 64-row tile (two 8 KB boxes)
 __device__ __forceinline__ uint32_t dswz(int r, int c) {
   return (uint32_t)(c >> 3) * kDBox + (uint32_t)r * 128u + ((uint32_t)((c & 7) ^ (r & 7)) << 4);
 }
-// K-major operand of 64 rows (the B of R^T: sigma(K) rows, 16 dk per step)
-__device__ __forceinline__ uint64_t dkmajor_desc(uint32_t tile, int kk) {
-  return smem_desc_sw128(tile, 16u, 1024u) + (uint64_t)((uint32_t)(kk >> 2) * (kDBox >> 4) + (uint32_t)(kk & 3) * 2u);
-}
-// MN-major operand of 64 K-rows x 128 (the B of dM^T: sigma(K) [t][dk], 16 tokens per step)
-__device__ __forceinline__ uint64_t dmnmajor_desc(uint32_t tile, int kk) {
+// MN-major operand of 64 K-rows (tokens) x 128 M/N columns, 16 tokens per step
+__device__ __forceinline__ uint64_t dmn_desc(uint32_t tile, int kk) {
   return smem_desc_sw128(tile, kDBox, 1024u) + (uint64_t)((uint32_t)kk * (2048u >> 4));
 }
-__device__ __forceinline__ float lds_bf16(uint32_t a) {
-  unsigned short v;
-  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
-  return __uint_as_float((uint32_t)v << 16);
+// Rows of M owned by CTA grp of G for the snapshot: k with k * G / 128 = grp.
+__device__ __forceinline__ int delta_row_lo(int grp, int G) { return (grp * 128 + G - 1) / G; }
+
+// Snapshot rows [r_lo, r_hi) of M_{s-1} (bf16 for the attention; fp32 when
+// asked, for the backward) and, from CTA 0, z_{s-1}, by `nthr` threads.
+__device__ __forceinline__ void delta_snapshot(const UpdArgs& a, const float* Mh, int bh, int s, int grp, int tid,
+                                               int nthr) {
+  const int c_lo = 16 * delta_row_lo(grp, a.G), c_hi = 16 * delta_row_lo(grp + 1, a.G);  // 16-byte bf16 chunks
+  __nv_bfloat16* snap = a.snapM + ((long long)bh * a.S + s) * 16384;
+  for (int ch = c_lo + tid; ch < c_hi; ch += nthr) {
+    const int r = ch >> 4, cc = ch & 15;
+    const float4 f0 = *reinterpret_cast<const float4*>(Mh + r * 128 + 8 * cc);
+    const float4 f1 = *reinterpret_cast<const float4*>(Mh + r * 128 + 8 * cc + 4);
+    if (a.snapM != nullptr)
+      *reinterpret_cast<uint4*>(snap + r * 128 + 8 * cc) = make_uint4(
+          pack_bf16x2(f0.x, f0.y), pack_bf16x2(f0.z, f0.w), pack_bf16x2(f1.x, f1.y), pack_bf16x2(f1.z, f1.w));
+    if (a.snapM32 != nullptr) {
+      float4* s32 = reinterpret_cast<float4*>(a.snapM32 + ((long long)bh * a.S + s) * 16384 + r * 128 + 8 * cc);
+      s32[0] = f0;
+      s32[1] = f1;
+    }
+  }
+  if (grp == 0 && tid < 128 && a.snapzw != nullptr)
+    a.snapzw[((long long)bh * a.S + s) * 128 + tid] = a.z[(long long)bh * 128 + tid];
 }
+
+// bf16 hi and lo parts of (x0, x1): hi = bf16(x), lo = bf16(x - hi)
+__device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  hi = pack_bf16x2(x0, x1);
+  float l0, l1;
+  fma2(l0, l1, bf16_lo(hi), bf16_hi(hi), -1.f, -1.f, x0, x1);
+  lo = pack_bf16x2(l0, l1);
+}
+
 
 __global__ void __launch_bounds__(kDeltaThreads, 1)
     delta_update_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                            const UpdArgs a) {
   using SL = DeltaSmem;
-  constexpr int KST = SL::KST, LST = SL::LST, VST = SL::VST;
+  constexpr int KST = SL::KST, VST = SL::VST, LST = SL::LST;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -108,256 +161,249 @@ __global__ void __launch_bounds__(kDeltaThreads, 1)
   const int t_end = min(n_s, t_begin + a.cpb * kTile);
   const int nch = t_begin < t_end ? (t_end - t_begin + kDChunk - 1) / kDChunk : 0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float* red = reinterpret_cast<float*>(gbase + SL::RED);
   const float* Mh = a.M + (long long)bh * 16384;
-
-  // Snapshot of M_{s-1}, z_{s-1} for the attention (and the backward): CTA
-  // grp writes slice grp.  The running M, z change only after the cluster
-  // barrier below, once every CTA of the head has read them.
-  {
-    const int per = (2048 + a.G - 1) / a.G;  // 16-byte chunks of the bf16 snapshot per CTA
-    const int c_lo = grp * per, c_hi = min(2048, c_lo + per);
-    __nv_bfloat16* snap = a.snapM + ((long long)bh * a.S + s) * 16384;
-    for (int ch = c_lo + (int)threadIdx.x; ch < c_hi; ch += blockDim.x) {
-      const int r = ch >> 4, cc = ch & 15;
-      const float4 f0 = *reinterpret_cast<const float4*>(Mh + r * 128 + 8 * cc);
-      const float4 f1 = *reinterpret_cast<const float4*>(Mh + r * 128 + 8 * cc + 4);
-      if (a.snapM != nullptr)
-        *reinterpret_cast<uint4*>(snap + r * 128 + 8 * cc) = make_uint4(
-            pack_bf16x2(f0.x, f0.y), pack_bf16x2(f0.z, f0.w), pack_bf16x2(f1.x, f1.y), pack_bf16x2(f1.z, f1.w));
-      if (a.snapM32 != nullptr) {
-        float4* s32 = reinterpret_cast<float4*>(a.snapM32 + ((long long)bh * a.S + s) * 16384 + r * 128 + 8 * cc);
-        s32[0] = f0;
-        s32[1] = f1;
-      }
-    }
-    if (grp == 0 && threadIdx.x < 128 && a.snapzw != nullptr)
-      a.snapzw[((long long)bh * a.S + s) * 128 + threadIdx.x] = a.z[(long long)bh * 128 + threadIdx.x];
+  const int per = (kDeltaE4 + a.G - 1) / a.G;  // float4 elements of [M | z] in a slice
+  const int e4_begin = grp * per, e4_end = min(kDeltaE4, e4_begin + per);  // this CTA's slice
+  auto has_tokens = [&](int g2) { return g2 * a.cpb * kTile < n_s; };   // CTA g2 of the head has chunks
+  auto bar = [&](int i) { return base + SL::BAR + 8u * (uint32_t)i; };
+  [[maybe_unused]] const bool t0 = threadIdx.x == 0;
+  DELTA_TRACE(t0, 3200);
+  if (threadIdx.x == 0) {
+    // receive barrier: this CTA's slice from every other CTA of the head
+    // with tokens, armed before this CTA's arrival on the cluster barrier
+    // (peers copy only after it)
+    int senders = 0;
+    for (int g2 = 0; g2 < a.G; ++g2) senders += g2 != grp && has_tokens(g2);
+    mbar_init(bar(D_RX), 1);
+    fence_barrier_init();
+    mbar_expect_tx(bar(D_RX), (uint32_t)(senders * (e4_end - e4_begin) * 16));
   }
+  // Launched as a programmatic dependent of the previous segment's update,
+  // whose outputs are M, z and their snapshots only: the next segment's grid
+  // may start its setup and its K, V loads now; every read or write of M, z
+  // and the snapshots comes after griddep_wait().
+  griddep_launch_dependents();
 
-  if (nch == 0) {  // group past the end of a short segment: contributes nothing
-    for (int e = threadIdx.x; e < 128 * 128 + 128; e += blockDim.x) red[e] = 0.f;
+  if (nch == 0) {
+    // a group past the end of a short segment: its snapshot slice; it sends nothing
+    griddep_wait();
+    delta_snapshot(a, Mh, bh, s, grp, threadIdx.x, blockDim.x);
+    cluster_arrive();
+    cluster_wait();
   } else {
-    auto bar = [&](int i) { return base + SL::BAR + 8u * (uint32_t)i; };
     auto sK = [&](int st) { return base + SL::K0 + (uint32_t)st * kDTile; };
-    auto sL = [&](int st) { return base + SL::KL0 + (uint32_t)st * kDTile; };
     auto sV = [&](int st) { return base + SL::V0 + (uint32_t)st * kDTile; };
-    const float* zs = reinterpret_cast<const float*>(gbase + SL::Z);
-    float* rinv = reinterpret_cast<float*>(gbase + SL::RINV);
+    auto sLo = [&](int st) { return base + SL::W0 + (uint32_t)(2 * st) * kDTile; };
+    auto sS = [&](int st) { return base + SL::W0 + (uint32_t)(2 * st + 1) * kDTile; };
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + SL::SLOT);
     if (threadIdx.x == 0) {
       for (int i = 0; i < KST; ++i) {
         mbar_init(bar(D_KF + i), 1);
         mbar_init(bar(D_KE + i), 1);
       }
-      for (int i = 0; i < LST; ++i) mbar_init(bar(D_LE + i), 1);
       for (int i = 0; i < VST; ++i) {
         mbar_init(bar(D_VF + i), 1);
-        mbar_init(bar(D_VE + i), 16);
+        mbar_init(bar(D_VE + i), 1);
       }
-      for (int i = 0; i < 2; ++i) {
+      for (int i = 0; i < LST; ++i) {
+        mbar_init(bar(D_LE + i), 1);
         mbar_init(bar(D_SK + i), 16);
-        mbar_init(bar(D_RF + i), 1);
-        mbar_init(bar(D_UR + i), 16);
-        mbar_init(bar(D_UE + i), 1);
       }
-      mbar_init(bar(D_MT), 16);
-      mbar_init(bar(D_DONE), 1);
+      mbar_init(bar(D_ACC), 1);
+      mbar_init(bar(D_GR), 16);
+      mbar_init(bar(D_FIN), 1);
       fence_barrier_init();
     }
-    if (threadIdx.x < 128) reinterpret_cast<float*>(gbase + SL::Z)[threadIdx.x] = a.z[(long long)bh * 128 + threadIdx.x];
     if (warp == 17) {
-      tmem_alloc(smem_u32(tmem_slot), 512);
+      tmem_alloc(smem_u32(tmem_slot), 256);
       tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    // TMEM columns: M^T (bf16 pairs) 0-63, R^T buffers 64-191, U^T buffers
-    // (hi 32 + lo 32 columns each) 192-319, dM^T 320-447
-    const uint32_t tMT = tmem, tD = tmem + 320u;
-    auto tR = [&](int rb) { return tmem + 64u + 64u * (uint32_t)rb; };
-    auto tU = [&](int ub) { return tmem + 192u + 64u * (uint32_t)ub; };
+    DELTA_TRACE(t0, 3202);
+    // TMEM columns: VM^T (then dM^T) 0-127, G 128-255
+    const uint32_t tVM = tmem, tG = tmem + 128u;
 
-    if (warp == 16) {
+    if (warp == 16 || warp == 18) {
+      // ------------------------------------------------------------ producers
+      // warp 16 loads K, warp 18 V: the K ring runs ahead of the V ring, whose
+      // stages the chunk products release later than the sigma pass needs
+      // the next keys
       if (lane == 0) {
-        // ---------------------------------------------------------- producer
-        prefetch_tensormap(&tm_k);
-        prefetch_tensormap(&tm_v);
-        for (int c = 0; c < nch; ++c) {
+        const bool kw = warp == 16;
+        const CUtensorMap* tm = kw ? &tm_k : &tm_v;
+        const int nst = kw ? KST : VST;
+        const int full = kw ? D_KF : D_VF, empty = kw ? D_KE : D_VE;
+        const uint32_t ring = kw ? base + SL::K0 : base + SL::V0;
+        prefetch_tensormap(tm);
+        auto load_chunk = [&](int c) {
           const int lt = (int)(seg_start + t_begin + (long long)c * kDChunk);
-          const int ks = c % KST, vs = c % VST;
-          if (c >= KST) mbar_wait(bar(D_KE + ks), ((c / KST) - 1) & 1);
-          mbar_expect_tx(bar(D_KF + ks), kDTile);
-          tma_load_4d(sK(ks), &tm_k, bar(D_KF + ks), 0, lt, h, b);
-          tma_load_4d(sK(ks) + kDBox, &tm_k, bar(D_KF + ks), 64, lt, h, b);
-          if (c >= VST) mbar_wait(bar(D_VE + vs), ((c / VST) - 1) & 1);
-          mbar_expect_tx(bar(D_VF + vs), kDTile);
-          tma_load_4d(sV(vs), &tm_v, bar(D_VF + vs), 0, lt, h, b);
-          tma_load_4d(sV(vs) + kDBox, &tm_v, bar(D_VF + vs), 64, lt, h, b);
-        }
+          const int st = c % nst;
+          if (c >= nst) mbar_wait_parked(bar(empty + st), ((c / nst) - 1) & 1);
+          mbar_expect_tx(bar(full + st), kDTile);
+          tma_load_4d(ring + (uint32_t)st * kDTile, tm, bar(full + st), 0, lt, h, b);
+          tma_load_4d(ring + (uint32_t)st * kDTile + kDBox, tm, bar(full + st), 64, lt, h, b);
+          DELTA_TRACE(!kw && c < 64, 3350 + c);
+        };
+        for (int c = 0; c < nch; ++c) load_chunk(c);
       }
+      __syncwarp();
+      if (warp == 18) {
+        // idle until the end: bring M_{s-1} (read by the epilogue) into L2
+        griddep_wait();
+        for (int i = lane; i < 512; i += 32) prefetch_l2(Mh + 32 * i);
+      }
+      cluster_arrive();  // every load lands before the chunk products complete
+      cluster_wait();
     } else if (warp == 17) {
       if (lane == 0) {
         // ---------------------------------------------------------- MMA issuer
-        constexpr uint32_t idesc_r = idesc_bf16(128, 64, 0, 0);   // A = M^T (TMEM), B = sigma(K)_hi K-major
-        constexpr uint32_t idesc_d = idesc_bf16(128, 128, 0, 1);  // A = U^T (TMEM), B = sigma(K) MN-major
-        mbar_wait(bar(D_MT), 0);
-        auto issue_r = [&](int c) {
-          const int rb = c & 1, ks = c % KST;
-          mbar_wait(bar(D_SK + rb), (c >> 1) & 1);
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) mma_ts(tR(rb), tMT + 8u * (uint32_t)kk, dkmajor_desc(sK(ks), kk), idesc_r, kk > 0 ? 1u : 0u);
-          mma_commit(bar(D_RF + rb));
-        };
-        issue_r(0);
+        constexpr uint32_t idesc_c = idesc_bf16(128, 128, 1, 1);  // chunk products: A, B MN-major
         for (int c = 0; c < nch; ++c) {
-          if (c + 1 < nch) issue_r(c + 1);
-          const int ub = c & 1, ks = c % KST, ls = c % LST;
-          mbar_wait(bar(D_UR + ub), (c >> 1) & 1);
+          const int ks = c % KST, vs = c % VST, ls = c % LST;
+          mbar_wait_parked(bar(D_SK + ls), (c / LST) & 1);
+          mbar_wait_parked(bar(D_VF + vs), (c / VST) & 1);
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t bH = dmnmajor_desc(sK(ks), kk), bL = dmnmajor_desc(sL(ls), kk);
-            const uint32_t aH = tU(ub) + 8u * (uint32_t)kk, aL = aH + 32u;
-            mma_ts(tD, aH, bH, idesc_d, (c > 0 || kk > 0) ? 1u : 0u);
-            mma_ts(tD, aH, bL, idesc_d, 1u);
-            mma_ts(tD, aL, bH, idesc_d, 1u);
+            const uint32_t acc = (c > 0 || kk > 0) ? 1u : 0u;
+            const uint64_t bH = dmn_desc(sK(ks), kk), bL = dmn_desc(sLo(ls), kk);
+            const uint64_t aV = dmn_desc(sV(vs), kk), aS = dmn_desc(sS(ls), kk);
+            mma_ss(tVM, aV, bH, idesc_c, acc);
+            mma_ss(tVM, aV, bL, idesc_c, 1u);
+            mma_ss(tG, aS, bH, idesc_c, acc);
           }
           mma_commit(bar(D_KE + ks));
+          mma_commit(bar(D_VE + vs));
           mma_commit(bar(D_LE + ls));
-          mma_commit(bar(D_UE + ub));
+          DELTA_TRACE(c < 64, 3280 + c);
         }
-        mma_commit(bar(D_DONE));
+        mma_commit(bar(D_ACC));
       }
+      __syncwarp();
+      cluster_arrive();  // the rings are released by the compute warps' arrivals after ACC
+      if (lane == 0) {
+        constexpr uint32_t idesc_f = idesc_bf16(128, 128, 1, 0);  // final: A = M^T MN-major, B = -G^T K-major
+        mbar_wait_parked(bar(D_GR), 0);
+        tc_fence_after();
+        const uint32_t gh = base + SL::GH, gl = base + SL::GL, mh = base + SL::MH, ml = base + SL::ML;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          mma_ss(tVM, mnmajor_desc(mh, kk), kmajor_desc(gh, kk), idesc_f, 1u);
+          mma_ss(tVM, mnmajor_desc(mh, kk), kmajor_desc(gl, kk), idesc_f, 1u);
+          mma_ss(tVM, mnmajor_desc(ml, kk), kmajor_desc(gh, kk), idesc_f, 1u);
+        }
+        mma_commit(bar(D_FIN));
+      }
+      __syncwarp();
+      cluster_wait();
     } else {
       // ------------------------------------------------------------ compute warps
       const int q = warp & 3, g = warp >> 2;
       const uint32_t lq = (uint32_t)(32 * q) << 16;  // this warp's TMEM lane quarter
-      const int d = 32 * q + lane;                   // U pass: value column = TMEM lane
-      {
-        // M_{s-1}^T into TMEM: lane d, column j = (M[2j][d], M[2j+1][d]) for
-        // this warp's 32 rows k of M
-        uint32_t mw[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int k = 32 * g + 2 * j;
-          mw[j] = pack_bf16x2(Mh[k * 128 + d], Mh[(k + 1) * 128 + d]);
-        }
-        tmem_st16(tMT + lq + 16u * (uint32_t)g, mw);
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(D_MT));
-      }
+      const int d = 32 * q + lane;                   // TMEM lane: a dv (M^T, dM^T) or dk (G) index
+      // M_{s-1} is needed only by the final product: the chunks start as
+      // soon as z_{s-1} (the previous segment's update) is available
+      griddep_wait();
+      if (grp == 0 && threadIdx.x < 128 && a.snapzw != nullptr)
+        a.snapzw[((long long)bh * a.S + s) * 128 + threadIdx.x] = a.z[(long long)bh * 128 + threadIdx.x];
+      DELTA_TRACE(t0, 3201);
       // sigma pass: row rr of the chunk, 16-byte chunks p (columns 8p..8p+7)
       // and 8 + p (columns 64 + 8p..)
       const int rr = 4 * warp + (lane >> 3), p = lane & 7;
-      float dz[16];
+      float zz[16], dz[16];
+      {
+        const float* zh = a.z + (long long)bh * 128;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) dz[i] = 0.f;
-      auto sigma_pass = [&](int c) {
-        const int ks = c % KST, ls = c % LST, rb = c & 1;
-        mbar_wait(bar(D_KF + ks), (c / KST) & 1);
-        const bool valid = t_begin + c * kDChunk + rr < t_end;
-        uint4 w[2], lo[2];
+        for (int i = 0; i < 16; ++i) {
+          zz[i] = zh[64 * (i >> 3) + 8 * p + (i & 7)];
+          dz[i] = 0.f;
+        }
+      }
+      // ring stages and phase parities of chunk c, advanced incrementally
+      int ks = 0, ls = 0;
+      uint32_t kph = 0, lph = 0;
+      for (int c = 0; c < nch; ++c) {
+        mbar_wait_parked(bar(D_KF + ks), kph);
+        DELTA_TRACE(t0 && c < 64, 3430 + c);
+        uint4 w[2];
         w[0] = lds128(sK(ks) + dswz(rr, p));
         w[1] = lds128(sK(ks) + dswz(rr, 8 + p));
-        float dp = 0.f;
+        // sigma = max(x, 0) + 2^(min(x, 0) log2 e), pairs of columns in f32x2
+        float sg[16];
+        float dp0 = 0.f, dp1 = 0.f;
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
-          const float4 za = *reinterpret_cast<const float4*>(zs + 64 * i + 8 * p);
-          const float4 zb = *reinterpret_cast<const float4*>(zs + 64 * i + 8 * p + 4);
-          const float zz[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
-          uint32_t* wp = reinterpret_cast<uint32_t*>(&w[i]);
-          uint32_t* lp = reinterpret_cast<uint32_t*>(&lo[i]);
+          const uint32_t* wp = reinterpret_cast<const uint32_t*>(&w[i]);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float s0 = valid ? elu1(bf16_lo(wp[e])) : 0.f;
-            const float s1 = valid ? elu1(bf16_hi(wp[e])) : 0.f;
-            dp = fmaf(s0, zz[2 * e], dp);
-            dp = fmaf(s1, zz[2 * e + 1], dp);
-            dz[8 * i + 2 * e] += s0;
-            dz[8 * i + 2 * e + 1] += s1;
-            const uint32_t hi = pack_bf16x2(s0, s1);
-            wp[e] = hi;
-            lp[e] = pack_bf16x2(s0 - bf16_lo(hi), s1 - bf16_hi(hi));
+            const int j = 8 * i + 2 * e;
+            const float x0 = bf16_lo(wp[e]), x1 = bf16_hi(wp[e]);
+            float m0, m1;
+            mul2(m0, m1, fminf(x0, 0.f), fminf(x1, 0.f), 1.4426950408889634f, 1.4426950408889634f);
+            add2(sg[j], sg[j + 1], fmaxf(x0, 0.f), fmaxf(x1, 0.f), ex2_approx(m0), ex2_approx(m1));
           }
         }
-        sts128(sK(ks) + dswz(rr, p), w[0]);
-        sts128(sK(ks) + dswz(rr, 8 + p), w[1]);
-        if (c >= LST) mbar_wait(bar(D_LE + ls), ((c / LST) - 1) & 1);  // dM(c - LST) released the lo buffer
-        sts128(sL(ls) + dswz(rr, p), lo[0]);
-        sts128(sL(ls) + dswz(rr, 8 + p), lo[1]);
+        if (t_begin + c * kDChunk + rr >= t_end) {  // a token past the segment's end (last chunk only)
+#pragma unroll
+          for (int j = 0; j < 16; ++j) sg[j] = 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < 16; j += 2) {
+          fma2(dp0, dp1, sg[j], sg[j + 1], zz[j], zz[j + 1], dp0, dp1);
+          add2(dz[j], dz[j + 1], dz[j], dz[j + 1], sg[j], sg[j + 1]);
+        }
         // den of the row: the 8 lanes of the row in a fixed butterfly (every lane gets the same sum)
+        float dp = dp0 + dp1;
         dp += __shfl_xor_sync(0xffffffffu, dp, 1);
         dp += __shfl_xor_sync(0xffffffffu, dp, 2);
         dp += __shfl_xor_sync(0xffffffffu, dp, 4);
-        if (p == 0) rinv[64 * ls + rr] = dp != 0.f ? 1.f / dp : 0.f;
+        const float rinv = dp != 0.f ? rcp_approx(dp) : 0.f;
+        uint4 hi[2], lo[2], sv[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          uint32_t* hp = reinterpret_cast<uint32_t*>(&hi[i]);
+          uint32_t* lp = reinterpret_cast<uint32_t*>(&lo[i]);
+          uint32_t* sp = reinterpret_cast<uint32_t*>(&sv[i]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float x0 = sg[8 * i + 2 * e], x1 = sg[8 * i + 2 * e + 1];
+            hp[e] = pack_bf16x2(x0, x1);
+            float l0, l1, s0, s1;
+            fma2(l0, l1, bf16_lo(hp[e]), bf16_hi(hp[e]), -1.f, -1.f, x0, x1);
+            lp[e] = pack_bf16x2(l0, l1);
+            mul2(s0, s1, x0, x1, rinv, rinv);
+            sp[e] = pack_bf16x2(s0, s1);
+          }
+        }
+        sts128(sK(ks) + dswz(rr, p), hi[0]);
+        sts128(sK(ks) + dswz(rr, 8 + p), hi[1]);
+        if (c >= LST) mbar_wait_parked(bar(D_LE + ls), lph ^ 1u);  // products of chunk c - LST are done
+        DELTA_TRACE(t0 && c < 64, 3500 + c);
+        sts128(sLo(ls) + dswz(rr, p), lo[0]);
+        sts128(sLo(ls) + dswz(rr, 8 + p), lo[1]);
+        sts128(sS(ls) + dswz(rr, p), sv[0]);
+        sts128(sS(ls) + dswz(rr, 8 + p), sv[1]);
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(D_SK + rb));
-      };
-      // U pass: value column d, tokens 16g..16g+15 of the chunk
-      auto u_pass = [&](int c) {
-        const int rb = c & 1, vs = c % VST;
-        mbar_wait(bar(D_SK + rb), (c >> 1) & 1);  // every warp's 1 / den of chunk c
-        mbar_wait(bar(D_RF + rb), (c >> 1) & 1);
-        tc_fence_after();
-        uint32_t r[16];
-        tmem_ld16(tR(rb) + lq + 16u * (uint32_t)g, r);
-        float ri[16];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float4 f = *reinterpret_cast<const float4*>(rinv + 64 * (c % LST) + 16 * g + 4 * i);
-          ri[4 * i] = f.x; ri[4 * i + 1] = f.y; ri[4 * i + 2] = f.z; ri[4 * i + 3] = f.w;
+        if (lane == 0) mbar_arrive(bar(D_SK + ls));
+        DELTA_TRACE(t0 && c < 64, 3210 + c);
+        if (++ks == KST) {
+          ks = 0;
+          kph ^= 1u;
         }
-        mbar_wait(bar(D_VF + vs), (c / VST) & 1);
-        float v[16];
-        const uint32_t vcol = (uint32_t)(d >> 6) * kDBox + (uint32_t)(d & 7) * 2u;
-#pragma unroll
-        for (int t = 0; t < 16; ++t) {
-          const int tt = 16 * g + t;
-          v[t] = lds_bf16(sV(vs) + vcol + (uint32_t)tt * 128u + ((uint32_t)(((d >> 3) & 7) ^ (tt & 7)) << 4));
+        if (++ls == LST) {
+          ls = 0;
+          lph ^= 1u;
         }
-        tmem_ld_wait();
-        uint32_t hw[8], lw[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float u0 = v[2 * j] - __uint_as_float(r[2 * j]) * ri[2 * j];
-          const float u1 = v[2 * j + 1] - __uint_as_float(r[2 * j + 1]) * ri[2 * j + 1];
-          hw[j] = pack_bf16x2(u0, u1);
-          lw[j] = pack_bf16x2(u0 - bf16_lo(hw[j]), u1 - bf16_hi(hw[j]));
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(D_VE + vs));  // every lane's V values are in registers
-        if (c >= 2) mbar_wait(bar(D_UE + rb), ((c >> 1) - 1) & 1);  // dM(c - 2) released the U buffer
-        tc_fence_after();
-        tmem_st8(tU(rb) + lq + 8u * (uint32_t)g, hw);
-        tmem_st8(tU(rb) + lq + 32u + 8u * (uint32_t)g, lw);
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(D_UR + rb));
-      };
-      sigma_pass(0);
-      for (int c = 0; c < nch; ++c) {
-        if (c + 1 < nch) sigma_pass(c + 1);
-        u_pass(c);
       }
-      mbar_wait(bar(D_DONE), 0);
+      mbar_wait_parked(bar(D_ACC), 0);
       tc_fence_after();
-      // every load and MMA of this CTA is complete: the rings hold the partial.
-      // dM[k][d] = dM^T[d][k]: lane d, columns k = 32g..32g+31
-      {
-        uint32_t rw[32];
-        tmem_ld32(tD + lq + 32u * (uint32_t)g, rw);
-        tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < 32; ++j) red[(32 * g + j) * 128 + d] = __uint_as_float(rw[j]);
-      }
+      __syncwarp();
+      cluster_arrive();  // every load and chunk product of this CTA is complete: the rings are free
+      DELTA_TRACE(t0, 3204);
       // dz: the 4 rows of the warp (lanes p, p + 8, p + 16, p + 24), then the 16 warps in order
       float* dzs = reinterpret_cast<float*>(gbase + SL::DZS);
 #pragma unroll
@@ -369,11 +415,101 @@ __global__ void __launch_bounds__(kDeltaThreads, 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i) dzs[warp * 128 + 64 * (i >> 3) + 8 * p + (i & 7)] = dz[i];
       }
+      // M_{s-1} for the final product and the snapshot: 16-byte chunks
+      // qq = tid + 512 i of the bf16 tiles (row k = qq / 16, columns
+      // 8 (qq % 16) ..).  M is still M_{s-1}: no CTA of the head reduces
+      // before this CTA's partial has reached it.
+      float4 mv[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int qq = threadIdx.x + 512 * i;
+        const float4* src = reinterpret_cast<const float4*>(Mh + (qq >> 4) * 128 + 8 * (qq & 15));
+        mv[2 * i] = src[0];
+        mv[2 * i + 1] = src[1];
+      }
+      // -G^T as the K-major B operand of the final product: row n = k holds
+      // -G[k][k'] along k', i.e. TMEM lane k of G; this warp writes columns
+      // 32g..32g+31
+      {
+        uint32_t rw[32];
+        tmem_ld32(tG + lq + 32u * (uint32_t)g, rw);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          uint4 vh, vl;
+          uint32_t* hp = reinterpret_cast<uint32_t*>(&vh);
+          uint32_t* lp = reinterpret_cast<uint32_t*>(&vl);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            split2(-__uint_as_float(rw[8 * i + 2 * e]), -__uint_as_float(rw[8 * i + 2 * e + 1]), hp[e], lp[e]);
+          sts128(base + SL::GH + swz_chunk(d, 4 * g + i), vh);
+          sts128(base + SL::GL + swz_chunk(d, 4 * g + i), vl);
+        }
+      }
+      // M^T as the MN-major A operand: row k of M, columns d contiguous, in
+      // hi and lo tiles; this CTA's rows of the snapshot from the same values
+      {
+        const int r_lo = delta_row_lo(grp, a.G), r_hi = delta_row_lo(grp + 1, a.G);
+        __nv_bfloat16* snap = a.snapM + ((long long)bh * a.S + s) * 16384;
+        float* snap32 = a.snapM32 + ((long long)bh * a.S + s) * 16384;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int qq = threadIdx.x + 512 * i, k = qq >> 4, cc = qq & 15;
+          const float4 f0 = mv[2 * i], f1 = mv[2 * i + 1];
+          uint4 vh, vl;
+          split2(f0.x, f0.y, vh.x, vl.x);
+          split2(f0.z, f0.w, vh.y, vl.y);
+          split2(f1.x, f1.y, vh.z, vl.z);
+          split2(f1.z, f1.w, vh.w, vl.w);
+          sts128(base + SL::MH + swz_chunk(k, cc), vh);
+          sts128(base + SL::ML + swz_chunk(k, cc), vl);
+          if (k >= r_lo && k < r_hi) {
+            if (a.snapM != nullptr) *reinterpret_cast<uint4*>(snap + k * 128 + 8 * cc) = vh;
+            if (a.snapM32 != nullptr) {
+              reinterpret_cast<float4*>(snap32 + k * 128 + 8 * cc)[0] = f0;
+              reinterpret_cast<float4*>(snap32 + k * 128 + 8 * cc)[1] = f1;
+            }
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(D_GR));
+      DELTA_TRACE(t0, 3205);
       named_bar_sync(1, 512);
-      if (threadIdx.x < 128) {
-        float t = 0.f;
-        for (int w2 = 0; w2 < 16; ++w2) t += dzs[w2 * 128 + threadIdx.x];
-        red[16384 + threadIdx.x] = t;
+      float dzt = 0.f;
+      if (threadIdx.x < 128)
+        for (int w2 = 0; w2 < 16; ++w2) dzt += dzs[w2 * 128 + threadIdx.x];
+      DELTA_TRACE(t0, 3206);
+      // dM[k][d] = dM^T[d][k]: lane d, columns k = 32g..32g+31, staged in
+      // this CTA's shared memory as [dM | dz]
+      mbar_wait_parked(bar(D_FIN), 0);
+      tc_fence_after();
+      float* red = reinterpret_cast<float*>(gbase + SL::RED);
+      {
+        uint32_t rw[32];
+        tmem_ld32(tVM + lq + 32u * (uint32_t)g, rw);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) red[(32 * g + j) * 128 + d] = __uint_as_float(rw[j]);
+        if (threadIdx.x < 128) red[16384 + threadIdx.x] = dzt;
+      }
+      fence_proxy_async_smem();  // the bulk copies read the staged partial
+      named_bar_sync(1, 512);
+      DELTA_TRACE(t0, 3207);
+      cluster_wait();  // every CTA of the cluster is past its chunks: its landing area is free
+      DELTA_TRACE(t0, 3208);
+      // slice r of the partial to CTA r (slot grp of its landing area); this
+      // CTA's own slice stays in place
+      const int r = threadIdx.x;
+      if (r < a.G && r != grp) {
+        const int len = min(per, kDeltaE4 - r * per);
+        bulk_copy_to_peer(mapa_shared(base + SL::LAND + 16u * (uint32_t)(grp * per), (uint32_t)r),
+                          base + SL::RED + 16u * (uint32_t)(r * per), (uint32_t)(16 * len),
+                          mapa_shared(bar(D_RX), (uint32_t)r));
+        bulk_commit();
+        bulk_wait_read();  // the source stays valid until it has been read
       }
     }
     tc_fence_before();
@@ -381,33 +517,47 @@ __global__ void __launch_bounds__(kDeltaThreads, 1)
     if (warp == 17) {
       __syncwarp();
       tc_fence_after();
-      tmem_dealloc(tmem, 512);
+      tmem_dealloc(tmem, 256);
     }
   }
   // ------------------------------------------------------------ cluster reduction
-  __syncthreads();
-  cluster_sync();  // every CTA of the head has staged its partial
+  // This CTA's slice of M, z (no other CTA writes it) is loaded while the
+  // partials land: at most 7 float4 per thread (a slice of <= 4128 float4).
+  auto state4 = [&](int e4) {
+    const int e = 4 * e4;
+    return e < 16384 ? reinterpret_cast<float4*>(&a.M[(long long)bh * 16384 + e])
+                     : reinterpret_cast<float4*>(&a.z[(long long)bh * 128 + (e - 16384)]);
+  };
+  constexpr int kIt = (kDeltaE4 + kDeltaThreads - 1) / kDeltaThreads;
+  float4 acc[kIt];
+  griddep_wait();  // (complete long since for the threads that read M above)
+#pragma unroll
+  for (int it = 0; it < kIt; ++it) {
+    const int e4 = e4_begin + (int)threadIdx.x + it * kDeltaThreads;
+    if (e4 < e4_end) acc[it] = *state4(e4);
+  }
+  mbar_wait_parked(bar(D_RX), 0);  // every other CTA's partial of this slice has landed
+  DELTA_TRACE(t0, 3209);
   {
-    constexpr int E4 = (128 * 128 + 128) / 4;  // float4 elements of [M | z]
-    const int per = (E4 + a.G - 1) / a.G;
-    const int e4_begin = grp * per, e4_end = min(E4, e4_begin + per);
-    const uint32_t red_addr = smem_u32(red);
-    for (int e4 = e4_begin + (int)threadIdx.x; e4 < e4_end; e4 += blockDim.x) {
-      const int e = 4 * e4;
-      float4* st = e < 16384 ? reinterpret_cast<float4*>(&a.M[(long long)bh * 16384 + e])
-                             : reinterpret_cast<float4*>(&a.z[(long long)bh * 128 + (e - 16384)]);
-      float4 acc = *st;
-      for (int g2 = 0; g2 < a.G; ++g2) {
-        const float4 v = ld_dsmem_f4(mapa_shared(red_addr + 16u * (uint32_t)e4, (uint32_t)g2));
-        acc.x += v.x;
-        acc.y += v.y;
-        acc.z += v.z;
-        acc.w += v.w;
+    const float4* lf = reinterpret_cast<const float4*>(gbase + SL::LAND);
+    const float4* own = reinterpret_cast<const float4*>(gbase + SL::RED);  // this CTA's partial (nch > 0)
+#pragma unroll
+    for (int it = 0; it < kIt; ++it) {
+      const int e4 = e4_begin + (int)threadIdx.x + it * kDeltaThreads;
+      if (e4 < e4_end) {
+        for (int g2 = 0; g2 < a.G; ++g2) {
+          if (g2 == grp ? nch == 0 : !has_tokens(g2)) continue;
+          const float4 v = g2 != grp ? lf[g2 * per + (e4 - e4_begin)] : own[e4];
+          acc[it].x += v.x;
+          acc[it].y += v.y;
+          acc[it].z += v.z;
+          acc[it].w += v.w;
+        }
+        *state4(e4) = acc[it];
       }
-      *st = acc;
     }
   }
-  cluster_sync();  // peers have finished reading this CTA's shared memory
+  DELTA_TRACE(t0, 3420);
 }
 
 }  // namespace tc
