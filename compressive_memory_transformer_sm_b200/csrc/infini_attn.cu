@@ -434,8 +434,8 @@ int set_tc_smem_limits() {
   if (ctx != 0 && std::find(done.begin(), done.end(), ctx) != done.end()) return INFINI_OK;
   if (cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kAttnSmem) !=
           cudaSuccess ||
-      cudaFuncSetAttribute(tc::mem_update_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)tc::UpdSmem<false>::BYTES) != cudaSuccess ||
+      cudaFuncSetAttribute(tc::mem_update_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)tc::UpdSmem::BYTES) != cudaSuccess ||
       cudaFuncSetAttribute(tc::delta_update_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)tc::DeltaSmem::BYTES) != cudaSuccess ||
       cudaFuncSetAttribute(tc::gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kGemmSmem) !=
@@ -561,7 +561,7 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale, c
     ua.seg0 = 0; ua.nseg = pl.S;
     {
       LaunchScope ls(kPhaseUpdate, p.stream);
-      tc::mem_update_tc_kernel<false><<<BH * pl.S * pl.G, tc::UpdWarps<false>::THREADS, tc::UpdSmem<false>::BYTES, p.stream>>>(
+      tc::mem_update_tc_kernel<<<BH * pl.S * pl.G, tc::UpdWarps::THREADS, tc::UpdSmem::BYTES, p.stream>>>(
           tm_k, tm_v, ua);
     }
     LaunchScope ls(kPhaseState, p.stream);
