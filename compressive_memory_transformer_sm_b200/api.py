@@ -30,6 +30,7 @@ NOALLOC_SCRATCH_BYTES = 32 << 20
 FLAG_FORCE_SIMT = 0x1
 FLAG_ATTN_SINGLE = 0x2
 FLAG_ATTN_PAIRS = 0x4
+FLAG_ATTN_SPLIT = 0x8
 
 EXPORTED = (
     "infini_attn_forward", "infini_attn_segment_step", "infini_attn_forward_ex", "infini_attn_workspace_size",

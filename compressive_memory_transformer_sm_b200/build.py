@@ -67,16 +67,19 @@ def check_register_split(ptxas_log: str, kernel: str = "attn_tc_kernel", want: i
     assuming it was launched with exactly `want` registers per thread; any other
     allocation could make a register increase wait forever, so refuse to build."""
     lines = ptxas_log.splitlines()
+    checked = 0
     for i, line in enumerate(lines):
-        if "Compiling entry function" in line and kernel in line:
+        if "Compiling entry function" in line and kernel in line:  # every instantiation
             for nxt in lines[i + 1:i + 6]:
                 if "Used" in nxt and "registers" in nxt:
                     used = int(nxt.split("Used")[1].split("registers")[0])
                     if used != want:
                         raise RuntimeError(f"{kernel} uses {used} registers per thread, its register split "
                                            f"assumes {want}: refusing to build")
-                    return
-    raise RuntimeError(f"ptxas report for {kernel} not found: cannot verify its register split")
+                    checked += 1
+                    break
+    if checked == 0:
+        raise RuntimeError(f"ptxas report for {kernel} not found: cannot verify its register split")
 
 
 if __name__ == "__main__":

@@ -432,8 +432,10 @@ int set_tc_smem_limits() {
   const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lk(mu);
   if (ctx != 0 && std::find(done.begin(), done.end(), ctx) != done.end()) return INFINI_OK;
-  if (cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kAttnSmem) !=
-          cudaSuccess ||
+  if (cudaFuncSetAttribute(tc::attn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)tc::kAttnSmem) != cudaSuccess ||
+      cudaFuncSetAttribute(tc::attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)tc::kAttnSmem) != cudaSuccess ||
       cudaFuncSetAttribute(tc::mem_update_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)tc::UpdSmem::BYTES) != cudaSuccess ||
       cudaFuncSetAttribute(tc::delta_update_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -625,9 +627,12 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale, c
   const long long NS = (long long)BH * pl.S;
   // Pairs of query tiles per CTA, unless that leaves SMs idle (short streaming steps):
   // then one query tile per CTA.
-  aa.single = NS * ((aa.T + 1) / 2) < sms ? 1 : 0;
+  // pairs of query tiles per item when they fill the GPU, else one tile per
+  // item with its key tiles split between the two softmax warpgroups
+  aa.single = NS * ((aa.T + 1) / 2) < sms ? 2 : 0;
   if (p.flags & INFINI_FLAG_ATTN_SINGLE) aa.single = 1;
   if (p.flags & INFINI_FLAG_ATTN_PAIRS) aa.single = 0;
+  if (p.flags & INFINI_FLAG_ATTN_SPLIT) aa.single = 2;
   aa.P = aa.single ? aa.T : (aa.T + 1) / 2;
   aa.GS = (int)std::max<long long>(1, std::min<long long>(NS, (sms + aa.P - 1) / aa.P));
   const long long groups = (NS + aa.GS - 1) / aa.GS;
@@ -640,8 +645,11 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale, c
   }
   {
     LaunchScope ls(kPhaseAttn, as);
-    tc::attn_tc_kernel<<<(unsigned)std::min<long long>(items, sms), tc::kAttnThreads, tc::kAttnSmem, as>>>(
-        tm_qa, tm_ka, tm_v, tm_mt, aa);
+    const unsigned grid = (unsigned)std::min<long long>(items, sms);
+    if (aa.single == 2)
+      tc::attn_tc_kernel<true><<<grid, tc::kAttnThreads, tc::kAttnSmem, as>>>(tm_qa, tm_ka, tm_v, tm_mt, aa);
+    else
+      tc::attn_tc_kernel<false><<<grid, tc::kAttnThreads, tc::kAttnSmem, as>>>(tm_qa, tm_ka, tm_v, tm_mt, aa);
   }
   const int rc = launch_status();
   join();

@@ -32,9 +32,12 @@ struct AttnArgs {
   __nv_bfloat16* out;
   unsigned int* work_counter;  // next unclaimed work item; zero at launch (items < 2^31)
   int B, H, S, T;         // T = query tiles per full segment
-  int P;                  // work items per full segment: ceil(T / 2) pairs, or T tiles when `single`
+  int P;                  // work items per full segment: ceil(T / 2) pairs, or T tiles (modes 1, 2)
   int GS;                 // segments per scheduling group
-  int single;             // 1: one query tile per work item (small grids), warpgroup 1 idle
+  // 0: a pair of query tiles per work item; 1: one query tile per item,
+  // warpgroup 1 idle; 2: one query tile per item, its key tiles split between
+  // the two warpgroups and their softmax states merged (small grids)
+  int single;
   long long L;
   int N;
   float scale_log2;       // softmax scale * log2(e)
@@ -120,6 +123,9 @@ static_assert(kAttnSmem <= 232448, "attention kernel exceeds 227 KB of shared me
 // Items are ordered by groups of GS segments (about one wave of items per
 // group, so the group's K/V stays in L2), heaviest pair first inside a group;
 // claiming them dynamically balances the CTAs.
+// kSplit: the split schedule (a.single == 2), compiled as its own kernel so
+// that the pair and single-tile schedules keep their code unchanged.
+template <bool kSplit>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_mt,
@@ -133,7 +139,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int NS = a.B * a.H * a.S;
   const int per_group = a.GS * a.P;
   const int total = ((NS + a.GS - 1) / a.GS) * per_group;  // the host keeps this below 2^31
-  const bool single = a.single != 0;
+  const bool single = !kSplit && a.single == 1;
+  constexpr bool split = kSplit;
   // Work item idx of the grouped heavy-first order -> (m, segment); false for
   // the padding of the last group and for tiles past the end of a short
   // (tail) segment.
@@ -146,16 +153,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int r = idx - grp * per_group;
     const int gsz = min(a.GS, NS - grp * a.GS);
     if (r >= gsz * a.P) return false;
-    it.m = a.P - 1 - r / gsz;  // pair index, or tile index when single
+    it.m = a.P - 1 - r / gsz;  // pair index, or tile index (modes 1, 2)
     it.seg = grp * a.GS + r % gsz;  // = bh * S + s
     const int bh = it.seg / a.S, s = it.seg % a.S;
     it.b = bh / a.H;
     it.h = bh % a.H;
     it.seg0 = (long long)s * a.N;
     it.n_s = (int)min((long long)a.N, a.L - it.seg0);
-    it.tq0 = single ? it.m : 2 * it.m;        // query tile of warpgroup 0 (warpgroup 1: tq0 + 1)
-    it.nk0 = it.tq0 + 1;                      // K/V tiles of query tile tq0
-    it.nk1 = it.tq0 + (single ? 1 : 2);       // K/V tiles of the item's last query tile
+    it.tq0 = single || split ? it.m : 2 * it.m;  // query tile of warpgroup 0 (pairs: warpgroup 1 has tq0 + 1)
+    if (split) {  // key tiles [0, nk0) to warpgroup 0, [nk0, nk0 + nk1) (with the diagonal) to warpgroup 1
+      it.nk0 = (it.tq0 + 1) / 2;
+      it.nk1 = it.tq0 + 1 - it.nk0;
+    } else {
+      it.nk0 = it.tq0 + 1;                    // K/V tiles of query tile tq0
+      it.nk1 = it.tq0 + (single ? 1 : 2);     // K/V tiles of the item's last query tile
+    }
     return it.tq0 * kTile < it.n_s;
   };
 
@@ -265,39 +277,78 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // a pending V never holds back the next K).  Q after the memory-read
         // products of the previous item, which read sigma(Q) from the Q
         // tiles: issued after K tile 0 of the new item.
-        for (int j = 0; j <= w.nk1; ++j) {
-          if (j < w.nk1) {
-            const int lk = (int)(w.seg0 + (long long)j * kTile);
-            if (!mbar_wait(kfree(gk), kph(gk) ^ 1u)) goto done;
-            mbar_expect_tx(kfull(gk), kTileBytes);
-            tma_load_4d(sKt(gk), &tm_k, kfull(gk), 0, lk, w.h, w.b);
-            tma_load_4d(sKt(gk) + kBox, &tm_k, kfull(gk), 64, lk, w.h, w.b);
-            gk = knext(gk, 1);
-            kn = min(kn + 1u, (uint32_t)kKStages);
-          }
-          if (j == 0) {
-            const uint32_t prev = (uint32_t)(it & 1) ^ 1u;  // previous item's phase (fresh: complete)
-            if (!mbar_wait(bar(B_MEM0), prev)) goto done;
-            if (!single && !mbar_wait(bar(B_MEM0 + 1), prev)) goto done;
-            const int lq = (int)(w.seg0 + (long long)w.tq0 * kTile);
-            mbar_expect_tx(bar(B_Q), (single ? 1 : 2) * kTileBytes);
-            tma_load_4d(sQ(0), &tm_q, bar(B_Q), 0, lq, w.h, w.b);
-            tma_load_4d(sQ(0) + kBox, &tm_q, bar(B_Q), 64, lq, w.h, w.b);
-            if (!single) {
-              tma_load_4d(sQ(1), &tm_q, bar(B_Q), 0, lq + kTile, w.h, w.b);
-              tma_load_4d(sQ(1) + kBox, &tm_q, bar(B_Q), 64, lq + kTile, w.h, w.b);
+        if (split) {
+          // Key tiles of the two warpgroups interleaved in both rings: step j
+          // loads warpgroup 0's tile j (j < nk0), then warpgroup 1's tile
+          // nk0 + j (j < nk1); V trails K by one step.  One Q tile.
+          for (int j = 0; j <= w.nk1; ++j) {
+            for (int kq = 0; kq < 2; ++kq) {
+              if (j >= (kq ? w.nk1 : w.nk0)) continue;
+              const int lk = (int)(w.seg0 + (long long)(kq ? w.nk0 + j : j) * kTile);
+              if (!mbar_wait(kfree(gk), kph(gk) ^ 1u)) goto done;
+              mbar_expect_tx(kfull(gk), kTileBytes);
+              tma_load_4d(sKt(gk), &tm_k, kfull(gk), 0, lk, w.h, w.b);
+              tma_load_4d(sKt(gk) + kBox, &tm_k, kfull(gk), 64, lk, w.h, w.b);
+              gk = knext(gk, 1);
+              kn = min(kn + 1u, (uint32_t)kKStages);
             }
-            ++nq;
-            ATTN_TRACE(true, 3072 + 16 * it + 2);
+            if (j == 0) {
+              const uint32_t prev = (uint32_t)(it & 1) ^ 1u;  // previous item's phase (fresh: complete)
+              if (!mbar_wait(bar(B_MEM0), prev)) goto done;
+              const int lq = (int)(w.seg0 + (long long)w.tq0 * kTile);
+              mbar_expect_tx(bar(B_Q), kTileBytes);
+              tma_load_4d(sQ(0), &tm_q, bar(B_Q), 0, lq, w.h, w.b);
+              tma_load_4d(sQ(0) + kBox, &tm_q, bar(B_Q), 64, lq, w.h, w.b);
+              ++nq;
+            }
+            if (j >= 1) {
+              for (int kq = 0; kq < 2; ++kq) {
+                if (j - 1 >= (kq ? w.nk1 : w.nk0)) continue;
+                const int lk = (int)(w.seg0 + (long long)(kq ? w.nk0 + j - 1 : j - 1) * kTile);
+                if (!mbar_wait(vfree(gv), vph(gv) ^ 1u)) goto done;
+                mbar_expect_tx(vfull(gv), kTileBytes);
+                tma_load_4d(sVt(gv), &tm_v, vfull(gv), 0, lk, w.h, w.b);
+                tma_load_4d(sVt(gv) + kBox, &tm_v, vfull(gv), 64, lk, w.h, w.b);
+                ++gv;
+                vn = min(vn + 1u, 2u);
+              }
+            }
           }
-          if (j >= 1) {
-            const int lk = (int)(w.seg0 + (long long)(j - 1) * kTile);
-            if (!mbar_wait(vfree(gv), vph(gv) ^ 1u)) goto done;
-            mbar_expect_tx(vfull(gv), kTileBytes);
-            tma_load_4d(sVt(gv), &tm_v, vfull(gv), 0, lk, w.h, w.b);
-            tma_load_4d(sVt(gv) + kBox, &tm_v, vfull(gv), 64, lk, w.h, w.b);
-            ++gv;
-            vn = min(vn + 1u, 2u);
+        } else {
+          for (int j = 0; j <= w.nk1; ++j) {
+            if (j < w.nk1) {
+              const int lk = (int)(w.seg0 + (long long)j * kTile);
+              if (!mbar_wait(kfree(gk), kph(gk) ^ 1u)) goto done;
+              mbar_expect_tx(kfull(gk), kTileBytes);
+              tma_load_4d(sKt(gk), &tm_k, kfull(gk), 0, lk, w.h, w.b);
+              tma_load_4d(sKt(gk) + kBox, &tm_k, kfull(gk), 64, lk, w.h, w.b);
+              gk = knext(gk, 1);
+              kn = min(kn + 1u, (uint32_t)kKStages);
+            }
+            if (j == 0) {
+              const uint32_t prev = (uint32_t)(it & 1) ^ 1u;  // previous item's phase (fresh: complete)
+              if (!mbar_wait(bar(B_MEM0), prev)) goto done;
+              if (!single && !mbar_wait(bar(B_MEM0 + 1), prev)) goto done;
+              const int lq = (int)(w.seg0 + (long long)w.tq0 * kTile);
+              mbar_expect_tx(bar(B_Q), (single ? 1 : 2) * kTileBytes);
+              tma_load_4d(sQ(0), &tm_q, bar(B_Q), 0, lq, w.h, w.b);
+              tma_load_4d(sQ(0) + kBox, &tm_q, bar(B_Q), 64, lq, w.h, w.b);
+              if (!single) {
+                tma_load_4d(sQ(1), &tm_q, bar(B_Q), 0, lq + kTile, w.h, w.b);
+                tma_load_4d(sQ(1) + kBox, &tm_q, bar(B_Q), 64, lq + kTile, w.h, w.b);
+              }
+              ++nq;
+              ATTN_TRACE(true, 3072 + 16 * it + 2);
+            }
+            if (j >= 1) {
+              const int lk = (int)(w.seg0 + (long long)(j - 1) * kTile);
+              if (!mbar_wait(vfree(gv), vph(gv) ^ 1u)) goto done;
+              mbar_expect_tx(vfull(gv), kTileBytes);
+              tma_load_4d(sVt(gv), &tm_v, vfull(gv), 0, lk, w.h, w.b);
+              tma_load_4d(sVt(gv) + kBox, &tm_v, vfull(gv), 64, lk, w.h, w.b);
+              ++gv;
+              vn = min(vn + 1u, 2u);
+            }
           }
         }
         // M_{s-1} (bf16 snapshot, [dk][dv]) enters the K ring after the item's K tiles.
@@ -367,6 +418,80 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (elect_one()) mma_commit(b);
           __syncwarp();
         };
+        if (split) {
+          // One query tile (Q_0) for both warpgroups; warpgroup k's key tile j
+          // sits at ring position kpos(k, j) of the item (the producer's order).
+          const uint32_t prev = (uint32_t)(it & 1) ^ 1u;
+          const int n0 = w.nk0, n1 = w.nk1;
+          auto kpos = [&](int k, int j) { return k == 0 ? 2 * j : j + min(j + 1, n0); };
+          auto issue_sq = [&](int k, uint32_t g) {  // S_k = Q_0 K^T
+            const uint64_t da = kmajor_base(sQi(0)), db = kmajor_base(sKt(g));
+            if (elect_one()) {
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk)
+                mma_ss(tmem + (uint32_t)k * 128u, da + kmajor_step(kk), db + kmajor_step(kk), idesc_kk, kk > 0 ? 1u : 0u);
+            }
+            __syncwarp();
+          };
+          mbar_wait(bar(B_Q), (uint32_t)(it & 1));
+#pragma unroll 1
+          for (int k = 0; k < 2; ++k) {
+            if ((k ? n1 : n0) == 0) continue;
+            const uint32_t g = knext(gk, kpos(k, 0));
+            mbar_wait(kfull(g), kph(g));
+            mbar_wait(bar(B_OF0 + k), prev);  // S_k(0) overwrites what the previous epilogue reads
+            tc_fence_after();
+            issue_sq(k, g);
+            commit(bar(B_SF0 + k));
+            commit(kfree(g));
+          }
+          for (int j = 0; j < n1; ++j) {
+#pragma unroll 1
+            for (int k = 0; k < 2; ++k) {
+              const int nk = k ? n1 : n0;
+              if (j >= nk) continue;
+              const uint32_t gvj = gv + (uint32_t)kpos(k, j);
+              uint32_t& nt = k ? nt1 : nt0;
+              mbar_wait(vfull(gvj), vph(gvj));
+              mbar_wait(bar(B_PH0 + k), nt & 1u);
+              tc_fence_after();
+              issue_pv_half(k, gvj, 0, j == 0);
+              mbar_wait(bar(B_PF0 + k), nt & 1u);
+              ++nt;
+              tc_fence_after();
+              issue_pv_half(k, gvj, 1, j == 0);
+              commit(vfree(gvj));
+              if (j + 1 < nk) {
+                const uint32_t gn = knext(gk, kpos(k, j + 1));
+                mbar_wait(kfull(gn), kph(gn));
+                issue_sq(k, gn);
+                commit(bar(B_SF0 + k));
+                commit(kfree(gn));
+              }
+            }
+          }
+          commit(bar(B_MEM0 + 1));  // every product of warpgroup 1 complete: its O is final
+          // memory read of the tile: sigma(Q_0) M_{s-1} into S_0's columns
+          const uint32_t gm = knext(gk, n0 + n1);
+          mbar_wait(kfull(gm), kph(gm));
+          mbar_wait(bar(B_OF0), prev);  // (no S_0 product waited for it when n0 = 0)
+          mbar_wait(bar(B_SQ0), (uint32_t)(it & 1));
+          tc_fence_after();
+          {
+            const uint64_t da = kmajor_base(sQi(0)), db = mnmajor_base(sKt(gm));
+            if (elect_one()) {
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk)
+                mma_ss(tmem, da + kmajor_step(kk), db + mnmajor_step(kk), idesc_mem, kk > 0 ? 1u : 0u);
+            }
+            __syncwarp();
+          }
+          commit(bar(B_MEM0));
+          commit(kfree(gm));
+          gk = knext(gm, 1);
+          gv += (uint32_t)(n0 + n1);
+          continue;
+        }
         const uint32_t prev = (uint32_t)(it & 1) ^ 1u;  // previous item's phase (fresh: complete)
         ATTN_TRACE(true, 2048 + 16 * it + 0);
         mbar_wait(bar(B_Q), (uint32_t)(it & 1));
@@ -463,7 +588,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (idx < 0) break;
       Item w;
       decode(idx, w);
-      const int nk = w.nk0 + k;  // its K/V tiles; the last one is its diagonal
+      // its K/V tiles; the last one is its diagonal (split: warpgroup 1's last)
+      const int nk = split ? (k ? w.nk1 : w.nk0) : w.nk0 + k;
       ATTN_TRACE(tr, 1024 * k + 16 * it + 0);
       ATTN_TRACE_VAL(tr, 1024 * k + 16 * it + 8, (unsigned long long)nk);
       const float zrow = a.snapz[(long long)w.seg * 128 + row];  // used after the loop
@@ -487,7 +613,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tmem_ld_wait();
         }
         ATTN_TRACE(tr && it == 0, 1024 * k + 512 + 8 * j + 2);
-        if (j == nk - 1) {  // diagonal tile: key e is visible to query row iff e <= row
+        if (j == nk - 1 && (!split || k == 1)) {  // diagonal tile: key e is visible to query row iff e <= row
 #pragma unroll
           for (int e = 0; e < 128; ++e)
             if (e > row) x[e] = __float_as_uint(-INFINITY);
@@ -555,6 +681,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         ATTN_TRACE(tr && it == 0, 1024 * k + 512 + 8 * j + 1);
       }
       ATTN_TRACE(tr, 1024 * k + 16 * it + 2);
+      if (split && k == 1) {
+        // warpgroup 1's row state (reference max, sum) for warpgroup 0's merge,
+        // in the Q_1 tile's space (unused with one query tile); its O stays in
+        // TMEM.  Warpgroup 0 reads them after the barrier and releases O_1.
+        float* ml = reinterpret_cast<float*>(gbase + kA_Q1);
+        ml[row] = m_ref;
+        ml[128 + row] = l;
+        named_bar_arrive(3, 256);
+        continue;
+      }
+      // Split: warpgroup 1's S products read Q_0 too; its arrival (after it
+      // has waited for every one of them) lets warpgroup 0 overwrite Q_0.
+      if (split) named_bar_sync(3, 256);
       // Every Q_k K^T product of the item has completed: overwrite this row of
       // Q_k with sigma(Q_k) (bf16) for the memory read, and form the fp32
       // denominator sigma(q) . z_{s-1} from the unrounded sigma.  (The z copy
@@ -616,6 +755,60 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_wait(bar(B_MEM0 + k), (uint32_t)(it & 1));  // also implies the last P V of tile k
       ATTN_TRACE(tr, 1024 * k + 16 * it + 4);
       tc_fence_after();
+      if (split) {
+        // Merge the two warpgroups' softmax states: reference maxima m0, m1
+        // (log2 units), sums l0, l1, unnormalised O_0, O_1 (TMEM; B_MEM0
+        // complete implies warpgroup 1's products complete):
+        // O = 2^(m0-m) O_0 + 2^(m1-m) O_1, l = 2^(m0-m) l0 + 2^(m1-m) l1.
+        // (warpgroup 1 stored m1, l1 before the barrier above.)
+        const float* ml = reinterpret_cast<const float*>(gbase + kA_Q1);
+        const float m1 = ml[row], l1 = ml[128 + row];
+        const bool has0 = w.nk0 > 0;  // warpgroup 0 had key tiles (O_0 written)
+        const float mx = has0 ? fmaxf(m_ref, m1) : m1;
+        const float a0 = has0 ? ex2_approx(m_ref - mx) : 0.f, a1 = ex2_approx(m1 - mx);
+        const float lt = a0 * l + a1 * l1;
+        const float gw = 1.f / (1.f + __expf(-a.beta[w.h]));
+        const float wdot = (1.f - gw) / lt;
+        const float wmem = den != 0.f ? gw / den : 0.f;
+        const int qrow = w.tq0 * kTile + row;
+        const bool valid = qrow < w.n_s;
+        uint4* dst = reinterpret_cast<uint4*>(a.out + w.b * a.os[0] + w.h * a.os[1] + (w.seg0 + qrow) * a.os[2]);
+        const uint32_t tO1 = tmem + lrow + 384u;
+#pragma unroll 1
+        for (int c8 = 0; c8 < 8; ++c8) {  // 16 columns at a time
+          uint32_t r0[16], r1[16], rm[16];
+          if (has0) tmem_ld16(tO + 16u * c8, r0);
+          tmem_ld16(tO1 + 16u * c8, r1);
+          tmem_ld16(tS + 16u * c8, rm);
+          tmem_ld_wait();
+          float o[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            o[e] = has0 ? fmaf(a0, __uint_as_float(r0[e]), a1 * __uint_as_float(r1[e])) : a1 * __uint_as_float(r1[e]);
+          uint32_t pk[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            pk[e] = pack_bf16x2(wmem * __uint_as_float(rm[2 * e]) + wdot * o[2 * e],
+                                wmem * __uint_as_float(rm[2 * e + 1]) + wdot * o[2 * e + 1]);
+          if (valid) {
+            dst[2 * c8] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            dst[2 * c8 + 1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          }
+          if (a.adot != nullptr && valid) {
+            const float inv_l = 1.f / lt;
+            float4* ad = reinterpret_cast<float4*>(a.adot + (((long long)w.b * a.H + w.h) * a.L + w.seg0 + qrow) * 128);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              ad[4 * c8 + e] = make_float4(o[4 * e] * inv_l, o[4 * e + 1] * inv_l, o[4 * e + 2] * inv_l, o[4 * e + 3] * inv_l);
+          }
+        }
+        if (a.lse2 != nullptr && valid) a.lse2[((long long)w.b * a.H + w.h) * a.L + w.seg0 + qrow] = mx + __log2f(lt);
+        // S_0, O_0 and O_1 are read out: the next item's products may overwrite them
+        tc_fence_before();
+        mbar_arrive(bar(B_OF0));
+        mbar_arrive(bar(B_OF0 + 1));
+        continue;
+      }
       const float gw = 1.f / (1.f + __expf(-a.beta[w.h]));
       const float wdot = (1.f - gw) / l;
       const float wmem = den != 0.f ? gw / den : 0.f;

@@ -75,11 +75,14 @@ extern "C" {
 /* infini_attn_params.flags: run the CUDA-core (SIMT) kernels even where the
  * tensor-core kernels apply -- a second GPU implementation, for testing */
 #define INFINI_FLAG_FORCE_SIMT 0x1
-/* tensor-core attention schedule: one query tile per CTA (the default for
- * grids that would otherwise leave SMs idle) or pairs of query tiles per CTA
- * (the default otherwise); these force one of them, for testing */
+/* tensor-core attention schedule: pairs of query tiles per CTA (the default
+ * for grids that fill the GPU), one query tile per CTA with its key tiles
+ * split between the CTA's two softmax warpgroups (the default for grids that
+ * would otherwise leave SMs idle, e.g. one segment), or one query tile per
+ * CTA on one warpgroup; these force one of them, for testing */
 #define INFINI_FLAG_ATTN_SINGLE 0x2
 #define INFINI_FLAG_ATTN_PAIRS 0x4
+#define INFINI_FLAG_ATTN_SPLIT 0x8
 
 enum {
   INFINI_OK = 0,

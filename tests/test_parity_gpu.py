@@ -110,7 +110,7 @@ BF16_SHAPES = [
 
 
 PATH_FLAGS = {"tensor-pairs": api.FLAG_ATTN_PAIRS, "tensor-single": api.FLAG_ATTN_SINGLE,
-              "simt": api.FLAG_FORCE_SIMT}
+              "tensor-split": api.FLAG_ATTN_SPLIT, "simt": api.FLAG_FORCE_SIMT}
 
 
 @pytest.mark.parametrize("shape", BF16_SHAPES)
