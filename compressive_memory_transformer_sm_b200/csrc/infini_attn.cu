@@ -59,9 +59,34 @@ std::atomic<int> g_profile_mask{0};
 struct EventPair {
   int phase;
   cudaEvent_t a, b;
+  unsigned long long ctx;  // the context the events belong to
 };
 std::mutex g_prof_mu;
 std::vector<EventPair> g_prof;
+// Timing events already read out, for reuse (an event belongs to the context
+// it was created in): creating two events per timed launch would add host time
+// to every timed call.
+std::vector<std::pair<unsigned long long, cudaEvent_t>> g_event_pool;
+unsigned long long current_context_id();
+
+cudaEvent_t take_timing_event(unsigned long long ctx) {
+  {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    for (size_t i = 0; i < g_event_pool.size(); ++i)
+      if (g_event_pool[i].first == ctx) {
+        cudaEvent_t e = g_event_pool[i].second;
+        g_event_pool[i] = g_event_pool.back();
+        g_event_pool.pop_back();
+        return e;
+      }
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  return e;
+}
 
 // Counts one kernel launch and, when its phase is being timed, brackets it
 // with events on `stream`.  Construct right before the launch, destroy
@@ -70,12 +95,17 @@ struct LaunchScope {
   int phase;
   cudaStream_t stream;
   cudaEvent_t a = nullptr, b = nullptr;
+  unsigned long long ctx = 0;
   LaunchScope(int ph, cudaStream_t st) : phase(ph), stream(st) {
     g_launches.fetch_add(1, std::memory_order_relaxed);
     if (g_profile_mask.load(std::memory_order_relaxed) & (1 << ph)) {
-      if (cudaEventCreate(&a) == cudaSuccess && cudaEventCreate(&b) == cudaSuccess) {
+      ctx = current_context_id();
+      a = take_timing_event(ctx);
+      b = a ? take_timing_event(ctx) : nullptr;
+      if (a && b) {
         cudaEventRecord(a, stream);
       } else {
+        if (a) cudaEventDestroy(a);
         a = b = nullptr;
       }
     }
@@ -84,7 +114,7 @@ struct LaunchScope {
     if (a && b) {
       cudaEventRecord(b, stream);
       std::lock_guard<std::mutex> lk(g_prof_mu);
-      g_prof.push_back({phase, a, b});
+      g_prof.push_back({phase, a, b, ctx});
     }
   }
 };
@@ -223,12 +253,47 @@ size_t extent_bytes(const long long st[3], int B, int H, long long L, int d, siz
 }
 
 int check_device(bool need_tc) {
+  (void)need_tc;
+  // the answer for a context does not change: asked once per context (and thread)
+  thread_local unsigned long long ok_ctx = 0;
+  const unsigned long long ctx = current_context_id();
+  if (ctx != 0 && ctx == ok_ctx) return INFINI_OK;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return INFINI_ERR_DEVICE;
   int major = 0;
   if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return INFINI_ERR_DEVICE;
-  (void)need_tc;
-  return major == 10 ? INFINI_OK : INFINI_ERR_DEVICE;
+  if (major != 10) return INFINI_ERR_DEVICE;
+  ok_ctx = ctx;
+  return INFINI_OK;
+}
+
+// The fork and join events of one-segment calls, created once per thread and
+// context (a pair shared between threads could interleave their records).
+bool fork_events(cudaEvent_t* ev_fork, cudaEvent_t* ev_join) {
+  struct Pair {
+    unsigned long long ctx;
+    cudaEvent_t fork, join;
+  };
+  thread_local std::vector<Pair> pairs;
+  const unsigned long long ctx = current_context_id();
+  if (ctx == 0) return false;
+  for (const Pair& e : pairs)
+    if (e.ctx == ctx) {
+      *ev_fork = e.fork;
+      *ev_join = e.join;
+      return true;
+    }
+  Pair e{ctx, nullptr, nullptr};
+  if (cudaEventCreateWithFlags(&e.fork, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&e.join, cudaEventDisableTiming) != cudaSuccess) {
+    if (e.fork) cudaEventDestroy(e.fork);
+    cudaGetLastError();
+    return false;
+  }
+  pairs.push_back(e);
+  *ev_fork = e.fork;
+  *ev_join = e.join;
+  return true;
 }
 
 int launch_status() { return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_LAUNCH; }
@@ -540,9 +605,8 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale, c
       state_kernel<<<sgrid, 256, 0, p.stream>>>(p.M, p.z, part, 128, 128, 1, 2, 0, 1, pl.G, nullptr, snapM16, snapz);
     }
     cudaStream_t side = side_stream();
-    if (side != nullptr && cudaEventCreateWithFlags(&ev_fork, cudaEventDisableTiming) == cudaSuccess &&
-        cudaEventCreateWithFlags(&ev_join, cudaEventDisableTiming) == cudaSuccess &&
-        cudaEventRecord(ev_fork, p.stream) == cudaSuccess && cudaStreamWaitEvent(side, ev_fork, 0) == cudaSuccess) {
+    if (side != nullptr && fork_events(&ev_fork, &ev_join) && cudaEventRecord(ev_fork, p.stream) == cudaSuccess &&
+        cudaStreamWaitEvent(side, ev_fork, 0) == cudaSuccess) {
       as = side;
     } else {
       cudaGetLastError();
@@ -550,14 +614,12 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale, c
     ua.snapM = nullptr;  // taken above: the update kernels skip it
     ua.snapzw = nullptr;
   }
-  // the caller's stream waits for the attention's stream; the events are released
+  // the caller's stream waits for the attention's stream
   auto join = [&]() {
     if (ev_join != nullptr && as != p.stream) {
       if (cudaEventRecord(ev_join, as) != cudaSuccess || cudaStreamWaitEvent(p.stream, ev_join, 0) != cudaSuccess)
         cudaGetLastError();
     }
-    if (ev_fork) cudaEventDestroy(ev_fork);
-    if (ev_join) cudaEventDestroy(ev_join);
   };
   if (!pl.delta) {
     ua.seg0 = 0; ua.nseg = pl.S;
@@ -1518,8 +1580,13 @@ int infini_attn_profile_read(double* ms, long long* launches, int reset) {
   }
   if (reset) {
     for (const EventPair& e : g_prof) {
-      cudaEventDestroy(e.a);
-      cudaEventDestroy(e.b);
+      if (e.ctx != 0) {  // back to the pool of their context
+        g_event_pool.emplace_back(e.ctx, e.a);
+        g_event_pool.emplace_back(e.ctx, e.b);
+      } else {
+        cudaEventDestroy(e.a);
+        cudaEventDestroy(e.b);
+      }
     }
     g_prof.clear();
   }
