@@ -1,7 +1,8 @@
-// The memory branch of the backward on CUDA cores, in fp32: the memory read's
-// gradient (Eq. 7), the update's (Eq. 8 / 9) and the sigma(X)^T [Y | y0]
-// partials that feed the memory-gradient chain (see bwd_simt.cuh for the
-// formulas).  Every product here is a small dense one per (b, h, segment) --
+// The memory branch of the backward on CUDA cores, in fp32: the update's
+// gradient (Eq. 8 / 9, for tensors the tensor-core kernels do not take; see
+// sm100_bwdmem.cuh for those and for the memory read's) and the
+// sigma(X)^T [Y | y0] partials that feed the memory-gradient chain (see
+// bwd_simt.cuh for the formulas).  Every product here is a small dense one per (b, h, segment) --
 // rows x 128 times 128 x 128 -- so each block stages its operands in shared
 // memory and computes them with a register-tiled block product: thread
 // (tx, ty) = (tid % 16, tid / 16) owns output rows 16 i + ty and columns
@@ -109,111 +110,6 @@ __device__ __forceinline__ void stage_sigma(float* __restrict__ dst, const T* __
     for (int e = threadIdx.x; e < rows_tile * 128; e += blockDim.x) {
       const int r = e >> 7, c = e & 127;
       dst[r * kMP + c] = (r < nrows && c < cols) ? elu1_accurate(to_f32(src[(long long)r * cols + c])) : 0.f;
-    }
-  }
-}
-
-// Memory read's backward for 128 query rows of one (b, h, segment):
-//   den = sigma(q) z, A_mem = sigma(q) M / den (product 1), the row terms
-//   D'_i = dO_i . A_dot_i and dO_i . (A_mem_i - A_dot_i) (for dbeta),
-//   d_num = g dO / den, d_den = -g dO . A_mem / den, and
-//   dq_mem = sigma'(q) (d_num M^T + d_den z) (product 2); zero where den = 0.
-template <typename T>
-__global__ void __launch_bounds__(256, 1)
-    bwd_qmem_kernel(const T* __restrict__ q, const T* __restrict__ dout, const float* __restrict__ adot,
-                    const float* __restrict__ beta, const float* __restrict__ snapM, const float* __restrict__ snapz,
-                    BwdGeo g, int blocks_per_seg, float* __restrict__ dq_mem, float* __restrict__ Dp,
-                    float* __restrict__ brow, float* __restrict__ dnum, float* __restrict__ dden) {
-  extern __shared__ float sm[];
-  const int dk = g.dk, dv = g.dv, tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
-  int idx = blockIdx.x;
-  const int blk = idx % blocks_per_seg;
-  idx /= blocks_per_seg;
-  const int s = idx % g.S;
-  const int bh = idx / g.S;
-  const int h = bh % g.H;
-  const long long seg_start = (long long)s * g.N;
-  const int n_s = (int)min((long long)g.N, g.L - seg_start);
-  const int r0 = blk * 128;
-  if (r0 >= n_s) return;
-  const int nr = min(128, n_s - r0);
-  const long long row0 = (long long)bh * g.L + seg_start + r0;
-  const float gw = 1.f / (1.f + expf(-beta[h]));
-  float* Ms = sm;                 // [128][kMP] M[i][j]
-  float* Sq = Ms + 128 * kMP;     // [128][kMP] sigma(q)[r][i]
-  float* W = Sq + 128 * kMP;      // [128][kMP] d_num[r][j]
-  float* zs = W + 128 * kMP;      // [128]
-  float* dens = zs + 128;         // [128]
-  float* ddens = dens + 128;      // [128]
-  const float* Mp = snapM + ((long long)bh * g.S + s) * dk * dv;
-  stage_f32(Ms, Mp, 128, dk, dv);
-  stage_sigma<T>(Sq, q + row0 * dk, 128, nr, dk);
-  if (tid < 128) zs[tid] = tid < dk ? snapz[((long long)bh * g.S + s) * dk + tid] : 0.f;
-  __syncthreads();
-  if (tid < 128) {
-    float d = 0.f;
-    for (int i = 0; i < dk; ++i) d = fmaf(Sq[tid * kMP + i], zs[i], d);
-    dens[tid] = d;
-  }
-  float acc[8][8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
-  mm_tile<8>(Sq, kMP, 1, Ms, kMP, 1, dk, acc, ty, tx);  // num = sigma(Q) M
-  __syncthreads();
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int r = 16 * i + ty;
-    const float den = dens[r];
-    float bt = 0.f, dp = 0.f, dd = 0.f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int c = 16 * j + tx;
-      float w = 0.f;
-      if (r < nr && c < dv) {
-        const long long o = (row0 + r) * dv + c;
-        const float dA = to_f32(dout[o]), ad = adot[o];
-        const float am = den != 0.f ? acc[i][j] / den : 0.f;
-        bt = fmaf(dA, am - ad, bt);
-        dp = fmaf(dA, ad, dp);
-        if (den != 0.f) {
-          w = gw * dA / den;
-          dd = fmaf(gw * dA, am, dd);
-        }
-        dnum[o] = w;
-      }
-      W[r * kMP + c] = w;
-    }
-    bt = row16_sum(bt);
-    dp = row16_sum(dp);
-    dd = row16_sum(dd);
-    const float d_den = den != 0.f ? -dd / den : 0.f;
-    if (tx == 0) {
-      ddens[r] = d_den;
-      if (r < nr) {
-        Dp[row0 + r] = dp;
-        brow[row0 + r] = bt;
-        dden[row0 + r] = d_den;
-      }
-    }
-  }
-  __syncthreads();
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
-  mm_tile<8>(W, kMP, 1, Ms, 1, kMP, dv, acc, ty, tx);  // d_num M^T
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int r = 16 * i + ty;
-    if (r >= nr) continue;
-    const float d_den = ddens[r];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int c = 16 * j + tx;
-      if (c < dk)
-        dq_mem[(row0 + r) * dk + c] = sigma_prime_of(Sq[r * kMP + c]) * fmaf(d_den, zs[c], acc[i][j]);
     }
   }
 }

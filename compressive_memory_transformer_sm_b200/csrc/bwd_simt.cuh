@@ -31,8 +31,8 @@
 //   sigma'(x) = 1 above zero, e^x at or below.
 //
 // Kernels (all deterministic: fixed summation orders, no atomics; the memory
-// branch's register-tiled products -- bwd_qmem_kernel, bwd_outer_kernel,
-// bwd_upd_kernel -- are in bwd_mem.cuh):
+// branch's register-tiled products -- bwd_outer_kernel, bwd_upd_kernel --
+// are in bwd_mem.cuh, their tensor-core forms in sm100_bwdmem.cuh):
 //   bwd_q_kernel     per (b, h, segment, 32 query rows): dq (local + memory
 //                    read), D, the dbeta row terms, d_num and d_den rows
 //   bwd_state_kernel the memory-gradient chain: a reverse scan of the

@@ -37,6 +37,7 @@
 #include "sm100_delta.cuh"
 #include "sm100_gemm.cuh"
 #include "sm100_bwd.cuh"
+#include "sm100_bwdmem.cuh"
 
 namespace infini {
 namespace {
@@ -510,6 +511,10 @@ int set_tc_smem_limits() {
       cudaFuncSetAttribute(tc::bwd_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kDQSmem) !=
           cudaSuccess ||
       cudaFuncSetAttribute(tc::bwd_dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kKVSmem) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(tc::bwd_qmem_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kQmSmem) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(tc::bwd_upd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kUpSmem) !=
           cudaSuccess)
     return INFINI_ERR_LAUNCH;
   if (ctx != 0) done.push_back(ctx);
@@ -955,14 +960,12 @@ int run_backward(const infini_attn_bwd_params& p, const BwdPlan& bp, char* ws) {
         !encode_bhld(&tm_v, p.v, p.B, p.H, p.L, cst[1]) || !encode_bhld(&tm_do, p.d_out, p.B, p.H, p.L, cst[1]))
       return INFINI_ERR_LAUNCH;
     if (set_tc_smem_limits() != INFINI_OK) return INFINI_ERR_LAUNCH;
-    // the memory read's backward and D' = dO . A_dot on CUDA cores
-    const size_t qm_smem = (size_t)(3 * 128 * kMP + 3 * 128) * 4;
-    cudaFuncSetAttribute(bwd_qmem_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qm_smem);
+    // the memory read's backward and D' = dO . A_dot (products on the tensor cores)
     {
-      LaunchScope ls(kPhaseBwd, st);
-      bwd_qmem_kernel<T><<<(unsigned)((long long)BH * f.S * bps), 256, qm_smem, st>>>(
-          q, dout, adot, p.beta, snapM, snapz, g, bps, dqmem,
-          Drow, brow, dnum, dden);
+      LaunchScope ls(kPhaseBwdTc, st);
+      tc::bwd_qmem_tc_kernel<<<(unsigned)((long long)BH * f.S * bps), tc::kQmThreads, tc::kQmSmem, st>>>(
+          reinterpret_cast<const __nv_bfloat16*>(q), reinterpret_cast<const __nv_bfloat16*>(dout), adot, p.beta,
+          snapM, snapz, p.B, p.H, f.S, p.N, p.L, bps, dqmem, Drow, brow, dnum, dden);
     }
     memset(&ta, 0, sizeof(ta));
     ta.lse2 = lse; ta.Dp = Drow; ta.beta = p.beta; ta.mem_q = dqmem;
@@ -1001,9 +1004,17 @@ int run_backward(const infini_attn_bwd_params& p, const BwdPlan& bp, char* ws) {
       bwd_state_kernel<<<sgrid, 256, 0, st>>>(nullptr, p.dM_S, p.dz_S, cpart, nullptr, dk, dv, f.S, 0, 0, bp.Gc, 0, gst,
                                               p.dM0, p.dz0);
     }
-    LaunchScope ls(kPhaseBwd, st);
-    bwd_upd_kernel<T><<<(unsigned)((long long)BH * f.S * bps64), 256, upd_smem, st>>>(
-        k, v, g, 0, gst, (long long)pst, (long long)f.S * pst, nullptr, nullptr, dkupd, dvupd, nullptr, nullptr, bps64);
+    if (bp.tc) {
+      LaunchScope ls(kPhaseBwdTc, st);
+      tc::bwd_upd_tc_kernel<<<(unsigned)((long long)BH * f.S * bps), tc::kQmThreads, tc::kUpSmem, st>>>(
+          reinterpret_cast<const __nv_bfloat16*>(k), reinterpret_cast<const __nv_bfloat16*>(v), p.B, p.H, f.S, p.N,
+          p.L, 0, gst, (long long)pst, (long long)f.S * pst, nullptr, nullptr, dkupd, dvupd, nullptr, nullptr, bps);
+    } else {
+      LaunchScope ls(kPhaseBwd, st);
+      bwd_upd_kernel<T><<<(unsigned)((long long)BH * f.S * bps64), 256, upd_smem, st>>>(
+          k, v, g, 0, gst, (long long)pst, (long long)f.S * pst, nullptr, nullptr, dkupd, dvupd, nullptr, nullptr,
+          bps64);
+    }
   } else {
     {
       LaunchScope ls(kPhaseBwd, st);
@@ -1011,7 +1022,12 @@ int run_backward(const infini_attn_bwd_params& p, const BwdPlan& bp, char* ws) {
                                               nullptr, nullptr, nullptr);
     }
     for (int s = f.S - 1; s >= 0; --s) {
-      {
+      if (bp.tc) {
+        LaunchScope ls(kPhaseBwdTc, st);
+        tc::bwd_upd_tc_kernel<<<(unsigned)((long long)BH * bps), tc::kQmThreads, tc::kUpSmem, st>>>(
+            reinterpret_cast<const __nv_bfloat16*>(k), reinterpret_cast<const __nv_bfloat16*>(v), p.B, p.H, f.S, p.N,
+            p.L, s, gst, 0, (long long)pst, snapM, snapz, dkupd, dvupd, dnumr, ddenr, bps);
+      } else {
         LaunchScope ls(kPhaseBwd, st);
         bwd_upd_kernel<T><<<(unsigned)((long long)BH * bps64), 256, upd_smem, st>>>(
             k, v, g, s, gst, 0, (long long)pst, snapM, snapz, dkupd, dvupd, dnumr, ddenr, bps64);
