@@ -52,7 +52,8 @@ from compressive_memory_transformer_sm_b200 import workloads as W  # noqa: E402
 METRIC = "Infini-attn fwd tokens/s per layer; TFLOP/s and % of B200 bf16 tensor peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FLUSH_BYTES = 1 << 30
-PHASE_NAMES = ("update", "state", "attention", "rope", "projections", "backward_cuda_cores", "backward_tensor")
+PHASE_NAMES = ("update", "state", "attention", "rope", "projections", "backward_cuda_cores", "backward_tensor",
+               "backward_memory_tensor")
 
 
 # ------------------------------------------------------------------ work model

@@ -39,7 +39,7 @@ EXPORTED = (
     "infini_attn_launch_count", "infini_attn_forward_noalloc",
     "infini_attn_layer_forward", "infini_attn_layer_workspace_size", "infini_attn_decode_step",
     "infini_attn_workspace_size_ex", "infini_attn_gemm_bf16", "infini_attn_backward",
-    "infini_attn_backward_workspace_size", "infini_attn_trim_workspace",
+    "infini_attn_backward_workspace_size", "infini_attn_trim_workspace", "infini_attn_last_cuda_error",
 )
 
 
@@ -76,6 +76,8 @@ lib.infini_attn_profile_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes
 lib.infini_attn_profile_read.restype = _i
 lib.infini_attn_launch_count.argtypes = []
 lib.infini_attn_launch_count.restype = _ll
+lib.infini_attn_last_cuda_error.argtypes = [ctypes.c_char_p, _i]
+lib.infini_attn_last_cuda_error.restype = _i
 lib.infini_attn_decode_step.argtypes = [_vp] * 9 + [_i] * 8 + [_vp]
 lib.infini_attn_decode_step.restype = _i
 lib.infini_attn_layer_forward.argtypes = [_vp] * 7 + [_i, _i, _l, _i, _i, _i, _vp, ctypes.c_size_t, _vp]
@@ -85,8 +87,8 @@ lib.infini_attn_layer_workspace_size.restype = ctypes.c_size_t
 lib.infini_attn_gemm_bf16.argtypes = [_vp, _vp, _vp, _l, _i, _i, _vp]
 lib.infini_attn_gemm_bf16.restype = _i
 
-PHASE_UPDATE, PHASE_STATE, PHASE_ATTN, PHASE_PRE, PHASE_PROJ, PHASE_BWD, PHASE_BWD_TC = 0, 1, 2, 3, 4, 5, 6
-PHASES = 7
+PHASE_UPDATE, PHASE_STATE, PHASE_ATTN, PHASE_PRE, PHASE_PROJ, PHASE_BWD, PHASE_BWD_TC, PHASE_BWD_MEM_TC = range(8)
+PHASES = 8
 
 
 class InfiniAttnParams(ctypes.Structure):
@@ -131,7 +133,18 @@ lib.infini_attn_trim_workspace.restype = _i
 class InfiniAttnError(RuntimeError):
     def __init__(self, code: int, where: str):
         self.code = code
-        super().__init__(f"{where}: {infini_attn_error_string(code)} ({code})")
+        detail = ""
+        if code == INFINI_ERR_LAUNCH:
+            err, name = infini_attn_last_cuda_error()
+            detail = f" [{name} ({err})]" if err else ""
+        super().__init__(f"{where}: {infini_attn_error_string(code)} ({code}){detail}")
+
+
+def infini_attn_last_cuda_error():
+    """(cudaError_t value, its name) behind the most recent INFINI_ERR_LAUNCH of this library; (0, ...) if none."""
+    buf = ctypes.create_string_buffer(64)
+    err = int(lib.infini_attn_last_cuda_error(buf, len(buf)))
+    return err, buf.value.decode()
 
 
 def infini_attn_error_string(code: int) -> str:
@@ -396,8 +409,10 @@ def infini_attn_profile_enable(phase_mask: int) -> int:
 
 
 def infini_attn_profile_read(reset: bool = True):
-    """Returns ([ms per phase], [timed launches per phase]) for phases update, state, attention and the
-    position-embedding pre-pass."""
+    """Returns ([ms per phase], [timed launches per phase]) for the phases PHASE_UPDATE ..
+    PHASE_BWD_MEM_TC (memory update, state, attention, position-embedding pre-pass, projections,
+    backward on CUDA cores, local attention's backward and memory branch's backward on the tensor
+    cores)."""
     ms = (ctypes.c_double * PHASES)()
     n = (_ll * PHASES)()
     rc = lib.infini_attn_profile_read(ms, n, 1 if reset else 0)

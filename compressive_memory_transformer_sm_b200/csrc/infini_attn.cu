@@ -21,6 +21,7 @@
 #include <algorithm>
 #include <cmath>
 #include <atomic>
+#include <cstdio>
 #include <mutex>
 #include <utility>
 #include <vector>
@@ -54,7 +55,7 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 // ------------------------------------------------------------ launch accounting
 enum Phase { kPhaseUpdate = 0, kPhaseState = 1, kPhaseAttn = 2, kPhasePre = 3, kPhaseProj = 4, kPhaseBwd = 5, kPhaseBwdTc = 6,
-             kPhases = 7 };
+             kPhaseBwdMemTc = 7, kPhases = 8 };
 std::atomic<long long> g_launches{0};
 std::atomic<int> g_profile_mask{0};
 struct EventPair {
@@ -297,7 +298,16 @@ bool fork_events(cudaEvent_t* ev_fork, cudaEvent_t* ev_join) {
   return true;
 }
 
-int launch_status() { return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_LAUNCH; }
+// The CUDA error behind the most recent INFINI_ERR_LAUNCH (any thread).
+std::atomic<int> g_last_cuda_error{0};
+int note_cuda_error(cudaError_t e) {
+  g_last_cuda_error.store((int)e);
+  return INFINI_ERR_LAUNCH;
+}
+int launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? INFINI_OK : note_cuda_error(e);
+}
 
 // What the local attention (Eq. 6) reads: q, k themselves, or their rotated
 // copies in the workspace when position embeddings are on (then qm is the
@@ -669,9 +679,11 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale, c
       ua.seg0 = s;
       cfg.numAttrs = s > 0 ? 2 : 1;
       LaunchScope ls(kPhaseUpdate, p.stream);
-      if (cudaLaunchKernelEx(&cfg, tc::delta_update_tc_kernel, tm_k64, tm_v64, ua) != cudaSuccess) {
+      const cudaError_t e = cudaLaunchKernelEx(&cfg, tc::delta_update_tc_kernel, tm_k64, tm_v64, ua);
+      if (e != cudaSuccess) {
+        cudaGetLastError();
         join();
-        return INFINI_ERR_LAUNCH;
+        return note_cuda_error(e);
       }
     }
   }
@@ -962,7 +974,7 @@ int run_backward(const infini_attn_bwd_params& p, const BwdPlan& bp, char* ws) {
     if (set_tc_smem_limits() != INFINI_OK) return INFINI_ERR_LAUNCH;
     // the memory read's backward and D' = dO . A_dot (products on the tensor cores)
     {
-      LaunchScope ls(kPhaseBwdTc, st);
+      LaunchScope ls(kPhaseBwdMemTc, st);
       tc::bwd_qmem_tc_kernel<<<(unsigned)((long long)BH * f.S * bps), tc::kQmThreads, tc::kQmSmem, st>>>(
           reinterpret_cast<const __nv_bfloat16*>(q), reinterpret_cast<const __nv_bfloat16*>(dout), adot, p.beta,
           snapM, snapz, p.B, p.H, f.S, p.N, p.L, bps, dqmem, Drow, brow, dnum, dden);
@@ -1005,7 +1017,7 @@ int run_backward(const infini_attn_bwd_params& p, const BwdPlan& bp, char* ws) {
                                               p.dM0, p.dz0);
     }
     if (bp.tc) {
-      LaunchScope ls(kPhaseBwdTc, st);
+      LaunchScope ls(kPhaseBwdMemTc, st);
       tc::bwd_upd_tc_kernel<<<(unsigned)((long long)BH * f.S * bps), tc::kQmThreads, tc::kUpSmem, st>>>(
           reinterpret_cast<const __nv_bfloat16*>(k), reinterpret_cast<const __nv_bfloat16*>(v), p.B, p.H, f.S, p.N,
           p.L, 0, gst, (long long)pst, (long long)f.S * pst, nullptr, nullptr, dkupd, dvupd, nullptr, nullptr, bps);
@@ -1023,7 +1035,7 @@ int run_backward(const infini_attn_bwd_params& p, const BwdPlan& bp, char* ws) {
     }
     for (int s = f.S - 1; s >= 0; --s) {
       if (bp.tc) {
-        LaunchScope ls(kPhaseBwdTc, st);
+        LaunchScope ls(kPhaseBwdMemTc, st);
         tc::bwd_upd_tc_kernel<<<(unsigned)((long long)BH * bps), tc::kQmThreads, tc::kUpSmem, st>>>(
             reinterpret_cast<const __nv_bfloat16*>(k), reinterpret_cast<const __nv_bfloat16*>(v), p.B, p.H, f.S, p.N,
             p.L, s, gst, 0, (long long)pst, snapM, snapz, dkupd, dvupd, dnumr, ddenr, bps);
@@ -1346,7 +1358,7 @@ int infini_attn_decode_step(const void* q_t, const void* k_t, const void* v_t, v
     }
     if (e != cudaSuccess) {
       cudaGetLastError();
-      return INFINI_ERR_LAUNCH;
+      return note_cuda_error(e);
     }
     if (!(fold || pos == N - 1)) return INFINI_OK;
     return decode_fold(k_cache, v_cache, beta, M, z, B, H, N, n, dk, dv, mode, stream);
@@ -1610,5 +1622,14 @@ int infini_attn_profile_read(double* ms, long long* launches, int reset) {
 }
 
 long long infini_attn_launch_count(void) { return g_launches.load(); }
+
+int infini_attn_last_cuda_error(char* name, int n) {
+  const int e = g_last_cuda_error.load();
+  if (name != nullptr && n > 0) {
+    const char* s = e != 0 ? cudaGetErrorName((cudaError_t)e) : "cudaSuccess";
+    std::snprintf(name, (size_t)n, "%s", s != nullptr ? s : "unknown");
+  }
+  return e;
+}
 
 }  // extern "C"

@@ -355,14 +355,15 @@ INFINI_API int infini_attn_selftest_timeout(unsigned limit_us, cudaStream_t stre
  * Kernel timing for benchmarks.  phase_mask selects phases (bit 0 = memory
  * update kernels, bit 1 = state/snapshot kernels, bit 2 = attention
  * kernel, bit 3 = position-embedding pre-pass, bit 4 = projection GEMMs of
- * the full layer, bit 5 = backward kernels on CUDA cores, bit 6 = backward
- * kernels on the tensor cores); while a bit is set, every
+ * the full layer, bit 5 = backward kernels on CUDA cores, bit 6 = the
+ * local attention's backward kernels on the tensor cores, bit 7 = the
+ * memory branch's backward kernels on the tensor cores); while a bit is set, every
  * launch of that phase is bracketed by two CUDA events recorded on the
  * launch's stream.  0 turns timing off.
  */
 INFINI_API int infini_attn_profile_enable(int phase_mask);
 /*
- * Synchronises the recorded events and adds, per phase p in 0..6, the
+ * Synchronises the recorded events and adds, per phase p in 0..7, the
  * elapsed milliseconds to ms[p] and the number of timed launches to
  * launches[p], for everything recorded since the last reset; reset != 0
  * then drops the records.  Either array may be NULL.
@@ -370,6 +371,13 @@ INFINI_API int infini_attn_profile_enable(int phase_mask);
 INFINI_API int infini_attn_profile_read(double* ms, long long* launches, int reset);
 /* Number of kernels this library has launched in this process (all phases). */
 INFINI_API long long infini_attn_launch_count(void);
+/*
+ * The cudaError_t value behind the most recent INFINI_ERR_LAUNCH returned by
+ * any call of this library in this process (0 if there was none), for
+ * diagnostics; its name (cudaGetErrorName) is copied into name[0..n-1],
+ * NUL-terminated, when name != NULL and n > 0.
+ */
+INFINI_API int infini_attn_last_cuda_error(char* name, int n);
 
 /* sizeof(infini_attn_params), for bindings that build the struct themselves. */
 INFINI_API size_t infini_attn_params_size(void);

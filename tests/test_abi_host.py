@@ -46,6 +46,16 @@ def test_error_strings():
     assert api.infini_attn_error_string(-99) == "unknown error code"
 
 
+def test_last_cuda_error_query():
+    # code and name agree (0 is cudaSuccess); a NULL buffer or a zero length
+    # is accepted and a short buffer is truncated, NUL-terminated
+    err, name = api.infini_attn_last_cuda_error()
+    assert isinstance(err, int) and name and (err == 0) == (name == "cudaSuccess")
+    assert api.lib.infini_attn_last_cuda_error(None, 0) == err
+    buf = ctypes.create_string_buffer(4)
+    assert api.lib.infini_attn_last_cuda_error(buf, len(buf)) == err and buf.value == name[:3].encode()
+
+
 def test_path_selection():
     assert api.infini_attn_path(128, 128, LINEAR, 0) == 1
     assert api.infini_attn_path(128, 128, DELTA, 0) == 1
