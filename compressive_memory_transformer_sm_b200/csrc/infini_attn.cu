@@ -525,6 +525,8 @@ int set_tc_smem_limits() {
       cudaFuncSetAttribute(tc::bwd_qmem_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kQmSmem) !=
           cudaSuccess ||
       cudaFuncSetAttribute(tc::bwd_upd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kUpSmem) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(tc::bwd_outer_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kOtSmem) !=
           cudaSuccess)
     return INFINI_ERR_LAUNCH;
   if (ctx != 0) done.push_back(ctx);
@@ -999,7 +1001,11 @@ int run_backward(const infini_attn_bwd_params& p, const BwdPlan& bp, char* ws) {
   // 3. the memory read's partials sigma(Q)^T [d_num | d_den] of every segment
   const size_t outer_smem = (size_t)(64 * kMP + 64 * 130) * 4;
   cudaFuncSetAttribute(bwd_outer_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)outer_smem);
-  {
+  if (bp.tc) {
+    LaunchScope ls(kPhaseBwdMemTc, st);
+    tc::bwd_outer_tc_kernel<<<(unsigned)((long long)BH * f.S * bp.Gc), tc::kOtThreads, tc::kOtSmem, st>>>(
+        reinterpret_cast<const __nv_bfloat16*>(q), dnum, dden, p.N, p.L, 0, f.S, bp.Gc, bp.cpbc, cpart);
+  } else {
     LaunchScope ls(kPhaseBwd, st);
     bwd_outer_kernel<T><<<(unsigned)((long long)BH * f.S * bp.Gc), 256, outer_smem, st>>>(q, dnum, dden, g, dv, 0, f.S,
                                                                                           bp.Gc, bp.cpbc, cpart);
@@ -1044,7 +1050,11 @@ int run_backward(const infini_attn_bwd_params& p, const BwdPlan& bp, char* ws) {
         bwd_upd_kernel<T><<<(unsigned)((long long)BH * bps64), 256, upd_smem, st>>>(
             k, v, g, s, gst, 0, (long long)pst, snapM, snapz, dkupd, dvupd, dnumr, ddenr, bps64);
       }
-      {
+      if (bp.tc) {
+        LaunchScope ls(kPhaseBwdMemTc, st);
+        tc::bwd_outer_tc_kernel<<<(unsigned)((long long)BH * bp.Gu), tc::kOtThreads, tc::kOtSmem, st>>>(
+            reinterpret_cast<const __nv_bfloat16*>(k), dnumr, ddenr, p.N, p.L, s, 1, bp.Gu, bp.cpbu, upart);
+      } else {
         LaunchScope ls(kPhaseBwd, st);
         bwd_outer_kernel<T><<<(unsigned)((long long)BH * bp.Gu), 256, outer_smem, st>>>(k, dnumr, ddenr, g, dv, s, 1,
                                                                                        bp.Gu, bp.cpbu, upart);

@@ -552,5 +552,204 @@ __global__ void __launch_bounds__(kQmThreads, 1)
   }
 }
 
+// The memory gradient's partial sums sigma(X)^T Y (dk x dv) and
+// sigma(X)^T y0 (dk) over the rows of one (b, h, segment, row group) on the
+// tensor cores, for bf16 X with d_key = d_value = 128: the quantity
+// bwd_outer_kernel (bwd_mem.cuh) computes on CUDA cores, same partial layout
+// [BH][nseg][G][dk * dv + dk].  X = Q with Y = d_num, y0 = d_den (the memory
+// read's terms, Eq. 7) or X = K with Y = d_num_r, y0 = d_den_r (the delta
+// rule's retrieval, Eq. 9).  Per 128-row block:
+//   sigma(X) (fp32, the accurate ELU + 1) and Y as bf16 hi + lo tiles, rows
+//   = the product's K index: sigma^T is the MN-major A operand, Y the MN-major
+//   B operand; D += s_hi^T Y_hi + s_hi^T Y_lo + s_lo^T Y_hi (~2^-16
+//   relative, fp32 in TMEM);
+//   y0's hi and lo parts as rows 0 and 1 of a 16-row K-major B tile (rows
+//   2-15 zero): Dz += (s_hi + s_lo)^T [y0_hi | y0_lo | 0], and
+//   sigma^T y0 = Dz[:, 0] + Dz[:, 1].
+// 256 threads: thread (row r = TMEM lane, half hh) stages columns
+// [64 hh, 64 hh + 64) of row r and writes row r's partial; thread 0 issues
+// the products.  A group with no rows writes a zero partial.
+constexpr int kOtThreads = 256;
+constexpr uint32_t kOtAH = 0, kOtAL = 32768, kOtYH = 65536, kOtYL = 98304;  // 128 x 128 bf16 tiles
+constexpr uint32_t kOtY0 = 131072;       // 16 x 128 bf16 K-major (two 2 KB boxes)
+constexpr uint32_t kOtBAR = kOtY0 + 4096;
+constexpr uint32_t kOtSLOT = kOtBAR + 16;
+constexpr uint32_t kOtSmem = kOtSLOT + 16 + 1024;
+
+__device__ __forceinline__ void sts16(uint32_t a, unsigned short v) {
+  asm volatile("st.shared.u16 [%0], %1;" ::"r"(a), "h"(v) : "memory");
+}
+
+__global__ void __launch_bounds__(kOtThreads, 1)
+    bwd_outer_tc_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ Y,
+                        const float* __restrict__ y0, int N, long long L, int seg0, int nseg, int G, int cpb,
+                        float* __restrict__ partial) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  int idx = blockIdx.x;
+  const int grp = idx % G;
+  idx /= G;
+  const int sl = idx % nseg;
+  const int bh = idx / nseg;
+  const long long seg_start = (long long)(seg0 + sl) * N;
+  const int n_s = (int)min((long long)N, L - seg_start);
+  const int t_begin = grp * cpb * 128;
+  const int t_end = min(n_s, t_begin + cpb * 128);
+  const int nblk = t_begin < t_end ? (t_end - t_begin + 127) / 128 : 0;
+  const uint32_t bar = base + kOtBAR;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kOtSLOT);
+  const int row = 32 * (warp & 3) + lane, hh = warp >> 2;  // row of the block (TMEM lane: dk index), column half
+  const uint32_t lq = (uint32_t)(32 * (warp & 3)) << 16;
+
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_barrier_init();
+  }
+  sts128(base + kOtY0 + 16u * (uint32_t)tid, make_uint4(0u, 0u, 0u, 0u));  // the y0 tile, 4 KB
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tD = tmem, tZ = tmem + 128u;
+
+#pragma unroll 1
+  for (int blk = 0; blk < nblk; ++blk) {
+    const int r0 = t_begin + 128 * blk;
+    const bool valid = row < t_end - r0;
+    const long long grow = (long long)bh * L + seg_start + r0 + row;
+    if (row < t_end - r0 - 128) {  // the next block's row: into L2 while this one is staged and multiplied
+      prefetch_l2(x + (grow + 128) * 128 + 64 * hh);
+      prefetch_l2(Y + (grow + 128) * 128 + 64 * hh);
+      prefetch_l2(Y + (grow + 128) * 128 + 64 * hh + 32);
+    }
+    if (blk > 0) {
+      mbar_wait(bar, (uint32_t)(blk - 1) & 1u);  // the previous block's products have read the tiles
+      tc_fence_after();
+    }
+    // sigma(x) of this thread's 64 columns
+#pragma unroll 2
+    for (int i = 0; i < 8; ++i) {
+      const int c = 8 * hh + i;
+      float v[8];
+      if (valid) {
+        const uint4 w = __ldg(reinterpret_cast<const uint4*>(x + grow * 128) + c);
+        const uint32_t wp[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          v[2 * e] = elu1_accurate(bf16_lo(wp[e]));
+          v[2 * e + 1] = elu1_accurate(bf16_hi(wp[e]));
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = 0.f;
+      }
+      uint4 hi, lo;
+      qm_split8(v, hi, lo);
+      sts128(base + kOtAH + swz_chunk(row, c), hi);
+      sts128(base + kOtAL + swz_chunk(row, c), lo);
+    }
+    // Y of this thread's 64 columns
+#pragma unroll 2
+    for (int i = 0; i < 8; ++i) {
+      const int c = 8 * hh + i;
+      float v[8];
+      if (valid) {
+        const float4 f0 = __ldg(reinterpret_cast<const float4*>(Y + grow * 128 + 8 * c));
+        const float4 f1 = __ldg(reinterpret_cast<const float4*>(Y + grow * 128 + 8 * c + 4));
+        v[0] = f0.x; v[1] = f0.y; v[2] = f0.z; v[3] = f0.w;
+        v[4] = f1.x; v[5] = f1.y; v[6] = f1.z; v[7] = f1.w;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = 0.f;
+      }
+      uint4 hi, lo;
+      qm_split8(v, hi, lo);
+      sts128(base + kOtYH + swz_chunk(row, c), hi);
+      sts128(base + kOtYL + swz_chunk(row, c), lo);
+    }
+    // y0 of this row: element (n, k = row) of the K-major tile, n = 0 (hi), 1 (lo)
+    if (hh == 0) {
+      const float v = valid ? y0[grow] : 0.f;
+      const __nv_bfloat16 vh = __float2bfloat16_rn(v);
+      const __nv_bfloat16 vl = __float2bfloat16_rn(v - __bfloat162float(vh));
+      const int c = row >> 3;
+#pragma unroll
+      for (int n = 0; n < 2; ++n) {
+        const uint32_t a = base + kOtY0 + (uint32_t)(c >> 3) * 2048u + (uint32_t)n * 128u +
+                           ((uint32_t)((c & 7) ^ n) << 4) + (uint32_t)(row & 7) * 2u;
+        sts16(a, __bfloat16_as_ushort(n == 0 ? vh : vl));
+      }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid == 0) {
+      constexpr uint32_t idesc = idesc_bf16(128, 128, 1, 1);  // A = sigma^T, B = Y: both MN-major
+      constexpr uint32_t idesc_z = idesc_bf16(128, 16, 1, 0);  // B = the y0 tile, K-major
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t acc = (blk > 0 || kk > 0) ? 1u : 0u;
+        const uint64_t aH = mnmajor_desc(base + kOtAH, kk), aL = mnmajor_desc(base + kOtAL, kk);
+        const uint64_t bH = mnmajor_desc(base + kOtYH, kk), bL = mnmajor_desc(base + kOtYL, kk);
+        const uint64_t bz = ones_desc(base + kOtY0, kk);
+        mma_ss(tD, aH, bH, idesc, acc);
+        mma_ss(tD, aH, bL, idesc, 1u);
+        mma_ss(tD, aL, bH, idesc, 1u);
+        mma_ss(tZ, aH, bz, idesc_z, acc);
+        mma_ss(tZ, aL, bz, idesc_z, 1u);
+      }
+      mma_commit(bar);
+    }
+  }
+  if (nblk > 0) {
+    mbar_wait(bar, (uint32_t)(nblk - 1) & 1u);
+    tc_fence_after();
+  }
+  // row `row` (a dk index) of the partial: columns [64 hh, 64 hh + 64), and
+  // (hh = 0) its sigma^T y0 entry
+  float* out = partial + (((long long)bh * nseg + sl) * G + grp) * (long long)(16384 + 128);
+#pragma unroll 1
+  for (int h2 = 0; h2 < 2; ++h2) {
+    const int c0 = 64 * hh + 32 * h2;
+    uint32_t v[32];
+    if (nblk > 0) {
+      tmem_ld32(tD + lq + (uint32_t)c0, v);
+      tmem_ld_wait();
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) v[e] = 0u;
+    }
+    float4* dst = reinterpret_cast<float4*>(out + row * 128 + c0);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]), __uint_as_float(v[4 * i + 2]),
+                           __uint_as_float(v[4 * i + 3]));
+  }
+  if (hh == 0) {
+    float zsum = 0.f;
+    if (nblk > 0) {
+      uint32_t v[16];
+      tmem_ld16(tZ + lq, v);
+      tmem_ld_wait();
+      zsum = __uint_as_float(v[0]) + __uint_as_float(v[1]);
+    }
+    out[16384 + row] = zsum;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
 }  // namespace tc
 }  // namespace infini
