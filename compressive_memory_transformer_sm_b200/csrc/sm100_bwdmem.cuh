@@ -79,6 +79,16 @@ __global__ void __launch_bounds__(kQmThreads, 1)
     mbar_init(bar, 1);
     fence_barrier_init();
   }
+  // this thread's q chunks now, and dO, A_dot (read after product 1) into L2
+  uint4 qw[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    qw[i] = valid ? __ldg(reinterpret_cast<const uint4*>(q + grow * 128) + 8 * hh + i) : make_uint4(0u, 0u, 0u, 0u);
+  if (valid) {
+    prefetch_l2(dout + grow * 128 + 64 * hh);
+    prefetch_l2(adot + grow * 128 + 64 * hh);
+    prefetch_l2(adot + grow * 128 + 64 * hh + 32);
+  }
   if (tid < 128) zs[tid] = snapz[((long long)bh * S + s) * 128 + tid];
   if (warp == 0) {
     tmem_alloc(smem_u32(tmem_slot), 256);
@@ -87,7 +97,7 @@ __global__ void __launch_bounds__(kQmThreads, 1)
   // M [dk][dv] (fp32) -> hi / lo tiles: 2048 chunks of 8 values, 8 per thread
   {
     const float* Mp = snapM + ((long long)bh * S + s) * 16384;
-#pragma unroll 2
+#pragma unroll
     for (int ch = tid; ch < 2048; ch += kQmThreads) {
       const int i = ch >> 4, c = ch & 15;
       const float4 f0 = __ldg(reinterpret_cast<const float4*>(Mp + i * 128 + 8 * c));
@@ -104,12 +114,12 @@ __global__ void __launch_bounds__(kQmThreads, 1)
   float den;
   {
     float dpart = 0.f;
-#pragma unroll 2
+#pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int c = 8 * hh + i;  // 16-byte chunk of the row
       float x[8];
       if (valid) {
-        const uint4 w = __ldg(reinterpret_cast<const uint4*>(q + grow * 128) + c);
+        const uint4 w = qw[i];
         const uint32_t wp[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -332,6 +342,12 @@ __global__ void __launch_bounds__(kQmThreads, 1)
     mbar_init(bar, 1);
     fence_barrier_init();
   }
+  // this thread's k chunks now, and v (read after the first products) into L2
+  uint4 kw[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    kw[i] = valid ? __ldg(reinterpret_cast<const uint4*>(k + grow * 128) + 8 * hh + i) : make_uint4(0u, 0u, 0u, 0u);
+  if (valid) prefetch_l2(v + grow * 128 + 64 * hh);
   if (tid < 128) {
     gz[tid] = gp[16384 + tid];
     zs[tid] = delta ? snapz[((long long)bh * S + s) * 128 + tid] : 0.f;
@@ -341,7 +357,7 @@ __global__ void __launch_bounds__(kQmThreads, 1)
     tmem_relinquish();
   }
   // G (and M) [dk][dv] fp32 -> hi / lo tiles
-#pragma unroll 2
+#pragma unroll
   for (int ch = tid; ch < 2048; ch += kQmThreads) {
     const int i = ch >> 4, c = ch & 15;
     float x[8];
@@ -367,12 +383,12 @@ __global__ void __launch_bounds__(kQmThreads, 1)
   // sigma(K) of this thread's 64 columns -> A tiles; partial den_k (delta)
   {
     float dpart = 0.f;
-#pragma unroll 2
+#pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int c = 8 * hh + i;
       float x[8];
       if (valid) {
-        const uint4 w = __ldg(reinterpret_cast<const uint4*>(k + grow * 128) + c);
+        const uint4 w = kw[i];
         const uint32_t wp[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -629,26 +645,31 @@ __global__ void __launch_bounds__(kOtThreads, 1)
       prefetch_l2(Y + (grow + 128) * 128 + 64 * hh);
       prefetch_l2(Y + (grow + 128) * 128 + 64 * hh + 32);
     }
+    // this thread's x and Y chunks, all loads issued before any store (and
+    // while the previous block's products run)
+    uint4 xw[8];
+    float4 yf[16];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      xw[i] = valid ? __ldg(reinterpret_cast<const uint4*>(x + grow * 128) + 8 * hh + i) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      yf[i] = valid ? __ldg(reinterpret_cast<const float4*>(Y + grow * 128 + 64 * hh) + i)
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
     if (blk > 0) {
       mbar_wait(bar, (uint32_t)(blk - 1) & 1u);  // the previous block's products have read the tiles
       tc_fence_after();
     }
-    // sigma(x) of this thread's 64 columns
-#pragma unroll 2
+    // sigma(x) of this thread's 64 columns (rows past the end: sigma = 0)
+#pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int c = 8 * hh + i;
       float v[8];
-      if (valid) {
-        const uint4 w = __ldg(reinterpret_cast<const uint4*>(x + grow * 128) + c);
-        const uint32_t wp[4] = {w.x, w.y, w.z, w.w};
+      const uint32_t wp[4] = {xw[i].x, xw[i].y, xw[i].z, xw[i].w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          v[2 * e] = elu1_accurate(bf16_lo(wp[e]));
-          v[2 * e + 1] = elu1_accurate(bf16_hi(wp[e]));
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) v[e] = 0.f;
+      for (int e = 0; e < 4; ++e) {
+        v[2 * e] = valid ? elu1_accurate(bf16_lo(wp[e])) : 0.f;
+        v[2 * e + 1] = valid ? elu1_accurate(bf16_hi(wp[e])) : 0.f;
       }
       uint4 hi, lo;
       qm_split8(v, hi, lo);
@@ -656,19 +677,11 @@ __global__ void __launch_bounds__(kOtThreads, 1)
       sts128(base + kOtAL + swz_chunk(row, c), lo);
     }
     // Y of this thread's 64 columns
-#pragma unroll 2
+#pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int c = 8 * hh + i;
-      float v[8];
-      if (valid) {
-        const float4 f0 = __ldg(reinterpret_cast<const float4*>(Y + grow * 128 + 8 * c));
-        const float4 f1 = __ldg(reinterpret_cast<const float4*>(Y + grow * 128 + 8 * c + 4));
-        v[0] = f0.x; v[1] = f0.y; v[2] = f0.z; v[3] = f0.w;
-        v[4] = f1.x; v[5] = f1.y; v[6] = f1.z; v[7] = f1.w;
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) v[e] = 0.f;
-      }
+      const float v[8] = {yf[2 * i].x, yf[2 * i].y, yf[2 * i].z, yf[2 * i].w,
+                          yf[2 * i + 1].x, yf[2 * i + 1].y, yf[2 * i + 1].z, yf[2 * i + 1].w};
       uint4 hi, lo;
       qm_split8(v, hi, lo);
       sts128(base + kOtYH + swz_chunk(row, c), hi);
