@@ -1024,7 +1024,7 @@ int run_backward(const infini_attn_bwd_params& p, const BwdPlan& bp, char* ws) {
     }
     if (bp.tc) {
       LaunchScope ls(kPhaseBwdMemTc, st);
-      tc::bwd_upd_tc_kernel<<<(unsigned)((long long)BH * f.S * bps), tc::kQmThreads, tc::kUpSmem, st>>>(
+      tc::bwd_upd_tc_kernel<<<(unsigned)((long long)BH * f.S * bps), tc::kUpThreads, tc::kUpSmem, st>>>(
           reinterpret_cast<const __nv_bfloat16*>(k), reinterpret_cast<const __nv_bfloat16*>(v), p.B, p.H, f.S, p.N,
           p.L, 0, gst, (long long)pst, (long long)f.S * pst, nullptr, nullptr, dkupd, dvupd, nullptr, nullptr, bps);
     } else {
@@ -1042,7 +1042,7 @@ int run_backward(const infini_attn_bwd_params& p, const BwdPlan& bp, char* ws) {
     for (int s = f.S - 1; s >= 0; --s) {
       if (bp.tc) {
         LaunchScope ls(kPhaseBwdMemTc, st);
-        tc::bwd_upd_tc_kernel<<<(unsigned)((long long)BH * bps), tc::kQmThreads, tc::kUpSmem, st>>>(
+        tc::bwd_upd_tc_kernel<<<(unsigned)((long long)BH * bps), tc::kUpThreads, tc::kUpSmem, st>>>(
             reinterpret_cast<const __nv_bfloat16*>(k), reinterpret_cast<const __nv_bfloat16*>(v), p.B, p.H, f.S, p.N,
             p.L, s, gst, 0, (long long)pst, snapM, snapz, dkupd, dvupd, dnumr, ddenr, bps);
       } else {

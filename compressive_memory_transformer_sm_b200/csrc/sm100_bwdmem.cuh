@@ -13,8 +13,8 @@
 // swizzle: the MN-major B operand of sigma(q) M and, read as K-major, the B
 // operand M^T of d_num M^T.  The A tiles hold sigma(q), then d_num.
 //
-// 256 threads: thread (row r = TMEM lane, half hh) handles columns
-// [64 hh, 64 hh + 64) of query row r; one thread issues the products.
+// 512 threads: thread (row r = TMEM lane, quarter qq) handles columns
+// [32 qq, 32 qq + 32) of query row r; one thread issues the products.
 #pragma once
 
 #include "sm100_common.cuh"
@@ -22,11 +22,11 @@
 namespace infini {
 namespace tc {
 
-constexpr int kQmThreads = 256;
+constexpr int kQmThreads = 512;
 constexpr uint32_t kQmAH = 0, kQmAL = 32768, kQmMH = 65536, kQmML = 98304;  // 128 x 128 bf16 tiles
 constexpr uint32_t kQmZ = 131072;        // z, 128 floats
-constexpr uint32_t kQmX = kQmZ + 512;    // [2 halves][128 rows] partial row sums (x4 quantities)
-constexpr uint32_t kQmBAR = kQmX + 4 * 1024;
+constexpr uint32_t kQmX = kQmZ + 512;    // [4 quantities][4 column quarters][128 rows] partial row sums
+constexpr uint32_t kQmBAR = kQmX + 8 * 1024;
 constexpr uint32_t kQmSLOT = kQmBAR + 16;
 constexpr uint32_t kQmSmem = kQmSLOT + 16 + 1024;
 
@@ -66,11 +66,12 @@ __global__ void __launch_bounds__(kQmThreads, 1)
   const long long row0 = (long long)bh * L + seg_start + r0;
   const float gw = 1.f / (1.f + expf(-beta[h]));
   float* zs = reinterpret_cast<float*>(gbase + kQmZ);
-  float* xs = reinterpret_cast<float*>(gbase + kQmX);  // [4 quantities][2 halves][128 rows]
+  float* xs = reinterpret_cast<float*>(gbase + kQmX);  // [den | d_den | dbeta | D'][4 quarters][128 rows]
   const uint32_t bar = base + kQmBAR;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kQmSLOT);
 
-  const int row = 32 * (warp & 3) + lane, hh = warp >> 2;  // query row (TMEM lane), column half
+  const int row = 32 * (warp & 3) + lane, qq = warp >> 2;  // query row (TMEM lane), column quarter
+  const int c0 = 32 * qq;                                   // first column of this thread
   const uint32_t lq = (uint32_t)(32 * (warp & 3)) << 16;
   const bool valid = row < nr;
   const long long grow = row0 + row;  // global row (meaningful when valid)
@@ -80,21 +81,20 @@ __global__ void __launch_bounds__(kQmThreads, 1)
     fence_barrier_init();
   }
   // this thread's q chunks now, and dO, A_dot (read after product 1) into L2
-  uint4 qw[8];
+  uint4 qw[4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
-    qw[i] = valid ? __ldg(reinterpret_cast<const uint4*>(q + grow * 128) + 8 * hh + i) : make_uint4(0u, 0u, 0u, 0u);
+  for (int i = 0; i < 4; ++i)
+    qw[i] = valid ? __ldg(reinterpret_cast<const uint4*>(q + grow * 128 + c0) + i) : make_uint4(0u, 0u, 0u, 0u);
   if (valid) {
-    prefetch_l2(dout + grow * 128 + 64 * hh);
-    prefetch_l2(adot + grow * 128 + 64 * hh);
-    prefetch_l2(adot + grow * 128 + 64 * hh + 32);
+    if ((qq & 1) == 0) prefetch_l2(dout + grow * 128 + c0);
+    prefetch_l2(adot + grow * 128 + c0);
   }
   if (tid < 128) zs[tid] = snapz[((long long)bh * S + s) * 128 + tid];
   if (warp == 0) {
     tmem_alloc(smem_u32(tmem_slot), 256);
     tmem_relinquish();
   }
-  // M [dk][dv] (fp32) -> hi / lo tiles: 2048 chunks of 8 values, 8 per thread
+  // M [dk][dv] (fp32) -> hi / lo tiles: 2048 chunks of 8 values, 4 per thread
   {
     const float* Mp = snapM + ((long long)bh * S + s) * 16384;
 #pragma unroll
@@ -110,25 +110,18 @@ __global__ void __launch_bounds__(kQmThreads, 1)
     }
   }
   __syncthreads();  // z staged
-  // sigma(q) of this thread's 64 columns -> A tiles; partial den
-  float den;
+  // sigma(q) of this thread's 32 columns -> A tiles; partial den
   {
     float dpart = 0.f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int c = 8 * hh + i;  // 16-byte chunk of the row
+    for (int i = 0; i < 4; ++i) {
+      const int c = 4 * qq + i;  // 16-byte chunk of the row
       float x[8];
-      if (valid) {
-        const uint4 w = qw[i];
-        const uint32_t wp[4] = {w.x, w.y, w.z, w.w};
+      const uint32_t wp[4] = {qw[i].x, qw[i].y, qw[i].z, qw[i].w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          x[2 * e] = elu1_accurate(bf16_lo(wp[e]));
-          x[2 * e + 1] = elu1_accurate(bf16_hi(wp[e]));
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] = 0.f;
+      for (int e = 0; e < 4; ++e) {
+        x[2 * e] = valid ? elu1_accurate(bf16_lo(wp[e])) : 0.f;
+        x[2 * e + 1] = valid ? elu1_accurate(bf16_hi(wp[e])) : 0.f;
       }
 #pragma unroll
       for (int e = 0; e < 8; ++e) dpart = fmaf(x[e], zs[8 * c + e], dpart);
@@ -137,7 +130,7 @@ __global__ void __launch_bounds__(kQmThreads, 1)
       sts128(base + kQmAH + swz_chunk(row, c), hi);
       sts128(base + kQmAL + swz_chunk(row, c), lo);
     }
-    xs[hh * 128 + row] = dpart;
+    xs[qq * 128 + row] = dpart;
   }
   fence_proxy_async_smem();
   tc_fence_before();
@@ -145,7 +138,12 @@ __global__ void __launch_bounds__(kQmThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tP1 = tmem, tP2 = tmem + 128u;
-  den = xs[row] + xs[128 + row];  // fixed order: columns 0-63, then 64-127
+  // a row quantity from its four column quarters, in a fixed order
+  auto rowsum = [&](int quantity) {
+    const float* x4 = xs + quantity * 512 + row;
+    return ((x4[0] + x4[128]) + x4[256]) + x4[384];
+  };
+  const float den = rowsum(0);
   // product 1: num = sigma(q) M (A K-major, B = M MN-major)
   if (tid == 0) {
     constexpr uint32_t idesc = idesc_bf16(128, 128, 0, 1);
@@ -161,75 +159,69 @@ __global__ void __launch_bounds__(kQmThreads, 1)
   }
   mbar_wait(bar, 0);
   tc_fence_after();
-  // row terms over this thread's 64 columns; d_num -> A tiles (product 1 has read them)
+  // row terms over this thread's 32 columns; d_num -> A tiles (product 1 has read them)
   float bt = 0.f, dp = 0.f, dd = 0.f;
   {
-#pragma unroll 1
-    for (int half = 0; half < 2; ++half) {
-      uint32_t nm[32];
-      tmem_ld32(tP1 + lq + (uint32_t)(64 * hh + 32 * half), nm);
-      tmem_ld_wait();
-      float dA[32], ad[32];
-      const int c0 = 64 * hh + 32 * half;  // first column
-      if (valid) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint4 w = __ldg(reinterpret_cast<const uint4*>(dout + grow * 128 + c0) + i);
-          const uint32_t wp[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            dA[8 * i + 2 * e] = bf16_lo(wp[e]);
-            dA[8 * i + 2 * e + 1] = bf16_hi(wp[e]);
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float4 f = __ldg(reinterpret_cast<const float4*>(adot + grow * 128 + c0) + i);
-          ad[4 * i] = f.x; ad[4 * i + 1] = f.y; ad[4 * i + 2] = f.z; ad[4 * i + 3] = f.w;
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 32; ++e) dA[e] = ad[e] = 0.f;
-      }
-      float w[32];
-#pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const float am = den != 0.f ? __uint_as_float(nm[e]) / den : 0.f;
-        bt = fmaf(dA[e], am - ad[e], bt);
-        dp = fmaf(dA[e], ad[e], dp);
-        w[e] = 0.f;
-        if (den != 0.f) {
-          w[e] = gw * dA[e] / den;
-          dd = fmaf(gw * dA[e], am, dd);
-        }
-      }
-      if (valid) {
-        float4* dst = reinterpret_cast<float4*>(dnum + grow * 128 + c0);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) dst[i] = make_float4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-      }
+    uint32_t nm[32];
+    tmem_ld32(tP1 + lq + (uint32_t)c0, nm);
+    tmem_ld_wait();
+    float dA[32], ad[32];
+    if (valid) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        uint4 hi, lo;
-        qm_split8(w + 8 * i, hi, lo);
-        sts128(base + kQmAH + swz_chunk(row, c0 / 8 + i), hi);
-        sts128(base + kQmAL + swz_chunk(row, c0 / 8 + i), lo);
+        const uint4 w = __ldg(reinterpret_cast<const uint4*>(dout + grow * 128 + c0) + i);
+        const uint32_t wp[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          dA[8 * i + 2 * e] = bf16_lo(wp[e]);
+          dA[8 * i + 2 * e + 1] = bf16_hi(wp[e]);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float4 f = __ldg(reinterpret_cast<const float4*>(adot + grow * 128 + c0) + i);
+        ad[4 * i] = f.x; ad[4 * i + 1] = f.y; ad[4 * i + 2] = f.z; ad[4 * i + 3] = f.w;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) dA[e] = ad[e] = 0.f;
+    }
+    float w[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const float am = den != 0.f ? __uint_as_float(nm[e]) / den : 0.f;
+      bt = fmaf(dA[e], am - ad[e], bt);
+      dp = fmaf(dA[e], ad[e], dp);
+      w[e] = 0.f;
+      if (den != 0.f) {
+        w[e] = gw * dA[e] / den;
+        dd = fmaf(gw * dA[e], am, dd);
       }
     }
+    if (valid) {
+      float4* dst = reinterpret_cast<float4*>(dnum + grow * 128 + c0);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) dst[i] = make_float4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint4 hi, lo;
+      qm_split8(w + 8 * i, hi, lo);
+      sts128(base + kQmAH + swz_chunk(row, 4 * qq + i), hi);
+      sts128(base + kQmAL + swz_chunk(row, 4 * qq + i), lo);
+    }
   }
-  // the two halves of each row: fixed order
-  xs[512 + hh * 128 + row] = bt;
-  xs[768 + hh * 128 + row] = dp;
-  xs[256 + hh * 128 + row] = dd;
+  xs[512 + qq * 128 + row] = dd;
+  xs[1024 + qq * 128 + row] = bt;
+  xs[1536 + qq * 128 + row] = dp;
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const float ddt = xs[256 + row] + xs[384 + row];
-  const float d_den = den != 0.f ? -ddt / den : 0.f;
-  if (hh == 0 && valid) {
-    Dp[grow] = xs[768 + row] + xs[896 + row];
-    brow[grow] = xs[512 + row] + xs[640 + row];
+  const float d_den = den != 0.f ? -rowsum(1) / den : 0.f;
+  if (qq == 0 && valid) {
+    Dp[grow] = rowsum(3);
+    brow[grow] = rowsum(2);
     dden[grow] = d_den;
   }
   // product 2: d_num M^T (A K-major, B = M read K-major)
@@ -248,17 +240,15 @@ __global__ void __launch_bounds__(kQmThreads, 1)
   mbar_wait(bar, 1);
   tc_fence_after();
   // dq_mem = sigma'(q) (d_num M^T + d_den z): sigma'(x) = 1 above zero, e^x at or below
-#pragma unroll 1
-  for (int half = 0; half < 2; ++half) {
+  {
     uint32_t pr[32];
-    tmem_ld32(tP2 + lq + (uint32_t)(64 * hh + 32 * half), pr);
+    tmem_ld32(tP2 + lq + (uint32_t)c0, pr);
     tmem_ld_wait();
-    const int c0 = 64 * hh + 32 * half;
     if (valid) {
       float o[32];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const uint4 w = __ldg(reinterpret_cast<const uint4*>(q + grow * 128 + c0) + i);
+        const uint4 w = __ldg(reinterpret_cast<const uint4*>(q + grow * 128 + c0) + i);  // L2
         const uint32_t wp[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -294,15 +284,18 @@ __global__ void __launch_bounds__(kQmThreads, 1)
 // fp32 operands in bf16 hi + lo parts (V is exact in bf16: two products for
 // V G^T).  G's and M's tiles are stored row-major [dk][dv]: the MN-major B
 // operand of sigma(K) G and sigma(K) M and, read as K-major, G^T and M^T.
-// The A tiles hold sigma(K), then U (or V), then d_num_r.
+// The A tiles hold sigma(K), then U (or V), then d_num_r.  512 threads:
+// thread (row r = TMEM lane, quarter qq) handles columns [32 qq, 32 qq + 32)
+// of key row r; one thread issues the products.
 constexpr uint32_t kUpAH = 0, kUpAL = 32768, kUpGH = 65536, kUpGL = 98304, kUpMH = 131072, kUpML = 163840;
 constexpr uint32_t kUpZ = 196608;           // gz, then z (2 x 128 floats)
-constexpr uint32_t kUpX = kUpZ + 1024;      // [2 quantities][2 halves][128 rows]
-constexpr uint32_t kUpBAR = kUpX + 2048;
+constexpr uint32_t kUpX = kUpZ + 1024;      // [2 quantities][4 column quarters][128 rows]
+constexpr uint32_t kUpBAR = kUpX + 4096;
 constexpr uint32_t kUpSLOT = kUpBAR + 16;
 constexpr uint32_t kUpSmem = kUpSLOT + 16 + 1024;
+constexpr int kUpThreads = 512;
 
-__global__ void __launch_bounds__(kQmThreads, 1)
+__global__ void __launch_bounds__(kUpThreads, 1)
     bwd_upd_tc_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v, int B, int H, int S,
                       int N, long long L, int seg0, const float* __restrict__ gstate, long long gstride_s,
                       long long gstride_bh, const float* __restrict__ snapM, const float* __restrict__ snapz,
@@ -328,10 +321,10 @@ __global__ void __launch_bounds__(kQmThreads, 1)
   const long long row0 = (long long)bh * L + seg_start + r0;
   float* gz = reinterpret_cast<float*>(gbase + kUpZ);
   float* zs = gz + 128;
-  float* xs = reinterpret_cast<float*>(gbase + kUpX);  // [den | d_den][2 halves][128 rows]
+  float* xs = reinterpret_cast<float*>(gbase + kUpX);  // [den | d_den][4 quarters][128 rows]
   const uint32_t bar = base + kUpBAR;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kUpSLOT);
-  const int row = 32 * (warp & 3) + lane, hh = warp >> 2;
+  const int row = 32 * (warp & 3) + lane, qq = warp >> 2;  // key row (TMEM lane), column quarter
   const uint32_t lq = (uint32_t)(32 * (warp & 3)) << 16;
   const bool valid = row < nr;
   const long long grow = row0 + row;
@@ -343,11 +336,11 @@ __global__ void __launch_bounds__(kQmThreads, 1)
     fence_barrier_init();
   }
   // this thread's k chunks now, and v (read after the first products) into L2
-  uint4 kw[8];
+  uint4 kw[4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
-    kw[i] = valid ? __ldg(reinterpret_cast<const uint4*>(k + grow * 128) + 8 * hh + i) : make_uint4(0u, 0u, 0u, 0u);
-  if (valid) prefetch_l2(v + grow * 128 + 64 * hh);
+  for (int i = 0; i < 4; ++i)
+    kw[i] = valid ? __ldg(reinterpret_cast<const uint4*>(k + grow * 128) + 4 * qq + i) : make_uint4(0u, 0u, 0u, 0u);
+  if (valid && (qq & 1) == 0) prefetch_l2(v + grow * 128 + 32 * qq);
   if (tid < 128) {
     gz[tid] = gp[16384 + tid];
     zs[tid] = delta ? snapz[((long long)bh * S + s) * 128 + tid] : 0.f;
@@ -358,7 +351,7 @@ __global__ void __launch_bounds__(kQmThreads, 1)
   }
   // G (and M) [dk][dv] fp32 -> hi / lo tiles
 #pragma unroll
-  for (int ch = tid; ch < 2048; ch += kQmThreads) {
+  for (int ch = tid; ch < 2048; ch += kUpThreads) {
     const int i = ch >> 4, c = ch & 15;
     float x[8];
     {
@@ -380,12 +373,12 @@ __global__ void __launch_bounds__(kQmThreads, 1)
     }
   }
   __syncthreads();  // gz, z staged
-  // sigma(K) of this thread's 64 columns -> A tiles; partial den_k (delta)
+  // sigma(K) of this thread's 32 columns -> A tiles; partial den_k (delta)
   {
     float dpart = 0.f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int c = 8 * hh + i;
+    for (int i = 0; i < 4; ++i) {
+      const int c = 4 * qq + i;
       float x[8];
       if (valid) {
         const uint4 w = kw[i];
@@ -406,7 +399,7 @@ __global__ void __launch_bounds__(kQmThreads, 1)
       sts128(base + kUpAH + swz_chunk(row, c), hi);
       sts128(base + kUpAL + swz_chunk(row, c), lo);
     }
-    xs[hh * 128 + row] = dpart;
+    xs[qq * 128 + row] = dpart;
   }
   fence_proxy_async_smem();
   tc_fence_before();
@@ -414,7 +407,12 @@ __global__ void __launch_bounds__(kQmThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tDU = tmem, tR = tmem + 128u, tDS = tmem + 256u;
-  const float den = delta ? xs[row] + xs[128 + row] : 0.f;
+  // a row quantity from its four column quarters, in a fixed order
+  auto rowsum = [&](int quantity) {
+    const float* x4 = xs + quantity * 512 + row;
+    return ((x4[0] + x4[128]) + x4[256]) + x4[384];
+  };
+  const float den = delta ? rowsum(0) : 0.f;
   // d (+)= A B in hi / lo parts: aH bH + aH bL (+ aL bH when `alo`); B MN-major or K-major
   auto issue3 = [&](uint32_t d, uint32_t aH, uint32_t aL, bool alo, uint32_t bH, uint32_t bL, bool bmn, bool acc0) {
     const uint32_t idesc = bmn ? idesc_bf16(128, 128, 0, 1) : idesc_bf16(128, 128, 0, 0);
@@ -437,9 +435,8 @@ __global__ void __launch_bounds__(kQmThreads, 1)
   tc_fence_after();
   // dU -> dv term; U = V (- R) -> A tiles; delta: d_num_r, d_den_r
   float dd = 0.f;
-#pragma unroll 1
-  for (int half = 0; half < 2; ++half) {
-    const int c0 = 64 * hh + 32 * half;
+  {
+    const int c0 = 32 * qq;
     uint32_t du[32], rr[32];
     tmem_ld32(tDU + lq + (uint32_t)c0, du);
     if (delta) tmem_ld32(tR + lq + (uint32_t)c0, rr);
@@ -487,13 +484,13 @@ __global__ void __launch_bounds__(kQmThreads, 1)
       if (delta) sts128(base + kUpAL + swz_chunk(row, c0 / 8 + i), lo);
     }
   }
-  if (delta) xs[256 + hh * 128 + row] = dd;
+  if (delta) xs[512 + qq * 128 + row] = dd;
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const float d_den = (delta && den != 0.f) ? (xs[256 + row] + xs[384 + row]) / den : 0.f;
-  if (delta && hh == 0 && valid) dden_r[grow] = d_den;
+  const float d_den = (delta && den != 0.f) ? rowsum(1) / den : 0.f;
+  if (delta && qq == 0 && valid) dden_r[grow] = d_den;
   // product 3: U G^T (linear: V G^T, V exact)
   if (tid == 0) {
     issue3(tDS, base + kUpAH, base + kUpAL, delta, base + kUpGH, base + kUpGL, false, false);
@@ -503,9 +500,8 @@ __global__ void __launch_bounds__(kQmThreads, 1)
   tc_fence_after();
   if (delta) {
     // product 4: d_num_r M^T into the same accumulator; d_num_r back from global (just written)
-#pragma unroll 1
-    for (int half = 0; half < 2; ++half) {
-      const int c0 = 64 * hh + 32 * half;
+    {
+      const int c0 = 32 * qq;
       float w[32];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -533,9 +529,8 @@ __global__ void __launch_bounds__(kQmThreads, 1)
     tc_fence_after();
   }
   // dk term: sigma'(k) (dsigma(K) + gz + d_den_r z)
-#pragma unroll 1
-  for (int half = 0; half < 2; ++half) {
-    const int c0 = 64 * hh + 32 * half;
+  {
+    const int c0 = 32 * qq;
     uint32_t ds[32];
     tmem_ld32(tDS + lq + (uint32_t)c0, ds);
     tmem_ld_wait();
@@ -582,10 +577,10 @@ __global__ void __launch_bounds__(kQmThreads, 1)
 //   y0's hi and lo parts as rows 0 and 1 of a 16-row K-major B tile (rows
 //   2-15 zero): Dz += (s_hi + s_lo)^T [y0_hi | y0_lo | 0], and
 //   sigma^T y0 = Dz[:, 0] + Dz[:, 1].
-// 256 threads: thread (row r = TMEM lane, half hh) stages columns
-// [64 hh, 64 hh + 64) of row r and writes row r's partial; thread 0 issues
-// the products.  A group with no rows writes a zero partial.
-constexpr int kOtThreads = 256;
+// 512 threads: thread (row r = TMEM lane, quarter qq) stages columns
+// [32 qq, 32 qq + 32) of row r and writes those of row r's partial; thread 0
+// issues the products.  A group with no rows writes a zero partial.
+constexpr int kOtThreads = 512;
 constexpr uint32_t kOtAH = 0, kOtAL = 32768, kOtYH = 65536, kOtYL = 98304;  // 128 x 128 bf16 tiles
 constexpr uint32_t kOtY0 = 131072;       // 16 x 128 bf16 K-major (two 2 KB boxes)
 constexpr uint32_t kOtBAR = kOtY0 + 4096;
@@ -617,14 +612,14 @@ __global__ void __launch_bounds__(kOtThreads, 1)
   const int nblk = t_begin < t_end ? (t_end - t_begin + 127) / 128 : 0;
   const uint32_t bar = base + kOtBAR;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kOtSLOT);
-  const int row = 32 * (warp & 3) + lane, hh = warp >> 2;  // row of the block (TMEM lane: dk index), column half
+  const int row = 32 * (warp & 3) + lane, qq = warp >> 2;  // row of the block (TMEM lane: dk index), column quarter
   const uint32_t lq = (uint32_t)(32 * (warp & 3)) << 16;
 
   if (tid == 0) {
     mbar_init(bar, 1);
     fence_barrier_init();
   }
-  sts128(base + kOtY0 + 16u * (uint32_t)tid, make_uint4(0u, 0u, 0u, 0u));  // the y0 tile, 4 KB
+  if (tid < 256) sts128(base + kOtY0 + 16u * (uint32_t)tid, make_uint4(0u, 0u, 0u, 0u));  // the y0 tile, 4 KB
   if (warp == 0) {
     tmem_alloc(smem_u32(tmem_slot), 256);
     tmem_relinquish();
@@ -641,29 +636,28 @@ __global__ void __launch_bounds__(kOtThreads, 1)
     const bool valid = row < t_end - r0;
     const long long grow = (long long)bh * L + seg_start + r0 + row;
     if (row < t_end - r0 - 128) {  // the next block's row: into L2 while this one is staged and multiplied
-      prefetch_l2(x + (grow + 128) * 128 + 64 * hh);
-      prefetch_l2(Y + (grow + 128) * 128 + 64 * hh);
-      prefetch_l2(Y + (grow + 128) * 128 + 64 * hh + 32);
+      if ((qq & 1) == 0) prefetch_l2(x + (grow + 128) * 128 + 32 * qq);
+      prefetch_l2(Y + (grow + 128) * 128 + 32 * qq);
     }
     // this thread's x and Y chunks, all loads issued before any store (and
     // while the previous block's products run)
-    uint4 xw[8];
-    float4 yf[16];
+    uint4 xw[4];
+    float4 yf[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      xw[i] = valid ? __ldg(reinterpret_cast<const uint4*>(x + grow * 128) + 4 * qq + i) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
     for (int i = 0; i < 8; ++i)
-      xw[i] = valid ? __ldg(reinterpret_cast<const uint4*>(x + grow * 128) + 8 * hh + i) : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-    for (int i = 0; i < 16; ++i)
-      yf[i] = valid ? __ldg(reinterpret_cast<const float4*>(Y + grow * 128 + 64 * hh) + i)
+      yf[i] = valid ? __ldg(reinterpret_cast<const float4*>(Y + grow * 128 + 32 * qq) + i)
                     : make_float4(0.f, 0.f, 0.f, 0.f);
     if (blk > 0) {
       mbar_wait(bar, (uint32_t)(blk - 1) & 1u);  // the previous block's products have read the tiles
       tc_fence_after();
     }
-    // sigma(x) of this thread's 64 columns (rows past the end: sigma = 0)
+    // sigma(x) of this thread's 32 columns (rows past the end: sigma = 0)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int c = 8 * hh + i;
+    for (int i = 0; i < 4; ++i) {
+      const int c = 4 * qq + i;
       float v[8];
       const uint32_t wp[4] = {xw[i].x, xw[i].y, xw[i].z, xw[i].w};
 #pragma unroll
@@ -676,10 +670,10 @@ __global__ void __launch_bounds__(kOtThreads, 1)
       sts128(base + kOtAH + swz_chunk(row, c), hi);
       sts128(base + kOtAL + swz_chunk(row, c), lo);
     }
-    // Y of this thread's 64 columns
+    // Y of this thread's 32 columns
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int c = 8 * hh + i;
+    for (int i = 0; i < 4; ++i) {
+      const int c = 4 * qq + i;
       const float v[8] = {yf[2 * i].x, yf[2 * i].y, yf[2 * i].z, yf[2 * i].w,
                           yf[2 * i + 1].x, yf[2 * i + 1].y, yf[2 * i + 1].z, yf[2 * i + 1].w};
       uint4 hi, lo;
@@ -688,7 +682,7 @@ __global__ void __launch_bounds__(kOtThreads, 1)
       sts128(base + kOtYL + swz_chunk(row, c), lo);
     }
     // y0 of this row: element (n, k = row) of the K-major tile, n = 0 (hi), 1 (lo)
-    if (hh == 0) {
+    if (qq == 0) {
       const float v = valid ? y0[grow] : 0.f;
       const __nv_bfloat16 vh = __float2bfloat16_rn(v);
       const __nv_bfloat16 vl = __float2bfloat16_rn(v - __bfloat162float(vh));
@@ -726,12 +720,11 @@ __global__ void __launch_bounds__(kOtThreads, 1)
     mbar_wait(bar, (uint32_t)(nblk - 1) & 1u);
     tc_fence_after();
   }
-  // row `row` (a dk index) of the partial: columns [64 hh, 64 hh + 64), and
-  // (hh = 0) its sigma^T y0 entry
+  // row `row` (a dk index) of the partial: columns [32 qq, 32 qq + 32), and
+  // (qq = 0) its sigma^T y0 entry
   float* out = partial + (((long long)bh * nseg + sl) * G + grp) * (long long)(16384 + 128);
-#pragma unroll 1
-  for (int h2 = 0; h2 < 2; ++h2) {
-    const int c0 = 64 * hh + 32 * h2;
+  {
+    const int c0 = 32 * qq;
     uint32_t v[32];
     if (nblk > 0) {
       tmem_ld32(tD + lq + (uint32_t)c0, v);
@@ -746,7 +739,7 @@ __global__ void __launch_bounds__(kOtThreads, 1)
       dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]), __uint_as_float(v[4 * i + 2]),
                            __uint_as_float(v[4 * i + 3]));
   }
-  if (hh == 0) {
+  if (qq == 0) {
     float zsum = 0.f;
     if (nblk > 0) {
       uint32_t v[16];
