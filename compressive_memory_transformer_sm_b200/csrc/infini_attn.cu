@@ -396,13 +396,13 @@ int run_simt(const infini_attn_params& p, const Plan& pl, char* ws, float scale,
     {
       LaunchScope ls(kPhaseState, p.stream);
       state_kernel<<<sgrid, 256, 0, p.stream>>>(p.M, p.z, part, p.dk, p.dv, pl.S, 0, 0, pl.S, pl.G, snapM, nullptr,
-                                                snapz);
+                                                snapz, nullptr);
     }
   } else {
     {
       LaunchScope ls(kPhaseState, p.stream);
       state_kernel<<<sgrid, 256, 0, p.stream>>>(p.M, p.z, part, p.dk, p.dv, pl.S, 2, 0, 1, pl.G, snapM, nullptr,
-                                                snapz);
+                                                snapz, nullptr);
     }
     for (int s = 0; s < pl.S; ++s) {
       {
@@ -412,7 +412,7 @@ int run_simt(const infini_attn_params& p, const Plan& pl, char* ws, float scale,
       }
       LaunchScope ls(kPhaseState, p.stream);
       state_kernel<<<sgrid, 256, 0, p.stream>>>(p.M, p.z, part, p.dk, p.dv, pl.S, 1, s, 1, pl.G, snapM, nullptr,
-                                                snapz);
+                                                snapz, nullptr);
     }
   }
   if (p.flags & kFlagUpdateOnly) return launch_status();
@@ -611,44 +611,48 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale, c
   ua.G = pl.G; ua.cpb = pl.cpb;
   // One segment (a streaming step): the attention reads only the snapshot of
   // (M_0, z_0), which the update never writes after its start, so once the
-  // snapshot is taken the attention runs on a second stream alongside the
-  // update; the caller's stream then waits for both (event fork and join).
-  cudaStream_t as = p.stream;  // the attention's stream
+  // snapshot is taken the update runs on a second stream and the attention
+  // follows the snapshot on the caller's stream, as a programmatic dependent
+  // (its setup overlaps the snapshot kernel; it reads nothing before the
+  // snapshot is complete); the caller's stream then waits for the update
+  // (event fork and join).  The snapshot kernel also zeroes the attention's
+  // work counter.
+  unsigned int* ctr = reinterpret_cast<unsigned int*>(ws + pl.off_ctr);
+  cudaStream_t us = p.stream;  // the update's stream
   cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
   const bool fork = pl.S == 1 && !(p.flags & kFlagUpdateOnly) && extra == nullptr;
   if (fork) {
     {
       LaunchScope ls(kPhaseState, p.stream);
-      state_kernel<<<sgrid, 256, 0, p.stream>>>(p.M, p.z, part, 128, 128, 1, 2, 0, 1, pl.G, nullptr, snapM16, snapz);
+      state_kernel<<<sgrid, 256, 0, p.stream>>>(p.M, p.z, part, 128, 128, 1, 2, 0, 1, pl.G, nullptr, snapM16, snapz, ctr);
     }
     cudaStream_t side = side_stream();
     if (side != nullptr && fork_events(&ev_fork, &ev_join) && cudaEventRecord(ev_fork, p.stream) == cudaSuccess &&
         cudaStreamWaitEvent(side, ev_fork, 0) == cudaSuccess) {
-      as = side;
+      us = side;
     } else {
       cudaGetLastError();
     }
     ua.snapM = nullptr;  // taken above: the update kernels skip it
     ua.snapzw = nullptr;
   }
-  // the caller's stream waits for the attention's stream
+  // the caller's stream waits for the update's stream
   auto join = [&]() {
-    if (ev_join != nullptr && as != p.stream) {
-      if (cudaEventRecord(ev_join, as) != cudaSuccess || cudaStreamWaitEvent(p.stream, ev_join, 0) != cudaSuccess)
+    if (ev_join != nullptr && us != p.stream) {
+      if (cudaEventRecord(ev_join, us) != cudaSuccess || cudaStreamWaitEvent(p.stream, ev_join, 0) != cudaSuccess)
         cudaGetLastError();
     }
   };
   if (!pl.delta) {
     ua.seg0 = 0; ua.nseg = pl.S;
     {
-      LaunchScope ls(kPhaseUpdate, p.stream);
-      tc::mem_update_tc_kernel<<<BH * pl.S * pl.G, tc::UpdWarps::THREADS, tc::UpdSmem::BYTES, p.stream>>>(
-          tm_k, tm_v, ua);
+      LaunchScope ls(kPhaseUpdate, us);
+      tc::mem_update_tc_kernel<<<BH * pl.S * pl.G, tc::UpdWarps::THREADS, tc::UpdSmem::BYTES, us>>>(tm_k, tm_v, ua);
     }
-    LaunchScope ls(kPhaseState, p.stream);
-    state_kernel<<<sgrid, 256, 0, p.stream>>>(p.M, p.z, part, 128, 128, pl.S, 0, 0, pl.S, pl.G,
+    LaunchScope ls(kPhaseState, us);
+    state_kernel<<<sgrid, 256, 0, us>>>(p.M, p.z, part, 128, 128, pl.S, 0, 0, pl.S, pl.G,
                                               extra ? extra->snapM32 : nullptr, fork ? nullptr : snapM16,
-                                              fork ? nullptr : snapz);
+                                              fork ? nullptr : snapz, nullptr);
   } else {
     ua.nseg = 1;
     // 64-token chunks: K and V maps with 64-row boxes
@@ -672,7 +676,7 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale, c
     cfg.gridDim = dim3(BH * pl.G);
     cfg.blockDim = dim3(tc::kDeltaThreads);
     cfg.dynamicSmemBytes = tc::DeltaSmem::BYTES;
-    cfg.stream = p.stream;
+    cfg.stream = us;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     for (int s = 0; s < pl.S; ++s) {
@@ -680,7 +684,7 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale, c
       // segment s, reduced inside each head's cluster into M, z
       ua.seg0 = s;
       cfg.numAttrs = s > 0 ? 2 : 1;
-      LaunchScope ls(kPhaseUpdate, p.stream);
+      LaunchScope ls(kPhaseUpdate, us);
       const cudaError_t e = cudaLaunchKernelEx(&cfg, tc::delta_update_tc_kernel, tm_k64, tm_v64, ua);
       if (e != cudaSuccess) {
         cudaGetLastError();
@@ -719,18 +723,32 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale, c
   const long long groups = (NS + aa.GS - 1) / aa.GS;
   // persistent: one CTA per SM, or one per work item when there are fewer
   const long long items = groups * aa.GS * aa.P;
-  aa.work_counter = reinterpret_cast<unsigned int*>(ws + pl.off_ctr);
-  if (items >= (1LL << 31) || cudaMemsetAsync(aa.work_counter, 0, sizeof(unsigned int), as) != cudaSuccess) {
+  aa.work_counter = ctr;
+  if (items >= (1LL << 31) ||
+      (!fork && cudaMemsetAsync(aa.work_counter, 0, sizeof(unsigned int), p.stream) != cudaSuccess)) {
     join();
     return items >= (1LL << 31) ? INFINI_ERR_UNSUPPORTED : INFINI_ERR_LAUNCH;
   }
   {
-    LaunchScope ls(kPhaseAttn, as);
-    const unsigned grid = (unsigned)std::min<long long>(items, sms);
-    if (aa.single == 2)
-      tc::attn_tc_kernel<true><<<grid, tc::kAttnThreads, tc::kAttnSmem, as>>>(tm_qa, tm_ka, tm_v, tm_mt, aa);
-    else
-      tc::attn_tc_kernel<false><<<grid, tc::kAttnThreads, tc::kAttnSmem, as>>>(tm_qa, tm_ka, tm_v, tm_mt, aa);
+    LaunchScope ls(kPhaseAttn, p.stream);
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3((unsigned)std::min<long long>(items, sms));
+    cfg.blockDim = dim3(tc::kAttnThreads);
+    cfg.dynamicSmemBytes = tc::kAttnSmem;
+    cfg.stream = p.stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = fork ? 1 : 0;  // after the snapshot kernel: a programmatic dependent
+    const cudaError_t e = aa.single == 2
+                              ? cudaLaunchKernelEx(&cfg, tc::attn_tc_kernel<true>, tm_qa, tm_ka, tm_v, tm_mt, aa)
+                              : cudaLaunchKernelEx(&cfg, tc::attn_tc_kernel<false>, tm_qa, tm_ka, tm_v, tm_mt, aa);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      join();
+      return note_cuda_error(e);
+    }
   }
   const int rc = launch_status();
   join();

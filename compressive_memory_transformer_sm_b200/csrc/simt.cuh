@@ -148,12 +148,15 @@ __global__ void __launch_bounds__(256) simt_update_kernel(const T* __restrict__ 
 //        in `partial`, store, and snapshot as segment s + 1 if it exists.
 //   op 2 (snapshot only): snapshot the state as segment s.
 // Snapshots are fp32 [BH][S][dk][dv] (snapM32) and/or, for the tensor-core
-// kernels, bf16 [BH][S][dk][dv] (snapM16); z snapshots fp32.
+// kernels, bf16 [BH][S][dk][dv] (snapM16); z snapshots fp32.  `counter`, when
+// given (op 2), is set to zero (the next attention launch's work counter); a
+// programmatic dependent launch may start as soon as every block has begun.
 __global__ void __launch_bounds__(256) state_kernel(float* __restrict__ M, float* __restrict__ z,
                                                     const float* __restrict__ partial, int dk, int dv, int S, int op,
                                                     int s, int nseg, int G, float* __restrict__ snapM32,
                                                     __nv_bfloat16* __restrict__ snapM16,
-                                                    float* __restrict__ snapz) {
+                                                    float* __restrict__ snapz, unsigned int* __restrict__ counter) {
+  griddep_launch_dependents();
   const int bh = blockIdx.y;
   const int e = blockIdx.x * 256 + threadIdx.x;
   const int E = dk * dv;
@@ -199,6 +202,7 @@ __global__ void __launch_bounds__(256) state_kernel(float* __restrict__ M, float
     if (s + 1 < S) snap(s + 1, acc);
   } else {
     snap(s, acc);
+    if (counter != nullptr && e == 0 && bh == 0) *counter = 0u;
   }
 }
 

@@ -225,6 +225,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // Launched as a programmatic dependent (after the snapshot of a streaming
+  // step), the setup above overlaps the previous kernel; nothing it wrote
+  // (the snapshots, the work counter) is read before this returns.
+  griddep_wait();
   // The CTA owns all 512 columns of the SM's tensor memory, so its block
   // starts at lane 0, column 0 and every TMEM address below is a constant.
   if (*tmem_slot != 0u) {  // not expected: report and leave
