@@ -621,6 +621,11 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale, c
   cudaStream_t us = p.stream;  // the update's stream
   cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
   const bool fork = pl.S == 1 && !(p.flags & kFlagUpdateOnly) && extra == nullptr;
+  // Otherwise the attention's work counter is zeroed before the update, so
+  // that the attention launch directly follows the update's last kernel (a
+  // programmatic dependent of it, like the streaming case's).
+  if (!fork && !(p.flags & kFlagUpdateOnly) && cudaMemsetAsync(ctr, 0, sizeof(unsigned int), p.stream) != cudaSuccess)
+    return note_cuda_error(cudaGetLastError());
   if (fork) {
     {
       LaunchScope ls(kPhaseState, p.stream);
@@ -724,10 +729,9 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale, c
   // persistent: one CTA per SM, or one per work item when there are fewer
   const long long items = groups * aa.GS * aa.P;
   aa.work_counter = ctr;
-  if (items >= (1LL << 31) ||
-      (!fork && cudaMemsetAsync(aa.work_counter, 0, sizeof(unsigned int), p.stream) != cudaSuccess)) {
+  if (items >= (1LL << 31)) {
     join();
-    return items >= (1LL << 31) ? INFINI_ERR_UNSUPPORTED : INFINI_ERR_LAUNCH;
+    return INFINI_ERR_UNSUPPORTED;
   }
   {
     LaunchScope ls(kPhaseAttn, p.stream);
@@ -740,7 +744,7 @@ int run_tc(const infini_attn_params& p, const Plan& pl, char* ws, float scale, c
     cfg.dynamicSmemBytes = tc::kAttnSmem;
     cfg.stream = p.stream;
     cfg.attrs = attr;
-    cfg.numAttrs = fork ? 1 : 0;  // after the snapshot kernel: a programmatic dependent
+    cfg.numAttrs = 1;  // a programmatic dependent of the kernel before it (snapshot, scan or update)
     const cudaError_t e = aa.single == 2
                               ? cudaLaunchKernelEx(&cfg, tc::attn_tc_kernel<true>, tm_qa, tm_ka, tm_v, tm_mt, aa)
                               : cudaLaunchKernelEx(&cfg, tc::attn_tc_kernel<false>, tm_qa, tm_ka, tm_v, tm_mt, aa);
