@@ -151,7 +151,10 @@ namespace infini {
 // memory, merges them in rank order (deterministic), adds the memory read
 // (Eq. 7) and the gate (Eq. 10) and writes the row; a second barrier keeps
 // every CTA's shared memory alive until rank 0 is done.  No global scratch.
-// CTA 0 also appends k_t, v_t to row n - 1 of the caches (no CTA reads it).
+// The memory read is spread the same way: CTA r forms sigma(q) M and
+// sigma(q) z over its slice of M's rows, before its key range, and rank 0
+// adds the slices in rank order.  CTA 0 also appends k_t, v_t to row n - 1 of
+// the caches (no CTA reads it).
 constexpr int kDecodeMaxSplits = 16;
 
 // q . k for one cached key row of dk elements: 16-byte vector loads when
@@ -198,8 +201,8 @@ __global__ void __launch_bounds__(256)
   __shared__ float qs[128];
   __shared__ float wm[8], wl[8], wacc[8][128];
   __shared__ __align__(16) float st[2 + 128];  // this range's state: m, l, o[dv]
+  __shared__ __align__(16) float mr[2][129];   // this slice's sigma(q) M [dv] and sigma(q) z, per thread half
   __shared__ float sq[128];
-  __shared__ float red[8];
   const int split = blockIdx.x, bh = blockIdx.y, splits = gridDim.x;
   const int h = bh % H;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -207,8 +210,39 @@ __global__ void __launch_bounds__(256)
     for (int i = tid; i < dk; i += 256) kc[((long long)bh * N + n - 1) * dk + i] = k_t[(long long)bh * dk + i];
     for (int i = tid; i < dv; i += 256) vc[((long long)bh * N + n - 1) * dv + i] = v_t[(long long)bh * dv + i];
   }
-  for (int i = tid; i < dk; i += 256) qs[i] = to_f32(q[(long long)bh * dk + i]);
+  for (int i = tid; i < dk; i += 256) {
+    qs[i] = to_f32(q[(long long)bh * dk + i]);
+    sq[i] = elu1_accurate(qs[i]);
+  }
   __syncthreads();
+  {
+    // the memory read over rows [i0, i1) of M, z: thread (column c, half hf)
+    // takes every other row; 16 independent sums keep 16 loads in flight
+    const int i0 = split * dk / splits, i1 = (split + 1) * dk / splits;
+    const int c = tid & 127, hf = tid >> 7;
+    const float* Mh = M + (long long)bh * dk * dv;
+    float nm[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) nm[u] = 0.f;
+    if (c < dv) {
+      int i = i0 + hf;
+      for (; i + 30 < i1; i += 32) {
+#pragma unroll
+        for (int u = 0; u < 16; ++u) nm[u] = fmaf(sq[i + 2 * u], Mh[(long long)(i + 2 * u) * dv + c], nm[u]);
+      }
+      for (int u = 0; i < i1; i += 2, ++u) nm[u & 15] = fmaf(sq[i], Mh[(long long)i * dv + c], nm[u & 15]);
+      float t = 0.f;
+#pragma unroll
+      for (int u = 0; u < 16; ++u) t += nm[u];
+      mr[hf][c] = t;
+    }
+    if (tid < 32) {  // sigma(q) z over the slice: lanes stride the rows, then the warp
+      float d = 0.f;
+      for (int i = i0 + tid; i < i1; i += 32) d = fmaf(sq[i], z[(long long)bh * dk + i], d);
+      d = warp_sum(d);
+      if (tid == 0) mr[0][128] = d;
+    }
+  }
   const int j0 = split * per, j1 = min(n, j0 + per);
   const T* kb = kc + (long long)bh * N * dk;
   const T* vb = vc + (long long)bh * N * dv;
@@ -265,44 +299,28 @@ __global__ void __launch_bounds__(256)
   }
   cluster_sync();  // every range's state is in its CTA's shared memory
   if (split == 0) {
-    // memory read: sigma(q), den = sigma(q) . z
-    const float* zh = z + (long long)bh * dk;
-    for (int i = tid; i < dk; i += 256) sq[i] = elu1_accurate(qs[i]);
-    __syncthreads();
-    float d = 0.f;
-    for (int i = tid; i < dk; i += 256) d = fmaf(sq[i], zh[i], d);
-    d = warp_sum(d);
-    if (lane == 0) red[warp] = d;
-    __syncthreads();
+    const uint32_t sbase = smem_u32(st), mbase = smem_u32(&mr[0][0]);
+    // den = sigma(q) . z: the slices in rank order
     float den = 0.f;
-    for (int w = 0; w < 8; ++w) den += red[w];
-    const uint32_t sbase = smem_u32(st);
+    for (int r = 0; r < splits; ++r) den += ld_dsmem_f32(mapa_shared(mbase + 4u * 128u, (uint32_t)r));
     float gm = -INFINITY;
     for (int r = 0; r < splits; ++r) gm = fmaxf(gm, ld_dsmem_f32(mapa_shared(sbase, (uint32_t)r)));
     float gl = 0.f;
     for (int r = 0; r < splits; ++r) {
       const uint32_t a = mapa_shared(sbase, (uint32_t)r);
-      const float mr = ld_dsmem_f32(a);
-      gl += mr == -INFINITY ? 0.f : ld_dsmem_f32(a + 4u) * expf(mr - gm);
+      const float mx = ld_dsmem_f32(a);
+      gl += mx == -INFINITY ? 0.f : ld_dsmem_f32(a + 4u) * expf(mx - gm);
     }
     const float g = 1.f / (1.f + expf(-beta[h]));
-    const float* Mh = M + (long long)bh * dk * dv;
     for (int c = tid; c < dv; c += 256) {
-      float o = 0.f;
+      float o = 0.f, num = 0.f;
       for (int r = 0; r < splits; ++r) {
         const uint32_t a = mapa_shared(sbase, (uint32_t)r);
-        const float mr = ld_dsmem_f32(a);
-        o += mr == -INFINITY ? 0.f : ld_dsmem_f32(a + 4u * (uint32_t)(2 + c)) * expf(mr - gm);
+        const float mx = ld_dsmem_f32(a);
+        o += mx == -INFINITY ? 0.f : ld_dsmem_f32(a + 4u * (uint32_t)(2 + c)) * expf(mx - gm);
+        const uint32_t b = mapa_shared(mbase + 4u * (uint32_t)c, (uint32_t)r);
+        num += ld_dsmem_f32(b) + ld_dsmem_f32(b + 4u * 129u);  // the slice's two halves
       }
-      // sigma(q) M column c: eight independent partial sums keep eight loads in flight
-      float nm[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      int i = 0;
-      for (; i + 8 <= dk; i += 8) {
-#pragma unroll
-        for (int u = 0; u < 8; ++u) nm[u] = fmaf(sq[i + u], Mh[(long long)(i + u) * dv + c], nm[u]);
-      }
-      for (; i < dk; ++i) nm[0] = fmaf(sq[i], Mh[(long long)i * dv + c], nm[0]);
-      const float num = ((nm[0] + nm[1]) + (nm[2] + nm[3])) + ((nm[4] + nm[5]) + (nm[6] + nm[7]));
       const float a_mem = den != 0.f ? num / den : 0.f;
       out[(long long)bh * dv + c] = from_f32<T>(g * a_mem + (1.f - g) * (o / gl));
     }
