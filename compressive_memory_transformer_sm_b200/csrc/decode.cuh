@@ -166,7 +166,7 @@ __device__ __forceinline__ float decode_dot(const float* qs, const T* kr, int dk
   if (vec) {
     const uint4* k4 = reinterpret_cast<const uint4*>(kr);
     if constexpr (sizeof(T) == 2) {
-#pragma unroll 4
+#pragma unroll 8
       for (int c = 0; c < dk / 8; ++c) {
         const uint4 w = __ldg(k4 + c);
         const uint32_t u[4] = {w.x, w.y, w.z, w.w};
@@ -177,7 +177,7 @@ __device__ __forceinline__ float decode_dot(const float* qs, const T* kr, int dk
         }
       }
     } else {
-#pragma unroll 4
+#pragma unroll 8
       for (int c = 0; c < dk / 4; ++c) {
         const float4 w = __ldg(reinterpret_cast<const float4*>(k4 + c));
         d = fmaf(qs[4 * c], w.x, d);
@@ -261,7 +261,7 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
     for (int c = 0; c < 4; ++c) acc[c] *= alpha;
     const int cnt = min(32, j1 - jb);
-#pragma unroll 4
+#pragma unroll 8
     for (int jj = 0; jj < cnt; ++jj) {
       const float pj = __shfl_sync(0xffffffffu, p, jj);
       const int key = jb + jj;
