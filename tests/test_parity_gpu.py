@@ -272,6 +272,32 @@ def test_workload_passkey_1m_streaming_delta():
     _sample_check_head(q, k, v, beta, out, M, z, 0, 3, w.N, DELTA, segments=[0, 1, 2, 255, S - 1])
 
 
+@pytest.mark.parametrize("shape", [(2, 3, 4 * 256 + 100, 256), (1, 2, 3 * 512, 512)])
+@pytest.mark.parametrize("mode", [LINEAR, DELTA])
+def test_segment_step_sequence_matches_forward(shape, mode):
+    """One segment_step call per segment (ragged last segment in the first shape), bf16 d = 128 on
+    the tensor cores (the update on the library's second stream, the attention on the caller's):
+    outputs and final state equal the oracle's whole-sequence forward."""
+    B, H, L, N = shape
+    q, k, v, beta = inputs(B, H, L, 128, 128, torch.bfloat16, 300 + L + mode)
+    M = torch.zeros(B, H, 128, 128, device=DEV)
+    z = torch.zeros(B, H, 128, device=DEV)
+    out = torch.full((B, H, L, 128), float("nan"), dtype=torch.bfloat16, device=DEV)
+    for s0 in range(0, L, N):
+        s1 = min(L, s0 + N)
+        o = torch.empty(B, H, s1 - s0, 128, dtype=torch.bfloat16, device=DEV)
+        api.infini_attn_segment_step(q[:, :, s0:s1].contiguous(), k[:, :, s0:s1].contiguous(),
+                                     v[:, :, s0:s1].contiguous(), beta, M, z, o, mode)
+        out[:, :, s0:s1] = o
+    torch.cuda.synchronize()
+    assert api.infini_attn_device_status() == api.INFINI_OK
+    wo, wM, wz = oracle(q, k, v, beta, N, mode)
+    what = f"segment_step {shape} mode={mode}"
+    assert_out(np64(out), wo, False, what + " out")
+    assert_state(np64(M), wM, False, what + " M")
+    assert_state(np64(z), wz, False, what + " z")
+
+
 def test_workload_8b_long_both_rules():
     w = W.LONG_8B
     q, k, v, beta = W.make_inputs(w, device=DEV)
