@@ -154,8 +154,8 @@ int make_plan(int B, int H, long long L, int N, int dk, int dv, int mode, int fl
     G = std::min<long long>(G, chunks_per_seg);
     // One segment with its attention (a streaming step): the update runs
     // alongside the attention, which sets the call's length, so it takes about
-    // an eighth of the SMs (as the delta rule's clusters of 2 do at 8 heads)
-    if (S == 1 && !p->delta && !(flags & kFlagUpdateOnly))
+    // an eighth of the SMs (two CTAs per head at 8 heads) and leaves the rest
+    if (S == 1 && !(flags & kFlagUpdateOnly))
       G = std::max<long long>(1, std::min<long long>(G, (kSms / 8) / units));
     cpb = (chunks_per_seg + G - 1) / G;
   } else {
