@@ -99,11 +99,14 @@ __global__ void __launch_bounds__(256) rope_kernel(const __grid_constant__ RopeA
   float cs[E / 2], sn[E / 2];
 #pragma unroll
   for (int e = 0; e < E / 2; ++e) rope_angle(pos, fr[j * (E / 2) + e], cs[e], sn[e]);
-  const T* q = static_cast<const T*>(a.q);
-  const T* k = static_cast<const T*>(a.k);
-  T* qr = static_cast<T*>(a.qr);
-  T* kr = static_cast<T*>(a.kr);
+  // the rotated copies are workspace buffers, never the inputs: with the
+  // pointers marked so, the loads of several heads are in flight together
+  const T* __restrict__ q = static_cast<const T*>(a.q);
+  const T* __restrict__ k = static_cast<const T*>(a.k);
+  T* __restrict__ qr = static_cast<T*>(a.qr);
+  T* __restrict__ kr = static_cast<T*>(a.kr);
   const int BH = a.B * a.H;
+#pragma unroll 4
   for (int bh = blockIdx.y; bh < BH; bh += gridDim.y) {
     const int b = bh / a.H, h = bh - b * a.H;
     const long long row = (long long)bh * a.L + t;
