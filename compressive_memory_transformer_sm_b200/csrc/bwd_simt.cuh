@@ -221,6 +221,10 @@ __global__ void __launch_bounds__(256) bwd_state_kernel(float* __restrict__ runn
                                                         const float* __restrict__ upart, int dk, int dv, int S, int op,
                                                         int s, int G, int Gu, float* __restrict__ gsnap,
                                                         float* __restrict__ out0, float* __restrict__ out0z) {
+  // as a programmatic dependent (the delta rule's reverse steps), nothing the
+  // previous kernel reads or writes is touched before it has completed
+  griddep_launch_dependents();
+  griddep_wait();
   const int bh = blockIdx.y;
   const int e = blockIdx.x * 256 + threadIdx.x;
   const int E = dk * dv;

@@ -1066,12 +1066,36 @@ int run_backward(const infini_attn_bwd_params& p, const BwdPlan& bp, char* ws) {
       bwd_state_kernel<<<sgrid, 256, 0, st>>>(gst, p.dM_S, p.dz_S, nullptr, nullptr, dk, dv, f.S, 2, 0, bp.Gc, 0,
                                               nullptr, nullptr, nullptr);
     }
+    // the reverse steps' launches as programmatic dependents of the one
+    // before (each waits for it before touching memory): their launch
+    // latency overlaps the previous kernel's tail
+    auto dependent = [&](auto kernel, dim3 grid, unsigned block, size_t smem, auto... args) {
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[0].val.programmaticStreamSerializationAllowed = 1;
+      cfg.gridDim = grid;
+      cfg.blockDim = dim3(block);
+      cfg.dynamicSmemBytes = smem;
+      cfg.stream = st;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+      if (e != cudaSuccess) {
+        cudaGetLastError();
+        note_cuda_error(e);
+      }
+      return e == cudaSuccess;
+    };
     for (int s = f.S - 1; s >= 0; --s) {
       if (bp.tc) {
         LaunchScope ls(kPhaseBwdMemTc, st);
-        tc::bwd_upd_tc_kernel<<<(unsigned)((long long)BH * bps), tc::kUpThreads, tc::kUpSmem, st>>>(
-            reinterpret_cast<const __nv_bfloat16*>(k), reinterpret_cast<const __nv_bfloat16*>(v), p.B, p.H, f.S, p.N,
-            p.L, s, gst, 0, (long long)pst, snapM, snapz, dkupd, dvupd, dnumr, ddenr, bps);
+        if (!dependent(tc::bwd_upd_tc_kernel, dim3((unsigned)((long long)BH * bps)), (unsigned)tc::kUpThreads,
+                       (size_t)tc::kUpSmem, reinterpret_cast<const __nv_bfloat16*>(k),
+                       reinterpret_cast<const __nv_bfloat16*>(v), p.B, p.H, f.S, p.N, p.L, s,
+                       static_cast<const float*>(gst), 0LL, (long long)pst, snapM, snapz, dkupd, dvupd, dnumr, ddenr,
+                       bps))
+          return INFINI_ERR_LAUNCH;
       } else {
         LaunchScope ls(kPhaseBwd, st);
         bwd_upd_kernel<T><<<(unsigned)((long long)BH * bps64), 256, upd_smem, st>>>(
@@ -1079,16 +1103,27 @@ int run_backward(const infini_attn_bwd_params& p, const BwdPlan& bp, char* ws) {
       }
       if (bp.tc) {
         LaunchScope ls(kPhaseBwdMemTc, st);
-        tc::bwd_outer_tc_kernel<<<(unsigned)((long long)BH * bp.Gu), tc::kOtThreads, tc::kOtSmem, st>>>(
-            reinterpret_cast<const __nv_bfloat16*>(k), dnumr, ddenr, p.N, p.L, s, 1, bp.Gu, bp.cpbu, upart);
+        if (!dependent(tc::bwd_outer_tc_kernel, dim3((unsigned)((long long)BH * bp.Gu)), (unsigned)tc::kOtThreads,
+                       (size_t)tc::kOtSmem, reinterpret_cast<const __nv_bfloat16*>(k),
+                       static_cast<const float*>(dnumr), static_cast<const float*>(ddenr), p.N, p.L, s, 1, bp.Gu,
+                       bp.cpbu, upart))
+          return INFINI_ERR_LAUNCH;
       } else {
         LaunchScope ls(kPhaseBwd, st);
         bwd_outer_kernel<T><<<(unsigned)((long long)BH * bp.Gu), 256, outer_smem, st>>>(k, dnumr, ddenr, g, dv, s, 1,
                                                                                        bp.Gu, bp.cpbu, upart);
       }
       LaunchScope ls(kPhaseBwd, st);
-      bwd_state_kernel<<<sgrid, 256, 0, st>>>(gst, nullptr, nullptr, cpart, upart, dk, dv, f.S, 1, s, bp.Gc, bp.Gu,
-                                              nullptr, nullptr, nullptr);
+      if (bp.tc) {
+        if (!dependent(bwd_state_kernel, sgrid, 256u, (size_t)0, gst, static_cast<const float*>(nullptr),
+                       static_cast<const float*>(nullptr), static_cast<const float*>(cpart),
+                       static_cast<const float*>(upart), dk, dv, f.S, 1, s, bp.Gc, bp.Gu, static_cast<float*>(nullptr),
+                       static_cast<float*>(nullptr), static_cast<float*>(nullptr)))
+          return INFINI_ERR_LAUNCH;
+      } else {
+        bwd_state_kernel<<<sgrid, 256, 0, st>>>(gst, nullptr, nullptr, cpart, upart, dk, dv, f.S, 1, s, bp.Gc, bp.Gu,
+                                                nullptr, nullptr, nullptr);
+      }
     }
     LaunchScope ls(kPhaseBwd, st);
     bwd_state_kernel<<<sgrid, 256, 0, st>>>(gst, nullptr, nullptr, nullptr, nullptr, dk, dv, f.S, 3, 0, 0, 0, nullptr,

@@ -307,6 +307,10 @@ __global__ void __launch_bounds__(kUpThreads, 1)
   uint8_t* gbase = smem_raw + (base - raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const bool delta = snapM != nullptr;
+  // as a programmatic dependent (the delta rule's reverse steps), nothing the
+  // previous kernel reads or writes is touched before it has completed
+  griddep_launch_dependents();
+  griddep_wait();
   int idx = blockIdx.x;
   const int blk = idx % blocks_per_seg;
   idx /= blocks_per_seg;
@@ -600,6 +604,10 @@ __global__ void __launch_bounds__(kOtThreads, 1)
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // as a programmatic dependent (the delta rule's reverse steps), nothing the
+  // previous kernel reads or writes is touched before it has completed
+  griddep_launch_dependents();
+  griddep_wait();
   int idx = blockIdx.x;
   const int grp = idx % G;
   idx /= G;
